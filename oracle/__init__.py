@@ -1,0 +1,117 @@
+"""fp64 CPU oracle for the selective state-space scan (S6).
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, by the smoke check in
+__graft_entry__.py and by the cpu_baseline / reference leg of bench.py, and by
+nothing in the product package.  It shares no code with the CUDA library.
+
+The arithmetic lives in ``ssm_oracle.c`` (plain C, fp64, OpenMP over the
+independent (batch, channel) rows); this module only compiles it with gcc and
+marshals numpy arrays to it.  Every array is converted to contiguous float64
+first, so bf16 / fp32 inputs enter the oracle exactly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ssm_oracle.c")
+_LIB = os.path.join(_HERE, "libssm_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (-O2, no fast-math, OpenMP); returns the .so path."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            i64, vp, ci = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
+            lib.oracle_selective_scan_f64.argtypes = [vp] * 8 + [ci, vp, vp, vp, i64, i64, i64, i64]
+            lib.oracle_selective_scan_f64.restype = ci
+            lib.oracle_state_update_f64.argtypes = [vp] * 9 + [ci, vp, i64, i64, i64]
+            lib.oracle_state_update_f64.restype = ci
+            lib.oracle_num_threads.restype = ci
+            lib.oracle_softplus_f64.argtypes = [ctypes.c_double]
+            lib.oracle_softplus_f64.restype = ctypes.c_double
+            lib.oracle_silu_f64.argtypes = [ctypes.c_double]
+            lib.oracle_silu_f64.restype = ctypes.c_double
+            _lib = lib
+    return _lib
+
+
+def _f64(a):
+    if a is None:
+        return None
+    if hasattr(a, "detach"):  # torch tensor -> numpy, exact upcast
+        a = a.detach().to("cpu")
+        import torch
+        a = a.to(torch.float64).numpy()
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def softplus(x: float) -> float:
+    return float(_load().oracle_softplus_f64(float(x)))
+
+
+def silu(x: float) -> float:
+    return float(_load().oracle_silu_f64(float(x)))
+
+
+def selective_scan(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True, h0=None):
+    """Forward scan.  Shapes: u/delta/z (b, d, L); B/C (b, N, L); A (d, N); D/delta_bias (d);
+    h0 (b, d, N) or None.  Returns (y (b, d, L), last_state (b, d, N)) as float64 arrays."""
+    u, delta, A, B, C = map(_f64, (u, delta, A, B, C))
+    D, z, delta_bias, h0 = map(_f64, (D, z, delta_bias, h0))
+    b, d, L = u.shape
+    n = A.shape[1]
+    assert delta.shape == u.shape and A.shape == (d, n) and B.shape == (b, n, L) and C.shape == (b, n, L)
+    assert z is None or z.shape == u.shape
+    assert h0 is None or h0.shape == (b, d, n)
+    y = np.empty((b, d, L), dtype=np.float64)
+    last = np.empty((b, d, n), dtype=np.float64)
+    rc = _load().oracle_selective_scan_f64(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                           _ptr(z), _ptr(delta_bias), int(bool(softplus)), _ptr(h0),
+                                           _ptr(y), _ptr(last), b, d, n, L)
+    if rc != 0:
+        raise ValueError("oracle_selective_scan_f64 rejected its arguments")
+    return y, last
+
+
+def state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True):
+    """One decode step.  state (b, d, N) is NOT modified; returns (y (b, d), new_state)."""
+    st = _f64(state).copy()
+    u, delta, A, B, C = map(_f64, (u, delta, A, B, C))
+    D, z, delta_bias = map(_f64, (D, z, delta_bias))
+    b, d, n = st.shape
+    assert u.shape == (b, d) and delta.shape == (b, d) and A.shape == (d, n)
+    assert B.shape == (b, n) and C.shape == (b, n)
+    y = np.empty((b, d), dtype=np.float64)
+    rc = _load().oracle_state_update_f64(_ptr(st), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
+                                         _ptr(D), _ptr(z), _ptr(delta_bias), int(bool(softplus)),
+                                         _ptr(y), b, d, n)
+    if rc != 0:
+        raise ValueError("oracle_state_update_f64 rejected its arguments")
+    return y, st

@@ -1,0 +1,19 @@
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a); run with -m gpu")
+
+
+@pytest.fixture(scope="session")
+def cuda_device():
+    import torch
+    assert torch.cuda.is_available(), "GPU test collected on a machine without CUDA"
+    return torch.device("cuda:0")

@@ -1,0 +1,335 @@
+"""Pins for the fp64 oracle: each checks it against something other than itself
+(hand-derived worked examples, closed forms, library routines, brute force), so
+that a dropped term, a wrong sign or index, or a transposed operand fails here.
+
+Pages cited (sections as printed):
+  [Eng]  "Mamba 选择性状态空间模型：亚二次复杂度大语言模型推理工程实践"
+  [Hist] "AI底层架构的一场革命：Mamba如何用「状态压缩」挑战Transformer的十年统治"
+  [Card] "Mamba与SSM状态空间模型：一张摘要卡读完万页档案"
+  [S4M]  "State Space Models 深度实战：从 S4 到 Mamba 的架构演进与 CUDA 优化"
+  [Tech] "Transformer架构遭遇颠覆性突破：Mamba模型如何用状态空间重新定义序列建模效率？"
+"""
+import glob
+import math
+import os
+import random
+
+import numpy as np
+import pytest
+import scipy.special
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _selective_case(rng, b=2, d=3, n=4, L=17, softplus=True, with_z=True, with_D=True, with_bias=True):
+    """Fully time-varying inputs; A varies in both d and n (d != n) so that a transposed
+    A index cannot pass."""
+    u = rng.standard_normal((b, d, L))
+    delta = 0.5 * rng.standard_normal((b, d, L))
+    A = -rng.uniform(0.1, 2.0, (d, n))
+    B = rng.standard_normal((b, n, L))
+    C = rng.standard_normal((b, n, L))
+    D = rng.standard_normal(d) if with_D else None
+    z = rng.standard_normal((b, d, L)) if with_z else None
+    bias = rng.uniform(-3, 0.5, d) if with_bias else None
+    return dict(u=u, delta=delta, A=A, B=B, C=C, D=D, z=z, delta_bias=bias, softplus=softplus)
+
+
+def _step_sizes(case):
+    x = case["delta"] + (0 if case["delta_bias"] is None else case["delta_bias"][None, :, None])
+    return np.logaddexp(0.0, x) if case["softplus"] else x
+
+
+# ---------------------------------------------------------------------------------------------
+# Worked examples derived by hand (tests/golden/*.txt, each with its citation)
+# ---------------------------------------------------------------------------------------------
+def _parse_golden(path):
+    out = {}
+    with open(path) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if not line:
+                continue
+            k, v = line.split(":", 1)
+            v = v.split()
+            out[k.strip()] = v[0] if k.strip() == "kind" else [float(x) for x in v]
+    return out
+
+
+@pytest.mark.parametrize("path", sorted(glob.glob(os.path.join(GOLDEN, "worked_*.txt"))),
+                         ids=lambda p: os.path.basename(p))
+def test_worked_examples(path):
+    g = _parse_golden(path)
+    n = int(g["dstate"][0])
+    sp = bool(g["softplus"][0])
+    A = np.array(g["A"]).reshape(1, n)
+    D = np.array(g["D"]) if "D" in g else None
+    bias = np.array(g["bias"]) if "bias" in g else None
+    if g["kind"] == "scan":
+        L = int(g["L"][0])
+        u = np.array(g["u"]).reshape(1, 1, L)
+        delta = np.array(g["delta"]).reshape(1, 1, L)
+        B = np.array([g[f"B{i}"] for i in range(n)]).reshape(1, n, L)
+        C = np.array([g[f"C{i}"] for i in range(n)]).reshape(1, n, L)
+        z = np.array(g["z"]).reshape(1, 1, L) if "z" in g else None
+        y, last = oracle.selective_scan(u, delta, A, B, C, D=D, z=z, delta_bias=bias, softplus=sp)
+        np.testing.assert_allclose(y.ravel(), g["y"], rtol=1e-14, atol=1e-14)
+        np.testing.assert_allclose(last.ravel(), g["last_state"], rtol=1e-14, atol=1e-14)
+    else:
+        st = np.array(g["state"]).reshape(1, 1, n)
+        y, new = oracle.state_update(st, np.array(g["u"]).reshape(1, 1), np.array(g["delta"]).reshape(1, 1),
+                                     A, np.array(g["B"]).reshape(1, n), np.array(g["C"]).reshape(1, n),
+                                     D=D, delta_bias=bias, softplus=sp)
+        np.testing.assert_allclose(y.ravel(), g["y"], rtol=1e-14)
+        np.testing.assert_allclose(new.ravel(), g["last_state"], rtol=1e-14)
+
+
+# ---------------------------------------------------------------------------------------------
+# Elementwise helpers against library routines
+# ---------------------------------------------------------------------------------------------
+def test_softplus_matches_logaddexp():
+    # softplus(x) = log(1 + e^x) = logaddexp(0, x)   ([Card] 选择性机制: Delta = Softplus(.))
+    xs = [-745.0, -200.0, -40.0, -20.0, -5.0, -1e-3, 0.0, 1e-8, 0.3, 5.0, 20.0, 40.0, 200.0, 700.0]
+    for x in xs:
+        assert oracle.softplus(x) == pytest.approx(float(np.logaddexp(0.0, x)), rel=1e-15, abs=1e-300)
+
+
+def test_silu_matches_expit():
+    # silu(z) = z * sigmoid(z)   ([Hist] Mamba Block 数据流)
+    for zv in [-700.0, -30.0, -2.5, -1e-6, 0.0, 1e-6, 0.7, 3.0, 30.0, 700.0]:
+        assert oracle.silu(zv) == pytest.approx(zv * float(scipy.special.expit(zv)), rel=1e-14, abs=1e-300)
+
+
+# ---------------------------------------------------------------------------------------------
+# P-A: A = 0 and constant Delta, B, C  =>  scaled prefix sum  ([Card] 离散化变换 / 线性扫描算法)
+# ---------------------------------------------------------------------------------------------
+def test_prefix_sum_when_A_is_zero():
+    rng = _rng(1)
+    b, d, n, L = 2, 3, 5, 300
+    u = rng.standard_normal((b, d, L))
+    c = 0.37
+    delta = np.full((b, d, L), c)
+    Bv = rng.standard_normal((b, n))
+    Cv = rng.standard_normal((b, n))
+    B = np.repeat(Bv[:, :, None], L, axis=2)
+    C = np.repeat(Cv[:, :, None], L, axis=2)
+    D = rng.standard_normal(d)
+    A = np.zeros((d, n))
+    y, last = oracle.selective_scan(u, delta, A, B, C, D=D, softplus=False)
+    cb = (Cv * Bv).sum(axis=1)  # (b,)
+    expect = c * cb[:, None, None] * np.cumsum(u, axis=2) + D[None, :, None] * u
+    np.testing.assert_allclose(y, expect, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(last, c * Bv[:, None, :] * u.sum(axis=2)[:, :, None], rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------------------------
+# P-B: LTI case  =>  y = K * u + D u,  K_j = sum_n C_n Abar_n^j Bbar_n
+#      ([Eng] §2.3; [S4M] 2.1; [Tech] 二.3 with kernel length L)
+# ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("L", [1, 64, 1000, 4096])
+def test_lti_equals_convolution(L):
+    rng = _rng(2 + L)
+    d, n = 3, 16
+    u = rng.standard_normal((1, d, L))
+    dt = np.array([0.003, 0.02, 0.15])
+    delta = np.repeat(dt[None, :, None], L, axis=2)
+    A = -np.arange(1, n + 1, dtype=np.float64)[None, :] * rng.uniform(0.5, 1.5, (d, 1))
+    Bv, Cv = rng.standard_normal(n), rng.standard_normal(n)
+    B = np.repeat(Bv[None, :, None], L, axis=2)
+    C = np.repeat(Cv[None, :, None], L, axis=2)
+    D = rng.standard_normal(d)
+    y, _ = oracle.selective_scan(u, delta, A, B, C, D=D, softplus=False)
+    j = np.arange(L)
+    for di in range(d):
+        abar = np.exp(dt[di] * A[di])                       # (n,)
+        K = (Cv[None, :] * abar[None, :] ** j[:, None] * (dt[di] * Bv)[None, :]).sum(axis=1)
+        direct = np.convolve(u[0, di], K)[:L]
+        m = 1 << (2 * L - 1).bit_length()
+        viafft = np.fft.irfft(np.fft.rfft(u[0, di], m) * np.fft.rfft(K, m), m)[:L]
+        np.testing.assert_allclose(y[0, di], direct + D[di] * u[0, di], rtol=1e-10, atol=1e-10)
+        np.testing.assert_allclose(y[0, di], viafft + D[di] * u[0, di], rtol=1e-9, atol=1e-9)
+
+
+# ---------------------------------------------------------------------------------------------
+# P-C / P-D: brute-force closed form  h_t = sum_{s<=t} (prod_{r=s+1..t} Abar_r) Bbar_s u_s,
+#            y_t = C_t h_t  ([Card] Mamba架构设计 closed form, with the C_t read-out)
+# ---------------------------------------------------------------------------------------------
+def _brute_force(case):
+    u, A, B, C = case["u"], case["A"], case["B"], case["C"]
+    b, d, L = u.shape
+    n = A.shape[1]
+    dt = _step_sizes(case)
+    y = np.zeros((b, d, L))
+    hL = np.zeros((b, d, n))
+    for bi in range(b):
+        for di in range(d):
+            abar = np.exp(dt[bi, di][:, None] * A[di][None, :])       # (L, n)
+            for t in range(L):
+                h = np.zeros(n)
+                for s in range(t + 1):
+                    decay = np.prod(abar[s + 1:t + 1], axis=0) if s < t else np.ones(n)
+                    h += decay * dt[bi, di, s] * B[bi, :, s] * u[bi, di, s]
+                yt = float(C[bi, :, t] @ h)
+                if case["D"] is not None:
+                    yt += case["D"][di] * u[bi, di, t]
+                if case["z"] is not None:
+                    zt = case["z"][bi, di, t]
+                    yt *= zt * scipy.special.expit(zt)
+                y[bi, di, t] = yt
+                if t == L - 1:
+                    hL[bi, di] = h
+    return y, hL
+
+
+@pytest.mark.parametrize("flags", [dict(), dict(with_z=False), dict(with_D=False, with_z=False, with_bias=False),
+                                   dict(softplus=False, with_bias=False)],
+                         ids=["full", "no_gate", "bare", "no_softplus"])
+def test_brute_force_closed_form(flags):
+    rng = _rng(3)
+    case = _selective_case(rng, **flags)
+    y, last = oracle.selective_scan(**case)
+    y_bf, h_bf = _brute_force(case)
+    np.testing.assert_allclose(y, y_bf, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(last, h_bf, rtol=1e-11, atol=1e-12)
+
+
+def test_initial_state_enters_as_decayed_carry():
+    # h_t = (prod_{r<=t} Abar_r) h_init + (zero-start scan)_t: the state continuation of [Eng] §7.2.
+    rng = _rng(4)
+    case = _selective_case(rng, with_z=False, with_D=False)
+    b, d, L = case["u"].shape
+    n = case["A"].shape[1]
+    h0 = rng.standard_normal((b, d, n))
+    y0, last0 = oracle.selective_scan(**case)
+    y1, last1 = oracle.selective_scan(**case, h0=h0)
+    dt = _step_sizes(case)
+    P = np.exp(np.cumsum(dt, axis=2)[:, :, :, None] * case["A"][None, :, None, :])  # (b,d,L,n)
+    extra_y = np.einsum("bdtn,bnt,bdn->bdt", P, case["C"], h0)
+    np.testing.assert_allclose(y1, y0 + extra_y, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(last1, last0 + P[:, :, -1, :] * h0, rtol=1e-11, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------------------------
+# P-E: two-step identity with constant Abar  ([Card] 线性扫描算法)
+# ---------------------------------------------------------------------------------------------
+def test_two_step_identity():
+    rng = _rng(5)
+    b, d, n = 2, 3, 4
+    A = -rng.uniform(0.1, 2.0, (d, n))
+    h0 = rng.standard_normal((b, d, n))
+    dt = 0.3
+    delta = np.full((b, d), dt)
+    x1, x2 = rng.standard_normal((b, d)), rng.standard_normal((b, d))
+    B1, B2 = rng.standard_normal((b, n)), rng.standard_normal((b, n))
+    C1 = rng.standard_normal((b, n))
+    _, h1 = oracle.state_update(h0, x1, delta, A, B1, C1, softplus=False)
+    _, h2 = oracle.state_update(h1, x2, delta, A, B2, C1, softplus=False)
+    abar = np.exp(dt * A)[None]
+    expect = abar ** 2 * h0 + abar * (dt * B1[:, None, :]) * x1[..., None] + (dt * B2[:, None, :]) * x2[..., None]
+    np.testing.assert_allclose(h2, expect, rtol=1e-13, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------------------------
+# P-F: the associative pair operator (a1,b1) (x) (a2,b2) = (a2 a1, a2 b1 + b2)  ([Eng] §4.1)
+#      folded under random bracketings equals the sequential recurrence's final state.
+# ---------------------------------------------------------------------------------------------
+def _combine(p, q):
+    return (q[0] * p[0], q[0] * p[1] + q[1])
+
+
+def _random_tree_fold(pairs, rnd):
+    items = list(pairs)
+    while len(items) > 1:
+        i = rnd.randrange(len(items) - 1)
+        items[i:i + 2] = [_combine(items[i], items[i + 1])]
+    return items[0]
+
+
+def test_pair_operator_bracketings_match_scan():
+    rng = _rng(6)
+    case = _selective_case(rng, b=1, d=2, n=4, L=41, with_z=False, with_D=False)
+    _, last = oracle.selective_scan(**case)
+    dt = _step_sizes(case)
+    rnd = random.Random(7)
+    for di in range(2):
+        a = np.exp(dt[0, di][:, None] * case["A"][di][None, :])                  # (L, n)
+        bb = dt[0, di][:, None] * case["B"][0].T * case["u"][0, di][:, None]     # (L, n)
+        pairs = [(a[t], bb[t]) for t in range(41)]
+        for _ in range(5):
+            P, H = _random_tree_fold(pairs, rnd)
+            np.testing.assert_allclose(H, last[0, di], rtol=1e-12, atol=1e-13)
+            np.testing.assert_allclose(P, np.exp(dt[0, di].sum() * case["A"][di]), rtol=1e-12)
+
+
+# ---------------------------------------------------------------------------------------------
+# P-G: L chained decode steps from zero state equal the forward scan  ([Card] 线性扫描算法;
+#      [Eng] §6.2 incremental one-step recurrence)
+# ---------------------------------------------------------------------------------------------
+def test_decode_chain_equals_scan():
+    rng = _rng(8)
+    case = _selective_case(rng, b=2, d=3, n=16, L=25)
+    y, last = oracle.selective_scan(**case)
+    b, d, L = case["u"].shape
+    st = np.zeros((b, d, 16))
+    for t in range(L):
+        yt, st = oracle.state_update(st, case["u"][:, :, t], case["delta"][:, :, t], case["A"],
+                                     case["B"][:, :, t], case["C"][:, :, t], D=case["D"],
+                                     z=case["z"][:, :, t], delta_bias=case["delta_bias"], softplus=True)
+        np.testing.assert_allclose(yt, y[:, :, t], rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(st, last, rtol=1e-13, atol=1e-14)
+
+
+# ---------------------------------------------------------------------------------------------
+# P-H: limits  ([Eng] §3.2; [Card] 离散化变换 / 选择性机制)
+# ---------------------------------------------------------------------------------------------
+def test_small_delta_freezes_state():
+    rng = _rng(9)
+    b, d, n = 2, 3, 8
+    A = -rng.uniform(0.1, 2.0, (d, n))
+    h0 = rng.standard_normal((b, d, n))
+    delta = np.full((b, d), -60.0)  # softplus(-60) ~ 8.8e-27
+    x = rng.standard_normal((b, d))
+    Bv, Cv = rng.standard_normal((b, n)), rng.standard_normal((b, n))
+    y, h1 = oracle.state_update(h0, x, delta, A, Bv, Cv, softplus=True)
+    np.testing.assert_allclose(h1, h0, rtol=1e-20, atol=1e-24)
+    np.testing.assert_allclose(y, np.einsum("bn,bdn->bd", Cv, h0), rtol=1e-14)
+
+
+def test_large_delta_resets_state():
+    rng = _rng(10)
+    case = _selective_case(rng, b=1, d=2, n=4, L=30, softplus=False, with_bias=False, with_z=False)
+    case["delta"] = np.full_like(case["delta"], 60.0)
+    case["A"] = -np.abs(case["A"]) - 1.0  # Abar <= e^-60
+    y, _ = oracle.selective_scan(**case)
+    expect = 60.0 * np.einsum("bnt,bnt,bdt->bdt", case["C"], case["B"], case["u"]) + case["D"][None, :, None] * case["u"]
+    np.testing.assert_allclose(y, expect, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------------------------
+# P-I: epilogue special cases  ([Eng] §2.2 D skip; [Hist] Mamba Block gate)
+# ---------------------------------------------------------------------------------------------
+def test_zero_B_gives_gated_skip():
+    rng = _rng(11)
+    case = _selective_case(rng, b=2, d=3, n=16, L=50)
+    case["B"] = np.zeros_like(case["B"])
+    case["D"] = np.ones(3)
+    y, last = oracle.selective_scan(**case)
+    z = case["z"]
+    np.testing.assert_allclose(y, case["u"] * z * scipy.special.expit(z), rtol=1e-14, atol=1e-300)
+    assert np.all(last == 0.0)
+
+
+def test_empty_and_degenerate_shapes():
+    rng = _rng(12)
+    case = _selective_case(rng, b=1, d=2, n=3, L=0)
+    y, last = oracle.selective_scan(**case)
+    assert y.shape == (1, 2, 0) and np.all(last == 0.0)
+    case = _selective_case(rng, b=0, d=2, n=3, L=5)
+    y, last = oracle.selective_scan(**case)
+    assert y.shape == (0, 2, 5)
