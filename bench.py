@@ -1,0 +1,456 @@
+#!/usr/bin/env python
+"""Benchmark of the selective scan (S6) on B200: Gelem/s (B*D*L per second).
+
+A step is one forward scan (the whole hot path: B/C staging, step sizes,
+discretisation, scan, output contraction, D skip, silu gate, final state) over the
+Mamba-2.8B-shaped layer workload (batch 4, d_inner 5120, d_state 16, L 2048, bf16
+I/O, fp32 state), inputs resident in HBM.  Inputs are synthetic and seeded.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+One JSON line is printed by rank 0.  With N > 1 (torchrun, one rank per GPU) every
+rank scans its own batch (independent sequences, no collective on the data path):
+weak scaling, value = elements of all ranks / max-over-ranks time.
+`--impl reference` times the fp64 CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import faulthandler
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "selective-scan Gelem/s (B*D*L per second), 1xB200"
+UNIT = "Gelem/s"
+SM_COUNT_NOMINAL = 148
+MUFU_EX2_PER_CLK_PER_SM = 16     # special-function unit lanes per SM per clock
+EXPS_PER_ELEMENT = 16            # exp(Delta*A[d,n]) for n = 0..15 per (b, d, t)
+SM_MAX_MHZ_FALLBACK = 1965.0
+HBM_GBS_FALLBACK = 6650.0
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return dict(hbm_gbs=float(j["hbm_gbs"]), sm_max_mhz=float(j.get("sm_max_mhz", SM_MAX_MHZ_FALLBACK)),
+                    source="measured")
+    return dict(hbm_gbs=HBM_GBS_FALLBACK, sm_max_mhz=SM_MAX_MHZ_FALLBACK, source="fallback")
+
+
+def scan_algorithmic_bytes(w: workloads.Workload) -> int:
+    """Bytes the method must move once: u, delta, z read and y written ((b,d,L) each),
+    B and C read ((b,16,L) each), final state written ((b,d,16) fp32), A/D/bias read."""
+    e = 2 if w.io == "bf16" else 4
+    bdl = w.batch * w.dim * w.seqlen
+    return (4 * bdl * e + 2 * w.batch * w.dstate * w.seqlen * e + w.batch * w.dim * w.dstate * 4
+            + w.dim * w.dstate * 4 + 2 * w.dim * 4)
+
+
+def decode_algorithmic_bytes(w: workloads.Workload) -> int:
+    """Per decode step: fp32 state read + written, u/delta/z read, y written ((b,d) each),
+    B/C read ((b,16) each), A/D/bias read."""
+    e = 2 if w.io == "bf16" else 4
+    bd = w.batch * w.dim
+    return (2 * bd * w.dstate * 4 + 4 * bd * e + 2 * w.batch * w.dstate * e + w.dim * w.dstate * 4 + 2 * w.dim * 4)
+
+
+# ----------------------------------------------------------------------------- clocks (NVML)
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML while the timed region runs."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            props = torch.cuda.get_device_properties(device_index)
+            dom, bus, devn = (getattr(props, k, None) for k in ("pci_domain_id", "pci_bus_id", "pci_device_id"))
+            if all(isinstance(v, int) for v in (dom, bus, devn)):
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(f"{dom:08X}:{bus:02X}:{devn:02X}.0".encode())
+            else:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._h = None
+
+    def _sample(self):
+        nv = self._nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+        try:
+            mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+        except Exception:
+            mask = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+        for bit, name in self.REASONS.items():
+            if mask & bit:
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                return
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+            if not self.samples:
+                self._sample()
+
+    def summary(self):
+        if self._h is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- distributed plumbing
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- measurements
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "selective_state_space_16_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_record(kernel: str, workload: str):
+    """dram bytes per launch from the committed ncu summary, if it was taken on the
+    current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        recs = json.load(f)
+    for r in recs:
+        if r.get("kernel") == kernel and r.get("workload") == workload and r.get("src_sha") == kernel_source_hash():
+            return r.get("dram_bytes_per_launch")
+    return None
+
+
+def time_forward(ssm, g, ws, steps, warmup, world, stream, clocks=None):
+    def call():
+        ssm.ssm_selective_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"],
+                                   True, g["y"], g["last"], ws, stream=stream)
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            call()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ctx = clocks if clocks is not None else _Null()
+    with ctx:
+        ev0.record(stream)
+        for _ in range(steps):
+            call()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    return ev0.elapsed_time(ev1) / 1e3  # seconds
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def forward_buffers(w, dev):
+    inp = workloads.workload_inputs(w)
+    g = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+    g["y"] = torch.empty_like(g["u"])
+    g["last"] = torch.empty(w.batch, w.dim, w.dstate, dtype=torch.float32, device=dev)
+    return inp, g
+
+
+def e2e_forward(ssm, w, inp, ws, steps, stream):
+    """Same metric through the public C-ABI call with HOST (pinned) buffers: every step
+    copies the inputs host->device, runs the scan and copies y and the final state back."""
+    names = ["u", "delta", "z", "B", "C", "A", "D", "delta_bias"]
+    host = {k: inp[k].pin_memory() for k in names}
+    dev = {k: torch.empty_like(host[k], device="cuda") for k in names}
+    y_d = torch.empty_like(dev["u"])
+    last_d = torch.empty(w.batch, w.dim, w.dstate, dtype=torch.float32, device="cuda")
+    y_h = torch.empty_like(host["u"]).pin_memory()
+    last_h = torch.empty(last_d.shape, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = y_h.numel() * y_h.element_size() + last_h.numel() * 4
+
+    def step():
+        for k in names:
+            dev[k].copy_(host[k], non_blocking=True)
+        ssm.ssm_selective_scan_fwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], dev["D"], dev["z"],
+                                   dev["delta_bias"], True, y_d, last_d, ws, stream=stream)
+        y_h.copy_(y_d, non_blocking=True)
+        last_h.copy_(last_d, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        step()
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(steps):
+            step()
+        ev1.record(stream)
+    torch.cuda.synchronize()
+    t = ev0.elapsed_time(ev1) / 1e3
+    return {"value": w.elements * steps / t / 1e9, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": steps}
+
+
+def measure_long(ssm, stream, steps=10):
+    w = workloads.WORKLOADS[3]
+    _, g = forward_buffers(w, "cuda")
+    ws = ssm.new_workspace(w.batch, w.dim, w.dstate, w.seqlen)
+    t = time_forward(ssm, g, ws, steps, 3, 1, stream)
+    ms = t / steps * 1e3
+    del g
+    return {"workload": w.name, "value": w.elements / (ms / 1e3) / 1e9, "unit": UNIT, "ms_per_step": ms,
+            "mufu_frac_of_nominal": None}
+
+
+def measure_decode(ssm, stream, pk):
+    w = workloads.WORKLOADS[4]
+    dec = workloads.workload_decode_inputs(w)
+    A, D, bias = dec["A"].cuda(), dec["D"].cuda(), dec["delta_bias"].cuda()
+    sets = [{k: v.cuda() for k, v in s.items()} for s in dec["sets"]]
+    state = dec["state0"].cuda()
+    y = torch.empty(w.batch, w.dim, dtype=torch.bfloat16, device="cuda")
+
+    def chain(n):
+        for i in range(n):
+            s = sets[i % workloads.POOL]
+            ssm.ssm_state_update(state, s["u"], s["delta"], A, s["B"], s["C"], D, s["z"], bias, True, y,
+                                 stream=stream)
+
+    with torch.cuda.stream(stream):
+        chain(20)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        chain(w.decode_steps)
+    with torch.cuda.stream(stream):  # replay() launches on the current stream
+        graph.replay()
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        graph.replay()
+        ev1.record(stream)
+    torch.cuda.synchronize()
+    t = ev0.elapsed_time(ev1) / 1e3
+    per_step = t / w.decode_steps
+    gbs = decode_algorithmic_bytes(w) / per_step / 1e9
+    del graph
+    return {"workload": w.name, "value": w.batch * w.dim / per_step / 1e9, "unit": "Gelem/s (B*D per step)",
+            "us_per_step": per_step * 1e6, "steps": w.decode_steps, "launch": "one CUDA graph of 1000 steps",
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "note": "state is 84 MB < 126 MB L2: see ncu dram bytes"}}
+
+
+def cpu_oracle_rate(w, budget_s: float, channels_cap=None):
+    """Time the fp64 oracle on a bounded prefix of the workload's channels.
+    Returns (Gelem/s, seconds, channels, threads)."""
+    import oracle
+    inp = workloads.workload_inputs(w) if w.decode_steps == 0 else None
+    b0 = inp["u"][0]
+    sub = lambda c: dict(u=b0[:c][None], delta=inp["delta"][0][:c][None], A=inp["A"][:c], B=inp["B"][0][None],
+                         C=inp["C"][0][None], D=inp["D"][:c], z=inp["z"][0][:c][None],
+                         delta_bias=inp["delta_bias"][:c])
+    c = 16
+    t0 = time.perf_counter()
+    oracle.selective_scan(**sub(c))
+    t_cal = time.perf_counter() - t0
+    per_ch = t_cal / c
+    c = max(16, min(w.dim if channels_cap is None else channels_cap, int(budget_s / max(per_ch, 1e-9))))
+    args = sub(c)
+    t0 = time.perf_counter()
+    oracle.selective_scan(**args)
+    dt = time.perf_counter() - t0
+    return c * w.seqlen / dt / 1e9, dt, c, oracle.num_threads()
+
+
+# ----------------------------------------------------------------------------- arms
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    w = workloads.WORKLOADS[workloads.HEADLINE]
+    import oracle
+    oracle.build()
+    inp = workloads.workload_inputs(w)
+    budget_per_step = max(0.02, 90.0 / max(1, args.steps + args.warmup))
+    b0 = inp["u"][0]
+
+    def sample(c):
+        return dict(u=b0[:c][None], delta=inp["delta"][0][:c][None], A=inp["A"][:c], B=inp["B"][0][None],
+                    C=inp["C"][0][None], D=inp["D"][:c], z=inp["z"][0][:c][None], delta_bias=inp["delta_bias"][:c])
+    t0 = time.perf_counter()
+    oracle.selective_scan(**sample(8))
+    per_ch = (time.perf_counter() - t0) / 8
+    c = max(1, min(w.dim, int(budget_per_step / max(per_ch, 1e-9))))
+    s = sample(c)
+    for _ in range(args.warmup):
+        oracle.selective_scan(**s)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.selective_scan(**s)
+    dt = time.perf_counter() - t0
+    elems = c * w.seqlen * args.steps
+    val = elems / dt / 1e9
+    desc = f"{c} of {w.dim} channels of batch row 0, full L={w.seqlen}, per step"
+    line = {"metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+            "impl": "reference",
+            "config": {"workload": w.name, "batch": w.batch, "d_inner": w.dim, "d_state": w.dstate,
+                       "seq_len": w.seqlen, "io": w.io, "sample": desc},
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_gpu(args, world, rank, local):
+    import selective_state_space_16_b200 as ssm
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    pk = peaks()
+    w = workloads.WORKLOADS[workloads.HEADLINE]
+    inp, g = forward_buffers(w, dev)
+    ws = ssm.new_workspace(w.batch, w.dim, w.dstate, w.seqlen)
+    stream = torch.cuda.Stream()
+    clocks = ClockSampler(local)
+    t = time_forward(ssm, g, ws, args.steps, args.warmup, world, stream, clocks)
+    t = max_over_ranks(t, world)
+    per_call = t / args.steps
+    value = w.elements * world * args.steps / t / 1e9
+    assert ssm.ssm_read_status(ws) == 0
+
+    sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
+    ex2_peak = sm_count * MUFU_EX2_PER_CLK_PER_SM * pk["sm_max_mhz"] * 1e6 / 1e9  # G ex2 / s
+    achieved_ex2 = EXPS_PER_ELEMENT * w.elements / per_call / 1e9
+    hbm_achieved = scan_algorithmic_bytes(w) / per_call / 1e9
+    clk = clocks.summary()
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": t / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32 (bf16 I/O, fp32 state and arithmetic)",
+            "data": "synthetic (seeded)",
+            "config": {"workload": w.name, "batch": w.batch, "d_inner": w.dim, "d_state": w.dstate,
+                       "seq_len": w.seqlen, "io": w.io, "per_rank": "one full batch per GPU",
+                       "l2": "inputs larger than L2 (338 MB per step vs 126 MB L2)", "parallelism": f"dp{world}"},
+            "roofline": {"bound": "alu", "achieved": achieved_ex2, "peak": ex2_peak, "unit": "Gex2/s",
+                         "frac": achieved_ex2 / ex2_peak,
+                         "traffic": traffic_record("scan_fwd_seq_kernel", w.name),
+                         "peak_source": f"{sm_count} SMs x {MUFU_EX2_PER_CLK_PER_SM} ex2/clk x "
+                                        f"{pk['sm_max_mhz']:.0f} MHz ({pk['source']} max clock)",
+                         "timed": "whole C-ABI call (B/C pack + scan kernels) per launch"},
+            "roofline_hbm": {"achieved": hbm_achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                             "frac": hbm_achieved / pk["hbm_gbs"], "peak_source": pk["source"],
+                             "algorithmic_bytes_per_step": scan_algorithmic_bytes(w)},
+            "clocks": clk,
+            "gpu_launches": 2 * args.steps}
+    if rank == 0:
+        e2e_steps = max(3, min(args.steps, 10))
+        line["e2e"] = e2e_forward(ssm, w, inp, ws, e2e_steps, stream)
+    if world == 1 and not args.skip_extra:
+        line["also"] = {"long": measure_long(ssm, stream), "decode": measure_decode(ssm, stream, pk)}
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        rate, secs, ch, cores = cpu_oracle_rate(w, args.cpu_budget)
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": f"{ch} of {w.dim} channels of batch row 0, full L={w.seqlen} "
+                                          f"({ch * w.seqlen} elements, {secs:.1f} s)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    faulthandler.enable()
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--skip-extra", action="store_true")
+    args = ap.parse_args()
+    world, rank, local = dist_setup(args.gpus) if args.impl == "native" else (
+        int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_gpu(args, world, rank, local)
+    finally:
+        if world > 1 and args.impl == "native":
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,154 @@
+/*
+ * ssm_scan.h -- C ABI of the B200 (sm_100a) selective state-space scan (S6) library.
+ *
+ * Sources (web pages on Mamba / selective state-space models; sections as printed):
+ *   [Eng]  "Mamba 选择性状态空间模型：亚二次复杂度大语言模型推理工程实践"
+ *          (www.ybb.press/ai-agent/15212.html)
+ *   [Hist] "AI底层架构的一场革命：Mamba如何用「状态压缩」挑战Transformer的十年统治"
+ *          (gitcode.csdn.net/6a278c3f662f9a54cb7b917b.html)
+ *   [Card] "Mamba与SSM状态空间模型：一张摘要卡读完万页档案"
+ *          (aiqz.cc/article/mamba-ssm-state-space-model.html)
+ *   [S4M]  "State Space Models 深度实战：从 S4 到 Mamba 的架构演进与 CUDA 优化"
+ *          (www.ybb.press/ai-applications/10137.html)
+ *
+ * The operation, for every batch row b and channel d (independent of each other):
+ *   Delta_t = softplus(delta[b,d,t] + delta_bias[d])          [Eng] §3.2, [Card] 选择性机制
+ *   h_t[n]  = exp(Delta_t*A[d,n]) * h_{t-1}[n] + Delta_t*B[b,n,t]*u[b,d,t]
+ *             (simplified discretisation Abar = exp(Delta A), Bbar = Delta B,
+ *              [Card] 离散化变换 and 选择性机制)
+ *   y_t     = (sum_n C[b,n,t]*h_t[n] + D[d]*u[b,d,t]) * silu(z[b,d,t])
+ *             ([Eng] §2.2 for C h + D x; [Hist] Mamba Block 数据流 for the SiLU gate)
+ *   h_{-1}  = 0; last_state = h_{L-1}                            [Eng] §4.2 and §7.2
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *     allocates no device memory and frees nothing.
+ *   - Layouts are dense row-major:  u, delta, z, y: (batch, dim, seqlen);
+ *     B, C: (batch, dstate, seqlen);  A: (dim, dstate) fp32;  D, delta_bias: (dim) fp32;
+ *     last_state / decode state: (batch, dim, dstate) fp32.
+ *   - io_dtype gives the element type of u, delta, z, B, C and y (fp32 or bf16).
+ *     A, D, delta_bias and the state are always fp32; arithmetic is fp32.
+ *   - Calls are asynchronous on `stream`; errors found before the launch are
+ *     returned; errors found on the device (a look-back wait that ran out) are
+ *     recorded in the workspace status word and read back by ssm_read_status().
+ *   - dstate must be 16 (SSM_ERR_UNSUPPORTED otherwise).
+ *   - Inputs are never modified, except `state` in ssm_state_update().
+ *   - A pointer to a tensor with zero elements (e.g. u when seqlen == 0) may be NULL.
+ */
+#ifndef SSM_SCAN_H
+#define SSM_SCAN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ABI-identical to cudaStream_t (both are `struct CUstream_st *`); NULL = legacy stream. */
+typedef struct CUstream_st* ssm_stream_t;
+
+typedef enum {
+    SSM_OK = 0,
+    SSM_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad dtype, misaligned pointer    */
+    SSM_ERR_UNSUPPORTED = 2,   /* dstate != 16, or the current device is not sm_100             */
+    SSM_ERR_LAUNCH = 3,        /* a CUDA call or kernel launch failed                           */
+    SSM_ERR_TIMEOUT = 4,       /* device: a bounded wait in the kernel gave up (see read_status) */
+    SSM_ERR_WORKSPACE = 5      /* workspace missing or smaller than ssm_selective_scan_workspace_size */
+} ssm_status_t;
+
+typedef enum { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype_t;
+
+/* Version of this ABI (incremented on any signature change). */
+int ssm_abi_version(void);
+
+/* Human-readable name of a status code (static string). */
+const char* ssm_status_string(ssm_status_t status);
+
+/*
+ * Bytes of device workspace ssm_selective_scan_fwd needs for these sizes (a multiple
+ * of 256).  The workspace holds a transposed fp32 copy of B and C, the status word
+ * and the flags and (prod Abar, h) pairs of the inter-CTA chunk carry.
+ * Returns 0 for invalid sizes.
+ */
+size_t ssm_selective_scan_workspace_size(int batch, int dim, int dstate, int64_t seqlen);
+
+/*
+ * Zero a workspace before its first use.  After that every call leaves the
+ * workspace ready for the next one (its counters and flag epochs are reset by the
+ * kernel itself), so this is needed once per allocation.
+ */
+ssm_status_t ssm_workspace_init(void* workspace, size_t workspace_bytes, ssm_stream_t stream);
+
+/*
+ * Full-sequence forward scan (the operation above).
+ *   u, delta, B, C, y       required; io_dtype elements.
+ *   A                        required; fp32 (dim, dstate).
+ *   D, delta_bias            optional fp32 (dim); NULL means 0.
+ *   z                        optional io_dtype (batch, dim, seqlen); NULL means no gate.
+ *   softplus                 nonzero: Delta = softplus(delta + bias); zero: Delta = delta + bias.
+ *   last_state               optional fp32 (batch, dim, dstate) output: the state after step seqlen-1
+ *                            (zeros when seqlen == 0).
+ *   workspace                device buffer of at least
+ *                            ssm_selective_scan_workspace_size(batch, dim, dstate, seqlen) bytes,
+ *                            256-byte aligned, zeroed once by ssm_workspace_init().  It must not be
+ *                            used by two calls that can overlap on the GPU.
+ * All tensor pointers must be 16-byte aligned.  Any seqlen >= 0 is accepted; when
+ * seqlen * sizeof(io element) is a multiple of 16 the tiles are staged with TMA,
+ * otherwise a direct-load kernel runs.
+ */
+ssm_status_t ssm_selective_scan_fwd(
+    const void* u, const void* delta, const float* A, const void* B, const void* C,
+    const float* D, const void* z, const float* delta_bias, int softplus,
+    void* y, float* last_state,
+    int batch, int dim, int dstate, int64_t seqlen, ssm_dtype_t io_dtype,
+    void* workspace, size_t workspace_bytes, ssm_stream_t stream);
+
+/* Kernel family for ssm_selective_scan_fwd_ex. */
+typedef enum {
+    SSM_ALGO_AUTO = 0,        /* pick by shape (what ssm_selective_scan_fwd does)              */
+    SSM_ALGO_SEQUENTIAL = 1,  /* each CTA walks all of L for its channels; carry in registers  */
+    SSM_ALGO_CHUNKED = 2,     /* L split into chunks across CTAs, joined by decoupled look-back */
+    SSM_ALGO_DIRECT = 3       /* no staging: direct global loads (any alignment of seqlen)     */
+} ssm_algo_t;
+
+typedef struct {
+    int algo;                  /* ssm_algo_t                                                      */
+    int lanes_per_channel;     /* SEQUENTIAL/DIRECT: lanes sharing one channel (2, 4, 8 or 16); 0 = auto */
+    uint32_t spin_limit;       /* CHUNKED: polls before a look-back wait gives up; 0 = default    */
+    int debug_skip_publish;    /* CHUNKED, tests only: chunk index whose CTAs never publish; -1 = off */
+} ssm_fwd_options_t;
+
+/* ssm_selective_scan_fwd with an explicit kernel choice (tuning and tests).  opts may be NULL. */
+ssm_status_t ssm_selective_scan_fwd_ex(
+    const void* u, const void* delta, const float* A, const void* B, const void* C,
+    const float* D, const void* z, const float* delta_bias, int softplus,
+    void* y, float* last_state,
+    int batch, int dim, int dstate, int64_t seqlen, ssm_dtype_t io_dtype,
+    void* workspace, size_t workspace_bytes, const ssm_fwd_options_t* opts, ssm_stream_t stream);
+
+/*
+ * One-token decode ([Card] 线性扫描算法: a fixed-size state update per token;
+ * [Eng] §6.2).  For every (b, d):  h[n] <- exp(Delta*A[d,n]) h[n] + Delta*B[b,n]*u[b,d],
+ * y[b,d] = (sum_n C[b,n] h[n] + D[d] u[b,d]) * silu(z[b,d]), with the fp32 state
+ * read, modified and written IN PLACE.
+ *   state       fp32 (batch, dim, dstate), in/out.
+ *   u, delta, z, y: io_dtype (batch, dim);  B, C: io_dtype (batch, dstate).
+ *   D, delta_bias, z optional as above.  No workspace.
+ */
+ssm_status_t ssm_state_update(
+    float* state, const void* u, const void* delta, const float* A, const void* B, const void* C,
+    const float* D, const void* z, const float* delta_bias, int softplus, void* y,
+    int batch, int dim, int dstate, ssm_dtype_t io_dtype, ssm_stream_t stream);
+
+/*
+ * Synchronise `stream`, return the device-side status recorded in `workspace` by the
+ * calls made since the last read (SSM_OK or SSM_ERR_TIMEOUT) and clear it.
+ */
+ssm_status_t ssm_read_status(void* workspace, ssm_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSM_SCAN_H */

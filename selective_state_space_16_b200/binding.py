@@ -1,0 +1,164 @@
+"""ctypes binding of the C ABI in include/ssm_scan.h.
+
+Argument marshalling only: every step of the scan runs in the CUDA kernels of
+libssm_scan.so.  Tensors are torch tensors used purely as device memory; the
+current torch CUDA stream is passed unless another stream is given.  If the
+library has not been built this module raises on first use -- there is no CPU
+fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libssm_scan.so")
+
+SSM_OK, SSM_ERR_INVALID_ARG, SSM_ERR_UNSUPPORTED, SSM_ERR_LAUNCH, SSM_ERR_TIMEOUT, SSM_ERR_WORKSPACE = range(6)
+SSM_F32, SSM_BF16 = 0, 1
+SSM_ALGO_AUTO, SSM_ALGO_SEQUENTIAL, SSM_ALGO_CHUNKED, SSM_ALGO_DIRECT = range(4)
+ALGOS = {"auto": SSM_ALGO_AUTO, "sequential": SSM_ALGO_SEQUENTIAL, "chunked": SSM_ALGO_CHUNKED,
+         "direct": SSM_ALGO_DIRECT}
+
+
+class SsmError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} (status {code})")
+
+
+class FwdOptions(ctypes.Structure):
+    _fields_ = [("algo", ctypes.c_int), ("lanes_per_channel", ctypes.c_int),
+                ("spin_limit", ctypes.c_uint32), ("debug_skip_publish", ctypes.c_int)]
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def load() -> ctypes.CDLL:
+    """Load libssm_scan.so (raises if it was not built: run __graft_entry__.build())."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(f"{LIB_PATH} is missing; build it with selective_state_space_16_b200/build.py")
+            lib = ctypes.CDLL(LIB_PATH)
+            vp, ci, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+            lib.ssm_abi_version.restype = ci
+            lib.ssm_status_string.argtypes = [ci]
+            lib.ssm_status_string.restype = ctypes.c_char_p
+            lib.ssm_selective_scan_workspace_size.argtypes = [ci, ci, ci, i64]
+            lib.ssm_selective_scan_workspace_size.restype = sz
+            lib.ssm_workspace_init.argtypes = [vp, sz, vp]
+            lib.ssm_workspace_init.restype = ci
+            fwd = [vp, vp, vp, vp, vp, vp, vp, vp, ci, vp, vp, ci, ci, ci, i64, ci, vp, sz]
+            lib.ssm_selective_scan_fwd.argtypes = fwd + [vp]
+            lib.ssm_selective_scan_fwd.restype = ci
+            lib.ssm_selective_scan_fwd_ex.argtypes = fwd + [ctypes.POINTER(FwdOptions), vp]
+            lib.ssm_selective_scan_fwd_ex.restype = ci
+            lib.ssm_state_update.argtypes = [vp] * 9 + [ci, vp, ci, ci, ci, ci, vp]
+            lib.ssm_state_update.restype = ci
+            lib.ssm_read_status.argtypes = [vp, vp]
+            lib.ssm_read_status.restype = ci
+            _lib = lib
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return load().ssm_status_string(int(code)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _io(t):
+    if t.dtype == torch.bfloat16:
+        return SSM_BF16
+    if t.dtype == torch.float32:
+        return SSM_F32
+    raise TypeError(f"unsupported I/O dtype {t.dtype}")
+
+
+def _check(code, where):
+    if code != SSM_OK:
+        raise SsmError(code, where)
+
+
+def ssm_selective_scan_workspace_size(batch: int, dim: int, dstate: int, seqlen: int) -> int:
+    return int(load().ssm_selective_scan_workspace_size(batch, dim, dstate, seqlen))
+
+
+def ssm_workspace_init(workspace, stream=None):
+    _check(load().ssm_workspace_init(_ptr(workspace), workspace.numel() * workspace.element_size(),
+                                     _stream(stream)), "ssm_workspace_init")
+
+
+def new_workspace(batch, dim, dstate, seqlen, device="cuda", stream=None):
+    """Allocate (with torch) and zero a workspace large enough for these sizes."""
+    n = max(ssm_selective_scan_workspace_size(batch, dim, dstate, seqlen), 256)
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    ssm_workspace_init(ws, stream)
+    return ws
+
+
+def ssm_selective_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus, y, last_state, workspace,
+                           stream=None, algo=None, lanes_per_channel=0, spin_limit=0, debug_skip_publish=-1,
+                           check=True):
+    """Marshal a forward-scan call.  u/delta/z/y: (b, d, L); B/C: (b, N, L); A: (d, N) fp32;
+    D/delta_bias: (d) fp32 or None; last_state: (b, d, N) fp32 or None; workspace: uint8."""
+    lib = load()
+    b, d, L = u.shape
+    n = A.shape[1]
+    args = [_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+            int(bool(softplus)), _ptr(y), _ptr(last_state), b, d, n, L, _io(u), _ptr(workspace),
+            workspace.numel() * workspace.element_size()]
+    if algo is None and lanes_per_channel == 0 and spin_limit == 0 and debug_skip_publish < 0:
+        code = lib.ssm_selective_scan_fwd(*args, _stream(stream))
+    else:
+        a = ALGOS[algo] if isinstance(algo, str) else (algo or SSM_ALGO_AUTO)
+        opts = FwdOptions(a, lanes_per_channel, spin_limit, debug_skip_publish)
+        code = lib.ssm_selective_scan_fwd_ex(*args, ctypes.byref(opts), _stream(stream))
+    if check:
+        _check(code, "ssm_selective_scan_fwd")
+    return code
+
+
+def ssm_state_update(state, u, delta, A, B, C, D, z, delta_bias, softplus, y, stream=None, check=True):
+    """Marshal a decode call.  state: (b, d, N) fp32 in/out; u/delta/z/y: (b, d); B/C: (b, N)."""
+    b, d, n = state.shape
+    code = load().ssm_state_update(_ptr(state), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                   _ptr(z), _ptr(delta_bias), int(bool(softplus)), _ptr(y), b, d, n, _io(u),
+                                   _stream(stream))
+    if check:
+        _check(code, "ssm_state_update")
+    return code
+
+
+def ssm_read_status(workspace, stream=None) -> int:
+    return int(load().ssm_read_status(_ptr(workspace), _stream(stream)))
+
+
+def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
+                       return_last_state=True, workspace=None, stream=None, **opts):
+    """Convenience wrapper: allocates y (u's dtype), last_state (fp32) and, if not given,
+    a workspace, then calls ssm_selective_scan_fwd.  Returns (y, last_state)."""
+    b, d, L = u.shape
+    n = A.shape[1]
+    y = torch.empty_like(u)
+    last = torch.empty((b, d, n), dtype=torch.float32, device=u.device) if return_last_state else None
+    if workspace is None:
+        workspace = new_workspace(b, d, n, L, device=u.device, stream=stream)
+    ssm_selective_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus, y, last, workspace,
+                           stream=stream, **opts)
+    return y, last

@@ -1,0 +1,190 @@
+// aux_kernels.cuh -- the kernels around the main forward scans:
+//   pack_bc_kernel      B, C (batch, 16, L) -> fp32 [batch][L][32] rows (B then C), so a
+//                       step's 16 B and 16 C values are one 128-byte row for broadcast reads;
+//   scan_fwd_direct     forward scan with direct global loads, for any seqlen / alignment;
+//   state_update_kernel the one-token decode step, fp32 state read-modified-written in place.
+//
+// Pages (sections as printed):
+//   [Eng]  "Mamba 选择性状态空间模型：亚二次复杂度大语言模型推理工程实践"
+//   [Card] "Mamba与SSM状态空间模型：一张摘要卡读完万页档案"
+//   [Hist] "AI底层架构的一场革命：Mamba如何用「状态压缩」挑战Transformer的十年统治"
+#pragma once
+
+#include "common.cuh"
+#include "scan_math.cuh"
+
+namespace ssm {
+
+// ---------------------------------------------------------------------------------------
+// B/C transpose into the workspace.  grid = (ceil(L/64), batch), 256 threads.
+// ---------------------------------------------------------------------------------------
+template <typename IO>
+__global__ void __launch_bounds__(256) pack_bc_kernel(const IO* __restrict__ B, const IO* __restrict__ C,
+                                                      float* __restrict__ bc, long long L) {
+    __shared__ float tile[32][65];
+    const int b = blockIdx.y;
+    const long long t0 = static_cast<long long>(blockIdx.x) * 64;
+    for (int idx = threadIdx.x; idx < 32 * 64; idx += 256) {
+        const int r = idx >> 6, c = idx & 63;
+        const long long t = t0 + c;
+        const IO* src = (r < 16) ? B : C;
+        tile[r][c] = (t < L) ? IoTraits<IO>::to_f32(src[(static_cast<long long>(b) * 16 + (r & 15)) * L + t]) : 0.f;
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < 32 * 64; idx += 256) {
+        const int c = idx >> 5, r = idx & 31;
+        const long long t = t0 + c;
+        if (t < L) bc[(static_cast<long long>(b) * L + t) * 32 + r] = tile[r][c];
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// Direct-load forward scan (fallback for seqlen whose rows are not 16-byte multiples).
+// G lanes per channel, NC = 16/G chains per lane, 128 threads per block.
+// Per step: h = exp(Delta A) h + Delta B u; y = C.h + D u; y *= silu(z)
+// ([Card] 选择性机制 and Python 演示; [Hist] Mamba Block 数据流).
+// ---------------------------------------------------------------------------------------
+struct DirectParams {
+    const void* u;
+    const void* delta;
+    const void* z;
+    const float* bc;       // packed [batch][L][32]
+    const float* A;
+    const float* D;
+    const float* bias;
+    void* y;
+    float* last_state;
+    int batch, dim;
+    long long L;
+    int softplus;
+};
+
+template <typename IO, int G>
+__global__ void __launch_bounds__(128) scan_fwd_direct_kernel(const DirectParams p) {
+    constexpr int NC = 16 / G;
+    const int lane = threadIdx.x & 31;
+    const int nl = lane % G;
+    const long long ch = (static_cast<long long>(blockIdx.x) * 128 + threadIdx.x) / G;  // flat (b, d)
+    const bool valid = ch < static_cast<long long>(p.batch) * p.dim;
+    const int b = valid ? static_cast<int>(ch / p.dim) : 0;
+    const int d = valid ? static_cast<int>(ch % p.dim) : 0;
+
+    const IO* u = static_cast<const IO*>(p.u) + ch * p.L;
+    const IO* dl = static_cast<const IO*>(p.delta) + ch * p.L;
+    const IO* z = p.z ? static_cast<const IO*>(p.z) + ch * p.L : nullptr;
+    IO* y = static_cast<IO*>(p.y) + ch * p.L;
+    const float* bcb = p.bc + static_cast<long long>(b) * p.L * 32;
+
+    float A2[NC], h[NC];
+#pragma unroll
+    for (int j = 0; j < NC; ++j) {
+        A2[j] = valid ? p.A[d * 16 + nl * NC + j] * kLog2e : 0.f;
+        h[j] = 0.f;
+    }
+    const float Dd = (valid && p.D) ? p.D[d] : 0.f;
+    const float bias = (valid && p.bias) ? p.bias[d] : 0.f;
+
+    for (long long t = 0; t < p.L; ++t) {
+        float ut = 0.f, dt = 0.f;
+        if (valid) {
+            ut = IoTraits<IO>::to_f32(u[t]);
+            dt = step_size(IoTraits<IO>::to_f32(dl[t]), bias, p.softplus != 0);
+        }
+        const float w = dt * ut;
+        const float* row = bcb + t * 32;
+        float acc = 0.f;
+#pragma unroll
+        for (int j = 0; j < NC; ++j) {
+            const float a = ex2_mufu(dt * A2[j]);
+            h[j] = fmaf(a, h[j], w * row[nl * NC + j]);
+            acc = fmaf(row[16 + nl * NC + j], h[j], acc);
+        }
+#pragma unroll
+        for (int m = G / 2; m >= 1; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m, 32);
+        if (valid && nl == 0) {
+            float v = fmaf(Dd, ut, acc);
+            if (z) v *= silu_f32(IoTraits<IO>::to_f32(z[t]));
+            y[t] = IoTraits<IO>::from_f32(v);
+        }
+    }
+    if (valid && p.last_state) {
+        float* dst = p.last_state + ch * 16 + nl * NC;
+#pragma unroll
+        for (int j = 0; j < NC; ++j) dst[j] = h[j];
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// One-token decode ([Card] 线性扫描算法: one fixed-size state update per token;
+// [Eng] §6.3: the states of a batch laid out on contiguous threads).
+// Four threads per (b, d), each owning 4 of the 16 fp32 state values (one 16-byte
+// vector), so a warp reads and writes 512 contiguous bytes of state.
+// ---------------------------------------------------------------------------------------
+struct DecodeParams {
+    float* state;
+    const void* u;
+    const void* delta;
+    const float* A;
+    const void* B;
+    const void* C;
+    const float* D;
+    const void* z;
+    const float* bias;
+    void* y;
+    int batch, dim;
+    int softplus;
+};
+
+template <typename IO>
+__global__ void __launch_bounds__(256) state_update_kernel(const DecodeParams p) {
+    const long long gid = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
+    const long long row = gid >> 2;  // flat (b, d)
+    const int q = static_cast<int>(gid & 3);
+    const bool valid = row < static_cast<long long>(p.batch) * p.dim;
+    const long long rr = valid ? row : 0;
+    const int b = static_cast<int>(rr / p.dim);
+    const int d = static_cast<int>(rr % p.dim);
+
+    float4 hv = make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 av = make_float4(0.f, 0.f, 0.f, 0.f);
+    float Bq[4] = {0.f, 0.f, 0.f, 0.f}, Cq[4] = {0.f, 0.f, 0.f, 0.f};
+    float ut = 0.f, dt = 0.f, zt = 0.f, Dd = 0.f;
+    if (valid) {
+        hv = *reinterpret_cast<const float4*>(p.state + rr * 16 + q * 4);
+        av = *reinterpret_cast<const float4*>(p.A + d * 16 + q * 4);
+        const IO* Bp = static_cast<const IO*>(p.B) + b * 16 + q * 4;
+        const IO* Cp = static_cast<const IO*>(p.C) + b * 16 + q * 4;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            Bq[j] = IoTraits<IO>::to_f32(Bp[j]);
+            Cq[j] = IoTraits<IO>::to_f32(Cp[j]);
+        }
+        ut = IoTraits<IO>::to_f32(static_cast<const IO*>(p.u)[rr]);
+        const float bias = p.bias ? p.bias[d] : 0.f;
+        dt = step_size(IoTraits<IO>::to_f32(static_cast<const IO*>(p.delta)[rr]), bias, p.softplus != 0);
+        if (p.z) zt = IoTraits<IO>::to_f32(static_cast<const IO*>(p.z)[rr]);
+        Dd = p.D ? p.D[d] : 0.f;
+    }
+    const float w = dt * ut;
+    float hs[4] = {hv.x, hv.y, hv.z, hv.w};
+    const float as[4] = {av.x, av.y, av.z, av.w};
+    float acc = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float a = ex2_mufu(dt * as[j] * kLog2e);
+        hs[j] = fmaf(a, hs[j], w * Bq[j]);
+        acc = fmaf(Cq[j], hs[j], acc);
+    }
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1, 32);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2, 32);
+    if (valid) {
+        *reinterpret_cast<float4*>(p.state + rr * 16 + q * 4) = make_float4(hs[0], hs[1], hs[2], hs[3]);
+        if (q == 0) {
+            float v = fmaf(Dd, ut, acc);
+            if (p.z) v *= silu_f32(zt);
+            static_cast<IO*>(p.y)[rr] = IoTraits<IO>::from_f32(v);
+        }
+    }
+}
+
+}  // namespace ssm

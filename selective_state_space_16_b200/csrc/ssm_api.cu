@@ -1,0 +1,342 @@
+// ssm_api.cu -- host side of the C ABI declared in include/ssm_scan.h: argument
+// validation, workspace layout, TMA tensor maps, kernel choice and launches.
+// Everything here is marshalling; every step of the scan runs in the kernels.
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/ssm_scan.h"
+#include "aux_kernels.cuh"
+#include "common.cuh"
+#include "scan_fwd_seq.cuh"
+
+namespace {
+
+using ssm::WorkspaceHeader;
+
+constexpr int kAbiVersion = 1;
+constexpr uint32_t kDefaultWaitLimit = 1u << 22;
+
+size_t round_up(size_t v, size_t m) { return (v + m - 1) / m * m; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Workspace layout: [header 256 B][B/C fp32 rows: batch * L * 128 B][chunk-carry region].
+struct WsLayout {
+    size_t bc_off, carry_off, total;
+};
+
+WsLayout ws_layout(int batch, int dim, int64_t L) {
+    WsLayout w{};
+    w.bc_off = sizeof(WorkspaceHeader);
+    w.carry_off = w.bc_off + round_up(static_cast<size_t>(batch) * static_cast<size_t>(L) * 128u, 256);
+    (void)dim;
+    w.total = w.carry_off;
+    return w;
+}
+
+// ------------------------------------------------------------------ driver entry point
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 3-D tiled map over a dense (d2, d1, d0) tensor with d0 innermost.
+bool make_map_3d(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* ptr, uint64_t d0, uint64_t d1,
+                 uint64_t d2, uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {d0, d1, d2};
+    const cuuint64_t strides[2] = {d0 * esize, d0 * d1 * esize};
+    const cuuint32_t box[3] = {b0, b1, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, dt, 3, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+ssm_status_t check_device(int* sm_count) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SSM_ERR_LAUNCH;
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return SSM_ERR_LAUNCH;
+    if (major != 10) return SSM_ERR_UNSUPPORTED;
+    if (sm_count && cudaDeviceGetAttribute(sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return SSM_ERR_LAUNCH;
+    return SSM_OK;
+}
+
+ssm_status_t launch_status() {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SSM_OK : SSM_ERR_LAUNCH;
+}
+
+// Per-device "max dynamic shared memory" opt-in, remembered per (kernel, device).
+bool ensure_smem_attr(const void* kernel, int bytes) {
+    static std::mutex mu;
+    static std::set<std::pair<const void*, int>> done;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    std::lock_guard<std::mutex> lk(mu);
+    if (done.count({kernel, dev})) return true;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+    done.insert({kernel, dev});
+    return true;
+}
+
+// ------------------------------------------------------------------ forward launches
+struct FwdArgs {
+    const void *u, *delta, *B, *C, *z;
+    const float *A, *D, *bias;
+    int softplus;
+    void* y;
+    float* last_state;
+    int batch, dim;
+    int64_t L;
+    ssm_dtype_t io;
+    uint8_t* ws;
+    cudaStream_t stream;
+    int sm_count;
+};
+
+template <typename IO, int G, int NW>
+ssm_status_t launch_seq(const FwdArgs& a) {
+    using Cfg = ssm::SeqCfg<IO, G, NW>;
+    constexpr int TC = Cfg::kTC;
+    constexpr auto sw128 = CU_TENSOR_MAP_SWIZZLE_128B;
+    const auto dt = ssm::IoTraits<IO>::kTmaType;
+    constexpr int es = ssm::IoTraits<IO>::kBytes;
+    CUtensorMap mu, mdl, mz, mbc, my;
+    const uint64_t L = static_cast<uint64_t>(a.L);
+    bool ok = make_map_3d(&mu, dt, es, a.u, L, a.dim, a.batch, TC, Cfg::kR, sw128) &&
+              make_map_3d(&mdl, dt, es, a.delta, L, a.dim, a.batch, TC, Cfg::kR, sw128) &&
+              make_map_3d(&my, dt, es, a.y, L, a.dim, a.batch, TC, Cfg::kCW, sw128) &&
+              make_map_3d(&mbc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.ws + ws_layout(a.batch, a.dim, a.L).bc_off, 32,
+                          L, a.batch, 32, TC, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (ok && a.z) ok = make_map_3d(&mz, dt, es, a.z, L, a.dim, a.batch, TC, Cfg::kR, sw128);
+    if (!a.z) mz = mu;
+    if (!ok) return SSM_ERR_LAUNCH;
+    auto kern = ssm::scan_fwd_seq_kernel<IO, G, NW>;
+    if (!ensure_smem_attr(reinterpret_cast<const void*>(kern), Cfg::kSmem)) return SSM_ERR_LAUNCH;
+    ssm::SeqParams p{};
+    p.A = a.A;
+    p.D = a.D;
+    p.bias = a.bias;
+    p.last_state = a.last_state;
+    p.hdr = reinterpret_cast<WorkspaceHeader*>(a.ws);
+    p.batch = a.batch;
+    p.dim = a.dim;
+    p.L = a.L;
+    p.tiles_per_batch = (a.dim + Cfg::kR - 1) / Cfg::kR;
+    p.softplus = a.softplus;
+    p.has_z = a.z != nullptr;
+    p.wait_limit = kDefaultWaitLimit;
+    const long long grid = static_cast<long long>(a.batch) * p.tiles_per_batch;
+    if (grid > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
+    kern<<<static_cast<unsigned>(grid), Cfg::kThreads, Cfg::kSmem, a.stream>>>(mu, mdl, mz, mbc, my, p);
+    return launch_status();
+}
+
+template <typename IO>
+ssm_status_t launch_direct(const FwdArgs& a) {
+    ssm::DirectParams p{};
+    p.u = a.u;
+    p.delta = a.delta;
+    p.z = a.z;
+    p.bc = reinterpret_cast<const float*>(a.ws + ws_layout(a.batch, a.dim, a.L).bc_off);
+    p.A = a.A;
+    p.D = a.D;
+    p.bias = a.bias;
+    p.y = a.y;
+    p.last_state = a.last_state;
+    p.batch = a.batch;
+    p.dim = a.dim;
+    p.L = a.L;
+    p.softplus = a.softplus;
+    constexpr int G = 2;
+    const long long threads = static_cast<long long>(a.batch) * a.dim * G;
+    const long long grid = (threads + 127) / 128;
+    if (grid > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
+    ssm::scan_fwd_direct_kernel<IO, G><<<static_cast<unsigned>(grid), 128, 0, a.stream>>>(p);
+    return launch_status();
+}
+
+template <typename IO>
+ssm_status_t launch_pack(const FwdArgs& a) {
+    const dim3 grid(static_cast<unsigned>((a.L + 63) / 64), static_cast<unsigned>(a.batch));
+    ssm::pack_bc_kernel<IO><<<grid, 256, 0, a.stream>>>(
+        static_cast<const IO*>(a.B), static_cast<const IO*>(a.C),
+        reinterpret_cast<float*>(a.ws + ws_layout(a.batch, a.dim, a.L).bc_off), a.L);
+    return launch_status();
+}
+
+// Lanes per channel for the sequential kernel: the candidate whose most-loaded SM
+// carries the fewest channel-steps (all CTAs of a candidate are resident at once),
+// with a small charge for the wider reduce-scatter of larger groups.
+int pick_lanes(int batch, int dim, int sm_count, bool bf16) {
+    struct Cand { int G, R, per_sm; double cost; };
+    const Cand cands[] = {{2, 48, 3, 1.00}, {4, 24, 5, 1.04}, {8, 16, 6, 1.10}};
+    int best = 2;
+    double best_t = 1e300;
+    for (const Cand& c : cands) {
+        if (!bf16 && c.G == 8) continue;
+        const long long ctas = static_cast<long long>(batch) * ((dim + c.R - 1) / c.R);
+        const long long waves = (ctas + static_cast<long long>(sm_count) * c.per_sm - 1) / (static_cast<long long>(sm_count) * c.per_sm);
+        const long long per_sm = (ctas + sm_count - 1) / sm_count;
+        const double t = static_cast<double>(per_sm) * c.R * c.cost * (waves > 1 ? 1.05 : 1.0);
+        if (t < best_t - 1e-9) { best_t = t; best = c.G; }
+    }
+    return best;
+}
+
+template <typename IO>
+ssm_status_t launch_forward(const FwdArgs& a, const ssm_fwd_options_t& o) {
+    ssm_status_t st = launch_pack<IO>(a);
+    if (st != SSM_OK) return st;
+    const bool tma_ok = (static_cast<uint64_t>(a.L) * ssm::IoTraits<IO>::kBytes) % 16 == 0 && aligned16(a.u) &&
+                        aligned16(a.delta) && aligned16(a.y) && (!a.z || aligned16(a.z));
+    int algo = o.algo;
+    if (algo == SSM_ALGO_AUTO || algo == SSM_ALGO_CHUNKED) algo = SSM_ALGO_SEQUENTIAL;
+    if (!tma_ok) algo = SSM_ALGO_DIRECT;
+    if (algo == SSM_ALGO_DIRECT) return launch_direct<IO>(a);
+    int G = o.lanes_per_channel;
+    if (G == 0) G = pick_lanes(a.batch, a.dim, a.sm_count, sizeof(IO) == 2);
+    switch (G) {
+        case 2: return launch_seq<IO, 2, 3>(a);
+        case 4: return launch_seq<IO, 4, 3>(a);
+        case 8:
+            if constexpr (sizeof(IO) == 2) return launch_seq<IO, 8, 4>(a);
+            return SSM_ERR_INVALID_ARG;
+        default: return SSM_ERR_INVALID_ARG;
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+int ssm_abi_version(void) { return kAbiVersion; }
+
+const char* ssm_status_string(ssm_status_t s) {
+    switch (s) {
+        case SSM_OK: return "ok";
+        case SSM_ERR_INVALID_ARG: return "invalid argument";
+        case SSM_ERR_UNSUPPORTED: return "unsupported configuration";
+        case SSM_ERR_LAUNCH: return "CUDA launch or runtime error";
+        case SSM_ERR_TIMEOUT: return "device wait timed out";
+        case SSM_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+size_t ssm_selective_scan_workspace_size(int batch, int dim, int dstate, int64_t seqlen) {
+    if (batch < 0 || dim < 0 || dstate != 16 || seqlen < 0) return 0;
+    return round_up(ws_layout(batch, dim, seqlen).total, 256);
+}
+
+ssm_status_t ssm_workspace_init(void* workspace, size_t workspace_bytes, ssm_stream_t stream) {
+    if (!workspace || workspace_bytes < sizeof(WorkspaceHeader)) return SSM_ERR_WORKSPACE;
+    return cudaMemsetAsync(workspace, 0, workspace_bytes, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? SSM_OK
+               : SSM_ERR_LAUNCH;
+}
+
+ssm_status_t ssm_selective_scan_fwd_ex(const void* u, const void* delta, const float* A, const void* B,
+                                       const void* C, const float* D, const void* z, const float* delta_bias,
+                                       int softplus, void* y, float* last_state, int batch, int dim, int dstate,
+                                       int64_t seqlen, ssm_dtype_t io_dtype, void* workspace,
+                                       size_t workspace_bytes, const ssm_fwd_options_t* opts, ssm_stream_t stream) {
+    if (batch < 0 || dim < 0 || seqlen < 0) return SSM_ERR_INVALID_ARG;
+    // Tensors with elements must have a pointer; zero-element tensors may be NULL.
+    const bool seq_elems = batch > 0 && dim > 0 && seqlen > 0;
+    if (seq_elems && (!u || !delta || !B || !C || !y)) return SSM_ERR_INVALID_ARG;
+    if (dim > 0 && !A) return SSM_ERR_INVALID_ARG;
+    if (io_dtype != SSM_F32 && io_dtype != SSM_BF16) return SSM_ERR_INVALID_ARG;
+    if (dstate != 16) return SSM_ERR_UNSUPPORTED;
+    const void* ptrs[] = {u, delta, A, B, C, D, z, delta_bias, y, last_state};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return SSM_ERR_INVALID_ARG;
+    ssm_fwd_options_t o{SSM_ALGO_AUTO, 0, 0, -1};
+    if (opts) o = *opts;
+    if (o.algo < SSM_ALGO_AUTO || o.algo > SSM_ALGO_DIRECT) return SSM_ERR_INVALID_ARG;
+    if (batch == 0 || dim == 0) return SSM_OK;
+    if (batch > 65535) return SSM_ERR_UNSUPPORTED;  // batch is a grid y-dimension of the B/C pack
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+        workspace_bytes < ssm_selective_scan_workspace_size(batch, dim, dstate, seqlen))
+        return SSM_ERR_WORKSPACE;
+    int sm_count = 0;
+    ssm_status_t st = check_device(&sm_count);
+    if (st != SSM_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (seqlen == 0) {
+        if (last_state &&
+            cudaMemsetAsync(last_state, 0, static_cast<size_t>(batch) * dim * 16 * sizeof(float), s) != cudaSuccess)
+            return SSM_ERR_LAUNCH;
+        return SSM_OK;
+    }
+    FwdArgs a{u, delta, B, C, z, A, D, delta_bias, softplus, y, last_state, batch, dim, seqlen, io_dtype,
+              static_cast<uint8_t*>(workspace), s, sm_count};
+    return io_dtype == SSM_BF16 ? launch_forward<__nv_bfloat16>(a, o) : launch_forward<float>(a, o);
+}
+
+ssm_status_t ssm_selective_scan_fwd(const void* u, const void* delta, const float* A, const void* B, const void* C,
+                                    const float* D, const void* z, const float* delta_bias, int softplus, void* y,
+                                    float* last_state, int batch, int dim, int dstate, int64_t seqlen,
+                                    ssm_dtype_t io_dtype, void* workspace, size_t workspace_bytes,
+                                    ssm_stream_t stream) {
+    return ssm_selective_scan_fwd_ex(u, delta, A, B, C, D, z, delta_bias, softplus, y, last_state, batch, dim,
+                                     dstate, seqlen, io_dtype, workspace, workspace_bytes, nullptr, stream);
+}
+
+ssm_status_t ssm_state_update(float* state, const void* u, const void* delta, const float* A, const void* B,
+                              const void* C, const float* D, const void* z, const float* delta_bias, int softplus,
+                              void* y, int batch, int dim, int dstate, ssm_dtype_t io_dtype, ssm_stream_t stream) {
+    if (batch < 0 || dim < 0) return SSM_ERR_INVALID_ARG;
+    if (batch > 0 && dim > 0 && (!state || !u || !delta || !A || !B || !C || !y)) return SSM_ERR_INVALID_ARG;
+    if (io_dtype != SSM_F32 && io_dtype != SSM_BF16) return SSM_ERR_INVALID_ARG;
+    if (dstate != 16) return SSM_ERR_UNSUPPORTED;
+    if (!aligned16(state) || !aligned16(A)) return SSM_ERR_INVALID_ARG;
+    if (batch == 0 || dim == 0) return SSM_OK;
+    ssm_status_t st = check_device(nullptr);
+    if (st != SSM_OK) return st;
+    ssm::DecodeParams p{state, u, delta, A, B, C, D, z, delta_bias, y, batch, dim, softplus};
+    const long long threads = static_cast<long long>(batch) * dim * 4;
+    const long long grid = (threads + 255) / 256;
+    if (grid > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (io_dtype == SSM_BF16)
+        ssm::state_update_kernel<__nv_bfloat16><<<static_cast<unsigned>(grid), 256, 0, s>>>(p);
+    else
+        ssm::state_update_kernel<float><<<static_cast<unsigned>(grid), 256, 0, s>>>(p);
+    return launch_status();
+}
+
+ssm_status_t ssm_read_status(void* workspace, ssm_stream_t stream) {
+    if (!workspace) return SSM_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SSM_ERR_LAUNCH;
+    uint32_t code = 0;
+    auto* hdr = static_cast<WorkspaceHeader*>(workspace);
+    if (cudaMemcpy(&code, &hdr->status, sizeof(code), cudaMemcpyDeviceToHost) != cudaSuccess) return SSM_ERR_LAUNCH;
+    if (code != 0 && cudaMemset(&hdr->status, 0, sizeof(uint32_t)) != cudaSuccess) return SSM_ERR_LAUNCH;
+    return static_cast<ssm_status_t>(code);
+}
+
+}  // extern "C"

@@ -1,0 +1,124 @@
+"""CPU-only checks of the C ABI: the library loads, exports every entry point that
+include/*.h declares, and rejects bad arguments before touching any device."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import selective_state_space_16_b200 as ssm
+from selective_state_space_16_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"\b(ssm_\w+)\s*\(", text):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from selective_state_space_16_b200 import build as b
+    b.build()
+    return ssm.load()
+
+
+def test_header_declares_entry_points():
+    names = _declared_functions()
+    for n in ["ssm_selective_scan_fwd", "ssm_state_update", "ssm_selective_scan_workspace_size",
+              "ssm_read_status", "ssm_selective_scan_fwd_ex", "ssm_workspace_init"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [n for n in _declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert lib.ssm_abi_version() == 1
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert binding.status_string(code)
+    assert "workspace" in binding.status_string(binding.SSM_ERR_WORKSPACE)
+
+
+def test_workspace_size(lib):
+    f = binding.ssm_selective_scan_workspace_size
+    assert f(4, 5120, 16, 2048) % 256 == 0
+    assert f(4, 5120, 16, 2048) >= 256 + 4 * 2048 * 128   # header + fp32 B/C rows
+    assert f(4, 5120, 8, 2048) == 0                      # dstate != 16
+    assert f(-1, 5, 16, 5) == 0
+
+
+P = ctypes.c_void_p
+
+
+def _fwd(lib, **kw):
+    args = dict(u=P(4096), delta=P(4096), A=P(4096), B=P(4096), C=P(4096), D=None, z=None, bias=None,
+                softplus=1, y=P(4096), last=None, batch=1, dim=1, dstate=16, L=8, io=binding.SSM_BF16,
+                ws=P(4096), wsb=1 << 20, stream=None)
+    args.update(kw)
+    return lib.ssm_selective_scan_fwd(*args.values())
+
+
+def test_forward_argument_validation(lib):
+    assert _fwd(lib, u=None) == binding.SSM_ERR_INVALID_ARG
+    assert _fwd(lib, y=None) == binding.SSM_ERR_INVALID_ARG
+    assert _fwd(lib, batch=-1) == binding.SSM_ERR_INVALID_ARG
+    assert _fwd(lib, L=-3) == binding.SSM_ERR_INVALID_ARG
+    assert _fwd(lib, io=7) == binding.SSM_ERR_INVALID_ARG
+    assert _fwd(lib, dstate=8) == binding.SSM_ERR_UNSUPPORTED
+    assert _fwd(lib, u=P(4098)) == binding.SSM_ERR_INVALID_ARG      # not 16-byte aligned
+    assert _fwd(lib, z=P(4100)) == binding.SSM_ERR_INVALID_ARG
+    assert _fwd(lib, batch=0) == binding.SSM_OK                      # empty: nothing launched
+    assert _fwd(lib, dim=0) == binding.SSM_OK
+    assert _fwd(lib, ws=None) == binding.SSM_ERR_WORKSPACE
+    assert _fwd(lib, wsb=16) == binding.SSM_ERR_WORKSPACE
+    assert _fwd(lib, ws=P(4096 + 16)) == binding.SSM_ERR_WORKSPACE   # not 256-byte aligned
+
+
+def test_forward_ex_rejects_unknown_algo(lib):
+    opts = binding.FwdOptions(99, 0, 0, -1)
+    rc = lib.ssm_selective_scan_fwd_ex(P(4096), P(4096), P(4096), P(4096), P(4096), None, None, None, 1,
+                                       P(4096), None, 1, 1, 16, 8, binding.SSM_BF16, P(4096), 1 << 20,
+                                       ctypes.byref(opts), None)
+    assert rc == binding.SSM_ERR_INVALID_ARG
+
+
+def test_decode_argument_validation(lib):
+    def call(**kw):
+        a = dict(state=P(4096), u=P(4096), delta=P(4096), A=P(4096), B=P(4096), C=P(4096), D=None, z=None,
+                 bias=None, softplus=1, y=P(4096), batch=2, dim=3, dstate=16, io=binding.SSM_F32, stream=None)
+        a.update(kw)
+        return lib.ssm_state_update(*a.values())
+    assert call(state=None) == binding.SSM_ERR_INVALID_ARG
+    assert call(state=P(4100)) == binding.SSM_ERR_INVALID_ARG
+    assert call(dstate=32) == binding.SSM_ERR_UNSUPPORTED
+    assert call(io=3) == binding.SSM_ERR_INVALID_ARG
+    assert call(batch=0) == binding.SSM_OK
+
+
+def test_read_status_needs_workspace(lib):
+    assert lib.ssm_read_status(None, None) == binding.SSM_ERR_WORKSPACE
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(binding, "_lib", None)
+    monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        binding.load()
+
+
+def test_product_package_does_not_import_oracle():
+    pkg = os.path.join(ROOT, "selective_state_space_16_b200")
+    for f in glob.glob(os.path.join(pkg, "**", "*.*"), recursive=True):
+        if f.endswith((".py", ".cu", ".cuh", ".h")):
+            txt = open(f).read()
+            assert "import oracle" not in txt and "from oracle" not in txt and "ssm_oracle" not in txt, f

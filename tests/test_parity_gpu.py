@@ -1,0 +1,153 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the same
+seeded inputs, element by element, with the spec's tolerances:
+  fp32 I/O: |x - x_ref| <= 1e-4 (1 + |x_ref|);  bf16 I/O: |x - x_ref| <= 2e-2 (1 + |x_ref|).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import selective_state_space_16_b200 as ssm
+import workloads
+from parity import TOL, assert_close, check_forward, gpu_forward, oracle_forward, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+# ------------------------------------------------------------------ kernel variants, ragged sizes
+VARIANTS = [("sequential", 2), ("sequential", 4), ("sequential", 8), ("direct", 0)]
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("algo,lanes", VARIANTS, ids=[f"{a}{g or ''}" for a, g in VARIANTS])
+def test_forward_variants_ragged(cuda_device, io, algo, lanes):
+    if io == "f32" and lanes == 8:
+        pytest.skip("8 lanes per channel needs 8 steps per 16-byte group (bf16)")
+    # 100 channels: not a multiple of any channel tile; L = 1000: not a multiple of a stage.
+    inp = workloads.scan_inputs(2, 100, 1000, io=io, seed=11)
+    check_forward(inp, algo=algo, lanes_per_channel=lanes, what=f"{algo}/{lanes}/{io}")
+
+
+@pytest.mark.parametrize("flags", [dict(with_z=False), dict(with_D=False), dict(with_bias=False),
+                                   dict(with_z=False, with_D=False, with_bias=False)],
+                         ids=["no_gate", "no_D", "no_bias", "bare"])
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_forward_optional_inputs(cuda_device, flags, io):
+    inp = workloads.scan_inputs(2, 64, 512, io=io, seed=12, **flags)
+    check_forward(inp, what=str(flags))
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_forward_softplus_off(cuda_device, io):
+    inp = workloads.scan_inputs(1, 48, 256, io=io, seed=13)
+    # With softplus off the step is delta + bias itself, so both are made positive here
+    # (the workload's bias is an inverse softplus, i.e. negative).
+    inp["delta"] = (inp["delta"].float().abs() * 0.5 + 0.01).to(inp["delta"].dtype)
+    inp["delta_bias"] = torch.linspace(0.0, 0.05, inp["delta_bias"].numel())
+    check_forward(inp, softplus=False, what="softplus off")
+
+
+@pytest.mark.parametrize("L", [1, 7, 8, 9, 63, 64, 65, 4095, 4096])
+def test_forward_edge_lengths(cuda_device, L):
+    inp = workloads.scan_inputs(2, 20, L, io="bf16", seed=14 + L)
+    check_forward(inp, what=f"L={L}")
+
+
+def test_forward_empty_sequence_gives_zero_state(cuda_device):
+    inp = workloads.scan_inputs(2, 20, 0, io="bf16", seed=15)
+    y, last = gpu_forward(inp)
+    assert y.numel() == 0 and torch.all(last == 0)
+
+
+def test_forward_single_channel(cuda_device):
+    check_forward(workloads.scan_inputs(1, 1, 300, io="f32", seed=16), what="b1 d1")
+
+
+def test_workspace_reuse_is_deterministic(cuda_device):
+    inp = workloads.scan_inputs(2, 96, 640, io="bf16", seed=17)
+    g = to_dev(inp, "cuda")
+    ws = ssm.new_workspace(2, 96, 16, 640)
+    y1, l1 = ssm.selective_scan_fwd(**g, workspace=ws)
+    y2, l2 = ssm.selective_scan_fwd(**g, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2) and torch.equal(l1, l2)
+    assert ssm.ssm_read_status(ws) == 0
+
+
+# ------------------------------------------------------------------ the five workloads, full size
+@pytest.mark.parametrize("idx", [0, 1, 2])
+def test_workload_full_size(cuda_device, idx):
+    w = workloads.WORKLOADS[idx]
+    check_forward(workloads.workload_inputs(w), what=w.name)
+
+
+def test_workload_long_sequence_sampled(cuda_device):
+    w = workloads.WORKLOADS[3]
+    inp = workloads.workload_inputs(w)
+    rng = np.random.default_rng(3)
+    channels = np.sort(rng.choice(w.batch * w.dim, size=384, replace=False))
+    check_forward(inp, channels=channels, what=w.name + " (sampled channels)")
+
+
+# ------------------------------------------------------------------ decode
+def _decode_gpu_step(state, s, dec, y):
+    ssm.ssm_state_update(state, s["u"], s["delta"], dec["A"], s["B"], s["C"], dec["D"], s["z"],
+                         dec["delta_bias"], True, y)
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_decode_small_chain(cuda_device, io):
+    dec = workloads.decode_inputs(3, 50, io=io, seed=21, pool=4)
+    g = dict(A=dec["A"].cuda(), D=dec["D"].cuda(), delta_bias=dec["delta_bias"].cuda())
+    state = dec["state0"].cuda()
+    st_ref = dec["state0"].double().numpy()
+    for step in range(12):
+        s = dec["sets"][step % 4]
+        sg = {k: v.cuda() for k, v in s.items()}
+        y = torch.empty_like(sg["u"])
+        _decode_gpu_step(state, sg, g, y)
+        y_ref, st_ref = oracle.state_update(st_ref, s["u"], s["delta"], dec["A"], s["B"], s["C"], D=dec["D"],
+                                            z=s["z"], delta_bias=dec["delta_bias"])
+        torch.cuda.synchronize()
+        assert_close(y, y_ref, io, f"decode y step {step}")
+        assert_close(state, st_ref, io, f"decode state step {step}")
+
+
+def test_decode_chain_equals_forward(cuda_device):
+    inp = workloads.scan_inputs(2, 40, 64, io="f32", seed=22)
+    y_fwd, last_fwd = gpu_forward(inp)
+    g = to_dev(inp, "cuda")
+    state = torch.zeros(2, 40, 16, device="cuda")
+    ys = []
+    for t in range(64):
+        y = torch.empty(2, 40, device="cuda")
+        ssm.ssm_state_update(state, g["u"][:, :, t].contiguous(), g["delta"][:, :, t].contiguous(), g["A"],
+                             g["B"][:, :, t].contiguous(), g["C"][:, :, t].contiguous(), g["D"],
+                             g["z"][:, :, t].contiguous(), g["delta_bias"], True, y)
+        ys.append(y)
+    torch.cuda.synchronize()
+    y_dec = torch.stack(ys, dim=2)
+    assert_close(y_dec, y_fwd.double().cpu().numpy(), "f32", "decode chain vs forward y")
+    assert_close(state, last_fwd.double().cpu().numpy(), "f32", "decode chain vs forward state")
+
+
+def test_decode_workload_full_size_sampled(cuda_device):
+    w = workloads.WORKLOADS[4]
+    dec = workloads.workload_decode_inputs(w)
+    g = dict(A=dec["A"].cuda(), D=dec["D"].cuda(), delta_bias=dec["delta_bias"].cuda())
+    sets = [{k: v.cuda() for k, v in s.items()} for s in dec["sets"]]
+    state = dec["state0"].cuda()
+    y = torch.empty(w.batch, w.dim, dtype=torch.bfloat16, device="cuda")
+    d0, k = 1234, 8  # sampled channels: every batch row, d in [d0, d0+k)
+    sl = slice(d0, d0 + k)
+    st_ref = dec["state0"][:, sl].double().numpy()
+    A, D, bias = dec["A"][sl], dec["D"][sl], dec["delta_bias"][sl]
+    for step in range(w.decode_steps):
+        s = dec["sets"][step % workloads.POOL]
+        _decode_gpu_step(state, sets[step % workloads.POOL], g, y)
+        y_ref, st_ref = oracle.state_update(st_ref, s["u"][:, sl], s["delta"][:, sl], A, s["B"], s["C"], D=D,
+                                            z=s["z"][:, sl], delta_bias=bias)
+        if step + 1 in (1, 10, w.decode_steps):
+            torch.cuda.synchronize()
+            assert_close(y[:, sl], y_ref, "bf16", f"decode y after {step + 1} steps")
+            assert_close(state[:, sl], st_ref, "bf16", f"decode state after {step + 1} steps")
