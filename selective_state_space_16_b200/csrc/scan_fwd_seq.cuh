@@ -1,9 +1,9 @@
 // scan_fwd_seq.cuh -- forward selective scan, "sequential" kernel family.
 //
-// Each CTA owns R channels of one batch row and walks the whole sequence; the state
-// of every (channel, n) chain stays in registers from t = 0 to t = L-1 and only the
-// final state is written to HBM ([Eng] §4.2: the state lives on chip and only h_N is
-// written back; [S4M] 3.3: state accumulated on chip, written once at the end).
+// Every (channel, n) chain is walked from t = 0 to t = L-1 by one lane, with the state
+// in registers the whole time; only the final state is written to HBM ([Eng] §4.2: the
+// state lives on chip and only h_N is written back; [S4M] 3.3: state accumulated on
+// chip, written once at the end).
 //
 // Pages (sections as printed):
 //   [Eng]  "Mamba 选择性状态空间模型：亚二次复杂度大语言模型推理工程实践"
@@ -11,19 +11,27 @@
 //   [S4M]  "State Space Models 深度实战：从 S4 到 Mamba 的架构演进与 CUDA 优化"
 //   [Hist] "AI底层架构的一场革命：Mamba如何用「状态压缩」挑战Transformer的十年统治"
 //
-// Work split.  G lanes share one channel; lane `nl` of the group holds the NC = 16/G
-// chains n = nl*NC .. nl*NC+NC-1 in registers.  Per step each lane computes
+// Work split.  Channels are grouped in tiles of 8 consecutive channels of one batch
+// row; the tiles are spread evenly over one persistent CTA per SM (each CTA takes a
+// contiguous range, so every SM carries the same number of channel-steps to within
+// one warp's share).  G lanes share a channel: lane `nl` of the group holds the
+// NC = 16/G chains n = nl*NC .. nl*NC+NC-1, for CPL channels of the same batch row
+// (CPL = 2 lets one load of a step's B/C rows serve two channels; the shared-memory
+// data path is the scarce resource of this kernel).  Per step each lane computes
 //   a = 2^(Delta * A[d,n] * log2 e),  h = a*h + (Delta*u)*B[n],  y_partial += C[n]*h
+// (simplified discretisation Abar = exp(Delta A), Bbar = Delta B: [Card] 离散化变换),
 // and the G partial sums of y_t = sum_n C_t[n] h_t[n] are combined by a shuffle
-// reduce-scatter over each 16-byte group of steps, so that every lane finishes the
-// epilogue (D skip, silu gate, rounding) of GS/G steps and no work is duplicated.
+// reduce-scatter over each 16-byte group of GS steps, so that every lane finishes the
+// epilogue (D skip, silu gate, rounding, store) of GS/G steps and nothing is evaluated
+// twice.  The step sizes Delta = softplus(delta + bias) of group q+1 are computed
+// (split over the G lanes) while group q is scanned, and exchanged by shuffles.
 //
-// Staging.  A producer warp streams each stage (TC steps = one 128-byte row per
-// channel) of u, delta, z for the CTA's R channels plus the stage's B/C (already
-// transposed to fp32 [t][32] in the workspace) into shared memory with TMA, two
-// stages deep, signalled through mbarriers.  u/delta/z/y tiles use the 128-byte
-// swizzle, so the per-lane 16-byte reads of one column hit distinct banks.
-// Outputs go through a per-warp shared-memory tile and a TMA store.
+// Staging.  A producer warp streams stage k (TC steps: one 128-byte row per channel)
+// of u, delta and z for all the CTA's tiles, plus the stage's B/C rows (transposed in
+// the workspace to fp32 [t][32]; at most two batch rows per CTA) into shared memory
+// with TMA, through a ring of S stages signalled by mbarriers.  The 8-row u/delta/z
+// boxes use the 128-byte swizzle, so the per-lane 16-byte reads of one column hit
+// distinct banks; B/C are read as broadcasts.
 #pragma once
 
 #include "common.cuh"
@@ -36,10 +44,13 @@ struct SeqParams {
     const float* D;        // (dim) or null
     const float* bias;     // (dim) or null
     float* last_state;     // (batch, dim, 16) or null
+    void* y;               // (batch, dim, L) IO
     WorkspaceHeader* hdr;  // status word
     int batch, dim;
     long long L;
-    int tiles_per_batch;
+    int tiles_per_batch;   // ceil(dim / 8), rounded up to the tiles one warp covers
+    long long total_tiles; // batch * tiles_per_batch
+    int max_tiles;         // tiles one CTA stages per round (sets the shared-memory layout)
     int softplus;
     int has_z;
     uint32_t wait_limit;
@@ -47,24 +58,32 @@ struct SeqParams {
 
 __host__ __device__ constexpr int round_up_i(int v, int m) { return (v + m - 1) / m * m; }
 
-template <typename IO, int G, int NW>
+template <typename IO, int G, int CPL>
 struct SeqCfg {
-    static constexpr int kNC = 16 / G;                       // chains per lane
-    static constexpr int kCW = 32 / G;                       // channels per warp
-    static constexpr int kR = NW * kCW;                      // channels per CTA
+    static constexpr int kNC = 16 / G;                       // chains per lane and channel
+    static constexpr int kCW = 32 / G;                       // channel groups per warp
+    static constexpr int kCPW = kCW * CPL;                   // channels per warp
+    static constexpr int kTPW = kCPW >= 8 ? kCPW / 8 : 1;    // tiles per warp (a warp never spans batches)
     static constexpr int kGS = 16 / IoTraits<IO>::kBytes;    // steps per 16-byte group
+    static constexpr int kPER = kGS / G;                     // epilogue steps per lane per group
     static constexpr int kTC = 128 / IoTraits<IO>::kBytes;   // steps per stage
     static constexpr int kNG = kTC / kGS;                    // groups per stage (8)
-    static constexpr int kStages = 2;
-    static constexpr int kTileLoad = kR * 128;               // bytes one u/delta/z box carries
-    static constexpr int kTile = round_up_i(kTileLoad, 1024);
-    static constexpr int kBC = kTC * 128;                    // fp32 [TC][32] B/C rows
-    static constexpr int kStage = 3 * kTile + round_up_i(kBC, 1024);
-    static constexpr int kOutWarp = round_up_i(kCW * 128, 1024);
-    static constexpr int kSmem = kStages * kStage + 2 * NW * kOutWarp + 1024;  // +1024: alignment slack
-    static constexpr int kThreads = (NW + 1) * 32;           // NW consumer warps + 1 producer warp
-    static_assert(G >= 2 && G <= kGS && (16 % G) == 0, "G lanes must split a 16-byte group");
-    static_assert(kNC % 2 == 0, "chains are processed in fp32 pairs");
+    static constexpr int kTileBytes = 1024;                  // 8 rows x 128 bytes (one swizzle atom)
+    static constexpr int kBC = kTC * 128;                    // fp32 [TC][32] B/C rows of one batch row
+    static constexpr int kMaxBatchRows = 2;                  // batch rows one CTA round may span
+    // consumer warps per CTA (sets the register budget through the launch bound)
+    static constexpr int kMaxWarps = CPL == 2 ? 12 : G == 2 ? 12 : G == 4 ? (sizeof(IO) == 2 ? 18 : 16) : 22;
+    static_assert((G == 2 || G == 4 || G == 8) && G <= kGS, "G is 2, 4 or 8 and splits a 16-byte group");
+    static_assert(CPL == 1 || CPL == 2, "one or two channels per lane");
+    static_assert(kCPW % 8 == 0 || 8 % kCPW == 0, "warps tile the 8-channel tiles");
+
+    __host__ __device__ static constexpr int warps_for(int tiles) { return (tiles * 8 + kCPW - 1) / kCPW; }
+    __host__ __device__ static constexpr int stage_bytes(int max_tiles) {
+        return 3 * max_tiles * kTileBytes + kMaxBatchRows * kBC;
+    }
+    __host__ __device__ static constexpr int smem_bytes(int max_tiles, int stages) {
+        return stages * stage_bytes(max_tiles) + 1024;  // +1024: alignment slack
+    }
 };
 
 __device__ __forceinline__ float2 f2(float x, float y) { return make_float2(x, y); }
@@ -89,211 +108,307 @@ __device__ __forceinline__ void load_run(const uint8_t* src, float (&out)[N]) {
     }
 }
 
-template <typename IO, int G, int NW>
-__global__ void __launch_bounds__((NW + 1) * 32)
+// Store N fp32 values as N consecutive IO elements at a naturally aligned address.
+template <typename IO, int N>
+__device__ __forceinline__ void store_run(IO* dst, const float (&v)[N]) {
+    if constexpr (sizeof(IO) == 2 && N == 4) {
+        *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+    } else if constexpr (sizeof(IO) == 2 && N == 2) {
+        *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(v[0], v[1]);
+    } else if constexpr (sizeof(IO) == 4 && N == 2) {
+        *reinterpret_cast<float2*>(dst) = make_float2(v[0], v[1]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < N; ++i) dst[i] = IoTraits<IO>::from_f32(v[i]);
+    }
+}
+
+template <typename IO, int G, int CPL, int S>
+__global__ void __launch_bounds__((SeqCfg<IO, G, CPL>::kMaxWarps + 1) * 32, 1)
 scan_fwd_seq_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_dl,
                     const __grid_constant__ CUtensorMap map_z, const __grid_constant__ CUtensorMap map_bc,
-                    const __grid_constant__ CUtensorMap map_y, const SeqParams p) {
-    using Cfg = SeqCfg<IO, G, NW>;
-    constexpr int NC = Cfg::kNC, CW = Cfg::kCW, R = Cfg::kR, GS = Cfg::kGS, TC = Cfg::kTC, NG = Cfg::kNG;
-    constexpr int S = Cfg::kStages;
+                    const SeqParams p) {
+    using Cfg = SeqCfg<IO, G, CPL>;
+    constexpr int NC = Cfg::kNC, CW = Cfg::kCW, CPW = Cfg::kCPW, GS = Cfg::kGS, TC = Cfg::kTC, NG = Cfg::kNG;
+    constexpr int PER = Cfg::kPER, ES = IoTraits<IO>::kBytes, TPW = Cfg::kTPW;
+    static_assert(S >= 2 && S <= 8, "ring depth");
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t full_bar[S], empty_bar[S];
     __shared__ int abort_flag;
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned base for the swizzled tiles (pointer arithmetic keeps the shared
+    // address space visible to the compiler).
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int b = blockIdx.x / p.tiles_per_batch;
-    const int d0 = (blockIdx.x % p.tiles_per_batch) * R;
-    const int nstages = static_cast<int>((p.L + TC - 1) / TC);
+    const int stage_bytes = Cfg::stage_bytes(p.max_tiles);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int producer_warp = blockDim.x / 32 - 1;
+    const int L32 = static_cast<int>(p.L);  // the host launches this kernel for L < 2^31 - 1024 only
+    const int nstages = (L32 + TC - 1) / TC;
 
-    if (tid == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&full_bar[s], 1);
-            mbar_init(&empty_bar[s], NW);
+    // This CTA's tiles: [t_begin, t_end) of the flat (batch row, 8-channel tile) order,
+    // cut at multiples of the tiles one warp covers (so no warp straddles two batch rows:
+    // tiles_per_batch is a multiple of TPW, padded with empty tiles past `dim`).
+    const long long units = p.total_tiles / TPW;
+    const long long t_begin = units * blockIdx.x / gridDim.x * TPW;
+    const long long t_end = units * (blockIdx.x + 1) / gridDim.x * TPW;
+
+    // Rounds of at most max_tiles tiles (one round for the shapes the host launches;
+    // more when the tiles do not fit in shared memory at once).
+    for (long long r_begin = t_begin; r_begin < t_end; r_begin += p.max_tiles) {
+        const int nt = static_cast<int>(min(static_cast<long long>(p.max_tiles), t_end - r_begin));
+        const int b_first = static_cast<int>(r_begin / p.tiles_per_batch);
+        const int nb = static_cast<int>((r_begin + nt - 1) / p.tiles_per_batch) - b_first + 1;  // 1 or 2
+        const int nwarps = Cfg::warps_for(nt);
+
+        if (threadIdx.x == 0) {
+            for (int s = 0; s < S; ++s) {
+                mbar_init(&full_bar[s], 1);
+                mbar_init(&empty_bar[s], nwarps);
+            }
+            abort_flag = 0;
+            mbar_fence_init();
         }
-        abort_flag = 0;
-        mbar_fence_init();
-    }
-    __syncthreads();
+        __syncthreads();
 
-    // ---------------------------------------------------------------- producer warp
-    if (warp == NW) {
-        if (lane != 0) return;
-        tma_prefetch_map(&map_u);
-        tma_prefetch_map(&map_dl);
-        tma_prefetch_map(&map_bc);
-        if (p.has_z) tma_prefetch_map(&map_z);
-        const uint32_t bytes = (p.has_z ? 3u : 2u) * Cfg::kTileLoad + Cfg::kBC;
-        for (int k = 0; k < nstages; ++k) {
-            const int s = k % S;
-            if (k >= S) {
-                if (!mbar_wait_bounded(&empty_bar[s], ((k / S) - 1) & 1, p.wait_limit)) {
-                    report_status(p.hdr, kDevTimeout, 1, blockIdx.x, k, p.wait_limit);
-                    abort_flag = 1;
-                    return;
+        if (warp == producer_warp) {
+            // ------------------------------------------------------------ producer
+            if (lane == 0) {
+                if (r_begin == t_begin) {
+                    tma_prefetch_map(&map_u);
+                    tma_prefetch_map(&map_dl);
+                    tma_prefetch_map(&map_bc);
+                    if (p.has_z) tma_prefetch_map(&map_z);
+                }
+                const uint32_t bytes = nt * (p.has_z ? 3u : 2u) * Cfg::kTileBytes + nb * Cfg::kBC;
+                for (int k = 0; k < nstages; ++k) {
+                    const int s = k % S;
+                    if (k >= S && !mbar_wait_bounded(&empty_bar[s], ((k / S) - 1) & 1, p.wait_limit)) {
+                        report_status(p.hdr, kDevTimeout, 1, blockIdx.x, k, p.wait_limit);
+                        atomicExch(&abort_flag, 1);
+                        break;
+                    }
+                    uint8_t* st = smem + s * stage_bytes;
+                    fence_proxy_async_smem();
+                    mbar_arrive_expect_tx(&full_bar[s], bytes);
+                    const int t0 = k * TC;
+                    for (int j = 0; j < nt; ++j) {
+                        const long long tile = r_begin + j;
+                        const int b = static_cast<int>(tile / p.tiles_per_batch);
+                        const int dd = static_cast<int>(tile % p.tiles_per_batch) * 8;
+                        tma_load_3d(st + j * Cfg::kTileBytes, &map_u, &full_bar[s], t0, dd, b);
+                        tma_load_3d(st + (p.max_tiles + j) * Cfg::kTileBytes, &map_dl, &full_bar[s], t0, dd, b);
+                        if (p.has_z)
+                            tma_load_3d(st + (2 * p.max_tiles + j) * Cfg::kTileBytes, &map_z, &full_bar[s], t0, dd, b);
+                    }
+                    for (int bb = 0; bb < nb; ++bb)
+                        tma_load_3d(st + 3 * p.max_tiles * Cfg::kTileBytes + bb * Cfg::kBC, &map_bc, &full_bar[s], 0,
+                                    t0, b_first + bb);
                 }
             }
-            uint8_t* st = smem + s * Cfg::kStage;
-            fence_proxy_async_smem();
-            mbar_arrive_expect_tx(&full_bar[s], bytes);
-            const int t0 = k * TC;
-            tma_load_3d(st, &map_u, &full_bar[s], t0, d0, b);
-            tma_load_3d(st + Cfg::kTile, &map_dl, &full_bar[s], t0, d0, b);
-            if (p.has_z) tma_load_3d(st + 2 * Cfg::kTile, &map_z, &full_bar[s], t0, d0, b);
-            tma_load_3d(st + 3 * Cfg::kTile, &map_bc, &full_bar[s], 0, t0, b);
-        }
-        return;
-    }
-
-    // ---------------------------------------------------------------- consumer warps
-    const int chw = lane / G;           // channel within the warp
-    const int nl = lane % G;            // which NC-chain slice of the channel this lane holds
-    const int row = warp * CW + chw;    // channel row within the CTA tile
-    const int d = d0 + row;
-    const bool valid = d < p.dim;
-
-    float A2[NC];
-    float h[NC];
+        } else if (warp < nwarps) {
+            // ------------------------------------------------------------ consumers
+            // Lane (cg, nl) holds the NC chains n = nl*NC .. of the channels cg + c*CW
+            // (c < CPL) of this warp's block of CPW channels; the CPL channels share the
+            // batch row, hence every B/C value the lane loads.
+            const int cg = lane / G;
+            const int nl = lane % G;
+            const int gbase = lane & ~(G - 1);   // first lane of this channel group
+            int j[CPL], row[CPL], d[CPL];
+            bool valid[CPL];
+            int b = 0;
 #pragma unroll
-    for (int j = 0; j < NC; ++j) {
-        A2[j] = valid ? p.A[d * 16 + nl * NC + j] * kLog2e : 0.f;
-        h[j] = 0.f;
-    }
-    const float Dd = (valid && p.D) ? p.D[d] : 0.f;
-    const float bias = (valid && p.bias) ? p.bias[d] : 0.f;
-    const bool softplus = p.softplus != 0;
-    const bool has_z = p.has_z != 0;
+            for (int c = 0; c < CPL; ++c) {
+                const int cl = warp * CPW + cg + c * CW;   // channel within the round's tiles
+                const bool in_round = cl < nt * 8;
+                j[c] = in_round ? cl / 8 : 0;
+                row[c] = cl % 8;
+                const long long tile = r_begin + j[c];
+                if (c == 0) b = static_cast<int>(tile / p.tiles_per_batch);
+                d[c] = static_cast<int>(tile % p.tiles_per_batch) * 8 + row[c];
+                valid[c] = in_round && d[c] < p.dim;
+            }
+            const int bcs = b - b_first;         // B/C slot of this batch row
 
-    for (int k = 0; k < nstages; ++k) {
-        const int s = k % S;
-        // The outcome of the bounded wait is made warp-uniform, so that a timeout can
-        // never leave part of the warp inside the full-mask shuffles below.
-        const bool ready = __all_sync(0xffffffffu, mbar_wait_bounded(&full_bar[s], (k / S) & 1, p.wait_limit));
-        if (!ready) {
-            if (lane == 0) report_status(p.hdr, kDevTimeout, 2, blockIdx.x, k, p.wait_limit);
-            break;
-        }
-        if (__any_sync(0xffffffffu, *(volatile int*)&abort_flag != 0)) break;
-        const uint8_t* st = smem + s * Cfg::kStage;
-        const uint8_t* tu = st;
-        const uint8_t* tdl = st + Cfg::kTile;
-        const uint8_t* tz = st + 2 * Cfg::kTile;
-        const float* bc = reinterpret_cast<const float*>(st + 3 * Cfg::kTile);
-        uint8_t* out = smem + S * Cfg::kStage + (warp * 2 + (k & 1)) * Cfg::kOutWarp;
+            float2 A2[CPL][NC / 2], h[CPL][NC / 2];
+            float Dd[CPL], bias[CPL];
+            IO* yrow[CPL];
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) {
+#pragma unroll
+                for (int jj = 0; jj < NC / 2; ++jj) {
+                    const float a0 = valid[c] ? p.A[d[c] * 16 + nl * NC + 2 * jj] : 0.f;
+                    const float a1 = valid[c] ? p.A[d[c] * 16 + nl * NC + 2 * jj + 1] : 0.f;
+                    A2[c][jj] = f2(a0 * kLog2e, a1 * kLog2e);
+                    h[c][jj] = f2(0.f, 0.f);
+                }
+                Dd[c] = (valid[c] && p.D) ? p.D[d[c]] : 0.f;
+                bias[c] = (valid[c] && p.bias) ? p.bias[d[c]] : 0.f;
+                yrow[c] = static_cast<IO*>(p.y) + (static_cast<long long>(b) * p.dim + (valid[c] ? d[c] : 0)) * p.L;
+            }
+            const bool softplus = p.softplus != 0;
+            const bool has_z = p.has_z != 0;
 
-        // The TMA store issued from this buffer two stages ago must have read it.
-        if (lane == 0) bulk_wait_read<1>();
-        __syncwarp();
+            auto stage_of = [&](int q) -> const uint8_t* { return smem + ((q / NG) % S) * stage_bytes; };
+            auto chunk_of = [&](int q, int c) -> int {
+                return j[c] * Cfg::kTileBytes + row[c] * 128 + (((q % NG) ^ row[c]) << 4);
+            };
 
-        const long long t_stage = static_cast<long long>(k) * TC;
+            // Bounded, warp-uniform wait for the stage that holds group q (a timeout can
+            // never leave part of the warp inside the full-mask shuffles).
+            auto wait_stage = [&](int q) -> bool {
+                const int k = q / NG;
+                const bool ok =
+                    __all_sync(0xffffffffu, mbar_wait_bounded(&full_bar[k % S], (k / S) & 1, p.wait_limit));
+                if (!ok && lane == 0) report_status(p.hdr, kDevTimeout, 2, blockIdx.x, k, p.wait_limit);
+                return ok && !__any_sync(0xffffffffu, *(volatile int*)&abort_flag != 0);
+            };
+
+            // Step sizes of group q: lane nl evaluates softplus for its PER steps
+            // i = r*G + nl of each of its channels (issued one group ahead of the scan).
+            auto prologue = [&](int q, float (&mine)[CPL][PER]) {
+                const uint8_t* dl = stage_of(q) + p.max_tiles * Cfg::kTileBytes;
+#pragma unroll
+                for (int c = 0; c < CPL; ++c)
+#pragma unroll
+                    for (int r = 0; r < PER; ++r) {
+                        const int i = r * G + nl;
+                        const float raw =
+                            IoTraits<IO>::to_f32(*reinterpret_cast<const IO*>(dl + chunk_of(q, c) + i * ES));
+                        mine[c][r] = (q * GS + i < L32) ? step_size(raw, bias[c], softplus) : 0.f;  // 0 past L
+                    }
+            };
+
+            // Scan, reduce-scatter and epilogue of group q.  The G lanes of a channel group
+            // exchange their step sizes by shuffles, so each lane has Delta and Delta*u of
+            // every step; one B/C load per step serves all CPL channels of the lane.
+            auto scan_group = [&](int q, const float (&mine)[CPL][PER]) {
+                const uint8_t* st = stage_of(q);
+                float uf[CPL][GS];
+#pragma unroll
+                for (int c = 0; c < CPL; ++c)
+                    Group16<IO>::unpack(*reinterpret_cast<const uint4*>(st + chunk_of(q, c)), uf[c]);
+                const float* bc = reinterpret_cast<const float*>(st + 3 * p.max_tiles * Cfg::kTileBytes +
+                                                                 bcs * Cfg::kBC) +
+                                  (q % NG) * GS * 32 + nl * NC;
+                float yp[CPL][GS];
+#pragma unroll
+                for (int i = 0; i < GS; ++i) {
+                    const float* bcr = bc + i * 32;
+                    float2 Bv[NC / 2], Cv[NC / 2];
+#pragma unroll
+                    for (int jj = 0; jj < NC / 2; ++jj) {
+                        if constexpr (NC >= 4) {
+                            const float4 Bq = *reinterpret_cast<const float4*>(bcr + (jj & ~1) * 2);
+                            const float4 Cq = *reinterpret_cast<const float4*>(bcr + 16 + (jj & ~1) * 2);
+                            Bv[jj] = (jj & 1) ? f2(Bq.z, Bq.w) : f2(Bq.x, Bq.y);
+                            Cv[jj] = (jj & 1) ? f2(Cq.z, Cq.w) : f2(Cq.x, Cq.y);
+                        } else {
+                            Bv[jj] = *reinterpret_cast<const float2*>(bcr + 2 * jj);
+                            Cv[jj] = *reinterpret_cast<const float2*>(bcr + 16 + 2 * jj);
+                        }
+                    }
+#pragma unroll
+                    for (int c = 0; c < CPL; ++c) {
+                        const float dti = __shfl_sync(0xffffffffu, mine[c][i / G], gbase | (i % G), 32);
+                        const float wi = dti * uf[c][i];
+                        const float2 dd = f2(dti, dti);
+                        const float2 ww = f2(wi, wi);
+                        float2 acc = f2(0.f, 0.f);
+#pragma unroll
+                        for (int jj = 0; jj < NC / 2; ++jj) {
+                            const float2 arg = __fmul2_rn(dd, A2[c][jj]);
+                            const float2 a = f2(ex2_mufu(arg.x), ex2_mufu(arg.y));
+                            h[c][jj] = __ffma2_rn(a, h[c][jj], __fmul2_rn(ww, Bv[jj]));
+                            acc = __ffma2_rn(Cv[jj], h[c][jj], acc);
+                        }
+                        yp[c][i] = acc.x + acc.y;
+                    }
+                }
+
+                // Reduce-scatter the G partial sums of each channel: afterwards lane nl holds
+                // the full y_t of steps nl*PER .. nl*PER+PER-1 in yp[c][0..PER-1].
+#pragma unroll
+                for (int m = G / 2, half = GS / 2; m >= 1; m >>= 1, half >>= 1) {
+                    const bool upper = (nl & m) != 0;
+#pragma unroll
+                    for (int c = 0; c < CPL; ++c)
+#pragma unroll
+                        for (int i = 0; i < half; ++i) {
+                            const float send = upper ? yp[c][i] : yp[c][i + half];
+                            const float keep = upper ? yp[c][i + half] : yp[c][i];
+                            yp[c][i] = keep + __shfl_xor_sync(0xffffffffu, send, m, 32);
+                        }
+                }
+
+                // Epilogue: D skip and silu gate ([Eng] §2.2; [Hist] Mamba Block), round, store.
+                const int t0 = q * GS + nl * PER;
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) {
+                    const int off = chunk_of(q, c) + nl * PER * ES;
+                    float ue[PER], ze[PER], yo[PER];
+                    load_run<IO, PER>(st + off, ue);
+                    if (has_z) load_run<IO, PER>(st + 2 * p.max_tiles * Cfg::kTileBytes + off, ze);
+#pragma unroll
+                    for (int r = 0; r < PER; ++r) {
+                        float v = fmaf(Dd[c], ue[r], yp[c][r]);
+                        if (has_z) v *= gate_silu<IO>(ze[r]);
+                        yo[r] = v;
+                    }
+                    if (valid[c]) {
+                        if (t0 + PER <= L32) {
+                            store_run<IO, PER>(yrow[c] + t0, yo);
+                        } else {
+#pragma unroll
+                            for (int r = 0; r < PER; ++r)
+                                if (t0 + r < L32) yrow[c][t0 + r] = IoTraits<IO>::from_f32(yo[r]);
+                        }
+                    }
+                }
+                // The last group of a stage releases the stage to the producer.
+                if (q % NG == NG - 1) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty_bar[(q / NG) % S]);
+                }
+            };
+
+            // Groups two per iteration with ping-pong step-size buffers: while group q is
+            // scanned the next group's step sizes are computed into the other buffer.
+            const int ngroups = nstages * NG;
+            float spA[CPL][PER], spB[CPL][PER];
+            bool alive = wait_stage(0);
+            if (alive) prologue(0, spA);
 #pragma unroll 1
-        for (int g = 0; g < NG; ++g) {
-            const int chunk = row * 128 + (g ^ (row & 7)) * 16;
-            float uf[GS];
-            Group16<IO>::unpack(*reinterpret_cast<const uint4*>(tu + chunk), uf);
-
-            // Step sizes: each of the G lanes evaluates softplus for the PER = GS/G steps
-            // i = q*G + nl of the group, then the group exchanges them by shuffles, so every
-            // lane has all GS step sizes and no softplus is evaluated twice.
-            constexpr int PER = GS / G;
-            float mine[PER];
-#pragma unroll
-            for (int q = 0; q < PER; ++q) {
-                const int i = q * G + nl;
-                const float raw = IoTraits<IO>::to_f32(
-                    *reinterpret_cast<const IO*>(tdl + chunk + i * IoTraits<IO>::kBytes));
-                const long long t = t_stage + g * GS + i;
-                mine[q] = (t < p.L) ? step_size(raw, bias, softplus) : 0.f;
-            }
-            float dt[GS];
-#pragma unroll
-            for (int i = 0; i < GS; ++i)
-                dt[i] = __shfl_sync(0xffffffffu, mine[i / G], (lane & ~(G - 1)) | (i % G), 32);
-
-            float yp[GS];
-#pragma unroll
-            for (int i = 0; i < GS; ++i) {
-                const float* bcr = bc + (g * GS + i) * 32;
-                const float w = dt[i] * uf[i];
-                const float2 dd = f2(dt[i], dt[i]);
-                const float2 ww = f2(w, w);
-                float2 acc = f2(0.f, 0.f);
-#pragma unroll
-                for (int j = 0; j < NC; j += 2) {
-                    // B and C of chains j, j+1 (8-byte aligned pairs; NC may be 2).
-                    const float2 Bp = *reinterpret_cast<const float2*>(bcr + nl * NC + j);
-                    const float2 Cp = *reinterpret_cast<const float2*>(bcr + 16 + nl * NC + j);
-                    const float2 arg = __fmul2_rn(dd, f2(A2[j], A2[j + 1]));
-                    const float2 a = f2(ex2_mufu(arg.x), ex2_mufu(arg.y));
-                    const float2 hn = __ffma2_rn(a, f2(h[j], h[j + 1]), __fmul2_rn(ww, Bp));
-                    h[j] = hn.x;
-                    h[j + 1] = hn.y;
-                    acc = __ffma2_rn(Cp, hn, acc);
+            for (int q = 0; alive && q < ngroups; q += 2) {
+                if (q + 1 < ngroups) {
+                    if ((q + 1) % NG == 0) alive = wait_stage(q + 1);
+                    if (alive) prologue(q + 1, spB);
                 }
-                yp[i] = acc.x + acc.y;
+                scan_group(q, spA);
+                if (!alive || q + 1 >= ngroups) break;
+                if (q + 2 < ngroups) {
+                    if ((q + 2) % NG == 0) alive = wait_stage(q + 2);
+                    if (alive) prologue(q + 2, spA);
+                }
+                scan_group(q + 1, spB);
             }
 
-            // Reduce-scatter the G partial sums: after it, lane nl holds the full
-            // y_t for steps nl*PER .. nl*PER+PER-1 of this group in yp[0..PER-1].
 #pragma unroll
-            for (int m = G / 2, half = GS / 2; m >= 1; m >>= 1, half >>= 1) {
-                const bool upper = (nl & m) != 0;
+            for (int c = 0; c < CPL; ++c)
+                if (valid[c] && p.last_state) {
+                    float* dst = p.last_state + (static_cast<long long>(b) * p.dim + d[c]) * 16 + nl * NC;
 #pragma unroll
-                for (int i = 0; i < half; ++i) {
-                    const float send = upper ? yp[i] : yp[i + half];
-                    const float keep = upper ? yp[i + half] : yp[i];
-                    yp[i] = keep + __shfl_xor_sync(0xffffffffu, send, m, 32);
+                    for (int jj = 0; jj < NC / 2; ++jj) *reinterpret_cast<float2*>(dst + 2 * jj) = h[c][jj];
                 }
-            }
-
-            // Epilogue: D skip and silu gate for this lane's PER steps, rounded to IO.
-            float ue[PER], ze[PER];
-            load_run<IO, PER>(tu + chunk + nl * PER * IoTraits<IO>::kBytes, ue);
-            if (has_z) load_run<IO, PER>(tz + chunk + nl * PER * IoTraits<IO>::kBytes, ze);
-            float yo[PER];
-#pragma unroll
-            for (int q = 0; q < PER; ++q) {
-                float v = fmaf(Dd, ue[q], yp[q]);
-                if (has_z) v *= silu_f32(ze[q]);
-                yo[q] = v;
-            }
-            uint8_t* orow = out + chw * 128 + ((g ^ (chw & 7)) * 16) + nl * PER * IoTraits<IO>::kBytes;
-            if constexpr (sizeof(IO) == 2) {
-                if constexpr (PER == 4) {
-                    *reinterpret_cast<uint2*>(orow) = make_uint2(pack_bf16x2(yo[0], yo[1]), pack_bf16x2(yo[2], yo[3]));
-                } else if constexpr (PER == 2) {
-                    *reinterpret_cast<uint32_t*>(orow) = pack_bf16x2(yo[0], yo[1]);
-                } else {
-                    *reinterpret_cast<__nv_bfloat16*>(orow) = __float2bfloat16_rn(yo[0]);
-                }
-            } else {
-                if constexpr (PER == 2) {
-                    *reinterpret_cast<float2*>(orow) = make_float2(yo[0], yo[1]);
-                } else {
-                    *reinterpret_cast<float*>(orow) = yo[0];
-                }
-            }
         }
-
-        // Release the input stage to the producer, then store this warp's output tile.
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty_bar[s]);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0 && d0 + warp * CW < p.dim) {  // a box wholly past `dim` has nothing to store
-            tma_store_3d(&map_y, out, static_cast<int>(t_stage), d0 + warp * CW, b);
-            bulk_commit();
-        }
-    }
-    if (lane == 0) bulk_wait_all<0>();
-
-    if (valid && p.last_state) {
-        float* dst = p.last_state + (static_cast<long long>(b) * p.dim + d) * 16 + nl * NC;
-#pragma unroll
-        for (int j = 0; j < NC; j += 4)
-            *reinterpret_cast<float4*>(dst + j) = make_float4(h[j], h[j + 1], h[j + 2], h[j + 3]);
+        // Every warp leaves the round before the barriers are re-initialised for the next.
+        __syncthreads();
+        if (threadIdx.x == 0)
+            for (int s = 0; s < S; ++s) {
+                mbar_inval(&full_bar[s]);
+                mbar_inval(&empty_bar[s]);
+            }
+        __syncthreads();
     }
 }
 

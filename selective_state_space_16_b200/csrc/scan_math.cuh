@@ -8,6 +8,8 @@
 
 #include <cuda_runtime.h>
 
+#include "poly_coeffs.cuh"
+
 namespace ssm {
 
 constexpr float kLog2e = 1.4426950408889634f;  // log2(e): exp(x) = 2^(x log2 e)
@@ -20,10 +22,18 @@ __device__ __forceinline__ float ex2_mufu(float x) {
 }
 
 // Step size Delta = softplus(x) with x = delta + bias ([Eng] §3.2: the bias sits inside
-// softplus; [Card] 选择性机制: softplus keeps the step positive).  Above x = 20 the
-// correction log1p(e^-x) < 2.1e-9 is below fp32 resolution of x, so x is returned.
+// softplus; [Card] 选择性机制: softplus keeps the step positive), evaluated as
+//   softplus(x) = max(x, 0) + log1p(e),  e = e^{-|x|} in (0, 1],
+// with log1p(e) = e * P(e) from a degree-8 polynomial fitted on [0, 1] (gen_poly.py;
+// relative error 2.3e-7 in fp32).  One special-function op (the exponential); for
+// x < -87 e flushes to zero and the result is 0 (the true value is below 1e-38).
 __device__ __forceinline__ float softplus_f32(float x) {
-    return x > 20.f ? x : log1pf(ex2_mufu(x * kLog2e));
+    constexpr float c[] = SSM_LOG1P_POLY;
+    const float e = ex2_mufu(-fabsf(x) * kLog2e);
+    float p = c[8];
+#pragma unroll
+    for (int i = 7; i >= 0; --i) p = fmaf(p, e, c[i]);
+    return fmaf(e, p, fmaxf(x, 0.f));
 }
 
 __device__ __forceinline__ float step_size(float raw, float bias, bool softplus) {
@@ -35,6 +45,24 @@ __device__ __forceinline__ float step_size(float raw, float bias, bool softplus)
 // For z -> -inf the denominator overflows to +inf and the result is 0.
 __device__ __forceinline__ float silu_f32(float z) {
     return __fdividef(z, 1.f + ex2_mufu(-z * kLog2e));
+}
+
+// silu(z) = z * sigmoid(z) with sigmoid(z) = (1 + tanh(z/2)) / 2 on the special-function
+// unit (tanh.approx, relative error <= 2^-11): one special-function op instead of two.
+// Used only where the gated output is rounded to bf16 (relative step 2^-8), so the
+// approximation stays below the output's own rounding.
+__device__ __forceinline__ float silu_tanh_f32(float z) {
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * z));
+    return z * fmaf(0.5f, t, 0.5f);
+}
+
+// The gate used for an output element type: accurate for fp32 outputs, the one-op
+// tanh form for bf16 outputs.
+template <typename IO>
+__device__ __forceinline__ float gate_silu(float z) {
+    if constexpr (sizeof(IO) == 2) return silu_tanh_f32(z);
+    else return silu_f32(z);
 }
 
 }  // namespace ssm

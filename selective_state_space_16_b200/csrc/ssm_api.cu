@@ -2,6 +2,8 @@
 // validation, workspace layout, TMA tensor maps, kernel choice and launches.
 // Everything here is marshalling; every step of the scan runs in the kernels.
 #include <cstdint>
+#include <algorithm>
+#include <cmath>
 #include <cstring>
 #include <mutex>
 #include <set>
@@ -88,15 +90,22 @@ ssm_status_t launch_status() {
     return e == cudaSuccess ? SSM_OK : SSM_ERR_LAUNCH;
 }
 
-// Per-device "max dynamic shared memory" opt-in, remembered per (kernel, device).
+// Opt a kernel into the largest dynamic shared memory per block the device allows next
+// to its static shared memory, once per (kernel, device); `bytes` is checked against it.
 bool ensure_smem_attr(const void* kernel, int bytes) {
     static std::mutex mu;
     static std::set<std::pair<const void*, int>> done;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    int dev = 0, optin = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+        return false;
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return false;
+    const int limit = optin - static_cast<int>(fa.sharedSizeBytes);  // static + dynamic <= opt-in maximum
+    if (bytes > limit) return false;
     std::lock_guard<std::mutex> lk(mu);
     if (done.count({kernel, dev})) return true;
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, limit) != cudaSuccess) return false;
     done.insert({kernel, dev});
     return true;
 }
@@ -116,41 +125,118 @@ struct FwdArgs {
     int sm_count;
 };
 
-template <typename IO, int G, int NW>
-ssm_status_t launch_seq(const FwdArgs& a) {
-    using Cfg = ssm::SeqCfg<IO, G, NW>;
+template <typename IO, int G, int CPL>
+const void* seq_kernel_ptr(int stages) {
+    switch (stages) {
+        case 2: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 2>);
+        case 3: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 3>);
+        default: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 4>);
+    }
+}
+
+// Launch plan of the sequential kernel: one persistent CTA per SM (two when the tiles
+// do not fit one CTA's warps), each taking an even share of the 8-channel tiles, with
+// as deep a TMA ring as shared memory allows.
+struct SeqPlan {
+    long long total_tiles = 0;
+    int tiles_per_batch = 0, grid = 0, max_tiles = 0, stages = 0, threads = 0, smem = 0, warps_per_sm = 0;
+    bool ok = false;
+};
+
+template <typename IO, int G, int CPL>
+SeqPlan plan_seq(const FwdArgs& a) {
+    using Cfg = ssm::SeqCfg<IO, G, CPL>;
+    SeqPlan pl;
+    pl.tiles_per_batch = ((a.dim + 7) / 8 + Cfg::kTPW - 1) / Cfg::kTPW * Cfg::kTPW;
+    pl.total_tiles = static_cast<long long>(a.batch) * pl.tiles_per_batch;
+    // At most kMaxWarps consumer warps, and a round may span at most two batch rows.
+    // (tiles are handed out in whole-warp units of kTPW tiles).
+    const int tiles_cap = std::min(Cfg::kMaxWarps * Cfg::kCPW / 8 / Cfg::kTPW * Cfg::kTPW,
+                                   pl.tiles_per_batch + Cfg::kTPW);
+    for (int per_sm = 1; per_sm <= 2 && !pl.ok; ++per_sm) {
+        const long long ctas = std::min<long long>(pl.total_tiles, static_cast<long long>(a.sm_count) * per_sm);
+        const long long units = pl.total_tiles / Cfg::kTPW;  // tiles in whole-warp units
+        int mt = static_cast<int>((units + ctas - 1) / ctas) * Cfg::kTPW;
+        if (mt > tiles_cap) {
+            if (per_sm == 1) continue;
+            mt = tiles_cap;  // several rounds per CTA
+        }
+        const int budget = (228 * 1024) / per_sm - 1024 - 256;  // per-CTA reserve and static barriers
+        const int stages = std::min(4, (budget - 1024) / Cfg::stage_bytes(mt));
+        if (stages < 2) continue;
+        const int threads = (Cfg::warps_for(mt) + 1) * 32;
+        const int smem = Cfg::smem_bytes(mt, stages);
+        const void* kern = seq_kernel_ptr<IO, G, CPL>(stages);
+        int occ = 0;
+        if (!ensure_smem_attr(kern, smem) ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, smem) != cudaSuccess || occ < per_sm)
+            continue;
+        pl.grid = static_cast<int>(ctas);
+        pl.max_tiles = mt;
+        pl.stages = stages;
+        pl.threads = threads;
+        pl.smem = smem;
+        pl.warps_per_sm = per_sm * Cfg::warps_for(mt);
+        pl.ok = true;
+    }
+    return pl;
+}
+
+// Relative time of a plan: tiles on the busiest SM, a per-element charge for the
+// variant, and a latency penalty below ~10 consumer warps per SM.
+template <typename IO, int G, int CPL>
+double predict_seq(const FwdArgs& a, const SeqPlan& pl) {
+    if (!pl.ok) return 1e300;
+    const long long per_sm_ctas = (pl.grid + a.sm_count - 1) / a.sm_count;
+    const double rounds = std::ceil(static_cast<double>(pl.total_tiles) / pl.grid / pl.max_tiles);
+    const double tiles = static_cast<double>(per_sm_ctas) * pl.max_tiles * rounds;
+    // Calibrated on B200 (bf16, d_state 16): ~10 resident consumer warps per SM hide the
+    // per-step latencies; two channels per lane or two lanes per channel halve the warps
+    // for the same tiles and measured slower at equal warp counts.
+    const double cost = CPL == 2 ? 1.3 : G == 8 ? 1.12 : 1.0;
+    const double hide = std::min(1.0, pl.warps_per_sm / 10.0);
+    return tiles * cost / hide;
+}
+
+template <typename IO, int G, int CPL>
+ssm_status_t launch_seq(const FwdArgs& a, const SeqPlan& pl) {
+    using Cfg = ssm::SeqCfg<IO, G, CPL>;
+    if (!pl.ok) return SSM_ERR_UNSUPPORTED;
     constexpr int TC = Cfg::kTC;
     constexpr auto sw128 = CU_TENSOR_MAP_SWIZZLE_128B;
     const auto dt = ssm::IoTraits<IO>::kTmaType;
     constexpr int es = ssm::IoTraits<IO>::kBytes;
-    CUtensorMap mu, mdl, mz, mbc, my;
+    CUtensorMap mu, mdl, mz, mbc;
     const uint64_t L = static_cast<uint64_t>(a.L);
-    bool ok = make_map_3d(&mu, dt, es, a.u, L, a.dim, a.batch, TC, Cfg::kR, sw128) &&
-              make_map_3d(&mdl, dt, es, a.delta, L, a.dim, a.batch, TC, Cfg::kR, sw128) &&
-              make_map_3d(&my, dt, es, a.y, L, a.dim, a.batch, TC, Cfg::kCW, sw128) &&
+    bool ok = make_map_3d(&mu, dt, es, a.u, L, a.dim, a.batch, TC, 8, sw128) &&
+              make_map_3d(&mdl, dt, es, a.delta, L, a.dim, a.batch, TC, 8, sw128) &&
               make_map_3d(&mbc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.ws + ws_layout(a.batch, a.dim, a.L).bc_off, 32,
                           L, a.batch, 32, TC, CU_TENSOR_MAP_SWIZZLE_NONE);
-    if (ok && a.z) ok = make_map_3d(&mz, dt, es, a.z, L, a.dim, a.batch, TC, Cfg::kR, sw128);
+    if (ok && a.z) ok = make_map_3d(&mz, dt, es, a.z, L, a.dim, a.batch, TC, 8, sw128);
     if (!a.z) mz = mu;
     if (!ok) return SSM_ERR_LAUNCH;
-    auto kern = ssm::scan_fwd_seq_kernel<IO, G, NW>;
-    if (!ensure_smem_attr(reinterpret_cast<const void*>(kern), Cfg::kSmem)) return SSM_ERR_LAUNCH;
     ssm::SeqParams p{};
     p.A = a.A;
     p.D = a.D;
     p.bias = a.bias;
     p.last_state = a.last_state;
+    p.y = a.y;
     p.hdr = reinterpret_cast<WorkspaceHeader*>(a.ws);
     p.batch = a.batch;
     p.dim = a.dim;
     p.L = a.L;
-    p.tiles_per_batch = (a.dim + Cfg::kR - 1) / Cfg::kR;
+    p.tiles_per_batch = pl.tiles_per_batch;
+    p.total_tiles = pl.total_tiles;
+    p.max_tiles = pl.max_tiles;
     p.softplus = a.softplus;
     p.has_z = a.z != nullptr;
     p.wait_limit = kDefaultWaitLimit;
-    const long long grid = static_cast<long long>(a.batch) * p.tiles_per_batch;
-    if (grid > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
-    kern<<<static_cast<unsigned>(grid), Cfg::kThreads, Cfg::kSmem, a.stream>>>(mu, mdl, mz, mbc, my, p);
+    if (a.L >= (1LL << 31) - 1024) return SSM_ERR_UNSUPPORTED;
+    switch (pl.stages) {
+        case 2: ssm::scan_fwd_seq_kernel<IO, G, CPL, 2><<<pl.grid, pl.threads, pl.smem, a.stream>>>(mu, mdl, mz, mbc, p); break;
+        case 3: ssm::scan_fwd_seq_kernel<IO, G, CPL, 3><<<pl.grid, pl.threads, pl.smem, a.stream>>>(mu, mdl, mz, mbc, p); break;
+        default: ssm::scan_fwd_seq_kernel<IO, G, CPL, 4><<<pl.grid, pl.threads, pl.smem, a.stream>>>(mu, mdl, mz, mbc, p); break;
+    }
     return launch_status();
 }
 
@@ -187,25 +273,6 @@ ssm_status_t launch_pack(const FwdArgs& a) {
     return launch_status();
 }
 
-// Lanes per channel for the sequential kernel: the candidate whose most-loaded SM
-// carries the fewest channel-steps (all CTAs of a candidate are resident at once),
-// with a small charge for the wider reduce-scatter of larger groups.
-int pick_lanes(int batch, int dim, int sm_count, bool bf16) {
-    struct Cand { int G, R, per_sm; double cost; };
-    const Cand cands[] = {{2, 48, 3, 1.00}, {4, 24, 5, 1.04}, {8, 16, 6, 1.10}};
-    int best = 2;
-    double best_t = 1e300;
-    for (const Cand& c : cands) {
-        if (!bf16 && c.G == 8) continue;
-        const long long ctas = static_cast<long long>(batch) * ((dim + c.R - 1) / c.R);
-        const long long waves = (ctas + static_cast<long long>(sm_count) * c.per_sm - 1) / (static_cast<long long>(sm_count) * c.per_sm);
-        const long long per_sm = (ctas + sm_count - 1) / sm_count;
-        const double t = static_cast<double>(per_sm) * c.R * c.cost * (waves > 1 ? 1.05 : 1.0);
-        if (t < best_t - 1e-9) { best_t = t; best = c.G; }
-    }
-    return best;
-}
-
 template <typename IO>
 ssm_status_t launch_forward(const FwdArgs& a, const ssm_fwd_options_t& o) {
     ssm_status_t st = launch_pack<IO>(a);
@@ -216,16 +283,27 @@ ssm_status_t launch_forward(const FwdArgs& a, const ssm_fwd_options_t& o) {
     if (algo == SSM_ALGO_AUTO || algo == SSM_ALGO_CHUNKED) algo = SSM_ALGO_SEQUENTIAL;
     if (!tma_ok) algo = SSM_ALGO_DIRECT;
     if (algo == SSM_ALGO_DIRECT) return launch_direct<IO>(a);
+    // Variants: (lanes per channel G, channels per lane CPL).  lanes_per_channel selects
+    // G explicitly (CPL = 1), or G = 4 with CPL = 2 when given as 42.
+    const SeqPlan p2 = plan_seq<IO, 2, 1>(a), p4 = plan_seq<IO, 4, 1>(a), p42 = plan_seq<IO, 4, 2>(a);
+    SeqPlan p8;
+    if constexpr (sizeof(IO) == 2) p8 = plan_seq<IO, 8, 1>(a);
     int G = o.lanes_per_channel;
-    if (G == 0) G = pick_lanes(a.batch, a.dim, a.sm_count, sizeof(IO) == 2);
-    switch (G) {
-        case 2: return launch_seq<IO, 2, 3>(a);
-        case 4: return launch_seq<IO, 4, 3>(a);
-        case 8:
-            if constexpr (sizeof(IO) == 2) return launch_seq<IO, 8, 4>(a);
-            return SSM_ERR_INVALID_ARG;
-        default: return SSM_ERR_INVALID_ARG;
+    if (G == 0) {
+        const double t[4] = {predict_seq<IO, 2, 1>(a, p2), predict_seq<IO, 4, 1>(a, p4),
+                             sizeof(IO) == 2 ? predict_seq<IO, 8, 1>(a, p8) : 1e300, predict_seq<IO, 4, 2>(a, p42)};
+        const int ids[4] = {2, 4, 8, 42};
+        int best = 1;
+        for (int i = 0; i < 4; ++i)
+            if (t[i] < t[best]) best = i;
+        G = ids[best];
     }
+    if (G == 2) return launch_seq<IO, 2, 1>(a, p2);
+    if (G == 4) return launch_seq<IO, 4, 1>(a, p4);
+    if (G == 42) return launch_seq<IO, 4, 2>(a, p42);
+    if constexpr (sizeof(IO) == 2)
+        if (G == 8) return launch_seq<IO, 8, 1>(a, p8);
+    return SSM_ERR_INVALID_ARG;
 }
 
 }  // namespace

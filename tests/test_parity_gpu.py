@@ -15,12 +15,13 @@ pytestmark = pytest.mark.gpu
 
 
 # ------------------------------------------------------------------ kernel variants, ragged sizes
-VARIANTS = [("sequential", 2), ("sequential", 4), ("sequential", 8), ("direct", 0)]
+VARIANTS = [("sequential", 2), ("sequential", 4), ("sequential", 8), ("sequential", 42), ("direct", 0)]
 
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
 @pytest.mark.parametrize("algo,lanes", VARIANTS, ids=[f"{a}{g or ''}" for a, g in VARIANTS])
 def test_forward_variants_ragged(cuda_device, io, algo, lanes):
+    # lanes: lanes per channel; 42 = 4 lanes per channel, each lane carrying two channels
     if io == "f32" and lanes == 8:
         pytest.skip("8 lanes per channel needs 8 steps per 16-byte group (bf16)")
     # 100 channels: not a multiple of any channel tile; L = 1000: not a multiple of a stage.
