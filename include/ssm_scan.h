@@ -54,7 +54,8 @@ typedef enum {
     SSM_ERR_UNSUPPORTED = 2,   /* dstate != 16, or the current device is not sm_100             */
     SSM_ERR_LAUNCH = 3,        /* a CUDA call or kernel launch failed                           */
     SSM_ERR_TIMEOUT = 4,       /* device: a bounded wait in the kernel gave up (see read_status) */
-    SSM_ERR_WORKSPACE = 5      /* workspace missing or smaller than ssm_selective_scan_workspace_size */
+    SSM_ERR_WORKSPACE = 5,     /* workspace missing or smaller than ssm_selective_scan_workspace_size */
+    SSM_ERR_SCRATCH_LIMIT = 6  /* the problem needs more than the fixed scratch of ssm_selective_scan_fwd_noalloc */
 } ssm_status_t;
 
 typedef enum { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype_t;
@@ -140,6 +141,37 @@ ssm_status_t ssm_state_update(
     float* state, const void* u, const void* delta, const float* A, const void* B, const void* C,
     const float* D, const void* z, const float* delta_bias, int softplus, void* y,
     int batch, int dim, int dstate, ssm_dtype_t io_dtype, ssm_stream_t stream);
+
+/*
+ * Forward scan that allocates nothing and takes no workspace.  The pages have no
+ * counterpart: this entry point exists for callers that are handed only their input
+ * and output buffers -- for example a plugin inside a host framework that owns all
+ * device memory and offers no allocator, or a latency-critical loop that cannot
+ * afford cudaMalloc, which may synchronise the whole device.  The caller still
+ * passes every input and output tensor, with the same meaning, layout and alignment
+ * rules as ssm_selective_scan_fwd.
+ *
+ * Its scratch (a 256-byte header plus the transposed fp32 copy of B and C, i.e.
+ * 256 + batch * seqlen * 128 bytes rounded up to 256) lives in one fixed array of
+ * SSM_NOALLOC_SCRATCH_BYTES (8 MiB) in the library's device memory: every GPU that
+ * loads the library holds that array until the process exits.  Problems that need
+ * more return SSM_ERR_SCRATCH_LIMIT before anything is launched.
+ *   - The first call on each device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any stream
+ *     capture begins.
+ *   - All calls share the one array: calls whose kernels can overlap on the GPU
+ *     (different streams, or different host threads) race on it.  Order them on one
+ *     stream or synchronise between them.
+ *   - Each call clears the header itself; the B/C region is fully rewritten before
+ *     it is read, so nothing left by an earlier call is used.
+ * Device-side timeouts are not reported (there is no workspace to read them from).
+ */
+#define SSM_NOALLOC_SCRATCH_BYTES (8u << 20)
+ssm_status_t ssm_selective_scan_fwd_noalloc(
+    const void* u, const void* delta, const float* A, const void* B, const void* C,
+    const float* D, const void* z, const float* delta_bias, int softplus,
+    void* y, float* last_state,
+    int batch, int dim, int dstate, int64_t seqlen, ssm_dtype_t io_dtype, ssm_stream_t stream);
 
 /*
  * Synchronise `stream`, return the device-side status recorded in `workspace` by the

@@ -8,6 +8,7 @@ from .binding import (  # noqa: F401
     selective_scan_fwd,
     ssm_read_status,
     ssm_selective_scan_fwd,
+    ssm_selective_scan_fwd_noalloc,
     ssm_selective_scan_workspace_size,
     ssm_state_update,
     ssm_workspace_init,

@@ -17,7 +17,9 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libssm_scan.so")
 
-SSM_OK, SSM_ERR_INVALID_ARG, SSM_ERR_UNSUPPORTED, SSM_ERR_LAUNCH, SSM_ERR_TIMEOUT, SSM_ERR_WORKSPACE = range(6)
+(SSM_OK, SSM_ERR_INVALID_ARG, SSM_ERR_UNSUPPORTED, SSM_ERR_LAUNCH, SSM_ERR_TIMEOUT, SSM_ERR_WORKSPACE,
+ SSM_ERR_SCRATCH_LIMIT) = range(7)
+NOALLOC_SCRATCH_BYTES = 8 << 20
 SSM_F32, SSM_BF16 = 0, 1
 SSM_ALGO_AUTO, SSM_ALGO_SEQUENTIAL, SSM_ALGO_CHUNKED, SSM_ALGO_DIRECT = range(4)
 ALGOS = {"auto": SSM_ALGO_AUTO, "sequential": SSM_ALGO_SEQUENTIAL, "chunked": SSM_ALGO_CHUNKED,
@@ -60,6 +62,8 @@ def load() -> ctypes.CDLL:
             lib.ssm_selective_scan_fwd.restype = ci
             lib.ssm_selective_scan_fwd_ex.argtypes = fwd + [ctypes.POINTER(FwdOptions), vp]
             lib.ssm_selective_scan_fwd_ex.restype = ci
+            lib.ssm_selective_scan_fwd_noalloc.argtypes = fwd[:16] + [vp]
+            lib.ssm_selective_scan_fwd_noalloc.restype = ci
             lib.ssm_state_update.argtypes = [vp] * 9 + [ci, vp, ci, ci, ci, ci, vp]
             lib.ssm_state_update.restype = ci
             lib.ssm_read_status.argtypes = [vp, vp]
@@ -131,6 +135,20 @@ def ssm_selective_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus, y, las
         code = lib.ssm_selective_scan_fwd_ex(*args, ctypes.byref(opts), _stream(stream))
     if check:
         _check(code, "ssm_selective_scan_fwd")
+    return code
+
+
+def ssm_selective_scan_fwd_noalloc(u, delta, A, B, C, D, z, delta_bias, softplus, y, last_state, stream=None,
+                                   check=True):
+    """Marshal a call of the forward scan that allocates nothing and takes no workspace
+    (its scratch is a fixed array inside the library; see include/ssm_scan.h)."""
+    b, d, L = u.shape
+    n = A.shape[1]
+    code = load().ssm_selective_scan_fwd_noalloc(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                                                 _ptr(delta_bias), int(bool(softplus)), _ptr(y), _ptr(last_state),
+                                                 b, d, n, L, _io(u), _stream(stream))
+    if check:
+        _check(code, "ssm_selective_scan_fwd_noalloc")
     return code
 
 

@@ -306,6 +306,26 @@ ssm_status_t launch_forward(const FwdArgs& a, const ssm_fwd_options_t& o) {
     return SSM_ERR_INVALID_ARG;
 }
 
+// Fixed scratch of ssm_selective_scan_fwd_noalloc (header + transposed B/C rows).  In
+// host code this name only stands for the array: its device address comes from
+// cudaGetSymbolAddress, looked up once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SSM_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on the current device (nullptr on failure).
+void* noalloc_scratch_ptr() {
+    static std::mutex mu;
+    static void* addr[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
 }  // namespace
 
 extern "C" {
@@ -320,6 +340,7 @@ const char* ssm_status_string(ssm_status_t s) {
         case SSM_ERR_LAUNCH: return "CUDA launch or runtime error";
         case SSM_ERR_TIMEOUT: return "device wait timed out";
         case SSM_ERR_WORKSPACE: return "workspace missing or too small";
+        case SSM_ERR_SCRATCH_LIMIT: return "problem larger than the fixed scratch of the no-allocation entry point";
     }
     return "unknown status";
 }
@@ -404,6 +425,44 @@ ssm_status_t ssm_state_update(float* state, const void* u, const void* delta, co
     else
         ssm::state_update_kernel<float><<<static_cast<unsigned>(grid), 256, 0, s>>>(p);
     return launch_status();
+}
+
+ssm_status_t ssm_selective_scan_fwd_noalloc(const void* u, const void* delta, const float* A, const void* B,
+                                             const void* C, const float* D, const void* z, const float* delta_bias,
+                                             int softplus, void* y, float* last_state, int batch, int dim, int dstate,
+                                             int64_t seqlen, ssm_dtype_t io_dtype, ssm_stream_t stream) {
+    if (batch < 0 || dim < 0 || seqlen < 0) return SSM_ERR_INVALID_ARG;
+    const bool seq_elems = batch > 0 && dim > 0 && seqlen > 0;
+    if (seq_elems && (!u || !delta || !B || !C || !y)) return SSM_ERR_INVALID_ARG;
+    if (dim > 0 && !A) return SSM_ERR_INVALID_ARG;
+    if (io_dtype != SSM_F32 && io_dtype != SSM_BF16) return SSM_ERR_INVALID_ARG;
+    if (dstate != 16) return SSM_ERR_UNSUPPORTED;
+    const void* ptrs[] = {u, delta, A, B, C, D, z, delta_bias, y, last_state};
+    for (const void* q : ptrs)
+        if (q && !aligned16(q)) return SSM_ERR_INVALID_ARG;
+    if (batch == 0 || dim == 0) return SSM_OK;
+    if (batch > 65535) return SSM_ERR_UNSUPPORTED;
+    if (ssm_selective_scan_workspace_size(batch, dim, dstate, seqlen) > SSM_NOALLOC_SCRATCH_BYTES)
+        return SSM_ERR_SCRATCH_LIMIT;
+    int sm_count = 0;
+    ssm_status_t st = check_device(&sm_count);
+    if (st != SSM_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (seqlen == 0) {
+        if (last_state &&
+            cudaMemsetAsync(last_state, 0, static_cast<size_t>(batch) * dim * 16 * sizeof(float), s) != cudaSuccess)
+            return SSM_ERR_LAUNCH;
+        return SSM_OK;
+    }
+    uint8_t* scratch = static_cast<uint8_t*>(noalloc_scratch_ptr());
+    if (!scratch) return SSM_ERR_LAUNCH;
+    // The header (status word) starts every call at zero; the B/C rows are rewritten in full.
+    if (cudaMemsetAsync(scratch, 0, sizeof(WorkspaceHeader), s) != cudaSuccess) return SSM_ERR_LAUNCH;
+    // Kernels whose scratch is only the header and the B/C rows (no look-back flags).
+    const ssm_fwd_options_t o{SSM_ALGO_SEQUENTIAL, 0, 0, -1};
+    FwdArgs a{u, delta, B, C, z, A, D, delta_bias, softplus, y, last_state, batch, dim, seqlen, io_dtype,
+              scratch, s, sm_count};
+    return io_dtype == SSM_BF16 ? launch_forward<__nv_bfloat16>(a, o) : launch_forward<float>(a, o);
 }
 
 ssm_status_t ssm_read_status(void* workspace, ssm_stream_t stream) {

@@ -44,7 +44,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in range(6):
+    for code in range(7):
         assert binding.status_string(code)
     assert "workspace" in binding.status_string(binding.SSM_ERR_WORKSPACE)
 
