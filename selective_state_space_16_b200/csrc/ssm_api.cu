@@ -15,6 +15,7 @@
 #include "../../include/ssm_scan.h"
 #include "aux_kernels.cuh"
 #include "common.cuh"
+#include "scan_fwd_chunked.cuh"
 #include "scan_fwd_seq.cuh"
 
 namespace {
@@ -23,22 +24,35 @@ using ssm::WorkspaceHeader;
 
 constexpr int kAbiVersion = 1;
 constexpr uint32_t kDefaultWaitLimit = 1u << 22;
+constexpr uint32_t kDefaultSpinLimit = 1u << 21;  // look-back polls (~64 ns sleep each)
 
 size_t round_up(size_t v, size_t m) { return (v + m - 1) / m * m; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Workspace layout: [header 256 B][B/C fp32 rows: batch * L * 128 B][chunk-carry region].
+// Workspace layout:
+//   [header 256 B][B/C fp32 rows: batch * L * 128 B]
+//   [look-back flags: keys * 4 B][aggregate h: keys * 256 B][aggregate sum Delta: keys * 16 B]
+//   [inclusive h: keys * 256 B]
+// with keys = (8-channel tiles) * 2 columns * ceil(L / 32) chunks (32 steps is the
+// shorter chunk of the two element types, so one size serves both).
 struct WsLayout {
-    size_t bc_off, carry_off, total;
+    size_t bc_off, flags_off, agg_off, sdt_off, incl_off, total;
+    long long keys;
 };
+
+constexpr int kMinChunk = 32;
 
 WsLayout ws_layout(int batch, int dim, int64_t L) {
     WsLayout w{};
+    const long long tiles = static_cast<long long>(batch) * ((dim + 7) / 8);
+    w.keys = tiles * 2 * ((L + kMinChunk - 1) / kMinChunk);
     w.bc_off = sizeof(WorkspaceHeader);
-    w.carry_off = w.bc_off + round_up(static_cast<size_t>(batch) * static_cast<size_t>(L) * 128u, 256);
-    (void)dim;
-    w.total = w.carry_off;
+    w.flags_off = w.bc_off + round_up(static_cast<size_t>(batch) * static_cast<size_t>(L) * 128u, 256);
+    w.agg_off = w.flags_off + round_up(static_cast<size_t>(w.keys) * 4u, 256);
+    w.sdt_off = w.agg_off + static_cast<size_t>(w.keys) * 256u;
+    w.incl_off = w.sdt_off + static_cast<size_t>(w.keys) * 16u;
+    w.total = w.incl_off + static_cast<size_t>(w.keys) * 256u;
     return w;
 }
 
@@ -241,6 +255,58 @@ ssm_status_t launch_seq(const FwdArgs& a, const SeqPlan& pl) {
 }
 
 template <typename IO>
+ssm_status_t launch_chunked(const FwdArgs& a, const ssm_fwd_options_t& o) {
+    using Cfg = ssm::ChunkCfg<IO>;
+    constexpr int TC = Cfg::kTC;
+    if (a.L >= (1LL << 31) - 1024) return SSM_ERR_UNSUPPORTED;
+    constexpr auto sw128 = CU_TENSOR_MAP_SWIZZLE_128B;
+    const auto dt = ssm::IoTraits<IO>::kTmaType;
+    constexpr int es = ssm::IoTraits<IO>::kBytes;
+    const WsLayout wl = ws_layout(a.batch, a.dim, a.L);
+    CUtensorMap mu, mdl, mz, mbc;
+    const uint64_t L = static_cast<uint64_t>(a.L);
+    bool ok = make_map_3d(&mu, dt, es, a.u, L, a.dim, a.batch, TC, 8, sw128) &&
+              make_map_3d(&mdl, dt, es, a.delta, L, a.dim, a.batch, TC, 8, sw128) &&
+              make_map_3d(&mbc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.ws + wl.bc_off, 32, L, a.batch, 32, TC,
+                          CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (ok && a.z) ok = make_map_3d(&mz, dt, es, a.z, L, a.dim, a.batch, TC, 8, sw128);
+    if (!a.z) mz = mu;
+    if (!ok) return SSM_ERR_LAUNCH;
+    auto kern = ssm::scan_fwd_chunked_kernel<IO>;
+    if (!ensure_smem_attr(reinterpret_cast<const void*>(kern), Cfg::kSmem)) return SSM_ERR_LAUNCH;
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, Cfg::kThreads, Cfg::kSmem) != cudaSuccess ||
+        occ < 1)
+        return SSM_ERR_LAUNCH;
+    ssm::ChunkParams p{};
+    p.A = a.A;
+    p.D = a.D;
+    p.bias = a.bias;
+    p.last_state = a.last_state;
+    p.y = a.y;
+    p.hdr = reinterpret_cast<WorkspaceHeader*>(a.ws);
+    p.flags = reinterpret_cast<uint32_t*>(a.ws + wl.flags_off);
+    p.pay_agg = reinterpret_cast<float*>(a.ws + wl.agg_off);
+    p.pay_sdt = reinterpret_cast<float*>(a.ws + wl.sdt_off);
+    p.pay_incl = reinterpret_cast<float*>(a.ws + wl.incl_off);
+    p.batch = a.batch;
+    p.dim = a.dim;
+    p.L = static_cast<int>(a.L);
+    p.tiles_per_batch = (a.dim + 7) / 8;
+    p.nchunks = static_cast<int>((a.L + TC - 1) / TC);
+    p.total_tiles = static_cast<long long>(a.batch) * p.tiles_per_batch;
+    p.total_units = p.total_tiles * p.nchunks;
+    p.softplus = a.softplus;
+    p.has_z = a.z != nullptr;
+    p.wait_limit = kDefaultWaitLimit;
+    p.spin_limit = o.spin_limit ? o.spin_limit : kDefaultSpinLimit;
+    p.debug_skip_chunk = o.debug_skip_publish;
+    const long long grid = std::min<long long>(p.total_units, static_cast<long long>(a.sm_count) * occ);
+    kern<<<static_cast<unsigned>(grid), Cfg::kThreads, Cfg::kSmem, a.stream>>>(mu, mdl, mz, mbc, p);
+    return launch_status();
+}
+
+template <typename IO>
 ssm_status_t launch_direct(const FwdArgs& a) {
     ssm::DirectParams p{};
     p.u = a.u;
@@ -280,9 +346,18 @@ ssm_status_t launch_forward(const FwdArgs& a, const ssm_fwd_options_t& o) {
     const bool tma_ok = (static_cast<uint64_t>(a.L) * ssm::IoTraits<IO>::kBytes) % 16 == 0 && aligned16(a.u) &&
                         aligned16(a.delta) && aligned16(a.y) && (!a.z || aligned16(a.z));
     int algo = o.algo;
-    if (algo == SSM_ALGO_AUTO || algo == SSM_ALGO_CHUNKED) algo = SSM_ALGO_SEQUENTIAL;
     if (!tma_ok) algo = SSM_ALGO_DIRECT;
     if (algo == SSM_ALGO_DIRECT) return launch_direct<IO>(a);
+    if (algo == SSM_ALGO_AUTO) {
+        // The sequential kernel is faster whenever the channels alone give each SM a few
+        // warps (measured on B200: at 5120 channels x 32768 steps it runs at ~1.8x the
+        // chunked kernel).  Split the sequence across CTAs only when fewer than 4 warps of
+        // 8-lane channels per SM would be resident, and the sequence is long.
+        const double warps_per_sm = static_cast<double>(a.batch) * a.dim * 8.0 / 32.0 / a.sm_count;
+        const long long chunks = (a.L + ssm::ChunkCfg<IO>::kTC - 1) / ssm::ChunkCfg<IO>::kTC;
+        algo = (warps_per_sm < 4.0 && chunks >= 64) ? SSM_ALGO_CHUNKED : SSM_ALGO_SEQUENTIAL;
+    }
+    if (algo == SSM_ALGO_CHUNKED) return launch_chunked<IO>(a, o);
     // Variants: (lanes per channel G, channels per lane CPL).  lanes_per_channel selects
     // G explicitly (CPL = 1), or G = 4 with CPL = 2 when given as 42.
     const SeqPlan p2 = plan_seq<IO, 2, 1>(a), p4 = plan_seq<IO, 4, 1>(a), p42 = plan_seq<IO, 4, 2>(a);

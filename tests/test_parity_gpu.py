@@ -15,7 +15,8 @@ pytestmark = pytest.mark.gpu
 
 
 # ------------------------------------------------------------------ kernel variants, ragged sizes
-VARIANTS = [("sequential", 2), ("sequential", 4), ("sequential", 8), ("sequential", 42), ("direct", 0)]
+VARIANTS = [("sequential", 2), ("sequential", 4), ("sequential", 8), ("sequential", 42), ("chunked", 0),
+            ("direct", 0)]
 
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
@@ -88,6 +89,54 @@ def test_workload_long_sequence_sampled(cuda_device):
     rng = np.random.default_rng(3)
     channels = np.sort(rng.choice(w.batch * w.dim, size=384, replace=False))
     check_forward(inp, channels=channels, what=w.name + " (sampled channels)")
+
+
+# ------------------------------------------------------------------ chunked scan (look-back)
+def test_chunked_headline_full_size(cuda_device):
+    w = workloads.WORKLOADS[2]
+    check_forward(workloads.workload_inputs(w), algo="chunked", what=w.name + " chunked")
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_chunked_many_chunks_few_channels(cuda_device, io):
+    # one tile, 70+ chunks: the look-back chain is long and the ragged last chunk is partial
+    inp = workloads.scan_inputs(1, 8, 4600 if io == "bf16" else 2300, io=io, seed=41)
+    check_forward(inp, algo="chunked", what=f"chunked long chain {io}")
+
+
+def test_chunked_workspace_reuse(cuda_device):
+    # Consecutive launches on one workspace (flag epochs and the ticket counter are reset
+    # by each launch).  The look-back combines a unit's predecessors in whatever order
+    # their states are published, so floating-point rounding may differ between launches:
+    # every launch must match the oracle, and launches must agree to rounding.
+    cpu = workloads.scan_inputs(2, 40, 1024, io="f32", seed=42)
+    inp = to_dev(cpu, "cuda")
+    ws = ssm.new_workspace(2, 40, 16, 1024)
+    outs = [ssm.selective_scan_fwd(**inp, workspace=ws, algo="chunked") for _ in range(3)]
+    torch.cuda.synchronize()
+    y_ref, last_ref = oracle_forward(cpu)
+    for y, last in outs:
+        assert_close(y, y_ref, "f32", "chunked relaunch y")
+        assert_close(last, last_ref, "f32", "chunked relaunch last_state")
+        assert torch.allclose(y, outs[0][0], rtol=1e-5, atol=1e-6)
+    assert ssm.ssm_read_status(ws) == 0
+
+
+def test_chunked_lookback_wait_is_bounded(cuda_device):
+    """Units of chunk 3 never publish: their successors' look-back waits must run out,
+    record SSM_ERR_TIMEOUT and let the kernel finish; the workspace then still serves
+    a normal call."""
+    cpu = workloads.scan_inputs(1, 16, 1024, io="bf16", seed=43)
+    inp = to_dev(cpu, "cuda")
+    ws = ssm.new_workspace(1, 16, 16, 1024)
+    ssm.selective_scan_fwd(**inp, workspace=ws, algo="chunked", spin_limit=2000, debug_skip_publish=3)
+    assert ssm.ssm_read_status(ws) == 4          # SSM_ERR_TIMEOUT, read back and cleared
+    assert ssm.ssm_read_status(ws) == 0
+    y, last = ssm.selective_scan_fwd(**inp, workspace=ws, algo="chunked")
+    torch.cuda.synchronize()
+    y_ref, last_ref = oracle_forward(cpu)
+    assert_close(y, y_ref, "bf16", "after timeout: y")
+    assert_close(last, last_ref, "bf16", "after timeout: last_state")
 
 
 # ------------------------------------------------------------------ decode
