@@ -190,10 +190,12 @@ def traffic_record(kernel: str, workload: str):
     return None
 
 
-def time_forward(ssm, g, ws, steps, warmup, world, stream, clocks=None):
+def time_forward(ssm, g, ws, steps, warmup, world, stream, clocks=None, opts=None):
+    opts = opts or {}
+
     def call():
         ssm.ssm_selective_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"],
-                                   True, g["y"], g["last"], ws, stream=stream)
+                                   True, g["y"], g["last"], ws, stream=stream, **opts)
     with torch.cuda.stream(stream):
         for _ in range(warmup):
             call()
@@ -229,54 +231,79 @@ def forward_buffers(w, dev):
     return inp, g
 
 
-def e2e_forward(ssm, w, inp, ws, steps, stream):
+def e2e_forward(ssm, w, inp, ws, steps, stream, nstreams=3):
     """Same metric through the public C-ABI call with HOST (pinned) buffers: every step
-    copies the inputs host->device, runs the scan and copies y and the final state back."""
-    names = ["u", "delta", "z", "B", "C", "A", "D", "delta_bias"]
+    copies all inputs host->device, runs the scan and copies y and the final state back.
+    The batch rows are pipelined over `nstreams` streams (row b+1's upload overlaps row b's
+    scan and download); each stream has its own workspace."""
+    names = ["u", "delta", "z", "B", "C"]
     host = {k: inp[k].pin_memory() for k in names}
+    wts = {k: inp[k].pin_memory() for k in ("A", "D", "delta_bias")}
     dev = {k: torch.empty_like(host[k], device="cuda") for k in names}
+    dw = {k: torch.empty_like(wts[k], device="cuda") for k in wts}
     y_d = torch.empty_like(dev["u"])
     last_d = torch.empty(w.batch, w.dim, w.dstate, dtype=torch.float32, device="cuda")
     y_h = torch.empty_like(host["u"]).pin_memory()
     last_h = torch.empty(last_d.shape, dtype=torch.float32).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    h2d = sum(t.numel() * t.element_size() for t in list(host.values()) + list(wts.values()))
     d2h = y_h.numel() * y_h.element_size() + last_h.numel() * 4
+    streams = [torch.cuda.Stream() for _ in range(nstreams)]
+    wss = [ssm.new_workspace(1, w.dim, w.dstate, w.seqlen) for _ in range(nstreams)]
 
     def step():
-        for k in names:
-            dev[k].copy_(host[k], non_blocking=True)
-        ssm.ssm_selective_scan_fwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], dev["D"], dev["z"],
-                                   dev["delta_bias"], True, y_d, last_d, ws, stream=stream)
-        y_h.copy_(y_d, non_blocking=True)
-        last_h.copy_(last_d, non_blocking=True)
+        with torch.cuda.stream(stream):
+            for k in wts:
+                dw[k].copy_(wts[k], non_blocking=True)
+        start = torch.cuda.Event()
+        start.record(stream)
+        for b in range(w.batch):
+            st = streams[b % nstreams]
+            st.wait_event(start)
+            with torch.cuda.stream(st):
+                for k in names:
+                    dev[k][b].copy_(host[k][b], non_blocking=True)
+                ssm.ssm_selective_scan_fwd(dev["u"][b:b + 1], dev["delta"][b:b + 1], dw["A"], dev["B"][b:b + 1],
+                                           dev["C"][b:b + 1], dw["D"], dev["z"][b:b + 1], dw["delta_bias"], True,
+                                           y_d[b:b + 1], last_d[b:b + 1], wss[b % nstreams], stream=st)
+                y_h[b].copy_(y_d[b], non_blocking=True)
+                last_h[b].copy_(last_d[b], non_blocking=True)
+        for st in streams:
+            stream.wait_stream(st)
 
-    with torch.cuda.stream(stream):
+    step()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(steps):
         step()
-        torch.cuda.synchronize()
-        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        ev0.record(stream)
-        for _ in range(steps):
-            step()
-        ev1.record(stream)
+    ev1.record(stream)
     torch.cuda.synchronize()
     t = ev0.elapsed_time(ev1) / 1e3
     return {"value": w.elements * steps / t / 1e9, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-            "d2h_bytes_per_step": int(d2h), "steps": steps}
+            "d2h_bytes_per_step": int(d2h), "steps": steps,
+            "pipeline": f"pinned host buffers; per batch row H2D, scan, D2H over {nstreams} streams"}
 
 
-def measure_long(ssm, stream, steps=10):
+def measure_long(ssm, stream, pk, steps=5):
+    """Long-sequence workload (batch 1, d_inner 5120, L 32768): the default kernel choice
+    and the chunked kernel (sequence split across CTAs, decoupled look-back)."""
     w = workloads.WORKLOADS[3]
     _, g = forward_buffers(w, "cuda")
     ws = ssm.new_workspace(w.batch, w.dim, w.dstate, w.seqlen)
-    t = time_forward(ssm, g, ws, steps, 3, 1, stream)
-    ms = t / steps * 1e3
+    out = {"workload": w.name, "unit": UNIT}
+    for name, opts in (("default", {}), ("chunked_lookback", {"algo": "chunked"})):
+        t = time_forward(ssm, g, ws, steps, 2, 1, stream, opts=opts)
+        ms = t / steps * 1e3
+        out[name] = {"value": w.elements / (ms / 1e3) / 1e9, "ms_per_step": ms,
+                     "hbm_frac": scan_algorithmic_bytes(w) / (ms / 1e3) / 1e9 / pk["hbm_gbs"]}
+    assert ssm.ssm_read_status(ws) == 0
     del g
-    return {"workload": w.name, "value": w.elements / (ms / 1e3) / 1e9, "unit": UNIT, "ms_per_step": ms,
-            "mufu_frac_of_nominal": None}
+    return out
 
 
-def measure_decode(ssm, stream, pk):
+def measure_decode(ssm, stream, pk, steps=None):
     w = workloads.WORKLOADS[4]
+    nsteps = steps or w.decode_steps
     dec = workloads.workload_decode_inputs(w)
     A, D, bias = dec["A"].cuda(), dec["D"].cuda(), dec["delta_bias"].cuda()
     sets = [{k: v.cuda() for k, v in s.items()} for s in dec["sets"]]
@@ -294,7 +321,7 @@ def measure_decode(ssm, stream, pk):
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
-        chain(w.decode_steps)
+        chain(nsteps)
     with torch.cuda.stream(stream):  # replay() launches on the current stream
         graph.replay()
         torch.cuda.synchronize()
@@ -304,65 +331,87 @@ def measure_decode(ssm, stream, pk):
         ev1.record(stream)
     torch.cuda.synchronize()
     t = ev0.elapsed_time(ev1) / 1e3
-    per_step = t / w.decode_steps
+    per_step = t / nsteps
     gbs = decode_algorithmic_bytes(w) / per_step / 1e9
     del graph
     return {"workload": w.name, "value": w.batch * w.dim / per_step / 1e9, "unit": "Gelem/s (B*D per step)",
-            "us_per_step": per_step * 1e6, "steps": w.decode_steps, "launch": "one CUDA graph of 1000 steps",
+            "us_per_step": per_step * 1e6, "steps": nsteps, "launch": f"one CUDA graph of {nsteps} steps",
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / pk["hbm_gbs"], "note": "state is 84 MB < 126 MB L2: see ncu dram bytes"}}
 
 
-def cpu_oracle_rate(w, budget_s: float, channels_cap=None):
-    """Time the fp64 oracle on a bounded prefix of the workload's channels.
-    Returns (Gelem/s, seconds, channels, threads)."""
+def _oracle_sample(inp, w, channels):
+    """The workload restricted to its first `channels` flat (batch, channel) rows, as a list
+    of per-batch-row oracle calls (whole batch rows first)."""
+    calls, left = [], channels
+    for b in range(w.batch):
+        if left <= 0:
+            break
+        c = min(left, w.dim)
+        calls.append(dict(u=inp["u"][b, :c][None], delta=inp["delta"][b, :c][None], A=inp["A"][:c],
+                          B=inp["B"][b][None], C=inp["C"][b][None], D=inp["D"][:c], z=inp["z"][b, :c][None],
+                          delta_bias=inp["delta_bias"][:c]))
+        left -= c
+    return calls
+
+
+def _plan_oracle_sample(inp, w, budget_s):
+    """Pick a sample of about `budget_s` seconds of oracle work: the whole workload repeated
+    `reps` times, or (when one pass is longer) its first `channels` rows once."""
     import oracle
-    inp = workloads.workload_inputs(w) if w.decode_steps == 0 else None
-    b0 = inp["u"][0]
-    sub = lambda c: dict(u=b0[:c][None], delta=inp["delta"][0][:c][None], A=inp["A"][:c], B=inp["B"][0][None],
-                         C=inp["C"][0][None], D=inp["D"][:c], z=inp["z"][0][:c][None],
-                         delta_bias=inp["delta_bias"][:c])
-    c = 16
+    probe = _oracle_sample(inp, w, 32)
     t0 = time.perf_counter()
-    oracle.selective_scan(**sub(c))
-    t_cal = time.perf_counter() - t0
-    per_ch = t_cal / c
-    c = max(16, min(w.dim if channels_cap is None else channels_cap, int(budget_s / max(per_ch, 1e-9))))
-    args = sub(c)
+    for c in probe:
+        oracle.selective_scan(**c)
+    per_row = (time.perf_counter() - t0) / 32
+    rows = w.batch * w.dim
+    if per_row * rows <= budget_s:
+        return rows, max(1, int(budget_s / (per_row * rows)))
+    return max(1, int(budget_s / per_row)), 1
+
+
+def cpu_oracle_rate(w, budget_s: float):
+    """Time the fp64 oracle on a bounded sample of the workload.
+    Returns (Gelem/s, seconds, description, threads)."""
+    import oracle
+    inp = workloads.workload_inputs(w)
+    rows, reps = _plan_oracle_sample(inp, w, budget_s)
+    calls = _oracle_sample(inp, w, rows)
     t0 = time.perf_counter()
-    oracle.selective_scan(**args)
+    for _ in range(reps):
+        for c in calls:
+            oracle.selective_scan(**c)
     dt = time.perf_counter() - t0
-    return c * w.seqlen / dt / 1e9, dt, c, oracle.num_threads()
+    elems = rows * w.seqlen * reps
+    what = "the whole workload" if rows == w.batch * w.dim else f"its first {rows} of {w.batch * w.dim} channels"
+    desc = f"{what} (L={w.seqlen}), {reps} pass(es): {elems} elements in {dt:.1f} s"
+    return elems / dt / 1e9, dt, desc, oracle.num_threads()
 
 
 # ----------------------------------------------------------------------------- arms
 def run_reference(args, world, rank):
+    """The fp64 CPU oracle on the host cores, on the headline workload: each step is a
+    bounded sample of it (the whole workload when K+W steps of it fit in ~2 minutes)."""
     if rank != 0:
         return
     w = workloads.WORKLOADS[workloads.HEADLINE]
     import oracle
     oracle.build()
     inp = workloads.workload_inputs(w)
-    budget_per_step = max(0.02, 90.0 / max(1, args.steps + args.warmup))
-    b0 = inp["u"][0]
-
-    def sample(c):
-        return dict(u=b0[:c][None], delta=inp["delta"][0][:c][None], A=inp["A"][:c], B=inp["B"][0][None],
-                    C=inp["C"][0][None], D=inp["D"][:c], z=inp["z"][0][:c][None], delta_bias=inp["delta_bias"][:c])
-    t0 = time.perf_counter()
-    oracle.selective_scan(**sample(8))
-    per_ch = (time.perf_counter() - t0) / 8
-    c = max(1, min(w.dim, int(budget_per_step / max(per_ch, 1e-9))))
-    s = sample(c)
+    budget_per_step = max(0.02, 120.0 / max(1, args.steps + args.warmup))
+    rows, _ = _plan_oracle_sample(inp, w, budget_per_step)
+    calls = _oracle_sample(inp, w, rows)
     for _ in range(args.warmup):
-        oracle.selective_scan(**s)
+        for c in calls:
+            oracle.selective_scan(**c)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.selective_scan(**s)
+        for c in calls:
+            oracle.selective_scan(**c)
     dt = time.perf_counter() - t0
-    elems = c * w.seqlen * args.steps
-    val = elems / dt / 1e9
-    desc = f"{c} of {w.dim} channels of batch row 0, full L={w.seqlen}, per step"
+    val = rows * w.seqlen * args.steps / dt / 1e9
+    what = "the whole workload" if rows == w.batch * w.dim else f"its first {rows} of {w.batch * w.dim} channels"
+    desc = f"{what} (L={w.seqlen}) per step"
     line = {"metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
@@ -418,14 +467,26 @@ def run_gpu(args, world, rank, local):
         e2e_steps = max(3, min(args.steps, 10))
         line["e2e"] = e2e_forward(ssm, w, inp, ws, e2e_steps, stream)
     if world == 1 and not args.skip_extra:
-        line["also"] = {"long": measure_long(ssm, stream), "decode": measure_decode(ssm, stream, pk)}
+        line["also"] = {"long": measure_long(ssm, stream, pk), "decode": measure_decode(ssm, stream, pk)}
     if rank == 0 and world == 1 and not args.skip_cpu:
-        rate, secs, ch, cores = cpu_oracle_rate(w, args.cpu_budget)
-        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
-                                "sample": f"{ch} of {w.dim} channels of batch row 0, full L={w.seqlen} "
-                                          f"({ch * w.seqlen} elements, {secs:.1f} s)"}
+        rate, secs, desc, cores = cpu_oracle_rate(w, args.cpu_budget)
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def run_profile_workload(args):
+    """Run only the long-sequence scan or the decode chain (for profiler captures)."""
+    import selective_state_space_16_b200 as ssm
+    torch.cuda.set_device(0)
+    stream = torch.cuda.Stream()
+    pk = peaks()
+    if args.workload == "long":
+        out = measure_long(ssm, stream, pk, steps=args.steps)
+    else:
+        w = workloads.WORKLOADS[4]
+        out = measure_decode(ssm, stream, pk, steps=args.steps)
+    print(json.dumps({"workload": args.workload, "result": out}), flush=True)
 
 
 def main():
@@ -438,12 +499,16 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-extra", action="store_true")
+    ap.add_argument("--workload", default="headline", choices=["headline", "long", "decode"],
+                    help="profiling runs: 'long' / 'decode' run only that workload a few times")
     args = ap.parse_args()
     world, rank, local = dist_setup(args.gpus) if args.impl == "native" else (
         int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.workload != "headline":
+            run_profile_workload(args)
         else:
             run_gpu(args, world, rank, local)
     finally:
