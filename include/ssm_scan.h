@@ -18,7 +18,8 @@
  *              [Card] 离散化变换 and 选择性机制)
  *   y_t     = (sum_n C[b,n,t]*h_t[n] + D[d]*u[b,d,t]) * silu(z[b,d,t])
  *             ([Eng] §2.2 for C h + D x; [Hist] Mamba Block 数据流 for the SiLU gate)
- *   h_{-1}  = 0; last_state = h_{L-1}                            [Eng] §4.2 and §7.2
+ *   h_{-1}  = 0 (or a given initial state, ssm_selective_scan_fwd_state);
+ *   last_state = h_{L-1}                                         [Eng] §4.2 and §7.2
  *
  * Conventions shared by every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller.  The library
@@ -115,7 +116,8 @@ typedef enum {
 
 typedef struct {
     int algo;                  /* ssm_algo_t                                                      */
-    int lanes_per_channel;     /* SEQUENTIAL/DIRECT: lanes sharing one channel (2, 4, 8 or 16); 0 = auto */
+    int lanes_per_channel;     /* SEQUENTIAL: lanes sharing one channel: 2, 4 or 8 (8: bf16 only), or 42 =
+                                  4 lanes per channel with each lane holding two channels; 0 = auto    */
     uint32_t spin_limit;       /* CHUNKED: polls before a look-back wait gives up; 0 = default    */
     int debug_skip_publish;    /* CHUNKED, tests only: chunk index whose CTAs never publish; -1 = off */
 } ssm_fwd_options_t;
@@ -125,6 +127,30 @@ ssm_status_t ssm_selective_scan_fwd_ex(
     const void* u, const void* delta, const float* A, const void* B, const void* C,
     const float* D, const void* z, const float* delta_bias, int softplus,
     void* y, float* last_state,
+    int batch, int dim, int dstate, int64_t seqlen, ssm_dtype_t io_dtype,
+    void* workspace, size_t workspace_bytes, const ssm_fwd_options_t* opts, ssm_stream_t stream);
+
+/*
+ * Forward scan from a given state instead of zero: state continuation across the
+ * blocks of an over-long sequence ([Eng] §7.2: block-wise processing must carry the
+ * state from one block into the next) and reuse of a cached prefix state ([Eng] §6.2).
+ * The recurrence above then starts from h_{-1} = initial_state, so that scanning
+ * steps [0, L1) and then [L1, L) with initial_state = the first call's last_state
+ * gives the scan of [0, L) (up to the fp32 state handed over).
+ *   initial_state  optional fp32 (batch, dim, dstate); NULL means zero, and the call is
+ *                  then ssm_selective_scan_fwd_ex.  Read only.  It must not overlap
+ *                  last_state (SSM_ERR_INVALID_ARG): with the sequence split across CTAs,
+ *                  a channel's initial state can still be read after another CTA has
+ *                  written that channel's final state.  Use two buffers to chain calls.
+ *   seqlen == 0    last_state receives a copy of initial_state (zeros if it is NULL).
+ *   opts           as for ssm_selective_scan_fwd_ex; may be NULL.
+ * Every other argument, the workspace rules and the errors are those of
+ * ssm_selective_scan_fwd.
+ */
+ssm_status_t ssm_selective_scan_fwd_state(
+    const void* u, const void* delta, const float* A, const void* B, const void* C,
+    const float* D, const void* z, const float* delta_bias, int softplus,
+    const float* initial_state, void* y, float* last_state,
     int batch, int dim, int dstate, int64_t seqlen, ssm_dtype_t io_dtype,
     void* workspace, size_t workspace_bytes, const ssm_fwd_options_t* opts, ssm_stream_t stream);
 

@@ -62,6 +62,8 @@ def load() -> ctypes.CDLL:
             lib.ssm_selective_scan_fwd.restype = ci
             lib.ssm_selective_scan_fwd_ex.argtypes = fwd + [ctypes.POINTER(FwdOptions), vp]
             lib.ssm_selective_scan_fwd_ex.restype = ci
+            lib.ssm_selective_scan_fwd_state.argtypes = fwd[:9] + [vp] + fwd[9:] + [ctypes.POINTER(FwdOptions), vp]
+            lib.ssm_selective_scan_fwd_state.restype = ci
             lib.ssm_selective_scan_fwd_noalloc.argtypes = fwd[:16] + [vp]
             lib.ssm_selective_scan_fwd_noalloc.restype = ci
             lib.ssm_state_update.argtypes = [vp] * 9 + [ci, vp, ci, ci, ci, ci, vp]
@@ -118,21 +120,28 @@ def new_workspace(batch, dim, dstate, seqlen, device="cuda", stream=None):
 
 def ssm_selective_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus, y, last_state, workspace,
                            stream=None, algo=None, lanes_per_channel=0, spin_limit=0, debug_skip_publish=-1,
-                           check=True):
+                           check=True, initial_state=None):
     """Marshal a forward-scan call.  u/delta/z/y: (b, d, L); B/C: (b, N, L); A: (d, N) fp32;
-    D/delta_bias: (d) fp32 or None; last_state: (b, d, N) fp32 or None; workspace: uint8."""
+    D/delta_bias: (d) fp32 or None; last_state: (b, d, N) fp32 or None; workspace: uint8;
+    initial_state: (b, d, N) fp32 or None (zero), through ssm_selective_scan_fwd_state."""
     lib = load()
     b, d, L = u.shape
     n = A.shape[1]
-    args = [_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
-            int(bool(softplus)), _ptr(y), _ptr(last_state), b, d, n, L, _io(u), _ptr(workspace),
+    head = [_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+            int(bool(softplus))]
+    tail = [_ptr(y), _ptr(last_state), b, d, n, L, _io(u), _ptr(workspace),
             workspace.numel() * workspace.element_size()]
-    if algo is None and lanes_per_channel == 0 and spin_limit == 0 and debug_skip_publish < 0:
-        code = lib.ssm_selective_scan_fwd(*args, _stream(stream))
+    default_opts = algo is None and lanes_per_channel == 0 and spin_limit == 0 and debug_skip_publish < 0
+    if default_opts and initial_state is None:
+        code = lib.ssm_selective_scan_fwd(*head, *tail, _stream(stream))
     else:
         a = ALGOS[algo] if isinstance(algo, str) else (algo or SSM_ALGO_AUTO)
         opts = FwdOptions(a, lanes_per_channel, spin_limit, debug_skip_publish)
-        code = lib.ssm_selective_scan_fwd_ex(*args, ctypes.byref(opts), _stream(stream))
+        if initial_state is None:
+            code = lib.ssm_selective_scan_fwd_ex(*head, *tail, ctypes.byref(opts), _stream(stream))
+        else:
+            code = lib.ssm_selective_scan_fwd_state(*head, _ptr(initial_state), *tail, ctypes.byref(opts),
+                                                    _stream(stream))
     if check:
         _check(code, "ssm_selective_scan_fwd")
     return code
@@ -168,9 +177,10 @@ def ssm_read_status(workspace, stream=None) -> int:
 
 
 def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
-                       return_last_state=True, workspace=None, stream=None, **opts):
+                       return_last_state=True, workspace=None, stream=None, initial_state=None, **opts):
     """Convenience wrapper: allocates y (u's dtype), last_state (fp32) and, if not given,
-    a workspace, then calls ssm_selective_scan_fwd.  Returns (y, last_state)."""
+    a workspace, then calls ssm_selective_scan_fwd (from initial_state when given).
+    Returns (y, last_state)."""
     b, d, L = u.shape
     n = A.shape[1]
     y = torch.empty_like(u)
@@ -178,5 +188,5 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
     if workspace is None:
         workspace = new_workspace(b, d, n, L, device=u.device, stream=stream)
     ssm_selective_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus, y, last, workspace,
-                           stream=stream, **opts)
+                           stream=stream, initial_state=initial_state, **opts)
     return y, last

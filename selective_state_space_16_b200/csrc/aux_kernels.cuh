@@ -52,6 +52,7 @@ struct DirectParams {
     const float* A;
     const float* D;
     const float* bias;
+    const float* h0;       // (batch, dim, 16) initial state or null (zero)
     void* y;
     float* last_state;
     int batch, dim;
@@ -79,7 +80,7 @@ __global__ void __launch_bounds__(128) scan_fwd_direct_kernel(const DirectParams
 #pragma unroll
     for (int j = 0; j < NC; ++j) {
         A2[j] = valid ? p.A[d * 16 + nl * NC + j] * kLog2e : 0.f;
-        h[j] = 0.f;
+        h[j] = (valid && p.h0) ? p.h0[ch * 16 + nl * NC + j] : 0.f;
     }
     const float Dd = (valid && p.D) ? p.D[d] : 0.f;
     const float bias = (valid && p.bias) ? p.bias[d] : 0.f;

@@ -73,6 +73,17 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     return false;
 }
 
+// As mbar_wait_bounded, sleeping ~128 ns between tries: for a waiter that is far ahead
+// (the producer of a ring), so that its polling does not take issue slots from the
+// warps it waits for.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t limit) {
+    for (uint32_t i = 0; i < limit; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        __nanosleep(128);
+    }
+    return false;
+}
+
 // ---------------------------------------------------------------------------------------
 // TMA (tensor-map bulk copies) and bulk groups
 // ---------------------------------------------------------------------------------------

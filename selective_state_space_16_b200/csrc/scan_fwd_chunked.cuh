@@ -52,6 +52,7 @@ struct ChunkParams {
     float* pay_agg;        // [key][4 channels][16]: h of the chunk with a zero carry-in
     float* pay_sdt;        // [key][4 channels]: sum of the chunk's step sizes
     float* pay_incl;       // [key][4 channels][16]: h at the end of the chunk
+    const float* h0;       // (batch, dim, 16) state before step 0, or null (zero)
     int batch, dim;
     int L;
     int tiles_per_batch;   // ceil(dim / 8)
@@ -306,7 +307,17 @@ scan_fwd_chunked_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_
                     sdt_u += sdt_sm[w * 8 + row];
                 }
                 const bool publish = (k != p.debug_skip_chunk);
+                // The state before step 0 (the carry-in of chunk 0) of this lane's 4 chains.
+                auto initial = [&]() -> float4 {
+                    return (p.h0 && valid) ? *reinterpret_cast<const float4*>(
+                                                 p.h0 + (static_cast<long long>(b) * p.dim + d) * 16 + nl * 4)
+                                           : make_float4(0.f, 0.f, 0.f, 0.f);
+                };
                 float hin[4] = {0.f, 0.f, 0.f, 0.f};
+                if (k == 0) {
+                    const float4 v = initial();
+                    hin[0] = v.x; hin[1] = v.y; hin[2] = v.z; hin[3] = v.w;
+                }
                 const bool have_spec = k > 0 && spec_ok[bi][wc] != 0;
                 if (have_spec) {
                     const float4 v = *reinterpret_cast<const float4*>(spec + bi * 128 + row * 16 + nl * 4);
@@ -364,9 +375,11 @@ scan_fwd_chunked_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_
                             hx[c] = fmaf(px[c], hv[c], hx[c]);
                             px[c] *= ex2_mufu(a2[c] * sj);
                         }
-                        if (kk == 0) {
+                        if (kk == 0) {  // walked back over every chunk: apply them to the initial state
+                            const float4 v = initial();
+                            const float h0v[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                            for (int c = 0; c < 4; ++c) hin[c] = hx[c];
+                            for (int c = 0; c < 4; ++c) hin[c] = fmaf(px[c], h0v[c], hx[c]);
                         }
                     }
                 }

@@ -43,6 +43,7 @@ struct SeqParams {
     const float* A;        // (dim, 16)
     const float* D;        // (dim) or null
     const float* bias;     // (dim) or null
+    const float* h0;       // (batch, dim, 16) initial state or null (zero)
     float* last_state;     // (batch, dim, 16) or null
     void* y;               // (batch, dim, L) IO
     WorkspaceHeader* hdr;  // status word
@@ -123,14 +124,222 @@ __device__ __forceinline__ void store_run(IO* dst, const float (&v)[N]) {
     }
 }
 
+// Consumer warp of the sequential kernel (HZ: the z gate is present).
+//
+// Lane (cg, nl) holds the NC chains n = nl*NC .. of the channels cg + c*CW (c < CPL) of
+// this warp's block of CPW channels; the CPL channels share the batch row, hence every
+// B/C value the lane loads.  The walk goes stage by stage, and the eight 16-byte groups
+// of a stage are unrolled (compile-time shared-memory offsets) with ping-pong step-size
+// buffers: the step sizes of group g+1 (for the last group: group 0 of the next stage,
+// after waiting for it) are computed while group g is scanned.
+template <typename IO, int G, int CPL, int S, bool HZ>
+__device__ __forceinline__ void seq_consumer(const uint8_t* smem, uint64_t* full_bar, uint64_t* empty_bar,
+                                             const int* abort_flag, const SeqParams& p, long long r_begin, int nt,
+                                             int b_first, int stage_bytes, int nstages, int L32) {
+    using Cfg = SeqCfg<IO, G, CPL>;
+    constexpr int NC = Cfg::kNC, CW = Cfg::kCW, CPW = Cfg::kCPW, GS = Cfg::kGS, TC = Cfg::kTC, NG = Cfg::kNG;
+    constexpr int PER = Cfg::kPER, ES = IoTraits<IO>::kBytes;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int cg = lane / G;
+    const int nl = lane % G;
+    const int gbase = lane & ~(G - 1);   // first lane of this channel group
+    int cbase[CPL], d[CPL];
+    bool valid[CPL];
+    int b = 0;
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+        const int cl = warp * CPW + cg + c * CW;   // channel within the round's tiles
+        const bool in_round = cl < nt * 8;
+        const int j = in_round ? cl / 8 : 0;
+        const int row = cl % 8;
+        const long long tile = r_begin + j;
+        if (c == 0) b = static_cast<int>(tile / p.tiles_per_batch);
+        d[c] = static_cast<int>(tile % p.tiles_per_batch) * 8 + row;
+        valid[c] = in_round && d[c] < p.dim;
+        // Byte offset of the lane's 16-byte chunk of group g inside a u/delta/z tile block:
+        // cbase ^ (g << 4) (the 128-byte swizzle XORs the chunk index with the row).
+        cbase[c] = j * Cfg::kTileBytes + row * 128 + (row << 4);
+    }
+    const int dl_off = p.max_tiles * Cfg::kTileBytes;
+    const int z_off = 2 * p.max_tiles * Cfg::kTileBytes;
+    const int bc_off = 3 * p.max_tiles * Cfg::kTileBytes + (b - b_first) * Cfg::kBC + nl * NC * 4;
+
+    float2 A2[CPL][NC / 2], h[CPL][NC / 2];
+    float Dd[CPL], bias[CPL];
+    IO* yrow[CPL];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+        const float* h0 = (valid[c] && p.h0) ? p.h0 + (static_cast<long long>(b) * p.dim + d[c]) * 16 + nl * NC
+                                             : nullptr;
+#pragma unroll
+        for (int jj = 0; jj < NC / 2; ++jj) {
+            const float a0 = valid[c] ? p.A[d[c] * 16 + nl * NC + 2 * jj] : 0.f;
+            const float a1 = valid[c] ? p.A[d[c] * 16 + nl * NC + 2 * jj + 1] : 0.f;
+            A2[c][jj] = f2(a0 * kLog2e, a1 * kLog2e);
+            h[c][jj] = h0 ? *reinterpret_cast<const float2*>(h0 + 2 * jj) : f2(0.f, 0.f);
+        }
+        Dd[c] = (valid[c] && p.D) ? p.D[d[c]] : 0.f;
+        bias[c] = (valid[c] && p.bias) ? p.bias[d[c]] : 0.f;
+        yrow[c] = static_cast<IO*>(p.y) + (static_cast<long long>(b) * p.dim + (valid[c] ? d[c] : 0)) * p.L;
+    }
+    const bool softplus = p.softplus != 0;
+    const uint32_t wait_limit = p.wait_limit;
+
+    // Bounded, warp-uniform wait for ring slot s (a timeout can never leave part of the
+    // warp inside the full-mask shuffles).
+    auto wait_full = [&](int s, uint32_t parity, int k) -> bool {
+        const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&full_bar[s], parity, wait_limit));
+        if (!ok && lane == 0) report_status(p.hdr, kDevTimeout, 2, blockIdx.x, k, wait_limit);
+        return ok && !__any_sync(0xffffffffu, *(volatile const int*)abort_flag != 0);
+    };
+
+    // Step sizes of group g (first step tg) of the stage at st: lane nl evaluates softplus
+    // for its PER steps i = r*G + nl of each of its channels.
+    auto prologue = [&](const uint8_t* st, int g, int tg, float (&mine)[CPL][PER]) {
+#pragma unroll
+        for (int c = 0; c < CPL; ++c)
+#pragma unroll
+            for (int r = 0; r < PER; ++r) {
+                const int i = r * G + nl;
+                const float raw = IoTraits<IO>::to_f32(
+                    *reinterpret_cast<const IO*>(st + dl_off + (cbase[c] ^ (g << 4)) + i * ES));
+                mine[c][r] = (tg + i < L32) ? step_size(raw, bias[c], softplus) : 0.f;  // 0 past L
+            }
+    };
+
+    // Scan, reduce-scatter and epilogue of group g (first step tg) of the stage at st.
+    auto scan_group = [&](const uint8_t* st, int g, int tg, const float (&mine)[CPL][PER]) {
+        float uf[CPL][GS];
+        int chunk[CPL];
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+            chunk[c] = cbase[c] ^ (g << 4);
+            Group16<IO>::unpack(*reinterpret_cast<const uint4*>(st + chunk[c]), uf[c]);
+        }
+        const float* bc = reinterpret_cast<const float*>(st + bc_off) + g * GS * 32;
+        float yp[CPL][GS];
+#pragma unroll
+        for (int i = 0; i < GS; ++i) {
+            const float* bcr = bc + i * 32;
+            float2 Bv[NC / 2], Cv[NC / 2];
+#pragma unroll
+            for (int jj = 0; jj < NC / 2; ++jj) {
+                if constexpr (NC >= 4) {
+                    const float4 Bq = *reinterpret_cast<const float4*>(bcr + (jj & ~1) * 2);
+                    const float4 Cq = *reinterpret_cast<const float4*>(bcr + 16 + (jj & ~1) * 2);
+                    Bv[jj] = (jj & 1) ? f2(Bq.z, Bq.w) : f2(Bq.x, Bq.y);
+                    Cv[jj] = (jj & 1) ? f2(Cq.z, Cq.w) : f2(Cq.x, Cq.y);
+                } else {
+                    Bv[jj] = *reinterpret_cast<const float2*>(bcr + 2 * jj);
+                    Cv[jj] = *reinterpret_cast<const float2*>(bcr + 16 + 2 * jj);
+                }
+            }
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) {
+                const float dti = __shfl_sync(0xffffffffu, mine[c][i / G], gbase | (i % G), 32);
+                const float wi = dti * uf[c][i];
+                const float2 dd = f2(dti, dti);
+                const float2 ww = f2(wi, wi);
+                float2 acc = f2(0.f, 0.f);
+#pragma unroll
+                for (int jj = 0; jj < NC / 2; ++jj) {
+                    const float2 arg = __fmul2_rn(dd, A2[c][jj]);
+                    const float2 a = f2(ex2_mufu(arg.x), ex2_mufu(arg.y));
+                    h[c][jj] = __ffma2_rn(a, h[c][jj], __fmul2_rn(ww, Bv[jj]));
+                    acc = __ffma2_rn(Cv[jj], h[c][jj], acc);
+                }
+                yp[c][i] = acc.x + acc.y;
+            }
+        }
+
+        // Reduce-scatter the G partial sums of each channel: afterwards lane nl holds
+        // the full y_t of steps nl*PER .. nl*PER+PER-1 in yp[c][0..PER-1].
+#pragma unroll
+        for (int m = G / 2, half = GS / 2; m >= 1; m >>= 1, half >>= 1) {
+            const bool upper = (nl & m) != 0;
+#pragma unroll
+            for (int c = 0; c < CPL; ++c)
+#pragma unroll
+                for (int i = 0; i < half; ++i) {
+                    const float send = upper ? yp[c][i] : yp[c][i + half];
+                    const float keep = upper ? yp[c][i + half] : yp[c][i];
+                    yp[c][i] = keep + __shfl_xor_sync(0xffffffffu, send, m, 32);
+                }
+        }
+
+        // Epilogue: D skip and silu gate ([Eng] §2.2; [Hist] Mamba Block), round, store.
+        const int t0 = tg + nl * PER;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+            const int off = chunk[c] + nl * PER * ES;
+            float ue[PER], ze[PER], yo[PER];
+            load_run<IO, PER>(st + off, ue);
+            if constexpr (HZ) load_run<IO, PER>(st + z_off + off, ze);
+#pragma unroll
+            for (int r = 0; r < PER; ++r) {
+                float v = fmaf(Dd[c], ue[r], yp[c][r]);
+                if constexpr (HZ) v *= gate_silu<IO>(ze[r]);
+                yo[r] = v;
+            }
+            if (valid[c]) {
+                if (t0 + PER <= L32) {
+                    store_run<IO, PER>(yrow[c] + t0, yo);
+                } else {
+#pragma unroll
+                    for (int r = 0; r < PER; ++r)
+                        if (t0 + r < L32) yrow[c][t0 + r] = IoTraits<IO>::from_f32(yo[r]);
+                }
+            }
+        }
+    };
+
+    float spA[CPL][PER], spB[CPL][PER];
+    const uint8_t* st = smem;
+    int slot = 0;
+    uint32_t parity = 0;
+    bool alive = wait_full(0, 0, 0);
+    if (alive) prologue(st, 0, 0, spA);
+#pragma unroll 1
+    for (int k = 0, tk = 0; alive && k < nstages; ++k, tk += TC) {
+#pragma unroll
+        for (int g = 0; g < NG; g += 2) {
+            prologue(st, g + 1, tk + (g + 1) * GS, spB);
+            scan_group(st, g, tk + g * GS, spA);
+            if (g + 2 < NG) {
+                prologue(st, g + 2, tk + (g + 2) * GS, spA);
+            } else if (k + 1 < nstages) {
+                const int sn = slot + 1 == S ? 0 : slot + 1;
+                alive = wait_full(sn, slot + 1 == S ? parity ^ 1u : parity, k + 1);
+                if (alive) prologue(smem + sn * stage_bytes, 0, tk + TC, spA);
+            }
+            scan_group(st, g + 1, tk + (g + 1) * GS, spB);
+        }
+        // The stage is consumed: release it to the producer.
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_bar[slot]);
+        if (++slot == S) {
+            slot = 0;
+            parity ^= 1u;
+        }
+        st = smem + slot * stage_bytes;
+    }
+
+#pragma unroll
+    for (int c = 0; c < CPL; ++c)
+        if (valid[c] && p.last_state) {
+            float* dst = p.last_state + (static_cast<long long>(b) * p.dim + d[c]) * 16 + nl * NC;
+#pragma unroll
+            for (int jj = 0; jj < NC / 2; ++jj) *reinterpret_cast<float2*>(dst + 2 * jj) = h[c][jj];
+        }
+}
+
 template <typename IO, int G, int CPL, int S>
 __global__ void __launch_bounds__((SeqCfg<IO, G, CPL>::kMaxWarps + 1) * 32, 1)
 scan_fwd_seq_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_dl,
                     const __grid_constant__ CUtensorMap map_z, const __grid_constant__ CUtensorMap map_bc,
                     const SeqParams p) {
     using Cfg = SeqCfg<IO, G, CPL>;
-    constexpr int NC = Cfg::kNC, CW = Cfg::kCW, CPW = Cfg::kCPW, GS = Cfg::kGS, TC = Cfg::kTC, NG = Cfg::kNG;
-    constexpr int PER = Cfg::kPER, ES = IoTraits<IO>::kBytes, TPW = Cfg::kTPW;
+    constexpr int TC = Cfg::kTC, TPW = Cfg::kTPW;
     static_assert(S >= 2 && S <= 8, "ring depth");
 
     extern __shared__ uint8_t smem_raw[];
@@ -183,7 +392,7 @@ scan_fwd_seq_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_cons
                 const uint32_t bytes = nt * (p.has_z ? 3u : 2u) * Cfg::kTileBytes + nb * Cfg::kBC;
                 for (int k = 0; k < nstages; ++k) {
                     const int s = k % S;
-                    if (k >= S && !mbar_wait_bounded(&empty_bar[s], ((k / S) - 1) & 1, p.wait_limit)) {
+                    if (k >= S && !mbar_wait_sleep(&empty_bar[s], ((k / S) - 1) & 1, p.wait_limit)) {
                         report_status(p.hdr, kDevTimeout, 1, blockIdx.x, k, p.wait_limit);
                         atomicExch(&abort_flag, 1);
                         break;
@@ -207,199 +416,12 @@ scan_fwd_seq_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_cons
                 }
             }
         } else if (warp < nwarps) {
-            // ------------------------------------------------------------ consumers
-            // Lane (cg, nl) holds the NC chains n = nl*NC .. of the channels cg + c*CW
-            // (c < CPL) of this warp's block of CPW channels; the CPL channels share the
-            // batch row, hence every B/C value the lane loads.
-            const int cg = lane / G;
-            const int nl = lane % G;
-            const int gbase = lane & ~(G - 1);   // first lane of this channel group
-            int j[CPL], row[CPL], d[CPL];
-            bool valid[CPL];
-            int b = 0;
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) {
-                const int cl = warp * CPW + cg + c * CW;   // channel within the round's tiles
-                const bool in_round = cl < nt * 8;
-                j[c] = in_round ? cl / 8 : 0;
-                row[c] = cl % 8;
-                const long long tile = r_begin + j[c];
-                if (c == 0) b = static_cast<int>(tile / p.tiles_per_batch);
-                d[c] = static_cast<int>(tile % p.tiles_per_batch) * 8 + row[c];
-                valid[c] = in_round && d[c] < p.dim;
-            }
-            const int bcs = b - b_first;         // B/C slot of this batch row
-
-            float2 A2[CPL][NC / 2], h[CPL][NC / 2];
-            float Dd[CPL], bias[CPL];
-            IO* yrow[CPL];
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) {
-#pragma unroll
-                for (int jj = 0; jj < NC / 2; ++jj) {
-                    const float a0 = valid[c] ? p.A[d[c] * 16 + nl * NC + 2 * jj] : 0.f;
-                    const float a1 = valid[c] ? p.A[d[c] * 16 + nl * NC + 2 * jj + 1] : 0.f;
-                    A2[c][jj] = f2(a0 * kLog2e, a1 * kLog2e);
-                    h[c][jj] = f2(0.f, 0.f);
-                }
-                Dd[c] = (valid[c] && p.D) ? p.D[d[c]] : 0.f;
-                bias[c] = (valid[c] && p.bias) ? p.bias[d[c]] : 0.f;
-                yrow[c] = static_cast<IO*>(p.y) + (static_cast<long long>(b) * p.dim + (valid[c] ? d[c] : 0)) * p.L;
-            }
-            const bool softplus = p.softplus != 0;
-            const bool has_z = p.has_z != 0;
-
-            auto stage_of = [&](int q) -> const uint8_t* { return smem + ((q / NG) % S) * stage_bytes; };
-            auto chunk_of = [&](int q, int c) -> int {
-                return j[c] * Cfg::kTileBytes + row[c] * 128 + (((q % NG) ^ row[c]) << 4);
-            };
-
-            // Bounded, warp-uniform wait for the stage that holds group q (a timeout can
-            // never leave part of the warp inside the full-mask shuffles).
-            auto wait_stage = [&](int q) -> bool {
-                const int k = q / NG;
-                const bool ok =
-                    __all_sync(0xffffffffu, mbar_wait_bounded(&full_bar[k % S], (k / S) & 1, p.wait_limit));
-                if (!ok && lane == 0) report_status(p.hdr, kDevTimeout, 2, blockIdx.x, k, p.wait_limit);
-                return ok && !__any_sync(0xffffffffu, *(volatile int*)&abort_flag != 0);
-            };
-
-            // Step sizes of group q: lane nl evaluates softplus for its PER steps
-            // i = r*G + nl of each of its channels (issued one group ahead of the scan).
-            auto prologue = [&](int q, float (&mine)[CPL][PER]) {
-                const uint8_t* dl = stage_of(q) + p.max_tiles * Cfg::kTileBytes;
-#pragma unroll
-                for (int c = 0; c < CPL; ++c)
-#pragma unroll
-                    for (int r = 0; r < PER; ++r) {
-                        const int i = r * G + nl;
-                        const float raw =
-                            IoTraits<IO>::to_f32(*reinterpret_cast<const IO*>(dl + chunk_of(q, c) + i * ES));
-                        mine[c][r] = (q * GS + i < L32) ? step_size(raw, bias[c], softplus) : 0.f;  // 0 past L
-                    }
-            };
-
-            // Scan, reduce-scatter and epilogue of group q.  The G lanes of a channel group
-            // exchange their step sizes by shuffles, so each lane has Delta and Delta*u of
-            // every step; one B/C load per step serves all CPL channels of the lane.
-            auto scan_group = [&](int q, const float (&mine)[CPL][PER]) {
-                const uint8_t* st = stage_of(q);
-                float uf[CPL][GS];
-#pragma unroll
-                for (int c = 0; c < CPL; ++c)
-                    Group16<IO>::unpack(*reinterpret_cast<const uint4*>(st + chunk_of(q, c)), uf[c]);
-                const float* bc = reinterpret_cast<const float*>(st + 3 * p.max_tiles * Cfg::kTileBytes +
-                                                                 bcs * Cfg::kBC) +
-                                  (q % NG) * GS * 32 + nl * NC;
-                float yp[CPL][GS];
-#pragma unroll
-                for (int i = 0; i < GS; ++i) {
-                    const float* bcr = bc + i * 32;
-                    float2 Bv[NC / 2], Cv[NC / 2];
-#pragma unroll
-                    for (int jj = 0; jj < NC / 2; ++jj) {
-                        if constexpr (NC >= 4) {
-                            const float4 Bq = *reinterpret_cast<const float4*>(bcr + (jj & ~1) * 2);
-                            const float4 Cq = *reinterpret_cast<const float4*>(bcr + 16 + (jj & ~1) * 2);
-                            Bv[jj] = (jj & 1) ? f2(Bq.z, Bq.w) : f2(Bq.x, Bq.y);
-                            Cv[jj] = (jj & 1) ? f2(Cq.z, Cq.w) : f2(Cq.x, Cq.y);
-                        } else {
-                            Bv[jj] = *reinterpret_cast<const float2*>(bcr + 2 * jj);
-                            Cv[jj] = *reinterpret_cast<const float2*>(bcr + 16 + 2 * jj);
-                        }
-                    }
-#pragma unroll
-                    for (int c = 0; c < CPL; ++c) {
-                        const float dti = __shfl_sync(0xffffffffu, mine[c][i / G], gbase | (i % G), 32);
-                        const float wi = dti * uf[c][i];
-                        const float2 dd = f2(dti, dti);
-                        const float2 ww = f2(wi, wi);
-                        float2 acc = f2(0.f, 0.f);
-#pragma unroll
-                        for (int jj = 0; jj < NC / 2; ++jj) {
-                            const float2 arg = __fmul2_rn(dd, A2[c][jj]);
-                            const float2 a = f2(ex2_mufu(arg.x), ex2_mufu(arg.y));
-                            h[c][jj] = __ffma2_rn(a, h[c][jj], __fmul2_rn(ww, Bv[jj]));
-                            acc = __ffma2_rn(Cv[jj], h[c][jj], acc);
-                        }
-                        yp[c][i] = acc.x + acc.y;
-                    }
-                }
-
-                // Reduce-scatter the G partial sums of each channel: afterwards lane nl holds
-                // the full y_t of steps nl*PER .. nl*PER+PER-1 in yp[c][0..PER-1].
-#pragma unroll
-                for (int m = G / 2, half = GS / 2; m >= 1; m >>= 1, half >>= 1) {
-                    const bool upper = (nl & m) != 0;
-#pragma unroll
-                    for (int c = 0; c < CPL; ++c)
-#pragma unroll
-                        for (int i = 0; i < half; ++i) {
-                            const float send = upper ? yp[c][i] : yp[c][i + half];
-                            const float keep = upper ? yp[c][i + half] : yp[c][i];
-                            yp[c][i] = keep + __shfl_xor_sync(0xffffffffu, send, m, 32);
-                        }
-                }
-
-                // Epilogue: D skip and silu gate ([Eng] §2.2; [Hist] Mamba Block), round, store.
-                const int t0 = q * GS + nl * PER;
-#pragma unroll
-                for (int c = 0; c < CPL; ++c) {
-                    const int off = chunk_of(q, c) + nl * PER * ES;
-                    float ue[PER], ze[PER], yo[PER];
-                    load_run<IO, PER>(st + off, ue);
-                    if (has_z) load_run<IO, PER>(st + 2 * p.max_tiles * Cfg::kTileBytes + off, ze);
-#pragma unroll
-                    for (int r = 0; r < PER; ++r) {
-                        float v = fmaf(Dd[c], ue[r], yp[c][r]);
-                        if (has_z) v *= gate_silu<IO>(ze[r]);
-                        yo[r] = v;
-                    }
-                    if (valid[c]) {
-                        if (t0 + PER <= L32) {
-                            store_run<IO, PER>(yrow[c] + t0, yo);
-                        } else {
-#pragma unroll
-                            for (int r = 0; r < PER; ++r)
-                                if (t0 + r < L32) yrow[c][t0 + r] = IoTraits<IO>::from_f32(yo[r]);
-                        }
-                    }
-                }
-                // The last group of a stage releases the stage to the producer.
-                if (q % NG == NG - 1) {
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&empty_bar[(q / NG) % S]);
-                }
-            };
-
-            // Groups two per iteration with ping-pong step-size buffers: while group q is
-            // scanned the next group's step sizes are computed into the other buffer.
-            const int ngroups = nstages * NG;
-            float spA[CPL][PER], spB[CPL][PER];
-            bool alive = wait_stage(0);
-            if (alive) prologue(0, spA);
-#pragma unroll 1
-            for (int q = 0; alive && q < ngroups; q += 2) {
-                if (q + 1 < ngroups) {
-                    if ((q + 1) % NG == 0) alive = wait_stage(q + 1);
-                    if (alive) prologue(q + 1, spB);
-                }
-                scan_group(q, spA);
-                if (!alive || q + 1 >= ngroups) break;
-                if (q + 2 < ngroups) {
-                    if ((q + 2) % NG == 0) alive = wait_stage(q + 2);
-                    if (alive) prologue(q + 2, spA);
-                }
-                scan_group(q + 1, spB);
-            }
-
-#pragma unroll
-            for (int c = 0; c < CPL; ++c)
-                if (valid[c] && p.last_state) {
-                    float* dst = p.last_state + (static_cast<long long>(b) * p.dim + d[c]) * 16 + nl * NC;
-#pragma unroll
-                    for (int jj = 0; jj < NC / 2; ++jj) *reinterpret_cast<float2*>(dst + 2 * jj) = h[c][jj];
-                }
+            if (p.has_z)
+                seq_consumer<IO, G, CPL, S, true>(smem, full_bar, empty_bar, &abort_flag, p, r_begin, nt, b_first,
+                                                  stage_bytes, nstages, L32);
+            else
+                seq_consumer<IO, G, CPL, S, false>(smem, full_bar, empty_bar, &abort_flag, p, r_begin, nt, b_first,
+                                                   stage_bytes, nstages, L32);
         }
         // Every warp leaves the round before the barriers are re-initialised for the next.
         __syncthreads();

@@ -129,6 +129,7 @@ struct FwdArgs {
     const void *u, *delta, *B, *C, *z;
     const float *A, *D, *bias;
     int softplus;
+    const float* h0;
     void* y;
     float* last_state;
     int batch, dim;
@@ -233,6 +234,7 @@ ssm_status_t launch_seq(const FwdArgs& a, const SeqPlan& pl) {
     p.A = a.A;
     p.D = a.D;
     p.bias = a.bias;
+    p.h0 = a.h0;
     p.last_state = a.last_state;
     p.y = a.y;
     p.hdr = reinterpret_cast<WorkspaceHeader*>(a.ws);
@@ -289,6 +291,7 @@ ssm_status_t launch_chunked(const FwdArgs& a, const ssm_fwd_options_t& o) {
     p.pay_agg = reinterpret_cast<float*>(a.ws + wl.agg_off);
     p.pay_sdt = reinterpret_cast<float*>(a.ws + wl.sdt_off);
     p.pay_incl = reinterpret_cast<float*>(a.ws + wl.incl_off);
+    p.h0 = a.h0;
     p.batch = a.batch;
     p.dim = a.dim;
     p.L = static_cast<int>(a.L);
@@ -316,6 +319,7 @@ ssm_status_t launch_direct(const FwdArgs& a) {
     p.A = a.A;
     p.D = a.D;
     p.bias = a.bias;
+    p.h0 = a.h0;
     p.y = a.y;
     p.last_state = a.last_state;
     p.batch = a.batch;
@@ -432,11 +436,12 @@ ssm_status_t ssm_workspace_init(void* workspace, size_t workspace_bytes, ssm_str
                : SSM_ERR_LAUNCH;
 }
 
-ssm_status_t ssm_selective_scan_fwd_ex(const void* u, const void* delta, const float* A, const void* B,
-                                       const void* C, const float* D, const void* z, const float* delta_bias,
-                                       int softplus, void* y, float* last_state, int batch, int dim, int dstate,
-                                       int64_t seqlen, ssm_dtype_t io_dtype, void* workspace,
-                                       size_t workspace_bytes, const ssm_fwd_options_t* opts, ssm_stream_t stream) {
+ssm_status_t ssm_selective_scan_fwd_state(const void* u, const void* delta, const float* A, const void* B,
+                                          const void* C, const float* D, const void* z, const float* delta_bias,
+                                          int softplus, const float* initial_state, void* y, float* last_state,
+                                          int batch, int dim, int dstate, int64_t seqlen, ssm_dtype_t io_dtype,
+                                          void* workspace, size_t workspace_bytes, const ssm_fwd_options_t* opts,
+                                          ssm_stream_t stream) {
     if (batch < 0 || dim < 0 || seqlen < 0) return SSM_ERR_INVALID_ARG;
     // Tensors with elements must have a pointer; zero-element tensors may be NULL.
     const bool seq_elems = batch > 0 && dim > 0 && seqlen > 0;
@@ -444,9 +449,16 @@ ssm_status_t ssm_selective_scan_fwd_ex(const void* u, const void* delta, const f
     if (dim > 0 && !A) return SSM_ERR_INVALID_ARG;
     if (io_dtype != SSM_F32 && io_dtype != SSM_BF16) return SSM_ERR_INVALID_ARG;
     if (dstate != 16) return SSM_ERR_UNSUPPORTED;
-    const void* ptrs[] = {u, delta, A, B, C, D, z, delta_bias, y, last_state};
+    const void* ptrs[] = {u, delta, A, B, C, D, z, delta_bias, initial_state, y, last_state};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return SSM_ERR_INVALID_ARG;
+    const size_t state_bytes = static_cast<size_t>(batch) * static_cast<size_t>(dim) * 16u * sizeof(float);
+    if (initial_state && last_state && state_bytes > 0) {
+        // The chunked kernel may still read a channel's initial state after another CTA
+        // has written that channel's final state, so the two must not overlap.
+        const uintptr_t a0 = reinterpret_cast<uintptr_t>(initial_state), a1 = reinterpret_cast<uintptr_t>(last_state);
+        if ((a0 <= a1 ? a1 - a0 : a0 - a1) < state_bytes) return SSM_ERR_INVALID_ARG;
+    }
     ssm_fwd_options_t o{SSM_ALGO_AUTO, 0, 0, -1};
     if (opts) o = *opts;
     if (o.algo < SSM_ALGO_AUTO || o.algo > SSM_ALGO_DIRECT) return SSM_ERR_INVALID_ARG;
@@ -459,15 +471,28 @@ ssm_status_t ssm_selective_scan_fwd_ex(const void* u, const void* delta, const f
     ssm_status_t st = check_device(&sm_count);
     if (st != SSM_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (seqlen == 0) {
-        if (last_state &&
-            cudaMemsetAsync(last_state, 0, static_cast<size_t>(batch) * dim * 16 * sizeof(float), s) != cudaSuccess)
-            return SSM_ERR_LAUNCH;
+    if (seqlen == 0) {  // no steps: the final state is the initial one
+        if (last_state) {
+            const cudaError_t e = initial_state
+                                      ? cudaMemcpyAsync(last_state, initial_state, state_bytes,
+                                                        cudaMemcpyDeviceToDevice, s)
+                                      : cudaMemsetAsync(last_state, 0, state_bytes, s);
+            if (e != cudaSuccess) return SSM_ERR_LAUNCH;
+        }
         return SSM_OK;
     }
-    FwdArgs a{u, delta, B, C, z, A, D, delta_bias, softplus, y, last_state, batch, dim, seqlen, io_dtype,
-              static_cast<uint8_t*>(workspace), s, sm_count};
+    FwdArgs a{u, delta, B, C, z, A, D, delta_bias, softplus, initial_state, y, last_state, batch, dim, seqlen,
+              io_dtype, static_cast<uint8_t*>(workspace), s, sm_count};
     return io_dtype == SSM_BF16 ? launch_forward<__nv_bfloat16>(a, o) : launch_forward<float>(a, o);
+}
+
+ssm_status_t ssm_selective_scan_fwd_ex(const void* u, const void* delta, const float* A, const void* B,
+                                       const void* C, const float* D, const void* z, const float* delta_bias,
+                                       int softplus, void* y, float* last_state, int batch, int dim, int dstate,
+                                       int64_t seqlen, ssm_dtype_t io_dtype, void* workspace,
+                                       size_t workspace_bytes, const ssm_fwd_options_t* opts, ssm_stream_t stream) {
+    return ssm_selective_scan_fwd_state(u, delta, A, B, C, D, z, delta_bias, softplus, nullptr, y, last_state, batch,
+                                        dim, dstate, seqlen, io_dtype, workspace, workspace_bytes, opts, stream);
 }
 
 ssm_status_t ssm_selective_scan_fwd(const void* u, const void* delta, const float* A, const void* B, const void* C,
@@ -535,7 +560,7 @@ ssm_status_t ssm_selective_scan_fwd_noalloc(const void* u, const void* delta, co
     if (cudaMemsetAsync(scratch, 0, sizeof(WorkspaceHeader), s) != cudaSuccess) return SSM_ERR_LAUNCH;
     // Kernels whose scratch is only the header and the B/C rows (no look-back flags).
     const ssm_fwd_options_t o{SSM_ALGO_SEQUENTIAL, 0, 0, -1};
-    FwdArgs a{u, delta, B, C, z, A, D, delta_bias, softplus, y, last_state, batch, dim, seqlen, io_dtype,
+    FwdArgs a{u, delta, B, C, z, A, D, delta_bias, softplus, nullptr, y, last_state, batch, dim, seqlen, io_dtype,
               scratch, s, sm_count};
     return io_dtype == SSM_BF16 ? launch_forward<__nv_bfloat16>(a, o) : launch_forward<float>(a, o);
 }

@@ -34,20 +34,22 @@ def assert_close(x, ref, io, what):
     return worst
 
 
-def gpu_forward(inp, dev="cuda", softplus=True, **opts):
+def gpu_forward(inp, dev="cuda", softplus=True, h0=None, **opts):
     g = to_dev(inp, dev)
     y, last = ssm.selective_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"],
-                                     g["delta_bias"], softplus=softplus, **opts)
+                                     g["delta_bias"], softplus=softplus,
+                                     initial_state=None if h0 is None else h0.to(dev), **opts)
     torch.cuda.synchronize()
     return y, last
 
 
-def oracle_forward(inp, softplus=True, channels=None):
+def oracle_forward(inp, softplus=True, channels=None, h0=None):
     """Full oracle, or only the listed flat channels (b*dim + d) when `channels` is given;
-    returns (y, last) restricted to those channels in that order."""
+    returns (y, last) restricted to those channels in that order.  h0: initial state
+    (b, d, N) or None (zero)."""
     if channels is None:
         return oracle.selective_scan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], D=inp["D"],
-                                     z=inp["z"], delta_bias=inp["delta_bias"], softplus=softplus)
+                                     z=inp["z"], delta_bias=inp["delta_bias"], softplus=softplus, h0=h0)
     b_, d_, L = inp["u"].shape
     ys, lasts = [], []
     channels = np.asarray(channels)
@@ -57,7 +59,8 @@ def oracle_forward(inp, softplus=True, channels=None):
                    B=inp["B"][bi][None], C=inp["C"][bi][None],
                    D=None if inp["D"] is None else inp["D"][ds],
                    z=None if inp["z"] is None else inp["z"][bi, ds][None],
-                   delta_bias=None if inp["delta_bias"] is None else inp["delta_bias"][ds])
+                   delta_bias=None if inp["delta_bias"] is None else inp["delta_bias"][ds],
+                   h0=None if h0 is None else h0[bi, ds][None])
         y, last = oracle.selective_scan(**sub, softplus=softplus)
         ys.append((bi, ds, y[0], last[0]))
     order = {(int(bi), int(d)): (y[i], last[i]) for bi, ds, y, last in ys for i, d in enumerate(ds)}
@@ -66,10 +69,10 @@ def oracle_forward(inp, softplus=True, channels=None):
     return yy, ll
 
 
-def check_forward(inp, softplus=True, channels=None, what="forward", **opts):
+def check_forward(inp, softplus=True, channels=None, what="forward", h0=None, **opts):
     io = io_of(inp["u"])
-    y, last = gpu_forward(inp, softplus=softplus, **opts)
-    y_ref, last_ref = oracle_forward(inp, softplus=softplus, channels=channels)
+    y, last = gpu_forward(inp, softplus=softplus, h0=h0, **opts)
+    y_ref, last_ref = oracle_forward(inp, softplus=softplus, channels=channels, h0=h0)
     if channels is not None:
         b_, d_, L = inp["u"].shape
         idx = torch.as_tensor(np.asarray(channels), device=y.device)

@@ -33,7 +33,8 @@ def lib():
 def test_header_declares_entry_points():
     names = _declared_functions()
     for n in ["ssm_selective_scan_fwd", "ssm_state_update", "ssm_selective_scan_workspace_size",
-              "ssm_read_status", "ssm_selective_scan_fwd_ex", "ssm_workspace_init"]:
+              "ssm_read_status", "ssm_selective_scan_fwd_ex", "ssm_workspace_init",
+              "ssm_selective_scan_fwd_state"]:
         assert n in names
 
 
@@ -90,6 +91,19 @@ def test_forward_ex_rejects_unknown_algo(lib):
                                        P(4096), None, 1, 1, 16, 8, binding.SSM_BF16, P(4096), 1 << 20,
                                        ctypes.byref(opts), None)
     assert rc == binding.SSM_ERR_INVALID_ARG
+
+
+def test_forward_state_argument_validation(lib):
+    def call(h0, last, batch=2, dim=3):
+        return lib.ssm_selective_scan_fwd_state(P(4096), P(4096), P(4096), P(4096), P(4096), None, None, None, 1,
+                                                h0, P(4096), last, batch, dim, 16, 8, binding.SSM_BF16, P(4096),
+                                                1 << 20, None, None)
+    state_bytes = 2 * 3 * 16 * 4
+    assert call(P(1 << 20), P(1 << 20)) == binding.SSM_ERR_INVALID_ARG                  # same buffer
+    assert call(P(1 << 20), P((1 << 20) + state_bytes - 16)) == binding.SSM_ERR_INVALID_ARG  # overlap
+    assert call(P((1 << 20) + state_bytes - 16), P(1 << 20)) == binding.SSM_ERR_INVALID_ARG
+    assert call(P((1 << 20) + 8), None) == binding.SSM_ERR_INVALID_ARG                  # misaligned
+    assert call(P(1 << 20), P((1 << 20) + state_bytes), batch=0) == binding.SSM_OK     # adjacent, empty
 
 
 def test_decode_argument_validation(lib):

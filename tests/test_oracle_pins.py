@@ -215,6 +215,24 @@ def test_initial_state_enters_as_decayed_carry():
     np.testing.assert_allclose(last1, last0 + P[:, :, -1, :] * h0, rtol=1e-11, atol=1e-12)
 
 
+def test_block_continuation_equals_whole_scan():
+    # Scanning [0, L1) and then [L1, L) from the first block's final state is the scan of
+    # [0, L) ([Eng] §7.2): the block split is invisible in y and in the final state.
+    rng = _rng(41)
+    case = _selective_case(rng)
+    L = case["u"].shape[2]
+    y, last = oracle.selective_scan(**case)
+    for cut in (1, L // 3, L - 1):
+        first = {k: (v[..., :cut] if k in ("u", "delta", "z", "B", "C") and v is not None else v)
+                 for k, v in case.items()}
+        second = {k: (v[..., cut:] if k in ("u", "delta", "z", "B", "C") and v is not None else v)
+                  for k, v in case.items()}
+        y1, h1 = oracle.selective_scan(**first)
+        y2, h2 = oracle.selective_scan(**second, h0=h1)
+        np.testing.assert_allclose(np.concatenate([y1, y2], axis=2), y, rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(h2, last, rtol=1e-12, atol=1e-13)
+
+
 # ---------------------------------------------------------------------------------------------
 # P-E: two-step identity with constant Abar  ([Card] 线性扫描算法)
 # ---------------------------------------------------------------------------------------------

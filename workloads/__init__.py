@@ -15,6 +15,8 @@ Recipe (per workload):
   delta_bias[d]  = inverse softplus of dt, dt log-uniform in [dt_min, dt_max]
                    (computed in fp64, stored fp32)
   softplus on.
+Scans that continue from a given state (initial_state) draw it ~ N(0, 1), fp32,
+shape (batch, dim, dstate), from their own seed.
 Decode workloads additionally draw an initial state ~ N(0, 1) of shape
 (batch, dim, dstate) in fp32 and a pool of POOL per-step input sets.
 """
@@ -73,6 +75,13 @@ def _bias_from_dt(gen, dim, dt_min, dt_max):
     r = torch.rand(dim, generator=gen, dtype=torch.float64).numpy()
     dt = np.exp(math.log(dt_min) + r * (math.log(dt_max) - math.log(dt_min)))
     return torch.from_numpy(np.log(np.expm1(dt))).to(torch.float32)
+
+
+def initial_state(batch, dim, dstate=16, seed=0, scale=1.0):
+    """Seeded fp32 initial state (batch, dim, dstate) ~ scale * N(0, 1), for scans that
+    continue from a given state."""
+    g = torch.Generator().manual_seed(seed)
+    return _randn(g, (batch, dim, dstate), scale).contiguous()
 
 
 def scan_inputs(batch, dim, seqlen, dstate=16, io="bf16", dt_min=1e-3, dt_max=1e-1, seed=0,
