@@ -45,6 +45,8 @@ def _load():
             lib.oracle_selective_scan_f64.restype = ci
             lib.oracle_state_update_f64.argtypes = [vp] * 9 + [ci, vp, i64, i64, i64]
             lib.oracle_state_update_f64.restype = ci
+            lib.oracle_selective_scan_bwd_f64.argtypes = [vp] * 8 + [ci] + [vp] * 12 + [i64, i64, i64, i64]
+            lib.oracle_selective_scan_bwd_f64.restype = ci
             lib.oracle_num_threads.restype = ci
             lib.oracle_softplus_f64.argtypes = [ctypes.c_double]
             lib.oracle_softplus_f64.restype = ctypes.c_double
@@ -115,3 +117,27 @@ def state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, soft
     if rc != 0:
         raise ValueError("oracle_state_update_f64 rejected its arguments")
     return y, st
+
+
+def selective_scan_bwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True, h0=None, dy=None,
+                       dlast=None):
+    """Gradients of L = sum(dy * y) + sum(dlast * last_state) for the forward scan with these
+    inputs.  Returns a dict of float64 arrays: du, ddelta (b, d, L); dA (d, N); dB, dC (b, N, L);
+    dD, ddelta_bias (d) (always, as if D / delta_bias were given); dz (b, d, L) or None;
+    dh0 (b, d, N) (the gradient with respect to the initial state, zero or h0)."""
+    u, delta, A, B, C = map(_f64, (u, delta, A, B, C))
+    D, z, delta_bias, h0, dy, dlast = map(_f64, (D, z, delta_bias, h0, dy, dlast))
+    b, d, L = u.shape
+    n = A.shape[1]
+    assert dy is not None and dy.shape == u.shape
+    assert dlast is None or dlast.shape == (b, d, n)
+    out = dict(du=np.empty((b, d, L)), ddelta=np.empty((b, d, L)), dA=np.empty((d, n)),
+               dB=np.empty((b, n, L)), dC=np.empty((b, n, L)), dD=np.empty(d), ddelta_bias=np.empty(d),
+               dz=np.empty((b, d, L)) if z is not None else None, dh0=np.empty((b, d, n)))
+    rc = _load().oracle_selective_scan_bwd_f64(
+        _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias), int(bool(softplus)),
+        _ptr(h0), _ptr(dy), _ptr(dlast), _ptr(out["du"]), _ptr(out["ddelta"]), _ptr(out["dA"]), _ptr(out["dB"]),
+        _ptr(out["dC"]), _ptr(out["dD"]), _ptr(out["dz"]), _ptr(out["ddelta_bias"]), _ptr(out["dh0"]), b, d, n, L)
+    if rc != 0:
+        raise ValueError("oracle_selective_scan_bwd_f64 rejected its arguments")
+    return out

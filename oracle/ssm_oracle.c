@@ -32,6 +32,12 @@
  * The state starts at zero unless h0 is given ([Eng] §7.2; [Card] Python 演示) and
  * the state after the last step is written to last_state ([Eng] §4.2).
  *
+ * The backward (oracle_selective_scan_bwd_f64) is the plain definition of the
+ * gradients of L = sum dy*y + sum dlast*last_state: the same forward loop, keeping
+ * every state, then the chain rule applied to each step in reverse order (the
+ * recompute-in-backward scheme of [Tech] 四.1 and [S4M] 3.3, here with everything
+ * kept).  It is pinned by finite differences of the forward scan.
+ *
  * Layouts (all contiguous, row-major): u, delta, z, y: (batch, dim, L);
  * B, C: (batch, dstate, L); A: (dim, dstate); D, delta_bias: (dim);
  * h0 / last_state / decode state: (batch, dim, dstate).
@@ -44,6 +50,11 @@
 #include <math.h>
 #include <stddef.h>
 #include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 /* softplus(x) = log(1 + e^x), written so that neither branch overflows. */
 static double softplus_f64(double x)
@@ -142,11 +153,176 @@ int oracle_state_update_f64(double* state, const double* u, const double* delta,
     return 0;
 }
 
+/* d silu / dz = sigmoid(z) * (1 + z * (1 - sigmoid(z))). */
+static double silu_grad_f64(double z)
+{
+    const double s = 1.0 / (1.0 + exp(-z));
+    return s * (1.0 + z * (1.0 - s));
+}
+
+/* d softplus / dx = sigmoid(x). */
+static double sigmoid_f64(double x)
+{
+    return x >= 0.0 ? 1.0 / (1.0 + exp(-x)) : exp(x) / (1.0 + exp(x));
+}
+
+/*
+ * Backward of one channel (b, d): the forward loop again, keeping every state, then
+ * the chain rule applied to it step by step in reverse order.  Per-channel outputs are
+ * written; the sums over channels (dB, dC) and over batch rows (dA, dD, ddelta_bias)
+ * are added into the caller's accumulators.
+ *   H: (L+1) x dstate scratch (H[0] = initial state, H[t+1] = state after step t);
+ *   Dt: L scratch (step sizes).
+ */
+static void channel_bwd(int64_t b, int64_t d, const double* u, const double* delta, const double* A,
+                        const double* B, const double* C, const double* D, const double* z,
+                        const double* delta_bias, int softplus, const double* h0, const double* dy,
+                        const double* dlast, double* du, double* ddelta, double* dz, double* dh0,
+                        double* accB, double* accC, double* accA, double* accD, double* accBias,
+                        int64_t dim, int64_t N, int64_t L, double* H, double* Dt)
+{
+    const int64_t row = b * dim + d;
+    const double Dd = D ? D[d] : 0.0;
+    for (int64_t n = 0; n < N; ++n) H[n] = h0 ? h0[row * N + n] : 0.0;
+    for (int64_t t = 0; t < L; ++t) {  /* forward, as oracle_selective_scan_f64 */
+        const double ut = u[row * L + t];
+        Dt[t] = step_size(delta[row * L + t], delta_bias, d, softplus);
+        for (int64_t n = 0; n < N; ++n)
+            H[(t + 1) * N + n] = exp(Dt[t] * A[d * N + n]) * H[t * N + n] + Dt[t] * B[(b * N + n) * L + t] * ut;
+    }
+    /* g[n] = dL/dh: the gradient reaching the state, starting from dL/d last_state. */
+    double g[256];
+    for (int64_t n = 0; n < N; ++n) g[n] = dlast ? dlast[row * N + n] : 0.0;
+    for (int64_t t = L - 1; t >= 0; --t) {
+        const double ut = u[row * L + t], dt = Dt[t];
+        /* y = v * silu(z), v = sum_n C h_t + D u */
+        double v = Dd * ut;
+        for (int64_t n = 0; n < N; ++n) v += C[(b * N + n) * L + t] * H[(t + 1) * N + n];
+        double dv = dy[row * L + t];
+        if (z) {
+            const double zt = z[row * L + t];
+            dz[row * L + t] = dy[row * L + t] * v * silu_grad_f64(zt);
+            dv *= silu_f64(zt);
+        }
+        accD[d] += dv * ut;
+        double dut = Dd * dv, ddt = 0.0;
+        for (int64_t n = 0; n < N; ++n) {
+            const double Bn = B[(b * N + n) * L + t], Cn = C[(b * N + n) * L + t];
+            const double hprev = H[t * N + n], abar = exp(dt * A[d * N + n]);
+            accC[n * L + t] += dv * H[(t + 1) * N + n];
+            g[n] += dv * Cn;                          /* dL/dh_t complete */
+            /* h_t = abar * h_{t-1} + dt * B * u */
+            ddt += g[n] * (A[d * N + n] * abar * hprev + Bn * ut);
+            accB[n * L + t] += g[n] * dt * ut;
+            dut += g[n] * dt * Bn;
+            accA[d * N + n] += g[n] * dt * abar * hprev;
+            g[n] *= abar;                             /* dL/dh_{t-1} through this step */
+        }
+        du[row * L + t] = dut;
+        const double x = delta[row * L + t] + (delta_bias ? delta_bias[d] : 0.0);
+        const double dx = softplus ? ddt * sigmoid_f64(x) : ddt;
+        ddelta[row * L + t] = dx;
+        accBias[d] += dx;
+    }
+    if (dh0)
+        for (int64_t n = 0; n < N; ++n) dh0[row * N + n] = g[n];
+}
+
+/*
+ * Gradients of the forward scan (reverse-mode differentiation of oracle_selective_scan_f64):
+ * given dy = dL/dy (batch, dim, L) and optionally dlast = dL/d last_state (batch, dim, N),
+ * writes dL/d of every input: du, ddelta, dz (batch, dim, L; dz only when z is given),
+ * dA (dim, N), dB, dC (batch, N, L), dD and ddelta_bias (dim; always written, as if D and
+ * delta_bias were present), dh0 (batch, dim, N; optional).  The sums over channels and
+ * batch rows are formed per thread and added in thread order, so a run is reproducible
+ * for a given thread count.  Returns 0, or -1 on a bad argument or allocation failure.
+ */
+int oracle_selective_scan_bwd_f64(const double* u, const double* delta, const double* A,
+                                  const double* B, const double* C, const double* D,
+                                  const double* z, const double* delta_bias, int softplus,
+                                  const double* h0, const double* dy, const double* dlast,
+                                  double* du, double* ddelta, double* dA, double* dB, double* dC,
+                                  double* dD, double* dz, double* ddelta_bias, double* dh0,
+                                  int64_t batch, int64_t dim, int64_t dstate, int64_t L)
+{
+    if (batch < 0 || dim < 0 || dstate < 1 || dstate > 256 || L < 0) return -1;
+    if (!u || !delta || !A || !B || !C || !dy || !du || !ddelta || !dA || !dB || !dC || !dD ||
+        !ddelta_bias || (z && !dz))
+        return -1;
+    const int64_t N = dstate;
+    int nth = 1;
+#ifdef _OPENMP
+    nth = omp_get_max_threads();
+#endif
+    if (nth > dim && dim > 0) nth = (int)dim;
+    if (nth < 1) nth = 1;
+    const size_t nl = (size_t)N * (size_t)L, dn = (size_t)dim * (size_t)N;
+    double* accB = calloc((size_t)nth * nl + 1, sizeof(double));
+    double* accC = calloc((size_t)nth * nl + 1, sizeof(double));
+    double* accA = calloc((size_t)nth * dn + 1, sizeof(double));
+    double* accD = calloc((size_t)nth * (size_t)dim + 1, sizeof(double));
+    double* accBias = calloc((size_t)nth * (size_t)dim + 1, sizeof(double));
+    int fail = !accB || !accC || !accA || !accD || !accBias;
+    for (int64_t b = 0; b < batch && !fail; ++b) {
+        memset(accB, 0, (size_t)nth * nl * sizeof(double));
+        memset(accC, 0, (size_t)nth * nl * sizeof(double));
+        #pragma omp parallel num_threads(nth)
+        {
+            int tid = 0;
+#ifdef _OPENMP
+            tid = omp_get_thread_num();
+#endif
+            double* H = malloc(((size_t)L + 1) * (size_t)N * sizeof(double));
+            double* Dt = malloc(((size_t)L + 1) * sizeof(double));
+            if (!H || !Dt) {
+                #pragma omp atomic write
+                fail = 1;
+            }
+            #pragma omp for schedule(static)
+            for (int64_t d = 0; d < dim; ++d)
+                if (H && Dt)
+                    channel_bwd(b, d, u, delta, A, B, C, D, z, delta_bias, softplus, h0, dy, dlast, du, ddelta,
+                                dz, dh0, accB + tid * nl, accC + tid * nl, accA + tid * dn, accD + tid * dim,
+                                accBias + tid * dim, dim, N, L, H, Dt);
+            free(H);
+            free(Dt);
+        }
+        for (size_t i = 0; i < nl; ++i) {
+            double sb = 0.0, sc = 0.0;
+            for (int k = 0; k < nth; ++k) {
+                sb += accB[k * nl + i];
+                sc += accC[k * nl + i];
+            }
+            dB[(size_t)b * nl + i] = sb;
+            dC[(size_t)b * nl + i] = sc;
+        }
+    }
+    for (size_t i = 0; i < dn && !fail; ++i) {
+        double s = 0.0;
+        for (int k = 0; k < nth; ++k) s += accA[k * dn + i];
+        dA[i] = s;
+    }
+    for (int64_t d = 0; d < dim && !fail; ++d) {
+        double sd = 0.0, sb = 0.0;
+        for (int k = 0; k < nth; ++k) {
+            sd += accD[k * dim + d];
+            sb += accBias[k * dim + d];
+        }
+        dD[d] = sd;
+        ddelta_bias[d] = sb;
+    }
+    free(accB);
+    free(accC);
+    free(accA);
+    free(accD);
+    free(accBias);
+    return fail ? -1 : 0;
+}
+
 /* Number of OpenMP threads the oracle will use (reported beside CPU timings). */
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP
-    extern int omp_get_max_threads(void);
     return omp_get_max_threads();
 #else
     return 1;

@@ -351,3 +351,57 @@ def test_empty_and_degenerate_shapes():
     case = _selective_case(rng, b=0, d=2, n=3, L=5)
     y, last = oracle.selective_scan(**case)
     assert y.shape == (0, 2, 5)
+
+
+# ---------------------------------------------------------------------------------------------
+# Backward: gradients of L = sum(dy * y) + sum(dlast * last_state) against central finite
+# differences of the forward scan (itself pinned above).  A dropped term, a wrong sign or a
+# transposed index in any gradient fails one element here.
+# ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("flags", [dict(), dict(softplus=False), dict(with_z=False, with_D=False, with_bias=False)],
+                         ids=["full", "softplus_off", "bare"])
+def test_backward_matches_finite_differences(flags):
+    rng = _rng(51)
+    case = _selective_case(rng, b=2, d=3, n=4, L=9, **flags)
+    if not case["softplus"]:  # keep the step positive (a decaying state) without softplus
+        case["delta"] = np.abs(case["delta"]) + 0.05
+        case["delta_bias"] = rng.uniform(0.0, 0.05, case["delta_bias"].shape)
+    b, d, L = case["u"].shape
+    n = case["A"].shape[1]
+    h0 = rng.standard_normal((b, d, n))
+    dy = rng.standard_normal((b, d, L))
+    dlast = rng.standard_normal((b, d, n))
+    grads = oracle.selective_scan_bwd(**case, h0=h0, dy=dy, dlast=dlast)
+
+    def loss(name, value):
+        c = dict(case, h0=h0)
+        c[name] = value
+        y, last = oracle.selective_scan(**c)
+        return float((dy * y).sum() + (dlast * last).sum())
+
+    eps = 1e-6
+    names = [("u", "du"), ("delta", "ddelta"), ("A", "dA"), ("B", "dB"), ("C", "dC"), ("h0", "dh0")]
+    names += [(k, "d" + k) for k in ("D", "z", "delta_bias") if case[k] is not None]
+    for name, key in names:
+        base = h0 if name == "h0" else case[name]
+        fd = np.zeros_like(base)
+        for idx in np.ndindex(base.shape):
+            hi, lo = base.copy(), base.copy()
+            hi[idx] += eps
+            lo[idx] -= eps
+            fd[idx] = (loss(name, hi) - loss(name, lo)) / (2 * eps)
+        np.testing.assert_allclose(grads[key], fd, rtol=1e-6, atol=1e-7 * (1 + np.abs(fd).max()), err_msg=name)
+    if case["z"] is None:
+        assert grads["dz"] is None
+
+
+def test_backward_is_linear_in_the_output_gradient():
+    rng = _rng(52)
+    case = _selective_case(rng)
+    b, d, L = case["u"].shape
+    dy1, dy2 = rng.standard_normal((b, d, L)), rng.standard_normal((b, d, L))
+    g1 = oracle.selective_scan_bwd(**case, dy=dy1)
+    g2 = oracle.selective_scan_bwd(**case, dy=dy2)
+    g12 = oracle.selective_scan_bwd(**case, dy=dy1 - 3.0 * dy2)
+    for k in ("du", "ddelta", "dA", "dB", "dC", "dD", "dz", "ddelta_bias", "dh0"):
+        np.testing.assert_allclose(g12[k], g1[k] - 3.0 * g2[k], rtol=1e-11, atol=1e-12, err_msg=k)
