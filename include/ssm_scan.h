@@ -155,6 +155,45 @@ ssm_status_t ssm_selective_scan_fwd_state(
     void* workspace, size_t workspace_bytes, const ssm_fwd_options_t* opts, ssm_stream_t stream);
 
 /*
+ * Backward of the forward scan: the gradients of a loss L with respect to every input,
+ * given dy = dL/dy and optionally dlast_state = dL/d last_state.  The forward is
+ * recomputed rather than stored ([Tech] 四.1: keep little in the forward pass and
+ * rebuild in the backward pass; [S4M] 3.3: forward and backward with the state kept on
+ * chip).  With g the gradient reaching h_t and v_t = sum_n C h_t + D u_t:
+ *   dz = dy v silu'(z);  dv = dy silu(z);  g += dv C_t;  dC_t += dv h_t;
+ *   dDelta_t = sum_n g (A a_t h_{t-1} + B_t u_t);  dB_t += g Delta_t u_t;
+ *   du_t = sum_n g Delta_t B_t + D dv;  dA += g Delta_t a_t h_{t-1};  g <- a_t g;
+ *   ddelta_t = dDelta_t sigmoid(delta_t + bias) (dDelta_t without softplus);
+ *   dD = sum dv u;  ddelta_bias = sum ddelta;  d initial_state = g after step 0.
+ * Inputs: as ssm_selective_scan_fwd_state (same values; initial_state may be NULL),
+ *   dy                io_dtype (batch, dim, seqlen), required.
+ *   dlast_state       optional fp32 (batch, dim, dstate); NULL means 0.
+ * Outputs (written, not accumulated; none may overlap another argument):
+ *   du, ddelta        io_dtype (batch, dim, seqlen), required.
+ *   dz                io_dtype (batch, dim, seqlen); required when z is given, else ignored.
+ *   dA                fp32 (dim, dstate), summed over batch rows and steps; required.
+ *   dB, dC            fp32 (batch, dstate, seqlen), summed over channels; required.
+ *   dD, ddelta_bias   optional fp32 (dim), summed over batch rows and steps (computed
+ *                     as if D / delta_bias were given, also when they are NULL).
+ *   dinitial_state    optional fp32 (batch, dim, dstate).
+ * Every sum is formed in a fixed order: repeated calls give identical results.
+ *   workspace         device buffer of at least ssm_selective_scan_bwd_workspace_size()
+ *                     bytes, 256-byte aligned; no initialisation needed; must not be used
+ *                     by two calls that can overlap on the GPU.
+ * Errors as ssm_selective_scan_fwd.  Any seqlen >= 0 and any 16-byte aligned pointers.
+ */
+size_t ssm_selective_scan_bwd_workspace_size(int batch, int dim, int dstate, int64_t seqlen);
+
+ssm_status_t ssm_selective_scan_bwd(
+    const void* u, const void* delta, const float* A, const void* B, const void* C,
+    const float* D, const void* z, const float* delta_bias, int softplus,
+    const float* initial_state, const void* dy, const float* dlast_state,
+    void* du, void* ddelta, float* dA, float* dB, float* dC, float* dD, void* dz,
+    float* ddelta_bias, float* dinitial_state,
+    int batch, int dim, int dstate, int64_t seqlen, ssm_dtype_t io_dtype,
+    void* workspace, size_t workspace_bytes, ssm_stream_t stream);
+
+/*
  * One-token decode ([Card] 线性扫描算法: a fixed-size state update per token;
  * [Eng] §6.2).  For every (b, d):  h[n] <- exp(Delta*A[d,n]) h[n] + Delta*B[b,n]*u[b,d],
  * y[b,d] = (sum_n C[b,n] h[n] + D[d] u[b,d]) * silu(z[b,d]), with the fp32 state

@@ -5,8 +5,11 @@ from .binding import (  # noqa: F401
     SsmError,
     load,
     new_workspace,
+    selective_scan_bwd,
     selective_scan_fwd,
     ssm_read_status,
+    ssm_selective_scan_bwd,
+    ssm_selective_scan_bwd_workspace_size,
     ssm_selective_scan_fwd,
     ssm_selective_scan_fwd_noalloc,
     ssm_selective_scan_workspace_size,

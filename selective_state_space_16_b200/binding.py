@@ -66,6 +66,10 @@ def load() -> ctypes.CDLL:
             lib.ssm_selective_scan_fwd_state.restype = ci
             lib.ssm_selective_scan_fwd_noalloc.argtypes = fwd[:16] + [vp]
             lib.ssm_selective_scan_fwd_noalloc.restype = ci
+            lib.ssm_selective_scan_bwd_workspace_size.argtypes = [ci, ci, ci, i64]
+            lib.ssm_selective_scan_bwd_workspace_size.restype = sz
+            lib.ssm_selective_scan_bwd.argtypes = [vp] * 8 + [ci] + [vp] * 12 + [ci, ci, ci, i64, ci, vp, sz, vp]
+            lib.ssm_selective_scan_bwd.restype = ci
             lib.ssm_state_update.argtypes = [vp] * 9 + [ci, vp, ci, ci, ci, ci, vp]
             lib.ssm_state_update.restype = ci
             lib.ssm_read_status.argtypes = [vp, vp]
@@ -159,6 +163,49 @@ def ssm_selective_scan_fwd_noalloc(u, delta, A, B, C, D, z, delta_bias, softplus
     if check:
         _check(code, "ssm_selective_scan_fwd_noalloc")
     return code
+
+
+def ssm_selective_scan_bwd_workspace_size(batch: int, dim: int, dstate: int, seqlen: int) -> int:
+    return int(load().ssm_selective_scan_bwd_workspace_size(batch, dim, dstate, seqlen))
+
+
+def ssm_selective_scan_bwd(u, delta, A, B, C, D, z, delta_bias, softplus, dy, du, ddelta, dA, dB, dC, dD, dz,
+                           ddelta_bias, workspace, initial_state=None, dlast_state=None, dinitial_state=None,
+                           stream=None, check=True):
+    """Marshal a backward call (shapes as the forward; dA (d, N), dB/dC (b, N, L) fp32;
+    dD/ddelta_bias (d) fp32 or None; dinitial_state (b, d, N) fp32 or None)."""
+    b, d, L = u.shape
+    n = A.shape[1]
+    code = load().ssm_selective_scan_bwd(
+        _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias), int(bool(softplus)),
+        _ptr(initial_state), _ptr(dy), _ptr(dlast_state), _ptr(du), _ptr(ddelta), _ptr(dA), _ptr(dB), _ptr(dC),
+        _ptr(dD), _ptr(dz), _ptr(ddelta_bias), _ptr(dinitial_state), b, d, n, L, _io(u), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    if check:
+        _check(code, "ssm_selective_scan_bwd")
+    return code
+
+
+def selective_scan_bwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True, dy=None,
+                       initial_state=None, dlast_state=None, workspace=None, stream=None):
+    """Convenience wrapper: allocates every gradient and, if not given, a workspace, then
+    calls ssm_selective_scan_bwd.  Returns a dict du, ddelta, dz (or None), dA, dB, dC, dD,
+    ddelta_bias, dinitial_state."""
+    b, d, L = u.shape
+    n = A.shape[1]
+    f32 = dict(dtype=torch.float32, device=u.device)
+    out = dict(du=torch.empty_like(u), ddelta=torch.empty_like(u), dz=torch.empty_like(u) if z is not None else None,
+               dA=torch.empty((d, n), **f32), dB=torch.empty((b, n, L), **f32), dC=torch.empty((b, n, L), **f32),
+               dD=torch.empty(d, **f32), ddelta_bias=torch.empty(d, **f32),
+               dinitial_state=torch.empty((b, d, n), **f32))
+    if workspace is None:
+        workspace = torch.empty(max(ssm_selective_scan_bwd_workspace_size(b, d, n, L), 256), dtype=torch.uint8,
+                                device=u.device)
+    ssm_selective_scan_bwd(u, delta, A, B, C, D, z, delta_bias, softplus, dy, out["du"], out["ddelta"], out["dA"],
+                           out["dB"], out["dC"], out["dD"], out["dz"], out["ddelta_bias"], workspace,
+                           initial_state=initial_state, dlast_state=dlast_state,
+                           dinitial_state=out["dinitial_state"], stream=stream)
+    return out
 
 
 def ssm_state_update(state, u, delta, A, B, C, D, z, delta_bias, softplus, y, stream=None, check=True):

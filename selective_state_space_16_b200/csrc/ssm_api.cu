@@ -17,6 +17,7 @@
 #include "common.cuh"
 #include "scan_fwd_chunked.cuh"
 #include "scan_fwd_seq.cuh"
+#include "scan_bwd.cuh"
 
 namespace {
 
@@ -385,6 +386,106 @@ ssm_status_t launch_forward(const FwdArgs& a, const ssm_fwd_options_t& o) {
     return SSM_ERR_INVALID_ARG;
 }
 
+// ------------------------------------------------------------------ backward
+// Backward workspace layout:
+//   [header 256 B][B/C fp32 rows: batch * L * 128 B][checkpoints: batch * nseg * dim * 64 B]
+//   [dB/dC per CTA: batch * ncta * L * 128 B][dA per batch row: batch * dim * 64 B]
+//   [dD per batch row: batch * dim * 4 B][ddelta_bias per batch row: batch * dim * 4 B]
+struct BwdLayout {
+    size_t bc_off, ckpt_off, dbc_off, dA_off, dD_off, dbias_off, total;
+    int nseg, ncta;
+};
+
+BwdLayout bwd_layout(int batch, int dim, int64_t L) {
+    BwdLayout w{};
+    w.nseg = static_cast<int>((L + ssm::kBwdSeg - 1) / ssm::kBwdSeg);
+    w.ncta = (dim + ssm::kBwdChannels - 1) / ssm::kBwdChannels;
+    const size_t B = static_cast<size_t>(batch), D = static_cast<size_t>(dim), Ls = static_cast<size_t>(L);
+    w.bc_off = sizeof(WorkspaceHeader);
+    w.ckpt_off = w.bc_off + round_up(B * Ls * 128u, 256);
+    w.dbc_off = w.ckpt_off + round_up(B * static_cast<size_t>(w.nseg) * D * 64u, 256);
+    w.dA_off = w.dbc_off + round_up(B * static_cast<size_t>(w.ncta) * Ls * 128u, 256);
+    w.dD_off = w.dA_off + round_up(B * D * 64u, 256);
+    w.dbias_off = w.dD_off + round_up(B * D * 4u, 256);
+    w.total = w.dbias_off + round_up(B * D * 4u, 256);
+    return w;
+}
+
+struct BwdArgs {
+    const void *u, *delta, *B, *C, *z, *dy;
+    const float *A, *D, *bias, *h0, *dlast;
+    int softplus;
+    void *du, *ddelta, *dz;
+    float *dA, *dB, *dC, *dD, *dbias, *dh0;
+    int batch, dim;
+    int64_t L;
+    uint8_t* ws;
+    cudaStream_t stream;
+};
+
+template <typename IO>
+ssm_status_t launch_backward(const BwdArgs& a) {
+    const BwdLayout wl = bwd_layout(a.batch, a.dim, a.L);
+    float* bc = reinterpret_cast<float*>(a.ws + wl.bc_off);
+    {
+        const dim3 grid(static_cast<unsigned>((a.L + 63) / 64), static_cast<unsigned>(a.batch));
+        ssm::pack_bc_kernel<IO><<<grid, 256, 0, a.stream>>>(static_cast<const IO*>(a.B), static_cast<const IO*>(a.C),
+                                                           bc, a.L);
+        if (cudaGetLastError() != cudaSuccess) return SSM_ERR_LAUNCH;
+    }
+    ssm::BwdParams p{};
+    p.u = a.u;
+    p.delta = a.delta;
+    p.z = a.z;
+    p.dy = a.dy;
+    p.bc = bc;
+    p.A = a.A;
+    p.D = a.D;
+    p.bias = a.bias;
+    p.h0 = a.h0;
+    p.dlast = a.dlast;
+    p.du = a.du;
+    p.ddelta = a.ddelta;
+    p.dz = a.dz;
+    p.dh0 = a.dh0;
+    p.ckpt = reinterpret_cast<float*>(a.ws + wl.ckpt_off);
+    p.dbc_part = reinterpret_cast<float*>(a.ws + wl.dbc_off);
+    p.dA_part = reinterpret_cast<float*>(a.ws + wl.dA_off);
+    p.dD_part = reinterpret_cast<float*>(a.ws + wl.dD_off);
+    p.dbias_part = reinterpret_cast<float*>(a.ws + wl.dbias_off);
+    p.batch = a.batch;
+    p.dim = a.dim;
+    p.L = a.L;
+    p.nseg = wl.nseg;
+    p.ncta = wl.ncta;
+    p.softplus = a.softplus;
+    constexpr int smem = ssm::kBwdWarps * ssm::kBwdSeg * 32 * (16 + 4);
+    auto kern = ssm::scan_bwd_kernel<IO>;
+    if (!ensure_smem_attr(reinterpret_cast<const void*>(kern), smem)) return SSM_ERR_LAUNCH;
+    kern<<<dim3(static_cast<unsigned>(wl.ncta), static_cast<unsigned>(a.batch)), ssm::kBwdWarps * 32, smem,
+           a.stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return SSM_ERR_LAUNCH;
+    ssm::BwdFinalParams f{};
+    f.dbc_part = p.dbc_part;
+    f.dA_part = p.dA_part;
+    f.dD_part = p.dD_part;
+    f.dbias_part = p.dbias_part;
+    f.dB = a.dB;
+    f.dC = a.dC;
+    f.dA = a.dA;
+    f.dD = a.dD;
+    f.dbias = a.dbias;
+    f.batch = a.batch;
+    f.dim = a.dim;
+    f.ncta = wl.ncta;
+    f.L = a.L;
+    ssm::scan_bwd_reduce_bc_kernel<<<dim3(static_cast<unsigned>((a.L + 31) / 32), static_cast<unsigned>(a.batch)), 256,
+                                     0, a.stream>>>(f);
+    const long long n = static_cast<long long>(a.dim) * 16;
+    ssm::scan_bwd_reduce_params_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, a.stream>>>(f);
+    return launch_status();
+}
+
 // Fixed scratch of ssm_selective_scan_fwd_noalloc (header + transposed B/C rows).  In
 // host code this name only stands for the array: its device address comes from
 // cudaGetSymbolAddress, looked up once per device.
@@ -563,6 +664,54 @@ ssm_status_t ssm_selective_scan_fwd_noalloc(const void* u, const void* delta, co
     FwdArgs a{u, delta, B, C, z, A, D, delta_bias, softplus, nullptr, y, last_state, batch, dim, seqlen, io_dtype,
               scratch, s, sm_count};
     return io_dtype == SSM_BF16 ? launch_forward<__nv_bfloat16>(a, o) : launch_forward<float>(a, o);
+}
+
+size_t ssm_selective_scan_bwd_workspace_size(int batch, int dim, int dstate, int64_t seqlen) {
+    if (batch < 0 || dim < 0 || dstate != 16 || seqlen < 0) return 0;
+    return round_up(bwd_layout(batch, dim, seqlen).total, 256);
+}
+
+ssm_status_t ssm_selective_scan_bwd(const void* u, const void* delta, const float* A, const void* B, const void* C,
+                                    const float* D, const void* z, const float* delta_bias, int softplus,
+                                    const float* initial_state, const void* dy, const float* dlast_state, void* du,
+                                    void* ddelta, float* dA, float* dB, float* dC, float* dD, void* dz,
+                                    float* ddelta_bias, float* dinitial_state, int batch, int dim, int dstate,
+                                    int64_t seqlen, ssm_dtype_t io_dtype, void* workspace, size_t workspace_bytes,
+                                    ssm_stream_t stream) {
+    if (batch < 0 || dim < 0 || seqlen < 0) return SSM_ERR_INVALID_ARG;
+    const bool seq_elems = batch > 0 && dim > 0 && seqlen > 0;
+    if (seq_elems && (!u || !delta || !B || !C || !dy || !du || !ddelta || !dB || !dC || (z && !dz)))
+        return SSM_ERR_INVALID_ARG;
+    if (dim > 0 && (!A || !dA)) return SSM_ERR_INVALID_ARG;
+    if (io_dtype != SSM_F32 && io_dtype != SSM_BF16) return SSM_ERR_INVALID_ARG;
+    if (dstate != 16) return SSM_ERR_UNSUPPORTED;
+    const void* ptrs[] = {u, delta, A, B, C, D, z, delta_bias, initial_state, dy, dlast_state, du, ddelta, dA, dB, dC,
+                          dD, dz, ddelta_bias, dinitial_state};
+    for (const void* q : ptrs)
+        if (q && !aligned16(q)) return SSM_ERR_INVALID_ARG;
+    if (batch == 0 || dim == 0) return SSM_OK;
+    if (batch > 65535) return SSM_ERR_UNSUPPORTED;
+    if (seqlen >= (1LL << 40)) return SSM_ERR_UNSUPPORTED;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+        workspace_bytes < ssm_selective_scan_bwd_workspace_size(batch, dim, dstate, seqlen))
+        return SSM_ERR_WORKSPACE;
+    ssm_status_t st = check_device(nullptr);
+    if (st != SSM_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (seqlen == 0) {  // no steps: only the state passes through
+        const size_t state_bytes = static_cast<size_t>(batch) * dim * 16 * sizeof(float);
+        cudaError_t e = cudaMemsetAsync(dA, 0, static_cast<size_t>(dim) * 16 * sizeof(float), s);
+        if (e == cudaSuccess && dD) e = cudaMemsetAsync(dD, 0, static_cast<size_t>(dim) * sizeof(float), s);
+        if (e == cudaSuccess && ddelta_bias)
+            e = cudaMemsetAsync(ddelta_bias, 0, static_cast<size_t>(dim) * sizeof(float), s);
+        if (e == cudaSuccess && dinitial_state)
+            e = dlast_state ? cudaMemcpyAsync(dinitial_state, dlast_state, state_bytes, cudaMemcpyDeviceToDevice, s)
+                            : cudaMemsetAsync(dinitial_state, 0, state_bytes, s);
+        return e == cudaSuccess ? SSM_OK : SSM_ERR_LAUNCH;
+    }
+    BwdArgs a{u, delta, B, C, z, dy, A, D, delta_bias, initial_state, dlast_state, softplus, du, ddelta, dz, dA, dB,
+              dC, dD, ddelta_bias, dinitial_state, batch, dim, seqlen, static_cast<uint8_t*>(workspace), s};
+    return io_dtype == SSM_BF16 ? launch_backward<__nv_bfloat16>(a) : launch_backward<float>(a);
 }
 
 ssm_status_t ssm_read_status(void* workspace, ssm_stream_t stream) {

@@ -136,3 +136,24 @@ def test_product_package_does_not_import_oracle():
         if f.endswith((".py", ".cu", ".cuh", ".h")):
             txt = open(f).read()
             assert "import oracle" not in txt and "from oracle" not in txt and "ssm_oracle" not in txt, f
+
+
+def test_backward_argument_validation(lib):
+    def call(**kw):
+        a = dict(u=P(4096), delta=P(4096), A=P(4096), B=P(4096), C=P(4096), D=None, z=None, bias=None, softplus=1,
+                 h0=None, dy=P(4096), dlast=None, du=P(4096), ddelta=P(4096), dA=P(4096), dB=P(4096), dC=P(4096),
+                 dD=None, dz=None, dbias=None, dh0=None, batch=2, dim=3, dstate=16, L=8, io=binding.SSM_BF16,
+                 ws=P(4096), wsb=1 << 30, stream=None)
+        a.update(kw)
+        return lib.ssm_selective_scan_bwd(*a.values())
+    assert call(dy=None) == binding.SSM_ERR_INVALID_ARG
+    assert call(dB=None) == binding.SSM_ERR_INVALID_ARG
+    assert call(z=P(4096)) == binding.SSM_ERR_INVALID_ARG            # z given, dz missing
+    assert call(dA=P(4104)) == binding.SSM_ERR_INVALID_ARG           # misaligned
+    assert call(dstate=32) == binding.SSM_ERR_UNSUPPORTED
+    assert call(batch=0) == binding.SSM_OK
+    assert call(ws=None) == binding.SSM_ERR_WORKSPACE
+    assert call(wsb=64) == binding.SSM_ERR_WORKSPACE
+    f = binding.ssm_selective_scan_bwd_workspace_size
+    assert f(4, 5120, 16, 2048) % 256 == 0 and f(4, 5120, 16, 2048) > 4 * 2048 * 128
+    assert f(1, 1, 8, 1) == 0
