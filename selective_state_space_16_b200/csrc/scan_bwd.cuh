@@ -22,17 +22,18 @@
 //   g <- a_t g  (the gradient reaching h_{t-1}); after step 0 it is d initial_state
 //   ddelta_t = dDelta_t sigmoid(delta_t + bias)   (softplus' ; 1 without softplus)
 //
-// Work split.  A CTA of 8 warps takes 64 consecutive channels of one batch row; a warp
+// Work split.  A CTA of 4 warps takes 32 consecutive channels of one batch row; a warp
 // takes 8 channels, 4 lanes per channel, each lane 4 of the 16 chains (as the forward
-// kernels).  Each warp first runs the forward over the whole sequence and stores the
-// state at the start of every 16-step segment (checkpoints, in the workspace).  Then it
-// walks the segments from the last to the first: it re-runs the segment from its
-// checkpoint, keeping h_{t-1} of the 16 steps in shared memory, forms v_t, dz_t and
-// dv_t, and runs the gradient recurrence backwards through the segment.
+// kernels), with the chain arithmetic in f32x2 pairs.  Each warp first runs the forward
+// over the whole sequence and stores the state at the start of every 8-step segment
+// (checkpoints, in the workspace).  Then it walks the segments from the last to the
+// first: it re-runs the segment from its checkpoint, keeping h_{t-1} and exp(Delta A) of
+// the 8 steps in shared memory, forms v_t, dz_t and dv_t, and runs the gradient
+// recurrence backwards through the segment.
 //   - Sums over the 16 chains (du, dDelta, v) are reduce-scattered over the 4 lanes of a
-//     channel, so that lane nl finishes steps 4nl .. 4nl+3 of the segment.
+//     channel, so that lane nl finishes steps 2nl, 2nl+1 of the segment.
 //   - Sums over channels (dB, dC) are reduce-scattered over the 8 channels of a warp,
-//     added over the CTA's 8 warps in a fixed order, and written per CTA to the
+//     added over the CTA's warps in a fixed order, and written per CTA to the
 //     workspace; a second kernel adds the CTAs of a batch row (fixed order: the result
 //     does not depend on scheduling).
 //   - dA, dD and ddelta_bias are summed over time in registers, written per batch row and
@@ -41,12 +42,16 @@
 
 #include "common.cuh"
 #include "scan_math.cuh"
+#include "scan_fwd_seq.cuh"  // f2
 
 namespace ssm {
 
-constexpr int kBwdSeg = 16;      // steps per segment (checkpoint interval)
-constexpr int kBwdWarps = 8;     // warps per CTA
+constexpr int kBwdSeg = 8;       // steps per segment (checkpoint interval)
+constexpr int kBwdWarps = 4;     // warps per CTA (5 CTAs per SM: every CTA resident at once)
 constexpr int kBwdChannels = kBwdWarps * 8;
+constexpr int kBwdRing = 4;      // segments of B/C rows in flight (cp.async ring)
+// dynamic shared memory of scan_bwd_kernel: h and decay stages, dB/dC stage, B/C ring
+constexpr int kBwdSmem = kBwdWarps * kBwdSeg * 32 * (16 + 16 + 4) + kBwdRing * kBwdSeg * 32 * 4;
 
 struct BwdParams {
     const void *u, *delta, *z, *dy;  // (batch, dim, L) IO
@@ -73,13 +78,16 @@ __device__ __forceinline__ float load_io(const void* base, long long i) {
 }
 
 template <typename IO>
-__global__ void __launch_bounds__(kBwdWarps * 32, 2) scan_bwd_kernel(const BwdParams p) {
-    constexpr int T = kBwdSeg, NC = 4, G = 4, PER = T / G;
+__global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdParams p) {
+    constexpr int T = kBwdSeg, G = 4, PER = T / G, R = kBwdRing;
     extern __shared__ float4 bwd_smem[];
-    // h_{t-1} of the segment's steps: [warp][step][lane] (16 bytes per lane and step)
+    // h_{t-1} and exp(Delta_t A) of the segment's steps: [warp][step][lane] (16 bytes each)
     float4* hstage = bwd_smem;
+    float4* astage = bwd_smem + kBwdWarps * T * 32;
     // per-warp dB/dC partials of the segment's steps: [warp][step][32 columns]
-    float* cstage = reinterpret_cast<float*>(bwd_smem + kBwdWarps * T * 32);
+    float* cstage = reinterpret_cast<float*>(bwd_smem + 2 * kBwdWarps * T * 32);
+    // ring of R segments of packed B/C rows (shared by the CTA: one batch row): [slot][step][32]
+    float* bcring = cstage + kBwdWarps * T * 32;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cg = lane >> 2, nl = lane & 3, gbase = lane & ~3;
@@ -87,109 +95,166 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 2) scan_bwd_kernel(const BwdPa
     const int d = blockIdx.x * kBwdChannels + warp * 8 + cg;
     const bool valid = d < p.dim;
     const int dd = valid ? d : 0;
-    const long long L = p.L;
-    const long long row = (static_cast<long long>(b) * p.dim + dd) * L;
-    const float* bcb = p.bc + static_cast<long long>(b) * L * 32 + nl * NC;
-    const bool softplus = p.softplus != 0;
-
-    float An[NC], A2[NC];
+    const int L = static_cast<int>(p.L);  // the host launches this kernel for L < 2^31 - 16 only
+    const long long row = (static_cast<long long>(b) * p.dim + dd) * p.L;
+    const IO* x_row = static_cast<const IO*>(p.delta) + row;
+    const IO* u_row = static_cast<const IO*>(p.u) + row;
+    const IO* dy_row = static_cast<const IO*>(p.dy) + row;
+    const IO* z_row = p.z ? static_cast<const IO*>(p.z) + row : nullptr;
+    IO* du_row = static_cast<IO*>(p.du) + row;
+    IO* ddelta_row = static_cast<IO*>(p.ddelta) + row;
+    IO* dz_row = p.dz ? static_cast<IO*>(p.dz) + row : nullptr;
+    const float* bcrow = p.bc + static_cast<long long>(b) * p.L * 32;
+    float* ckrow = p.ckpt + (static_cast<long long>(b) * p.nseg * p.dim + dd) * 16 + nl * 4;  // segment stride dim*16
+    const long long ckstride = static_cast<long long>(p.dim) * 16;
+    int srcl[4];  // lanes of this channel, by step owner
 #pragma unroll
-    for (int j = 0; j < NC; ++j) {
-        An[j] = valid ? p.A[dd * 16 + nl * NC + j] : 0.f;
-        A2[j] = An[j] * kLog2e;
+    for (int k = 0; k < 4; ++k) srcl[k] = gbase | k;
+    const bool softplus = p.softplus != 0;
+    const bool has_z = p.z != nullptr;
+
+    float2 An[2], A2[2];  // A of the lane's 4 chains as pairs; A2 = A log2(e)
+    {
+        const float4 a = valid ? *reinterpret_cast<const float4*>(p.A + dd * 16 + nl * 4) : make_float4(0, 0, 0, 0);
+        An[0] = f2(a.x, a.y);
+        An[1] = f2(a.z, a.w);
+        A2[0] = f2(a.x * kLog2e, a.y * kLog2e);
+        A2[1] = f2(a.z * kLog2e, a.w * kLog2e);
     }
     const float Dd = (valid && p.D) ? p.D[dd] : 0.f;
     const float bias = (valid && p.bias) ? p.bias[dd] : 0.f;
-    const long long srow = (static_cast<long long>(b) * p.dim + dd) * 16 + nl * NC;  // state row of this lane
+    const long long srow = (static_cast<long long>(b) * p.dim + dd) * 16 + nl * 4;  // state row of this lane
+    auto ld4 = [](const float* q) { const float4 v = *reinterpret_cast<const float4*>(q); return v; };
+    auto lo = [](float4 v) { return f2(v.x, v.y); };
+    auto hi = [](float4 v) { return f2(v.z, v.w); };
+    auto decay = [&](float dti, int j) {
+        const float2 arg = __fmul2_rn(f2(dti, dti), A2[j]);
+        return f2(ex2_mufu(arg.x), ex2_mufu(arg.y));
+    };
+    auto ckpt_at = [&](int s) { return ckrow + s * ckstride; };
 
-    // Step sizes, inputs of the lane's own steps 4nl .. 4nl+3 of segment s (0 past L).
-    auto own_inputs = [&](long long t0, float (&dt)[PER], float (&uo)[PER], float (&xo)[PER]) {
+    // B/C rows of segment `seg` into ring slot `slot` (threads 0..63, 16 bytes each; zero
+    // past L); every thread commits a group, so that group counts agree across threads.
+    auto issue_bc = [&](int seg, int slot) {
+        if (threadIdx.x < T * 8 && seg >= 0 && seg < p.nseg) {
+            const int i = threadIdx.x >> 3, part = threadIdx.x & 7;
+            const int t = seg * T + i;
+            const bool in = t < L;
+            cp_async_16(bcring + (slot * T + i) * 32 + part * 4, in ? bcrow + static_cast<long long>(t) * 32 + part * 4 : bcrow,
+                        in ? 16u : 0u);
+        }
+        cp_async_commit();
+    };
+
+    // Raw inputs of the lane's own steps 2nl, 2nl+1 of segment seg: delta, u, dy, z.
+    struct Raw {
+        float x[PER], u[PER], dy[PER], z[PER];
+    };
+    auto load_raw = [&](int seg, bool with_grad, Raw& r) {
 #pragma unroll
-        for (int r = 0; r < PER; ++r) {
-            const long long t = t0 + nl * PER + r;
-            const bool in = valid && t < L;
-            const float raw = in ? load_io<IO>(p.delta, row + t) : 0.f;
-            xo[r] = raw + bias;
-            dt[r] = in ? step_size(raw, bias, softplus) : 0.f;
-            uo[r] = in ? load_io<IO>(p.u, row + t) : 0.f;
+        for (int k = 0; k < PER; ++k) {
+            const int t = seg * T + nl * PER + k;
+            const bool in = valid && seg >= 0 && t < L;
+            r.x[k] = in ? IoTraits<IO>::to_f32(x_row[t]) : 0.f;
+            r.u[k] = in ? IoTraits<IO>::to_f32(u_row[t]) : 0.f;
+            r.dy[k] = (in && with_grad) ? IoTraits<IO>::to_f32(dy_row[t]) : 0.f;
+            r.z[k] = (in && with_grad && has_z) ? IoTraits<IO>::to_f32(z_row[t]) : 0.f;
+        }
+    };
+    auto step_sizes = [&](int seg, const Raw& r, float (&dt)[PER]) {
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            const int t = seg * T + nl * PER + k;
+            dt[k] = (valid && t < L) ? step_size(r.x[k], bias, softplus) : 0.f;
         }
     };
 
     // ------------------------------------------------------------ forward sweep, checkpoints
-    float h[NC];
+    float2 h[2];
     {
-        const float4 h0 = (valid && p.h0) ? *reinterpret_cast<const float4*>(p.h0 + srow) : make_float4(0, 0, 0, 0);
-        h[0] = h0.x; h[1] = h0.y; h[2] = h0.z; h[3] = h0.w;
+        const float4 h0 = (valid && p.h0) ? ld4(p.h0 + srow) : make_float4(0, 0, 0, 0);
+        h[0] = lo(h0);
+        h[1] = hi(h0);
     }
+    for (int r = 0; r < R - 1; ++r) issue_bc(r, r);
+    Raw nxt;
+    load_raw(0, false, nxt);
     for (int s = 0; s < p.nseg; ++s) {
-        const long long t0 = static_cast<long long>(s) * T;
-        if (valid)
-            *reinterpret_cast<float4*>(p.ckpt + ((static_cast<long long>(b) * p.nseg + s) * p.dim + dd) * 16 +
-                                       nl * NC) = make_float4(h[0], h[1], h[2], h[3]);
-        float dt[PER], uo[PER], xo[PER];
-        own_inputs(t0, dt, uo, xo);
+        const Raw cur = nxt;
+        load_raw(s + 1, false, nxt);  // next segment's inputs, in flight during this one
+        __syncthreads();              // every warp is done with the slot refilled below
+        issue_bc(s + R - 1, (s + R - 1) % R);
+        cp_async_wait<R - 1>();
+        __syncthreads();              // segment s's B/C rows are visible to every warp
+        if (valid) *reinterpret_cast<float4*>(ckpt_at(s)) = make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
+        float dt[PER];
+        step_sizes(s, cur, dt);
+        const float* bcs = bcring + (s % R) * T * 32 + nl * 4;
 #pragma unroll
         for (int i = 0; i < T; ++i) {
-            const float dti = __shfl_sync(0xffffffffu, dt[i % PER], gbase | (i / PER));
-            const float ui = __shfl_sync(0xffffffffu, uo[i % PER], gbase | (i / PER));
-            const long long t = t0 + i;
-            const float4 Bq = t < L ? *reinterpret_cast<const float4*>(bcb + t * 32) : make_float4(0, 0, 0, 0);
-            const float Bv[NC] = {Bq.x, Bq.y, Bq.z, Bq.w};
-            const float w = dti * ui;
-#pragma unroll
-            for (int j = 0; j < NC; ++j) h[j] = fmaf(ex2_mufu(dti * A2[j]), h[j], w * Bv[j]);
+            const float dti = __shfl_sync(0xffffffffu, dt[i % PER], srcl[i / PER]);
+            const float ui = __shfl_sync(0xffffffffu, cur.u[i % PER], srcl[i / PER]);
+            const float4 Bq = ld4(bcs + i * 32);
+            const float2 ww = f2(dti * ui, dti * ui);
+            h[0] = __ffma2_rn(decay(dti, 0), h[0], __fmul2_rn(ww, lo(Bq)));
+            h[1] = __ffma2_rn(decay(dti, 1), h[1], __fmul2_rn(ww, hi(Bq)));
         }
     }
+    cp_async_wait<0>();
+    __syncthreads();
 
     // ------------------------------------------------------------ reverse sweep
-    float g[NC];
+    float2 g[2], dA_acc[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
     {
-        const float4 gl = (valid && p.dlast) ? *reinterpret_cast<const float4*>(p.dlast + srow) : make_float4(0, 0, 0, 0);
-        g[0] = gl.x; g[1] = gl.y; g[2] = gl.z; g[3] = gl.w;
+        const float4 gl = (valid && p.dlast) ? ld4(p.dlast + srow) : make_float4(0, 0, 0, 0);
+        g[0] = lo(gl);
+        g[1] = hi(gl);
     }
-    float dA_acc[NC] = {0.f, 0.f, 0.f, 0.f};
     float dD_acc = 0.f, dbias_acc = 0.f;
     float4* hst = hstage + warp * T * 32;
+    float4* ast = astage + warp * T * 32;
     float* cst = cstage + warp * T * 32;
-    const int col = (cg >> 2) * 16 + nl * NC + (cg & 3);  // dB/dC column this lane ends with
+    const int col = (cg >> 2) * 16 + nl * 4 + (cg & 3);  // dB/dC column this lane ends with
 
-    for (int s = p.nseg - 1; s >= 0; --s) {
-        const long long t0 = static_cast<long long>(s) * T;
-        float dt[PER], uo[PER], xo[PER];
-        own_inputs(t0, dt, uo, xo);
+    // k-th segment of the walk is s = nseg - 1 - k, in ring slot k % R.
+    for (int r = 0; r < R - 1; ++r) issue_bc(p.nseg - 1 - r, r);
+    load_raw(p.nseg - 1, true, nxt);
+    float4 ck_nxt = valid ? ld4(ckpt_at(p.nseg - 1)) : make_float4(0, 0, 0, 0);
+    for (int k = 0; k < p.nseg; ++k) {
+        const int s = p.nseg - 1 - k;
+        const int t0 = s * T;
+        const Raw cur = nxt;
+        const float4 ck = ck_nxt;
+        load_raw(s - 1, true, nxt);
+        if (valid && s > 0) ck_nxt = ld4(ckpt_at(s - 1));
+        __syncthreads();
+        issue_bc(s - (R - 1), (k + R - 1) % R);
+        cp_async_wait<R - 1>();
+        __syncthreads();
+        const float* bcs = bcring + (k % R) * T * 32 + nl * 4;
+        float dt[PER];
+        step_sizes(s, cur, dt);
 
-        // Re-run the segment from its checkpoint: h_{t-1} of each step to shared memory,
-        // the lane's part of sum_n C_t h_t per step.
-        float hs[NC];
-        {
-            const float4 c = valid ? *reinterpret_cast<const float4*>(
-                                         p.ckpt + ((static_cast<long long>(b) * p.nseg + s) * p.dim + dd) * 16 + nl * NC)
-                                   : make_float4(0, 0, 0, 0);
-            hs[0] = c.x; hs[1] = c.y; hs[2] = c.z; hs[3] = c.w;
-        }
+        // Re-run the segment from its checkpoint: h_{t-1} and exp(Delta A) of each step to
+        // shared memory, the lane's part of sum_n C_t h_t per step.
+        float2 hs[2] = {lo(ck), hi(ck)};
         float vp[T];
 #pragma unroll
         for (int i = 0; i < T; ++i) {
-            const float dti = __shfl_sync(0xffffffffu, dt[i % PER], gbase | (i / PER));
-            const float ui = __shfl_sync(0xffffffffu, uo[i % PER], gbase | (i / PER));
-            const long long t = t0 + i;
-            float4 Bq = make_float4(0, 0, 0, 0), Cq = make_float4(0, 0, 0, 0);
-            if (t < L) {
-                Bq = *reinterpret_cast<const float4*>(bcb + t * 32);
-                Cq = *reinterpret_cast<const float4*>(bcb + t * 32 + 16);
-            }
-            hst[i * 32 + lane] = make_float4(hs[0], hs[1], hs[2], hs[3]);
-            const float Bv[NC] = {Bq.x, Bq.y, Bq.z, Bq.w}, Cv[NC] = {Cq.x, Cq.y, Cq.z, Cq.w};
-            const float w = dti * ui;
-            float acc = 0.f;
-#pragma unroll
-            for (int j = 0; j < NC; ++j) {
-                hs[j] = fmaf(ex2_mufu(dti * A2[j]), hs[j], w * Bv[j]);
-                acc = fmaf(Cv[j], hs[j], acc);
-            }
-            vp[i] = acc;
+            const float dti = __shfl_sync(0xffffffffu, dt[i % PER], srcl[i / PER]);
+            const float ui = __shfl_sync(0xffffffffu, cur.u[i % PER], srcl[i / PER]);
+            const float4 Bq = ld4(bcs + i * 32), Cq = ld4(bcs + i * 32 + 16);
+            const float2 a0 = decay(dti, 0), a1 = decay(dti, 1);
+            hst[i * 32 + lane] = make_float4(hs[0].x, hs[0].y, hs[1].x, hs[1].y);
+            ast[i * 32 + lane] = make_float4(a0.x, a0.y, a1.x, a1.y);
+            const float2 ww = f2(dti * ui, dti * ui);
+            hs[0] = __ffma2_rn(a0, hs[0], __fmul2_rn(ww, lo(Bq)));
+            hs[1] = __ffma2_rn(a1, hs[1], __fmul2_rn(ww, hi(Bq)));
+            const float2 acc = __ffma2_rn(hi(Cq), hs[1], __fmul2_rn(lo(Cq), hs[0]));
+            vp[i] = acc.x + acc.y;
         }
-        // Reduce-scatter over the 4 lanes: lane nl gets sum_n C h of its steps 4nl.. 4nl+3.
+        // Reduce-scatter over the 4 lanes (upper lane bit first): lane nl ends with the
+        // sums of its own steps 2nl, 2nl+1.
 #pragma unroll
         for (int m = 2, half = T / 2; m >= 1; m >>= 1, half >>= 1) {
             const bool upper = (nl & m) != 0;
@@ -200,73 +265,62 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 2) scan_bwd_kernel(const BwdPa
                 vp[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
             }
         }
-        // vp[r] now belongs to step 4*nl' + r, nl' = the lane's position after the
-        // scatter: lower half -> first half of the steps.  With the upper bit taken first
-        // (m = 2: steps 8..15 to lanes 2,3), then m = 1, lane nl holds steps nl*4 + r.
         float dv[PER], dzv[PER];
 #pragma unroll
         for (int r = 0; r < PER; ++r) {
-            const long long t = t0 + nl * PER + r;
-            const bool in = valid && t < L;
-            const float v = fmaf(Dd, uo[r], vp[r]);
-            const float dyv = in ? load_io<IO>(p.dy, row + t) : 0.f;
-            if (p.z) {
-                const float zt = in ? load_io<IO>(p.z, row + t) : 0.f;
+            const float v = fmaf(Dd, cur.u[r], vp[r]);
+            if (has_z) {
+                const float zt = cur.z[r];
                 const float sg = sigmoid_f32(zt);
-                dv[r] = dyv * zt * sg;
-                dzv[r] = dyv * v * sg * fmaf(zt, 1.f - sg, 1.f);
+                dv[r] = cur.dy[r] * zt * sg;
+                dzv[r] = cur.dy[r] * v * sg * fmaf(zt, 1.f - sg, 1.f);
             } else {
-                dv[r] = dyv;
+                dv[r] = cur.dy[r];
                 dzv[r] = 0.f;
             }
-            dD_acc = fmaf(dv[r], uo[r], dD_acc);
+            dD_acc = fmaf(dv[r], cur.u[r], dD_acc);
         }
         __syncwarp();
 
         // Gradient recurrence backwards through the segment.
-        float hn[NC] = {hs[0], hs[1], hs[2], hs[3]};  // h_t of the step being processed
+        float2 hn[2] = {hs[0], hs[1]};  // h_t of the step being processed
         float ddt[T], dup[T];
 #pragma unroll
         for (int i = T - 1; i >= 0; --i) {
-            const float dti = __shfl_sync(0xffffffffu, dt[i % PER], gbase | (i / PER));
-            const float ui = __shfl_sync(0xffffffffu, uo[i % PER], gbase | (i / PER));
-            const float dvi = __shfl_sync(0xffffffffu, dv[i % PER], gbase | (i / PER));
-            const long long t = t0 + i;
-            float4 Bq = make_float4(0, 0, 0, 0), Cq = make_float4(0, 0, 0, 0);
-            if (t < L) {
-                Bq = *reinterpret_cast<const float4*>(bcb + t * 32);
-                Cq = *reinterpret_cast<const float4*>(bcb + t * 32 + 16);
-            }
-            const float Bv[NC] = {Bq.x, Bq.y, Bq.z, Bq.w}, Cv[NC] = {Cq.x, Cq.y, Cq.z, Cq.w};
-            const float4 hq = hst[i * 32 + lane];
-            const float hp[NC] = {hq.x, hq.y, hq.z, hq.w};
-            const float w = dti * ui;
-            float vals[2 * NC];  // dB (this channel's part) then dC
-            float sdt = 0.f, sdu = 0.f;
+            const float dti = __shfl_sync(0xffffffffu, dt[i % PER], srcl[i / PER]);
+            const float ui = __shfl_sync(0xffffffffu, cur.u[i % PER], srcl[i / PER]);
+            const float dvi = __shfl_sync(0xffffffffu, dv[i % PER], srcl[i / PER]);
+            const float4 Bq = ld4(bcs + i * 32), Cq = ld4(bcs + i * 32 + 16);
+            const float4 hq = hst[i * 32 + lane], aq = ast[i * 32 + lane];
+            const float2 Bv[2] = {lo(Bq), hi(Bq)}, Cv[2] = {lo(Cq), hi(Cq)};
+            const float2 hp[2] = {lo(hq), hi(hq)}, av[2] = {lo(aq), hi(aq)};
+            const float2 dv2 = f2(dvi, dvi), dt2 = f2(dti, dti), u2 = f2(ui, ui);
+            const float2 w2 = f2(dti * ui, dti * ui);
+            float2 sdt = f2(0.f, 0.f), sdu = f2(0.f, 0.f), dB[2], dC[2];
 #pragma unroll
-            for (int j = 0; j < NC; ++j) {
-                const float a = ex2_mufu(dti * A2[j]);
-                g[j] = fmaf(dvi, Cv[j], g[j]);
-                vals[NC + j] = dvi * hn[j];
-                const float ah = a * hp[j];
-                dA_acc[j] = fmaf(g[j] * dti, ah, dA_acc[j]);
-                sdt = fmaf(g[j], fmaf(An[j], ah, Bv[j] * ui), sdt);
-                sdu = fmaf(g[j], Bv[j], sdu);
-                vals[j] = g[j] * w;
-                g[j] *= a;
+            for (int j = 0; j < 2; ++j) {
+                g[j] = __ffma2_rn(dv2, Cv[j], g[j]);
+                dC[j] = __fmul2_rn(dv2, hn[j]);
+                const float2 ah = __fmul2_rn(av[j], hp[j]);
+                dA_acc[j] = __ffma2_rn(__fmul2_rn(g[j], dt2), ah, dA_acc[j]);
+                sdt = __ffma2_rn(g[j], __ffma2_rn(An[j], ah, __fmul2_rn(Bv[j], u2)), sdt);
+                sdu = __ffma2_rn(g[j], Bv[j], sdu);
+                dB[j] = __fmul2_rn(g[j], w2);
+                g[j] = __fmul2_rn(g[j], av[j]);
                 hn[j] = hp[j];
             }
-            ddt[i] = sdt;
-            dup[i] = sdu * dti;
+            ddt[i] = sdt.x + sdt.y;
+            dup[i] = (sdu.x + sdu.y) * dti;
             // dB/dC: reduce-scatter the 8 values over the warp's 8 channels (lane bits 4, 3, 2).
+            float vals[8] = {dB[0].x, dB[0].y, dB[1].x, dB[1].y, dC[0].x, dC[0].y, dC[1].x, dC[1].y};
 #pragma unroll
-            for (int m = 16, half = NC; m >= 4; m >>= 1, half >>= 1) {
+            for (int m = 16, half = 4; m >= 4; m >>= 1, half >>= 1) {
                 const bool upper = (lane & m) != 0;
 #pragma unroll
-                for (int k = 0; k < half; ++k) {
-                    const float send = upper ? vals[k] : vals[k + half];
-                    const float keep = upper ? vals[k + half] : vals[k];
-                    vals[k] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+                for (int q = 0; q < half; ++q) {
+                    const float send = upper ? vals[q] : vals[q + half];
+                    const float keep = upper ? vals[q + half] : vals[q];
+                    vals[q] = keep + __shfl_xor_sync(0xffffffffu, send, m);
                 }
             }
             cst[i * 32 + col] = vals[0];
@@ -287,34 +341,33 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 2) scan_bwd_kernel(const BwdPa
         }
 #pragma unroll
         for (int r = 0; r < PER; ++r) {
-            const long long t = t0 + nl * PER + r;
+            const int t = t0 + nl * PER + r;
             if (valid && t < L) {
-                const float dx = softplus ? ddt[r] * sigmoid_f32(xo[r]) : ddt[r];
+                const float dx = softplus ? ddt[r] * sigmoid_f32(cur.x[r] + bias) : ddt[r];
                 dbias_acc += dx;
-                static_cast<IO*>(p.ddelta)[row + t] = IoTraits<IO>::from_f32(dx);
-                static_cast<IO*>(p.du)[row + t] = IoTraits<IO>::from_f32(fmaf(Dd, dv[r], dup[r]));
-                if (p.z) static_cast<IO*>(p.dz)[row + t] = IoTraits<IO>::from_f32(dzv[r]);
+                ddelta_row[t] = IoTraits<IO>::from_f32(dx);
+                du_row[t] = IoTraits<IO>::from_f32(fmaf(Dd, dv[r], dup[r]));
+                if (has_z) dz_row[t] = IoTraits<IO>::from_f32(dzv[r]);
             }
         }
 
         // CTA sum of the warps' dB/dC partials (fixed order), one row per step.
         __syncthreads();
-        for (int k = threadIdx.x; k < T * 32; k += blockDim.x) {
-            const int i = k >> 5, c = k & 31;
-            const long long t = t0 + i;
+        for (int q = threadIdx.x; q < T * 32; q += blockDim.x) {
+            const int i = q >> 5, c = q & 31;
+            const int t = t0 + i;
             float sum = 0.f;
 #pragma unroll
             for (int w = 0; w < kBwdWarps; ++w) sum += cstage[(w * T + i) * 32 + c];
-            if (t < L)
-                p.dbc_part[((static_cast<long long>(b) * p.ncta + blockIdx.x) * L + t) * 32 + c] = sum;
+            if (t < L) p.dbc_part[((static_cast<long long>(b) * p.ncta + blockIdx.x) * p.L + t) * 32 + c] = sum;
         }
-        __syncthreads();
     }
+    cp_async_wait<0>();
 
     // Per-channel results: d initial_state, and the time sums of dA, dD, ddelta_bias.
     if (valid) {
-        if (p.dh0) *reinterpret_cast<float4*>(p.dh0 + srow) = make_float4(g[0], g[1], g[2], g[3]);
-        *reinterpret_cast<float4*>(p.dA_part + srow) = make_float4(dA_acc[0], dA_acc[1], dA_acc[2], dA_acc[3]);
+        if (p.dh0) *reinterpret_cast<float4*>(p.dh0 + srow) = make_float4(g[0].x, g[0].y, g[1].x, g[1].y);
+        *reinterpret_cast<float4*>(p.dA_part + srow) = make_float4(dA_acc[0].x, dA_acc[0].y, dA_acc[1].x, dA_acc[1].y);
     }
 #pragma unroll
     for (int m = 1; m <= 2; m <<= 1) {
@@ -328,11 +381,9 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 2) scan_bwd_kernel(const BwdPa
 }
 
 // ---------------------------------------------------------------------------------------
-// Second kernel: the sums over the CTAs of a batch row (dB, dC, transposed to (b, N, L))
-// and over batch rows (dA, dD, ddelta_bias), in a fixed order.
-// grid.x = ceil(L / 32) time tiles, grid.y = batch; 256 threads.  Block (0, 0) extra work
-// is avoided: dA/dD/dbias are done by a separate small launch of the same kernel with
-// grid.y = 0 semantics handled by `param_pass`.
+// Second pass: the sums over the CTAs of a batch row (dB, dC, transposed to (b, N, L);
+// grid (ceil(L / 32), batch)) and over batch rows (dA, dD, ddelta_bias; one thread per
+// output), each in a fixed order.
 // ---------------------------------------------------------------------------------------
 struct BwdFinalParams {
     const float* dbc_part;

@@ -459,7 +459,7 @@ ssm_status_t launch_backward(const BwdArgs& a) {
     p.nseg = wl.nseg;
     p.ncta = wl.ncta;
     p.softplus = a.softplus;
-    constexpr int smem = ssm::kBwdWarps * ssm::kBwdSeg * 32 * (16 + 4);
+    constexpr int smem = ssm::kBwdSmem;
     auto kern = ssm::scan_bwd_kernel<IO>;
     if (!ensure_smem_attr(reinterpret_cast<const void*>(kern), smem)) return SSM_ERR_LAUNCH;
     kern<<<dim3(static_cast<unsigned>(wl.ncta), static_cast<unsigned>(a.batch)), ssm::kBwdWarps * 32, smem,
@@ -691,7 +691,7 @@ ssm_status_t ssm_selective_scan_bwd(const void* u, const void* delta, const floa
         if (q && !aligned16(q)) return SSM_ERR_INVALID_ARG;
     if (batch == 0 || dim == 0) return SSM_OK;
     if (batch > 65535) return SSM_ERR_UNSUPPORTED;
-    if (seqlen >= (1LL << 40)) return SSM_ERR_UNSUPPORTED;
+    if (seqlen >= (1LL << 31) - 1024) return SSM_ERR_UNSUPPORTED;  // steps are 32-bit in the kernel
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
         workspace_bytes < ssm_selective_scan_bwd_workspace_size(batch, dim, dstate, seqlen))
         return SSM_ERR_WORKSPACE;
