@@ -166,26 +166,37 @@ def max_over_ranks(x: float, world: int) -> float:
 
 
 # ----------------------------------------------------------------------------- measurements
-def kernel_source_hash() -> str:
+# The device sources each kernel family is compiled from (its traffic record stays valid
+# while these files are unchanged).
+KERNEL_SOURCES = {
+    "scan_fwd_seq_kernel": ["common.cuh", "scan_math.cuh", "poly_coeffs.cuh", "scan_fwd_seq.cuh"],
+    "scan_fwd_chunked_kernel": ["common.cuh", "scan_math.cuh", "poly_coeffs.cuh", "scan_fwd_seq.cuh",
+                                "scan_fwd_chunked.cuh"],
+    "state_update_kernel": ["common.cuh", "scan_math.cuh", "poly_coeffs.cuh", "aux_kernels.cuh"],
+    "scan_bwd_kernel": ["common.cuh", "scan_math.cuh", "poly_coeffs.cuh", "scan_fwd_seq.cuh", "scan_bwd.cuh"],
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "selective_state_space_16_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(f.encode() + fh.read())
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
 
 
 def traffic_record(kernel: str, workload: str):
     """dram bytes per launch from the committed ncu summary, if it was taken on the
-    current kernel sources (else None)."""
+    current sources of that kernel (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         recs = json.load(f)
     for r in recs:
-        if r.get("kernel") == kernel and r.get("workload") == workload and r.get("src_sha") == kernel_source_hash():
+        if (r.get("kernel") == kernel and r.get("workload") == workload and
+                r.get("src_sha") == kernel_source_hash(kernel)):
             return r.get("dram_bytes_per_launch")
     return None
 
@@ -296,6 +307,7 @@ def measure_long(ssm, stream, pk, steps=5):
         ms = t / steps * 1e3
         out[name] = {"value": w.elements / (ms / 1e3) / 1e9, "ms_per_step": ms,
                      "hbm_frac": scan_algorithmic_bytes(w) / (ms / 1e3) / 1e9 / pk["hbm_gbs"]}
+    out["chunked_lookback"]["traffic"] = traffic_record("scan_fwd_chunked_kernel", w.name)
     assert ssm.ssm_read_status(ws) == 0
     del g
     return out
@@ -337,7 +349,50 @@ def measure_decode(ssm, stream, pk, steps=None):
     return {"workload": w.name, "value": w.batch * w.dim / per_step / 1e9, "unit": "Gelem/s (B*D per step)",
             "us_per_step": per_step * 1e6, "steps": nsteps, "launch": f"one CUDA graph of {nsteps} steps",
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / pk["hbm_gbs"], "note": "state is 84 MB < 126 MB L2: see ncu dram bytes"}}
+                         "frac": gbs / pk["hbm_gbs"], "note": "state is 84 MB < 126 MB L2: see ncu dram bytes",
+                         "traffic": traffic_record("state_update_kernel", w.name)}}
+
+
+def measure_backward(ssm, stream, pk, steps=5):
+    """Backward of the headline workload (gradients of every input for a seeded N(0, 1) dy),
+    timed with CUDA events on the launching stream; inputs larger than L2."""
+    w = workloads.WORKLOADS[workloads.HEADLINE]
+    _, g = forward_buffers(w, "cuda")
+    gen = torch.Generator().manual_seed(77)
+    dy = torch.randn(w.batch, w.dim, w.seqlen, generator=gen).to(torch.bfloat16).cuda()
+    ws = torch.empty(ssm.ssm_selective_scan_bwd_workspace_size(w.batch, w.dim, w.dstate, w.seqlen),
+                     dtype=torch.uint8, device="cuda")
+    f32 = dict(dtype=torch.float32, device="cuda")
+    du, ddelta, dz = torch.empty_like(g["u"]), torch.empty_like(g["u"]), torch.empty_like(g["u"])
+    dA, dD, dbias = torch.empty(w.dim, w.dstate, **f32), torch.empty(w.dim, **f32), torch.empty(w.dim, **f32)
+    dB, dC = torch.empty(w.batch, w.dstate, w.seqlen, **f32), torch.empty(w.batch, w.dstate, w.seqlen, **f32)
+
+    def call():
+        ssm.ssm_selective_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"], True,
+                                   dy, du, ddelta, dA, dB, dC, dD, dz, dbias, ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            call()
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(steps):
+            call()
+        ev1.record(stream)
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1) / steps
+    # algorithmic bytes: u, delta, z, dy read and du, ddelta, dz written (2 B each), B/C read,
+    # dB/dC written (fp32), A/D/bias and their gradients
+    nbytes = w.elements * 14 + w.batch * w.dstate * w.seqlen * (2 * 2 + 2 * 4) + w.dim * (w.dstate + 2) * 8
+    gbs = nbytes / (ms / 1e3) / 1e9
+    del g
+    return {"workload": w.name, "value": w.elements / (ms / 1e3) / 1e9, "unit": UNIT, "ms_per_step": ms,
+            "gradients": "du, ddelta, dz, dA, dB, dC, dD, ddelta_bias", "launches_per_step": 4,
+            "hbm": {"achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
+                    "algorithmic_bytes_per_step": nbytes,
+                    "traffic": traffic_record("scan_bwd_kernel", w.name)},
+            "ex2_per_element": "32 (the forward once with checkpoints, each segment once more) + 2 sigmoid + 2 softplus"}
 
 
 def _oracle_sample(inp, w, channels):
@@ -467,7 +522,8 @@ def run_gpu(args, world, rank, local):
         e2e_steps = max(3, min(args.steps, 10))
         line["e2e"] = e2e_forward(ssm, w, inp, ws, e2e_steps, stream)
     if world == 1 and not args.skip_extra:
-        line["also"] = {"long": measure_long(ssm, stream, pk), "decode": measure_decode(ssm, stream, pk)}
+        line["also"] = {"long": measure_long(ssm, stream, pk), "decode": measure_decode(ssm, stream, pk),
+                        "backward": measure_backward(ssm, stream, pk)}
     if rank == 0 and world == 1 and not args.skip_cpu:
         rate, secs, desc, cores = cpu_oracle_rate(w, args.cpu_budget)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
@@ -483,6 +539,8 @@ def run_profile_workload(args):
     pk = peaks()
     if args.workload == "long":
         out = measure_long(ssm, stream, pk, steps=args.steps)
+    elif args.workload == "backward":
+        out = measure_backward(ssm, stream, pk, steps=args.steps)
     else:
         w = workloads.WORKLOADS[4]
         out = measure_decode(ssm, stream, pk, steps=args.steps)
@@ -499,8 +557,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-extra", action="store_true")
-    ap.add_argument("--workload", default="headline", choices=["headline", "long", "decode"],
-                    help="profiling runs: 'long' / 'decode' run only that workload a few times")
+    ap.add_argument("--workload", default="headline", choices=["headline", "long", "decode", "backward"],
+                    help="profiling runs: 'long' / 'decode' / 'backward' run only that workload a few times")
     args = ap.parse_args()
     world, rank, local = dist_setup(args.gpus) if args.impl == "native" else (
         int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
