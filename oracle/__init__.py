@@ -45,6 +45,10 @@ def _load():
             lib.oracle_selective_scan_f64.restype = ci
             lib.oracle_state_update_f64.argtypes = [vp] * 9 + [ci, vp, i64, i64, i64]
             lib.oracle_state_update_f64.restype = ci
+            lib.oracle_selective_scan_zoh_f64.argtypes = [vp] * 8 + [ci, vp, vp, vp, i64, i64, i64, i64, ci]
+            lib.oracle_selective_scan_zoh_f64.restype = ci
+            lib.oracle_state_update_zoh_f64.argtypes = [vp] * 9 + [ci, vp, i64, i64, i64, ci]
+            lib.oracle_state_update_zoh_f64.restype = ci
             lib.oracle_selective_scan_bwd_f64.argtypes = [vp] * 8 + [ci] + [vp] * 12 + [i64, i64, i64, i64]
             lib.oracle_selective_scan_bwd_f64.restype = ci
             lib.oracle_num_threads.restype = ci
@@ -82,9 +86,10 @@ def silu(x: float) -> float:
     return float(_load().oracle_silu_f64(float(x)))
 
 
-def selective_scan(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True, h0=None):
+def selective_scan(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True, h0=None, zoh=False):
     """Forward scan.  Shapes: u/delta/z (b, d, L); B/C (b, N, L); A (d, N); D/delta_bias (d);
-    h0 (b, d, N) or None.  Returns (y (b, d, L), last_state (b, d, N)) as float64 arrays."""
+    h0 (b, d, N) or None; zoh: zero-order-hold input weight instead of Delta*B.
+    Returns (y (b, d, L), last_state (b, d, N)) as float64 arrays."""
     u, delta, A, B, C = map(_f64, (u, delta, A, B, C))
     D, z, delta_bias, h0 = map(_f64, (D, z, delta_bias, h0))
     b, d, L = u.shape
@@ -94,15 +99,15 @@ def selective_scan(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=
     assert h0 is None or h0.shape == (b, d, n)
     y = np.empty((b, d, L), dtype=np.float64)
     last = np.empty((b, d, n), dtype=np.float64)
-    rc = _load().oracle_selective_scan_f64(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
-                                           _ptr(z), _ptr(delta_bias), int(bool(softplus)), _ptr(h0),
-                                           _ptr(y), _ptr(last), b, d, n, L)
+    rc = _load().oracle_selective_scan_zoh_f64(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                               _ptr(z), _ptr(delta_bias), int(bool(softplus)), _ptr(h0),
+                                               _ptr(y), _ptr(last), b, d, n, L, int(bool(zoh)))
     if rc != 0:
         raise ValueError("oracle_selective_scan_f64 rejected its arguments")
     return y, last
 
 
-def state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True):
+def state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True, zoh=False):
     """One decode step.  state (b, d, N) is NOT modified; returns (y (b, d), new_state)."""
     st = _f64(state).copy()
     u, delta, A, B, C = map(_f64, (u, delta, A, B, C))
@@ -111,9 +116,9 @@ def state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, soft
     assert u.shape == (b, d) and delta.shape == (b, d) and A.shape == (d, n)
     assert B.shape == (b, n) and C.shape == (b, n)
     y = np.empty((b, d), dtype=np.float64)
-    rc = _load().oracle_state_update_f64(_ptr(st), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
-                                         _ptr(D), _ptr(z), _ptr(delta_bias), int(bool(softplus)),
-                                         _ptr(y), b, d, n)
+    rc = _load().oracle_state_update_zoh_f64(_ptr(st), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
+                                             _ptr(D), _ptr(z), _ptr(delta_bias), int(bool(softplus)),
+                                             _ptr(y), b, d, n, int(bool(zoh)))
     if rc != 0:
         raise ValueError("oracle_state_update_f64 rejected its arguments")
     return y, st

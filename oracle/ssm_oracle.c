@@ -68,6 +68,20 @@ static double silu_f64(double z)
     return z / (1.0 + exp(-z));
 }
 
+/*
+ * Input weight of one chain for one step.  Simplified discretisation: Bbar = Delta*B
+ * ([Card] 离散化变换).  Zero-order hold ([Eng] §2.2): Bbar = (Delta A)^-1 (exp(Delta A) - 1) Delta B
+ * = expm1(Delta A) / A * B for a diagonal A, whose limit as A -> 0 is Delta*B.  (The page prints
+ * the ZOH weight without the Delta in front of B; the reading here is the one that reduces to
+ * Delta*B for small Delta*A, as the simplified form on the other pages does.)
+ */
+static double input_weight(double dt, double a, double b, int zoh)
+{
+    if (!zoh) return dt * b;
+    const double x = dt * a;
+    return x == 0.0 ? dt * b : expm1(x) / a * b;
+}
+
 /* Step size for one (b, d, t): Delta = softplus(delta + bias) ([Eng] §3.2). */
 static double step_size(double delta_raw, const double* delta_bias, int64_t d, int softplus)
 {
@@ -80,11 +94,28 @@ static double step_size(double delta_raw, const double* delta_bias, int64_t d, i
  * (b, d), as in the sequential scans of [S4M] 5.2 and [Card] Python 演示.
  * Returns 0 on success, -1 on a bad argument.
  */
+int oracle_selective_scan_zoh_f64(const double* u, const double* delta, const double* A,
+                                  const double* B, const double* C, const double* D,
+                                  const double* z, const double* delta_bias, int softplus,
+                                  const double* h0, double* y, double* last_state,
+                                  int64_t batch, int64_t dim, int64_t dstate, int64_t L, int zoh);
+
 int oracle_selective_scan_f64(const double* u, const double* delta, const double* A,
                               const double* B, const double* C, const double* D,
                               const double* z, const double* delta_bias, int softplus,
                               const double* h0, double* y, double* last_state,
                               int64_t batch, int64_t dim, int64_t dstate, int64_t L)
+{
+    return oracle_selective_scan_zoh_f64(u, delta, A, B, C, D, z, delta_bias, softplus, h0, y, last_state,
+                                         batch, dim, dstate, L, 0);
+}
+
+/* As oracle_selective_scan_f64, with the zero-order-hold input weight when zoh != 0. */
+int oracle_selective_scan_zoh_f64(const double* u, const double* delta, const double* A,
+                                  const double* B, const double* C, const double* D,
+                                  const double* z, const double* delta_bias, int softplus,
+                                  const double* h0, double* y, double* last_state,
+                                  int64_t batch, int64_t dim, int64_t dstate, int64_t L, int zoh)
 {
     if (batch < 0 || dim < 0 || dstate < 1 || dstate > 256 || L < 0) return -1;
     if (!u || !delta || !A || !B || !C || !y) return -1;
@@ -103,7 +134,7 @@ int oracle_selective_scan_f64(const double* u, const double* delta, const double
                 double yt = 0.0;
                 for (int64_t n = 0; n < dstate; ++n) {
                     const double abar = exp(dt * A[d * dstate + n]);
-                    const double bbar = dt * B[(b * dstate + n) * L + t];
+                    const double bbar = input_weight(dt, A[d * dstate + n], B[(b * dstate + n) * L + t], zoh);
                     h[n] = abar * h[n] + bbar * ut;
                     yt += C[(b * dstate + n) * L + t] * h[n];
                 }
@@ -124,11 +155,28 @@ int oracle_selective_scan_f64(const double* u, const double* delta, const double
  * state: (batch, dim, dstate) in/out; u, delta, z, y: (batch, dim);
  * B, C: (batch, dstate).
  */
+int oracle_state_update_zoh_f64(double* state, const double* u, const double* delta,
+                                const double* A, const double* B, const double* C,
+                                const double* D, const double* z, const double* delta_bias,
+                                int softplus, double* y,
+                                int64_t batch, int64_t dim, int64_t dstate, int zoh);
+
 int oracle_state_update_f64(double* state, const double* u, const double* delta,
                             const double* A, const double* B, const double* C,
                             const double* D, const double* z, const double* delta_bias,
                             int softplus, double* y,
                             int64_t batch, int64_t dim, int64_t dstate)
+{
+    return oracle_state_update_zoh_f64(state, u, delta, A, B, C, D, z, delta_bias, softplus, y, batch, dim,
+                                       dstate, 0);
+}
+
+/* As oracle_state_update_f64, with the zero-order-hold input weight when zoh != 0. */
+int oracle_state_update_zoh_f64(double* state, const double* u, const double* delta,
+                                const double* A, const double* B, const double* C,
+                                const double* D, const double* z, const double* delta_bias,
+                                int softplus, double* y,
+                                int64_t batch, int64_t dim, int64_t dstate, int zoh)
 {
     if (batch < 0 || dim < 0 || dstate < 1 || dstate > 256) return -1;
     if (!state || !u || !delta || !A || !B || !C || !y) return -1;
@@ -142,7 +190,8 @@ int oracle_state_update_f64(double* state, const double* u, const double* delta,
             double yt = 0.0;
             for (int64_t n = 0; n < dstate; ++n) {
                 double* h = &state[row * dstate + n];
-                *h = exp(dt * A[d * dstate + n]) * (*h) + dt * B[b * dstate + n] * ut;
+                *h = exp(dt * A[d * dstate + n]) * (*h) +
+                     input_weight(dt, A[d * dstate + n], B[b * dstate + n], zoh) * ut;
                 yt += C[b * dstate + n] * (*h);
             }
             yt += (D ? D[d] : 0.0) * ut;

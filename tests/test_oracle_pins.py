@@ -405,3 +405,77 @@ def test_backward_is_linear_in_the_output_gradient():
     g12 = oracle.selective_scan_bwd(**case, dy=dy1 - 3.0 * dy2)
     for k in ("du", "ddelta", "dA", "dB", "dC", "dD", "dz", "ddelta_bias", "dh0"):
         np.testing.assert_allclose(g12[k], g1[k] - 3.0 * g2[k], rtol=1e-11, atol=1e-12, err_msg=k)
+
+
+# ---------------------------------------------------------------------------------------------
+# Zero-order hold ([Eng] §2.2): the discretisation of h' = A h + B x with the input held over
+# each step.  Pinned against a fine fourth-order Runge-Kutta integration of that ODE.
+# ---------------------------------------------------------------------------------------------
+def _rk4_zoh_reference(case):
+    u, A, B, C = case["u"], case["A"], case["B"], case["C"]
+    b, d, L = u.shape
+    n = A.shape[1]
+    dt = _step_sizes(case)
+    y = np.zeros((b, d, L))
+    last = np.zeros((b, d, n))
+    sub = 400
+    for bi in range(b):
+        for di in range(d):
+            h = np.zeros(n)
+            a = A[di]
+            for t in range(L):
+                drive = B[bi, :, t] * u[bi, di, t]           # held over the step
+                f = lambda hh: a * hh + drive
+                step = dt[bi, di, t] / sub
+                for _ in range(sub):
+                    k1 = f(h)
+                    k2 = f(h + 0.5 * step * k1)
+                    k3 = f(h + 0.5 * step * k2)
+                    k4 = f(h + step * k3)
+                    h = h + step / 6.0 * (k1 + 2 * k2 + 2 * k3 + k4)
+                yt = C[bi, :, t] @ h + (case["D"][di] if case["D"] is not None else 0.0) * u[bi, di, t]
+                if case["z"] is not None:
+                    zt = case["z"][bi, di, t]
+                    yt *= zt / (1.0 + np.exp(-zt))
+                y[bi, di, t] = yt
+            last[bi, di] = h
+    return y, last
+
+
+def test_zoh_matches_integrated_ode():
+    rng = _rng(61)
+    case = _selective_case(rng, b=1, d=2, n=3, L=6)
+    y, last = oracle.selective_scan(**case, zoh=True)
+    y_ref, last_ref = _rk4_zoh_reference(case)
+    np.testing.assert_allclose(y, y_ref, rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(last, last_ref, rtol=1e-9, atol=1e-11)
+    # ... and it is not the simplified discretisation
+    y_s, _ = oracle.selective_scan(**case)
+    assert np.abs(y_s - y).max() > 1e-3
+
+
+def test_zoh_limits():
+    rng = _rng(62)
+    case = _selective_case(rng)
+    # A = 0: the hold weight is exactly Delta*B, as the simplified discretisation
+    c0 = dict(case, A=np.zeros_like(case["A"]))
+    np.testing.assert_array_equal(oracle.selective_scan(**c0, zoh=True)[0], oracle.selective_scan(**c0)[0])
+    # small Delta A: ZOH -> simplified, with a relative gap of order Delta*|A|
+    cs = dict(case, delta=np.full_like(case["delta"], -20.0), delta_bias=None)   # softplus(-20) ~ 2e-9
+    y_z, h_z = oracle.selective_scan(**cs, zoh=True)
+    y_s, h_s = oracle.selective_scan(**cs)
+    np.testing.assert_allclose(h_z, h_s, rtol=1e-7, atol=1e-20)
+
+
+def test_zoh_decode_chain_equals_scan():
+    rng = _rng(63)
+    case = _selective_case(rng, L=8)
+    y, last = oracle.selective_scan(**case, zoh=True)
+    b, d, L = case["u"].shape
+    state = np.zeros((b, d, case["A"].shape[1]))
+    for t in range(L):
+        yt, state = oracle.state_update(state, case["u"][..., t], case["delta"][..., t], case["A"], case["B"][..., t],
+                                        case["C"][..., t], D=case["D"], z=case["z"][..., t],
+                                        delta_bias=case["delta_bias"], softplus=case["softplus"], zoh=True)
+        np.testing.assert_allclose(yt, y[..., t], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(state, last, rtol=1e-12, atol=1e-13)
