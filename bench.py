@@ -353,6 +353,19 @@ def measure_decode(ssm, stream, pk, steps=None):
                          "traffic": traffic_record("state_update_kernel", w.name)}}
 
 
+def measure_zoh(ssm, stream, pk, steps=10):
+    """Headline workload with the zero-order-hold discretisation (sequential kernel)."""
+    w = workloads.WORKLOADS[workloads.HEADLINE]
+    _, g = forward_buffers(w, "cuda")
+    ws = ssm.new_workspace(w.batch, w.dim, w.dstate, w.seqlen)
+    t = time_forward(ssm, g, ws, steps, 3, 1, stream, opts={"zoh": True})
+    ms = t / steps * 1e3
+    assert ssm.ssm_read_status(ws) == 0
+    del g
+    return {"workload": w.name, "discretization": "zero-order hold", "value": w.elements / (ms / 1e3) / 1e9,
+            "unit": UNIT, "ms_per_step": ms}
+
+
 def measure_backward(ssm, stream, pk, steps=5):
     """Backward of the headline workload (gradients of every input for a seeded N(0, 1) dy),
     timed with CUDA events on the launching stream; inputs larger than L2."""
@@ -523,7 +536,7 @@ def run_gpu(args, world, rank, local):
         line["e2e"] = e2e_forward(ssm, w, inp, ws, e2e_steps, stream)
     if world == 1 and not args.skip_extra:
         line["also"] = {"long": measure_long(ssm, stream, pk), "decode": measure_decode(ssm, stream, pk),
-                        "backward": measure_backward(ssm, stream, pk)}
+                        "backward": measure_backward(ssm, stream, pk), "zoh": measure_zoh(ssm, stream, pk)}
     if rank == 0 and world == 1 and not args.skip_cpu:
         rate, secs, desc, cores = cpu_oracle_rate(w, args.cpu_budget)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}

@@ -114,12 +114,24 @@ typedef enum {
     SSM_ALGO_DIRECT = 3       /* no staging: direct global loads (any alignment of seqlen)     */
 } ssm_algo_t;
 
+/*
+ * Discretisation of the continuous system ([Eng] §2.2).  SIMPLIFIED (the default): Abar = exp(Delta A),
+ * Bbar = Delta B ([Card] 离散化变换).  ZOH: the zero-order hold, Bbar = (Delta A)^-1 (exp(Delta A) - 1)
+ * Delta B = expm1(Delta A)/A * B for the diagonal A (Delta B when A = 0).  ZOH is supported by the
+ * sequential and direct forward kernels and by decode; SSM_ALGO_CHUNKED and the backward return
+ * SSM_ERR_UNSUPPORTED for it.
+ */
+typedef enum { SSM_DISC_SIMPLIFIED = 0, SSM_DISC_ZOH = 1 } ssm_discretization_t;
+
+/* Options of the forward entry points.  Zero-initialise the whole struct: zero means the
+ * default for every field (changed in ABI version 2: the discretization field was added). */
 typedef struct {
     int algo;                  /* ssm_algo_t                                                      */
     int lanes_per_channel;     /* SEQUENTIAL: lanes sharing one channel: 2, 4 or 8 (8: bf16 only), or 42 =
                                   4 lanes per channel with each lane holding two channels; 0 = auto    */
     uint32_t spin_limit;       /* CHUNKED: polls before a look-back wait gives up; 0 = default    */
     int debug_skip_publish;    /* CHUNKED, tests only: chunk index whose CTAs never publish; -1 = off */
+    int discretization;        /* ssm_discretization_t; 0 = SSM_DISC_SIMPLIFIED                   */
 } ssm_fwd_options_t;
 
 /* ssm_selective_scan_fwd with an explicit kernel choice (tuning and tests).  opts may be NULL. */
@@ -206,6 +218,13 @@ ssm_status_t ssm_state_update(
     float* state, const void* u, const void* delta, const float* A, const void* B, const void* C,
     const float* D, const void* z, const float* delta_bias, int softplus, void* y,
     int batch, int dim, int dstate, ssm_dtype_t io_dtype, ssm_stream_t stream);
+
+/* ssm_state_update with an explicit discretisation (ssm_discretization_t). */
+ssm_status_t ssm_state_update_ex(
+    float* state, const void* u, const void* delta, const float* A, const void* B, const void* C,
+    const float* D, const void* z, const float* delta_bias, int softplus, void* y,
+    int batch, int dim, int dstate, ssm_dtype_t io_dtype, ssm_discretization_t discretization,
+    ssm_stream_t stream);
 
 /*
  * Forward scan that allocates nothing and takes no workspace.  The pages have no

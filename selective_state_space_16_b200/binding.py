@@ -32,9 +32,13 @@ class SsmError(RuntimeError):
         super().__init__(f"{where}: {status_string(code)} (status {code})")
 
 
+SSM_DISC_SIMPLIFIED, SSM_DISC_ZOH = 0, 1
+
+
 class FwdOptions(ctypes.Structure):
     _fields_ = [("algo", ctypes.c_int), ("lanes_per_channel", ctypes.c_int),
-                ("spin_limit", ctypes.c_uint32), ("debug_skip_publish", ctypes.c_int)]
+                ("spin_limit", ctypes.c_uint32), ("debug_skip_publish", ctypes.c_int),
+                ("discretization", ctypes.c_int)]
 
 
 _lib = None
@@ -72,6 +76,8 @@ def load() -> ctypes.CDLL:
             lib.ssm_selective_scan_bwd.restype = ci
             lib.ssm_state_update.argtypes = [vp] * 9 + [ci, vp, ci, ci, ci, ci, vp]
             lib.ssm_state_update.restype = ci
+            lib.ssm_state_update_ex.argtypes = [vp] * 9 + [ci, vp, ci, ci, ci, ci, ci, vp]
+            lib.ssm_state_update_ex.restype = ci
             lib.ssm_read_status.argtypes = [vp, vp]
             lib.ssm_read_status.restype = ci
             _lib = lib
@@ -124,10 +130,11 @@ def new_workspace(batch, dim, dstate, seqlen, device="cuda", stream=None):
 
 def ssm_selective_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus, y, last_state, workspace,
                            stream=None, algo=None, lanes_per_channel=0, spin_limit=0, debug_skip_publish=-1,
-                           check=True, initial_state=None):
+                           check=True, initial_state=None, zoh=False):
     """Marshal a forward-scan call.  u/delta/z/y: (b, d, L); B/C: (b, N, L); A: (d, N) fp32;
     D/delta_bias: (d) fp32 or None; last_state: (b, d, N) fp32 or None; workspace: uint8;
-    initial_state: (b, d, N) fp32 or None (zero), through ssm_selective_scan_fwd_state."""
+    initial_state: (b, d, N) fp32 or None (zero), through ssm_selective_scan_fwd_state;
+    zoh: zero-order-hold discretisation instead of the simplified one."""
     lib = load()
     b, d, L = u.shape
     n = A.shape[1]
@@ -135,12 +142,14 @@ def ssm_selective_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus, y, las
             int(bool(softplus))]
     tail = [_ptr(y), _ptr(last_state), b, d, n, L, _io(u), _ptr(workspace),
             workspace.numel() * workspace.element_size()]
-    default_opts = algo is None and lanes_per_channel == 0 and spin_limit == 0 and debug_skip_publish < 0
+    default_opts = (algo is None and lanes_per_channel == 0 and spin_limit == 0 and debug_skip_publish < 0
+                    and not zoh)
     if default_opts and initial_state is None:
         code = lib.ssm_selective_scan_fwd(*head, *tail, _stream(stream))
     else:
         a = ALGOS[algo] if isinstance(algo, str) else (algo or SSM_ALGO_AUTO)
-        opts = FwdOptions(a, lanes_per_channel, spin_limit, debug_skip_publish)
+        opts = FwdOptions(a, lanes_per_channel, spin_limit, debug_skip_publish,
+                          SSM_DISC_ZOH if zoh else SSM_DISC_SIMPLIFIED)
         if initial_state is None:
             code = lib.ssm_selective_scan_fwd_ex(*head, *tail, ctypes.byref(opts), _stream(stream))
         else:
@@ -208,12 +217,16 @@ def selective_scan_bwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
     return out
 
 
-def ssm_state_update(state, u, delta, A, B, C, D, z, delta_bias, softplus, y, stream=None, check=True):
-    """Marshal a decode call.  state: (b, d, N) fp32 in/out; u/delta/z/y: (b, d); B/C: (b, N)."""
+def ssm_state_update(state, u, delta, A, B, C, D, z, delta_bias, softplus, y, stream=None, check=True, zoh=False):
+    """Marshal a decode call.  state: (b, d, N) fp32 in/out; u/delta/z/y: (b, d); B/C: (b, N);
+    zoh: zero-order-hold discretisation (ssm_state_update_ex)."""
     b, d, n = state.shape
-    code = load().ssm_state_update(_ptr(state), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
-                                   _ptr(z), _ptr(delta_bias), int(bool(softplus)), _ptr(y), b, d, n, _io(u),
-                                   _stream(stream))
+    args = [_ptr(state), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+            int(bool(softplus)), _ptr(y), b, d, n, _io(u)]
+    if zoh:
+        code = load().ssm_state_update_ex(*args, SSM_DISC_ZOH, _stream(stream))
+    else:
+        code = load().ssm_state_update(*args, _stream(stream))
     if check:
         _check(code, "ssm_state_update")
     return code

@@ -58,6 +58,7 @@ struct DirectParams {
     int batch, dim;
     long long L;
     int softplus;
+    int zoh;  // zero-order-hold input weight instead of Delta*B
 };
 
 template <typename IO, int G>
@@ -76,10 +77,12 @@ __global__ void __launch_bounds__(128) scan_fwd_direct_kernel(const DirectParams
     IO* y = static_cast<IO*>(p.y) + ch * p.L;
     const float* bcb = p.bc + static_cast<long long>(b) * p.L * 32;
 
-    float A2[NC], h[NC];
+    float A2[NC], invA[NC], h[NC];
 #pragma unroll
     for (int j = 0; j < NC; ++j) {
-        A2[j] = valid ? p.A[d * 16 + nl * NC + j] * kLog2e : 0.f;
+        const float a = valid ? p.A[d * 16 + nl * NC + j] : 0.f;
+        A2[j] = a * kLog2e;
+        invA[j] = 1.f / a;
         h[j] = (valid && p.h0) ? p.h0[ch * 16 + nl * NC + j] : 0.f;
     }
     const float Dd = (valid && p.D) ? p.D[d] : 0.f;
@@ -96,8 +99,11 @@ __global__ void __launch_bounds__(128) scan_fwd_direct_kernel(const DirectParams
         float acc = 0.f;
 #pragma unroll
         for (int j = 0; j < NC; ++j) {
-            const float a = ex2_mufu(dt * A2[j]);
-            h[j] = fmaf(a, h[j], w * row[nl * NC + j]);
+            const float y = dt * A2[j];
+            const float a = ex2_mufu(y);
+            const float Bn = row[nl * NC + j];
+            const float beta = p.zoh ? zoh_beta(y, a, w * Bn, ut * Bn * invA[j]) : w * Bn;
+            h[j] = fmaf(a, h[j], beta);
             acc = fmaf(row[16 + nl * NC + j], h[j], acc);
         }
 #pragma unroll
@@ -134,6 +140,7 @@ struct DecodeParams {
     void* y;
     int batch, dim;
     int softplus;
+    int zoh;  // zero-order-hold input weight instead of Delta*B
 };
 
 template <typename IO>
@@ -172,8 +179,10 @@ __global__ void __launch_bounds__(256) state_update_kernel(const DecodeParams p)
     float acc = 0.f;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        const float a = ex2_mufu(dt * as[j] * kLog2e);
-        hs[j] = fmaf(a, hs[j], w * Bq[j]);
+        const float y = dt * as[j] * kLog2e;
+        const float a = ex2_mufu(y);
+        const float beta = p.zoh ? zoh_beta(y, a, w * Bq[j], ut * Bq[j] / as[j]) : w * Bq[j];
+        hs[j] = fmaf(a, hs[j], beta);
         acc = fmaf(Cq[j], hs[j], acc);
     }
     acc += __shfl_xor_sync(0xffffffffu, acc, 1, 32);

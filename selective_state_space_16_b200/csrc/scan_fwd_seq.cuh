@@ -19,7 +19,8 @@
 // (CPL = 2 lets one load of a step's B/C rows serve two channels; the shared-memory
 // data path is the scarce resource of this kernel).  Per step each lane computes
 //   a = 2^(Delta * A[d,n] * log2 e),  h = a*h + (Delta*u)*B[n],  y_partial += C[n]*h
-// (simplified discretisation Abar = exp(Delta A), Bbar = Delta B: [Card] 离散化变换),
+// (simplified discretisation Abar = exp(Delta A), Bbar = Delta B: [Card] 离散化变换; with ZOH the
+// zero-order-hold weight of [Eng] §2.2, see zoh_beta2),
 // and the G partial sums of y_t = sum_n C_t[n] h_t[n] are combined by a shuffle
 // reduce-scatter over each 16-byte group of GS steps, so that every lane finishes the
 // epilogue (D skip, silu gate, rounding, store) of GS/G steps and nothing is evaluated
@@ -132,7 +133,7 @@ __device__ __forceinline__ void store_run(IO* dst, const float (&v)[N]) {
 // of a stage are unrolled (compile-time shared-memory offsets) with ping-pong step-size
 // buffers: the step sizes of group g+1 (for the last group: group 0 of the next stage,
 // after waiting for it) are computed while group g is scanned.
-template <typename IO, int G, int CPL, int S, bool HZ>
+template <typename IO, int G, int CPL, int S, bool HZ, bool ZOH>
 __device__ __forceinline__ void seq_consumer(const uint8_t* smem, uint64_t* full_bar, uint64_t* empty_bar,
                                              const int* abort_flag, const SeqParams& p, long long r_begin, int nt,
                                              int b_first, int stage_bytes, int nstages, int L32) {
@@ -165,6 +166,7 @@ __device__ __forceinline__ void seq_consumer(const uint8_t* smem, uint64_t* full
     const int bc_off = 3 * p.max_tiles * Cfg::kTileBytes + (b - b_first) * Cfg::kBC + nl * NC * 4;
 
     float2 A2[CPL][NC / 2], h[CPL][NC / 2];
+    float2 invA[CPL][ZOH ? NC / 2 : 1];  // 1 / A (zero-order hold only)
     float Dd[CPL], bias[CPL];
     IO* yrow[CPL];
 #pragma unroll
@@ -176,6 +178,7 @@ __device__ __forceinline__ void seq_consumer(const uint8_t* smem, uint64_t* full
             const float a0 = valid[c] ? p.A[d[c] * 16 + nl * NC + 2 * jj] : 0.f;
             const float a1 = valid[c] ? p.A[d[c] * 16 + nl * NC + 2 * jj + 1] : 0.f;
             A2[c][jj] = f2(a0 * kLog2e, a1 * kLog2e);
+            if constexpr (ZOH) invA[c][jj] = f2(1.f / a0, 1.f / a1);
             h[c][jj] = h0 ? *reinterpret_cast<const float2*>(h0 + 2 * jj) : f2(0.f, 0.f);
         }
         Dd[c] = (valid[c] && p.D) ? p.D[d[c]] : 0.f;
@@ -245,7 +248,11 @@ __device__ __forceinline__ void seq_consumer(const uint8_t* smem, uint64_t* full
                 for (int jj = 0; jj < NC / 2; ++jj) {
                     const float2 arg = __fmul2_rn(dd, A2[c][jj]);
                     const float2 a = f2(ex2_mufu(arg.x), ex2_mufu(arg.y));
-                    h[c][jj] = __ffma2_rn(a, h[c][jj], __fmul2_rn(ww, Bv[jj]));
+                    float2 beta = __fmul2_rn(ww, Bv[jj]);
+                    if constexpr (ZOH)
+                        beta = zoh_beta2(arg, a, beta,
+                                         __fmul2_rn(__fmul2_rn(f2(uf[c][i], uf[c][i]), Bv[jj]), invA[c][jj]));
+                    h[c][jj] = __ffma2_rn(a, h[c][jj], beta);
                     acc = __ffma2_rn(Cv[jj], h[c][jj], acc);
                 }
                 yp[c][i] = acc.x + acc.y;
@@ -333,7 +340,7 @@ __device__ __forceinline__ void seq_consumer(const uint8_t* smem, uint64_t* full
         }
 }
 
-template <typename IO, int G, int CPL, int S>
+template <typename IO, int G, int CPL, int S, bool ZOH = false>
 __global__ void __launch_bounds__((SeqCfg<IO, G, CPL>::kMaxWarps + 1) * 32, 1)
 scan_fwd_seq_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_dl,
                     const __grid_constant__ CUtensorMap map_z, const __grid_constant__ CUtensorMap map_bc,
@@ -417,11 +424,11 @@ scan_fwd_seq_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_cons
             }
         } else if (warp < nwarps) {
             if (p.has_z)
-                seq_consumer<IO, G, CPL, S, true>(smem, full_bar, empty_bar, &abort_flag, p, r_begin, nt, b_first,
-                                                  stage_bytes, nstages, L32);
+                seq_consumer<IO, G, CPL, S, true, ZOH>(smem, full_bar, empty_bar, &abort_flag, p, r_begin, nt,
+                                                       b_first, stage_bytes, nstages, L32);
             else
-                seq_consumer<IO, G, CPL, S, false>(smem, full_bar, empty_bar, &abort_flag, p, r_begin, nt, b_first,
-                                                   stage_bytes, nstages, L32);
+                seq_consumer<IO, G, CPL, S, false, ZOH>(smem, full_bar, empty_bar, &abort_flag, p, r_begin, nt,
+                                                        b_first, stage_bytes, nstages, L32);
         }
         // Every warp leaves the round before the barriers are re-initialised for the next.
         __syncthreads();

@@ -41,6 +41,32 @@ __device__ __forceinline__ float step_size(float raw, float bias, bool softplus)
     return softplus ? softplus_f32(x) : x;
 }
 
+// Zero-order-hold input weight ([Eng] §2.2): Bbar = (Delta A)^-1 (exp(Delta A) - 1) Delta B
+// = Delta B phi(Delta A), phi(x) = (e^x - 1) / x, for a diagonal A (phi -> 1 as A -> 0).
+// With y = Delta A log2(e) and a = 2^y already at hand, the weight times u is
+//   |y| >= kZohSmall:  (a - 1) * (u B / A)              (no cancellation: |a - 1| > 0.06)
+//   |y| <  kZohSmall:  (Delta u B) * phi, phi = 1 + x/2 + x^2/6 + x^3/24  (x = y ln 2;
+//                      truncation error x^4/120 < 1.3e-7 relative at |x| = 1/16)
+// Both are formed and one is selected, so A = 0 (u B / A infinite) never reaches the result.
+constexpr float kZohSmall = 0.0901684400f;  // log2(e) / 16: |Delta A| < 1/16
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kZohP1 = kLn2 / 2.f, kZohP2 = kLn2 * kLn2 / 6.f, kZohP3 = kLn2 * kLn2 * kLn2 / 24.f;
+
+__device__ __forceinline__ float zoh_beta(float y, float a, float wB, float uB_over_A) {
+    const float phi = fmaf(fmaf(fmaf(kZohP3, y, kZohP2), y, kZohP1), y, 1.f);
+    return fabsf(y) < kZohSmall ? wB * phi : (a - 1.f) * uB_over_A;
+}
+
+// The same for a pair of chains (f32x2 arithmetic).
+__device__ __forceinline__ float2 zoh_beta2(float2 y, float2 a, float2 wB, float2 uB_over_A) {
+    const float2 phi = __ffma2_rn(__ffma2_rn(__ffma2_rn(make_float2(kZohP3, kZohP3), y, make_float2(kZohP2, kZohP2)), y,
+                                             make_float2(kZohP1, kZohP1)),
+                                  y, make_float2(1.f, 1.f));
+    const float2 small = __fmul2_rn(wB, phi);
+    const float2 big = __fmul2_rn(__fadd2_rn(a, make_float2(-1.f, -1.f)), uB_over_A);
+    return make_float2(fabsf(y.x) < kZohSmall ? small.x : big.x, fabsf(y.y) < kZohSmall ? small.y : big.y);
+}
+
 // silu(z) = z / (1 + e^-z), the SiLU gate of the Mamba block ([Hist] Mamba Block 数据流).
 // For z -> -inf the denominator overflows to +inf and the result is 0.
 __device__ __forceinline__ float silu_f32(float z) {

@@ -23,7 +23,7 @@ namespace {
 
 using ssm::WorkspaceHeader;
 
-constexpr int kAbiVersion = 1;
+constexpr int kAbiVersion = 2;
 constexpr uint32_t kDefaultWaitLimit = 1u << 22;
 constexpr uint32_t kDefaultSpinLimit = 1u << 21;  // look-back polls (~64 ns sleep each)
 
@@ -131,6 +131,7 @@ struct FwdArgs {
     const float *A, *D, *bias;
     int softplus;
     const float* h0;
+    int zoh;
     void* y;
     float* last_state;
     int batch, dim;
@@ -141,12 +142,12 @@ struct FwdArgs {
     int sm_count;
 };
 
-template <typename IO, int G, int CPL>
+template <typename IO, int G, int CPL, bool ZOH>
 const void* seq_kernel_ptr(int stages) {
     switch (stages) {
-        case 2: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 2>);
-        case 3: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 3>);
-        default: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 4>);
+        case 2: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 2, ZOH>);
+        case 3: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 3, ZOH>);
+        default: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 4, ZOH>);
     }
 }
 
@@ -159,7 +160,7 @@ struct SeqPlan {
     bool ok = false;
 };
 
-template <typename IO, int G, int CPL>
+template <typename IO, int G, int CPL, bool ZOH = false>
 SeqPlan plan_seq(const FwdArgs& a) {
     using Cfg = ssm::SeqCfg<IO, G, CPL>;
     SeqPlan pl;
@@ -182,7 +183,7 @@ SeqPlan plan_seq(const FwdArgs& a) {
         if (stages < 2) continue;
         const int threads = (Cfg::warps_for(mt) + 1) * 32;
         const int smem = Cfg::smem_bytes(mt, stages);
-        const void* kern = seq_kernel_ptr<IO, G, CPL>(stages);
+        const void* kern = seq_kernel_ptr<IO, G, CPL, ZOH>(stages);
         int occ = 0;
         if (!ensure_smem_attr(kern, smem) ||
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, smem) != cudaSuccess || occ < per_sm)
@@ -214,7 +215,7 @@ double predict_seq(const FwdArgs& a, const SeqPlan& pl) {
     return tiles * cost / hide;
 }
 
-template <typename IO, int G, int CPL>
+template <typename IO, int G, int CPL, bool ZOH = false>
 ssm_status_t launch_seq(const FwdArgs& a, const SeqPlan& pl) {
     using Cfg = ssm::SeqCfg<IO, G, CPL>;
     if (!pl.ok) return SSM_ERR_UNSUPPORTED;
@@ -250,9 +251,9 @@ ssm_status_t launch_seq(const FwdArgs& a, const SeqPlan& pl) {
     p.wait_limit = kDefaultWaitLimit;
     if (a.L >= (1LL << 31) - 1024) return SSM_ERR_UNSUPPORTED;
     switch (pl.stages) {
-        case 2: ssm::scan_fwd_seq_kernel<IO, G, CPL, 2><<<pl.grid, pl.threads, pl.smem, a.stream>>>(mu, mdl, mz, mbc, p); break;
-        case 3: ssm::scan_fwd_seq_kernel<IO, G, CPL, 3><<<pl.grid, pl.threads, pl.smem, a.stream>>>(mu, mdl, mz, mbc, p); break;
-        default: ssm::scan_fwd_seq_kernel<IO, G, CPL, 4><<<pl.grid, pl.threads, pl.smem, a.stream>>>(mu, mdl, mz, mbc, p); break;
+        case 2: ssm::scan_fwd_seq_kernel<IO, G, CPL, 2, ZOH><<<pl.grid, pl.threads, pl.smem, a.stream>>>(mu, mdl, mz, mbc, p); break;
+        case 3: ssm::scan_fwd_seq_kernel<IO, G, CPL, 3, ZOH><<<pl.grid, pl.threads, pl.smem, a.stream>>>(mu, mdl, mz, mbc, p); break;
+        default: ssm::scan_fwd_seq_kernel<IO, G, CPL, 4, ZOH><<<pl.grid, pl.threads, pl.smem, a.stream>>>(mu, mdl, mz, mbc, p); break;
     }
     return launch_status();
 }
@@ -327,6 +328,7 @@ ssm_status_t launch_direct(const FwdArgs& a) {
     p.dim = a.dim;
     p.L = a.L;
     p.softplus = a.softplus;
+    p.zoh = a.zoh;
     constexpr int G = 2;
     const long long threads = static_cast<long long>(a.batch) * a.dim * G;
     const long long grid = (threads + 127) / 128;
@@ -353,6 +355,8 @@ ssm_status_t launch_forward(const FwdArgs& a, const ssm_fwd_options_t& o) {
     int algo = o.algo;
     if (!tma_ok) algo = SSM_ALGO_DIRECT;
     if (algo == SSM_ALGO_DIRECT) return launch_direct<IO>(a);
+    if (a.zoh && algo == SSM_ALGO_CHUNKED) return SSM_ERR_UNSUPPORTED;  // simplified discretisation only
+    if (algo == SSM_ALGO_AUTO && a.zoh) algo = SSM_ALGO_SEQUENTIAL;
     if (algo == SSM_ALGO_AUTO) {
         // The sequential kernel is faster whenever the channels alone give each SM a few
         // warps (measured on B200: at 5120 channels x 32768 steps it runs at ~1.8x the
@@ -364,7 +368,18 @@ ssm_status_t launch_forward(const FwdArgs& a, const ssm_fwd_options_t& o) {
     }
     if (algo == SSM_ALGO_CHUNKED) return launch_chunked<IO>(a, o);
     // Variants: (lanes per channel G, channels per lane CPL).  lanes_per_channel selects
-    // G explicitly (CPL = 1), or G = 4 with CPL = 2 when given as 42.
+    // G explicitly (CPL = 1), or G = 4 with CPL = 2 when given as 42.  The zero-order-hold
+    // weight is built into the 4- and 8-lane variants only.
+    if (a.zoh) {
+        const SeqPlan z4 = plan_seq<IO, 4, 1, true>(a);
+        if constexpr (sizeof(IO) == 2) {
+            const SeqPlan z8 = plan_seq<IO, 8, 1, true>(a);
+            const bool use8 = o.lanes_per_channel == 8 ||
+                              (o.lanes_per_channel == 0 && predict_seq<IO, 8, 1>(a, z8) < predict_seq<IO, 4, 1>(a, z4));
+            if (use8) return launch_seq<IO, 8, 1, true>(a, z8);
+        }
+        return launch_seq<IO, 4, 1, true>(a, z4);
+    }
     const SeqPlan p2 = plan_seq<IO, 2, 1>(a), p4 = plan_seq<IO, 4, 1>(a), p42 = plan_seq<IO, 4, 2>(a);
     SeqPlan p8;
     if constexpr (sizeof(IO) == 2) p8 = plan_seq<IO, 8, 1>(a);
@@ -560,9 +575,10 @@ ssm_status_t ssm_selective_scan_fwd_state(const void* u, const void* delta, cons
         const uintptr_t a0 = reinterpret_cast<uintptr_t>(initial_state), a1 = reinterpret_cast<uintptr_t>(last_state);
         if ((a0 <= a1 ? a1 - a0 : a0 - a1) < state_bytes) return SSM_ERR_INVALID_ARG;
     }
-    ssm_fwd_options_t o{SSM_ALGO_AUTO, 0, 0, -1};
+    ssm_fwd_options_t o{SSM_ALGO_AUTO, 0, 0, -1, SSM_DISC_SIMPLIFIED};
     if (opts) o = *opts;
     if (o.algo < SSM_ALGO_AUTO || o.algo > SSM_ALGO_DIRECT) return SSM_ERR_INVALID_ARG;
+    if (o.discretization != SSM_DISC_SIMPLIFIED && o.discretization != SSM_DISC_ZOH) return SSM_ERR_INVALID_ARG;
     if (batch == 0 || dim == 0) return SSM_OK;
     if (batch > 65535) return SSM_ERR_UNSUPPORTED;  // batch is a grid y-dimension of the B/C pack
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
@@ -582,8 +598,8 @@ ssm_status_t ssm_selective_scan_fwd_state(const void* u, const void* delta, cons
         }
         return SSM_OK;
     }
-    FwdArgs a{u, delta, B, C, z, A, D, delta_bias, softplus, initial_state, y, last_state, batch, dim, seqlen,
-              io_dtype, static_cast<uint8_t*>(workspace), s, sm_count};
+    FwdArgs a{u, delta, B, C, z, A, D, delta_bias, softplus, initial_state, o.discretization == SSM_DISC_ZOH, y,
+              last_state, batch, dim, seqlen, io_dtype, static_cast<uint8_t*>(workspace), s, sm_count};
     return io_dtype == SSM_BF16 ? launch_forward<__nv_bfloat16>(a, o) : launch_forward<float>(a, o);
 }
 
@@ -608,7 +624,16 @@ ssm_status_t ssm_selective_scan_fwd(const void* u, const void* delta, const floa
 ssm_status_t ssm_state_update(float* state, const void* u, const void* delta, const float* A, const void* B,
                               const void* C, const float* D, const void* z, const float* delta_bias, int softplus,
                               void* y, int batch, int dim, int dstate, ssm_dtype_t io_dtype, ssm_stream_t stream) {
+    return ssm_state_update_ex(state, u, delta, A, B, C, D, z, delta_bias, softplus, y, batch, dim, dstate, io_dtype,
+                               SSM_DISC_SIMPLIFIED, stream);
+}
+
+ssm_status_t ssm_state_update_ex(float* state, const void* u, const void* delta, const float* A, const void* B,
+                                 const void* C, const float* D, const void* z, const float* delta_bias, int softplus,
+                                 void* y, int batch, int dim, int dstate, ssm_dtype_t io_dtype,
+                                 ssm_discretization_t discretization, ssm_stream_t stream) {
     if (batch < 0 || dim < 0) return SSM_ERR_INVALID_ARG;
+    if (discretization != SSM_DISC_SIMPLIFIED && discretization != SSM_DISC_ZOH) return SSM_ERR_INVALID_ARG;
     if (batch > 0 && dim > 0 && (!state || !u || !delta || !A || !B || !C || !y)) return SSM_ERR_INVALID_ARG;
     if (io_dtype != SSM_F32 && io_dtype != SSM_BF16) return SSM_ERR_INVALID_ARG;
     if (dstate != 16) return SSM_ERR_UNSUPPORTED;
@@ -616,7 +641,8 @@ ssm_status_t ssm_state_update(float* state, const void* u, const void* delta, co
     if (batch == 0 || dim == 0) return SSM_OK;
     ssm_status_t st = check_device(nullptr);
     if (st != SSM_OK) return st;
-    ssm::DecodeParams p{state, u, delta, A, B, C, D, z, delta_bias, y, batch, dim, softplus};
+    ssm::DecodeParams p{state, u, delta, A, B, C, D, z, delta_bias, y, batch, dim, softplus,
+                        discretization == SSM_DISC_ZOH};
     const long long threads = static_cast<long long>(batch) * dim * 4;
     const long long grid = (threads + 255) / 256;
     if (grid > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
@@ -660,9 +686,9 @@ ssm_status_t ssm_selective_scan_fwd_noalloc(const void* u, const void* delta, co
     // The header (status word) starts every call at zero; the B/C rows are rewritten in full.
     if (cudaMemsetAsync(scratch, 0, sizeof(WorkspaceHeader), s) != cudaSuccess) return SSM_ERR_LAUNCH;
     // Kernels whose scratch is only the header and the B/C rows (no look-back flags).
-    const ssm_fwd_options_t o{SSM_ALGO_SEQUENTIAL, 0, 0, -1};
-    FwdArgs a{u, delta, B, C, z, A, D, delta_bias, softplus, nullptr, y, last_state, batch, dim, seqlen, io_dtype,
-              scratch, s, sm_count};
+    const ssm_fwd_options_t o{SSM_ALGO_SEQUENTIAL, 0, 0, -1, SSM_DISC_SIMPLIFIED};
+    FwdArgs a{u, delta, B, C, z, A, D, delta_bias, softplus, nullptr, 0, y, last_state, batch, dim, seqlen,
+              io_dtype, scratch, s, sm_count};
     return io_dtype == SSM_BF16 ? launch_forward<__nv_bfloat16>(a, o) : launch_forward<float>(a, o);
 }
 

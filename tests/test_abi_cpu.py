@@ -41,7 +41,7 @@ def test_header_declares_entry_points():
 def test_library_exports_every_declared_symbol(lib):
     missing = [n for n in _declared_functions() if not hasattr(lib, n)]
     assert not missing, missing
-    assert lib.ssm_abi_version() == 1
+    assert lib.ssm_abi_version() == 2
 
 
 def test_status_strings(lib):
@@ -86,7 +86,7 @@ def test_forward_argument_validation(lib):
 
 
 def test_forward_ex_rejects_unknown_algo(lib):
-    opts = binding.FwdOptions(99, 0, 0, -1)
+    opts = binding.FwdOptions(99, 0, 0, -1, 0)
     rc = lib.ssm_selective_scan_fwd_ex(P(4096), P(4096), P(4096), P(4096), P(4096), None, None, None, 1,
                                        P(4096), None, 1, 1, 16, 8, binding.SSM_BF16, P(4096), 1 << 20,
                                        ctypes.byref(opts), None)
@@ -117,6 +117,8 @@ def test_decode_argument_validation(lib):
     assert call(dstate=32) == binding.SSM_ERR_UNSUPPORTED
     assert call(io=3) == binding.SSM_ERR_INVALID_ARG
     assert call(batch=0) == binding.SSM_OK
+    assert lib.ssm_state_update_ex(P(4096), P(4096), P(4096), P(4096), P(4096), P(4096), None, None, None, 1,
+                                   P(4096), 2, 3, 16, binding.SSM_F32, 5, None) == binding.SSM_ERR_INVALID_ARG
 
 
 def test_read_status_needs_workspace(lib):
