@@ -32,7 +32,10 @@
  *   - Calls are asynchronous on `stream`; errors found before the launch are
  *     returned; errors found on the device (a look-back wait that ran out) are
  *     recorded in the workspace status word and read back by ssm_read_status().
- *   - dstate must be 16 (SSM_ERR_UNSUPPORTED otherwise).
+ *   - dstate: the forward scan and decode take 16 (the tuned kernels) or 32, 64, 128, 256 (one
+ *     warp per channel; bound by the exponential unit, N per element).  The backward, the
+ *     chunked kernel and the no-allocation entry point take 16 only.  Other values return
+ *     SSM_ERR_UNSUPPORTED.
  *   - Inputs are never modified, except `state` in ssm_state_update().
  *   - A pointer to a tensor with zero elements (e.g. u when seqlen == 0) may be NULL.
  */
@@ -52,7 +55,7 @@ typedef struct CUstream_st* ssm_stream_t;
 typedef enum {
     SSM_OK = 0,
     SSM_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad dtype, misaligned pointer    */
-    SSM_ERR_UNSUPPORTED = 2,   /* dstate != 16, or the current device is not sm_100             */
+    SSM_ERR_UNSUPPORTED = 2,   /* dstate not supported by the call, or the device is not sm_100 */
     SSM_ERR_LAUNCH = 3,        /* a CUDA call or kernel launch failed                           */
     SSM_ERR_TIMEOUT = 4,       /* device: a bounded wait in the kernel gave up (see read_status) */
     SSM_ERR_WORKSPACE = 5,     /* workspace missing or smaller than ssm_selective_scan_workspace_size */
@@ -70,7 +73,7 @@ const char* ssm_status_string(ssm_status_t status);
 /*
  * Bytes of device workspace ssm_selective_scan_fwd needs for these sizes (a multiple
  * of 256).  The workspace holds a transposed fp32 copy of B and C, the status word
- * and the flags and (prod Abar, h) pairs of the inter-CTA chunk carry.
+ * and (dstate 16) the flags and (prod Abar, h) pairs of the inter-CTA chunk carry.
  * Returns 0 for invalid sizes.
  */
 size_t ssm_selective_scan_workspace_size(int batch, int dim, int dstate, int64_t seqlen);

@@ -18,6 +18,7 @@
 #include "scan_fwd_chunked.cuh"
 #include "scan_fwd_seq.cuh"
 #include "scan_bwd.cuh"
+#include "scan_fwd_wide.cuh"
 
 namespace {
 
@@ -28,6 +29,10 @@ constexpr uint32_t kDefaultWaitLimit = 1u << 22;
 constexpr uint32_t kDefaultSpinLimit = 1u << 21;  // look-back polls (~64 ns sleep each)
 
 size_t round_up(size_t v, size_t m) { return (v + m - 1) / m * m; }
+
+// d_state values of the forward scan and decode: 16 (the tuned kernels) and the wider states
+// of scan_fwd_wide.cuh.
+bool dstate_supported(int n) { return n == 16 || n == 32 || n == 64 || n == 128 || n == 256; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -401,6 +406,56 @@ ssm_status_t launch_forward(const FwdArgs& a, const ssm_fwd_options_t& o) {
     return SSM_ERR_INVALID_ARG;
 }
 
+// ------------------------------------------------------------------ wider states
+template <typename IO, int N>
+ssm_status_t launch_wide_n(const FwdArgs& a) {
+    float* bc = reinterpret_cast<float*>(a.ws + sizeof(WorkspaceHeader));
+    const dim3 pgrid(static_cast<unsigned>((a.L + 31) / 32), static_cast<unsigned>(a.batch), 2 * N / 32);
+    ssm::pack_bc_wide_kernel<IO><<<pgrid, dim3(32, 8), 0, a.stream>>>(static_cast<const IO*>(a.B),
+                                                                    static_cast<const IO*>(a.C), bc, a.L, N);
+    if (cudaGetLastError() != cudaSuccess) return SSM_ERR_LAUNCH;
+    ssm::WideParams p{};
+    p.u = a.u;
+    p.delta = a.delta;
+    p.z = a.z;
+    p.bc = bc;
+    p.A = a.A;
+    p.D = a.D;
+    p.bias = a.bias;
+    p.h0 = a.h0;
+    p.y = a.y;
+    p.last_state = a.last_state;
+    p.batch = a.batch;
+    p.dim = a.dim;
+    p.L = a.L;
+    p.softplus = a.softplus;
+    p.zoh = a.zoh;
+    constexpr int cpb = 8 * ssm::WideCfg<N>::kCPW;  // channels per block of 8 warps
+    const long long grid = (static_cast<long long>(a.batch) * a.dim + cpb - 1) / cpb;
+    if (grid > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
+    ssm::scan_fwd_wide_kernel<IO, N><<<static_cast<unsigned>(grid), 256, 0, a.stream>>>(p);
+    return launch_status();
+}
+
+template <typename IO>
+ssm_status_t launch_wide(const FwdArgs& a, int n) {
+    switch (n) {
+        case 32: return launch_wide_n<IO, 32>(a);
+        case 64: return launch_wide_n<IO, 64>(a);
+        case 128: return launch_wide_n<IO, 128>(a);
+        case 256: return launch_wide_n<IO, 256>(a);
+    }
+    return SSM_ERR_UNSUPPORTED;
+}
+
+template <typename IO, int N>
+void launch_decode_wide(float* state, const void* u, const void* delta, const float* A, const void* B, const void* C,
+                        const float* D, const void* z, const float* bias, int softplus, void* y, int batch, int dim,
+                        int zoh, unsigned grid, cudaStream_t s) {
+    ssm::state_update_wide_kernel<IO, N><<<grid, 256, 0, s>>>(A, D, bias, state, u, delta, B, C, z, y, batch, dim,
+                                                             softplus, zoh);
+}
+
 // ------------------------------------------------------------------ backward
 // Backward workspace layout:
 //   [header 256 B][B/C fp32 rows: batch * L * 128 B][checkpoints: batch * nseg * dim * 64 B]
@@ -541,7 +596,10 @@ const char* ssm_status_string(ssm_status_t s) {
 }
 
 size_t ssm_selective_scan_workspace_size(int batch, int dim, int dstate, int64_t seqlen) {
-    if (batch < 0 || dim < 0 || dstate != 16 || seqlen < 0) return 0;
+    if (batch < 0 || dim < 0 || !dstate_supported(dstate) || seqlen < 0) return 0;
+    if (dstate != 16)  // header + B/C rows of 2 * dstate fp32 per step
+        return sizeof(WorkspaceHeader) +
+               round_up(static_cast<size_t>(batch) * static_cast<size_t>(seqlen) * 8u * dstate, 256);
     return round_up(ws_layout(batch, dim, seqlen).total, 256);
 }
 
@@ -564,11 +622,11 @@ ssm_status_t ssm_selective_scan_fwd_state(const void* u, const void* delta, cons
     if (seq_elems && (!u || !delta || !B || !C || !y)) return SSM_ERR_INVALID_ARG;
     if (dim > 0 && !A) return SSM_ERR_INVALID_ARG;
     if (io_dtype != SSM_F32 && io_dtype != SSM_BF16) return SSM_ERR_INVALID_ARG;
-    if (dstate != 16) return SSM_ERR_UNSUPPORTED;
+    if (!dstate_supported(dstate)) return SSM_ERR_UNSUPPORTED;
     const void* ptrs[] = {u, delta, A, B, C, D, z, delta_bias, initial_state, y, last_state};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return SSM_ERR_INVALID_ARG;
-    const size_t state_bytes = static_cast<size_t>(batch) * static_cast<size_t>(dim) * 16u * sizeof(float);
+    const size_t state_bytes = static_cast<size_t>(batch) * static_cast<size_t>(dim) * dstate * sizeof(float);
     if (initial_state && last_state && state_bytes > 0) {
         // The chunked kernel may still read a channel's initial state after another CTA
         // has written that channel's final state, so the two must not overlap.
@@ -600,6 +658,10 @@ ssm_status_t ssm_selective_scan_fwd_state(const void* u, const void* delta, cons
     }
     FwdArgs a{u, delta, B, C, z, A, D, delta_bias, softplus, initial_state, o.discretization == SSM_DISC_ZOH, y,
               last_state, batch, dim, seqlen, io_dtype, static_cast<uint8_t*>(workspace), s, sm_count};
+    if (dstate != 16) {
+        if (o.algo == SSM_ALGO_CHUNKED) return SSM_ERR_UNSUPPORTED;  // d_state 16 only
+        return io_dtype == SSM_BF16 ? launch_wide<__nv_bfloat16>(a, dstate) : launch_wide<float>(a, dstate);
+    }
     return io_dtype == SSM_BF16 ? launch_forward<__nv_bfloat16>(a, o) : launch_forward<float>(a, o);
 }
 
@@ -636,11 +698,34 @@ ssm_status_t ssm_state_update_ex(float* state, const void* u, const void* delta,
     if (discretization != SSM_DISC_SIMPLIFIED && discretization != SSM_DISC_ZOH) return SSM_ERR_INVALID_ARG;
     if (batch > 0 && dim > 0 && (!state || !u || !delta || !A || !B || !C || !y)) return SSM_ERR_INVALID_ARG;
     if (io_dtype != SSM_F32 && io_dtype != SSM_BF16) return SSM_ERR_INVALID_ARG;
-    if (dstate != 16) return SSM_ERR_UNSUPPORTED;
+    if (!dstate_supported(dstate)) return SSM_ERR_UNSUPPORTED;
     if (!aligned16(state) || !aligned16(A)) return SSM_ERR_INVALID_ARG;
     if (batch == 0 || dim == 0) return SSM_OK;
     ssm_status_t st = check_device(nullptr);
     if (st != SSM_OK) return st;
+    if (dstate != 16) {
+        const int tpc = std::min(dstate / 4, 32);  // threads per channel
+        const long long threads = static_cast<long long>(batch) * dim * tpc;
+        const long long grid = (threads + 255) / 256;
+        if (grid > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
+        cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+        const int zoh = discretization == SSM_DISC_ZOH;
+        const unsigned g = static_cast<unsigned>(grid);
+#define SSM_DECODE_WIDE(IO_T)                                                                                        \
+    switch (dstate) {                                                                                                \
+        case 32: launch_decode_wide<IO_T, 32>(state, u, delta, A, B, C, D, z, delta_bias, softplus, y, batch, dim, zoh, g, s); break; \
+        case 64: launch_decode_wide<IO_T, 64>(state, u, delta, A, B, C, D, z, delta_bias, softplus, y, batch, dim, zoh, g, s); break; \
+        case 128: launch_decode_wide<IO_T, 128>(state, u, delta, A, B, C, D, z, delta_bias, softplus, y, batch, dim, zoh, g, s); break; \
+        default: launch_decode_wide<IO_T, 256>(state, u, delta, A, B, C, D, z, delta_bias, softplus, y, batch, dim, zoh, g, s); break; \
+    }
+        if (io_dtype == SSM_BF16) {
+            SSM_DECODE_WIDE(__nv_bfloat16)
+        } else {
+            SSM_DECODE_WIDE(float)
+        }
+#undef SSM_DECODE_WIDE
+        return launch_status();
+    }
     ssm::DecodeParams p{state, u, delta, A, B, C, D, z, delta_bias, y, batch, dim, softplus,
                         discretization == SSM_DISC_ZOH};
     const long long threads = static_cast<long long>(batch) * dim * 4;

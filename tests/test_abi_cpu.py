@@ -54,7 +54,9 @@ def test_workspace_size(lib):
     f = binding.ssm_selective_scan_workspace_size
     assert f(4, 5120, 16, 2048) % 256 == 0
     assert f(4, 5120, 16, 2048) >= 256 + 4 * 2048 * 128   # header + fp32 B/C rows
-    assert f(4, 5120, 8, 2048) == 0                      # dstate != 16
+    assert f(4, 5120, 8, 2048) == 0                      # dstate not supported
+    assert f(2, 64, 128, 100) >= 256 + 2 * 100 * 8 * 128 # wider state: B/C rows of 2N fp32
+    assert f(2, 64, 48, 100) == 0
     assert f(-1, 5, 16, 5) == 0
 
 
@@ -76,6 +78,7 @@ def test_forward_argument_validation(lib):
     assert _fwd(lib, L=-3) == binding.SSM_ERR_INVALID_ARG
     assert _fwd(lib, io=7) == binding.SSM_ERR_INVALID_ARG
     assert _fwd(lib, dstate=8) == binding.SSM_ERR_UNSUPPORTED
+    assert _fwd(lib, dstate=48) == binding.SSM_ERR_UNSUPPORTED
     assert _fwd(lib, u=P(4098)) == binding.SSM_ERR_INVALID_ARG      # not 16-byte aligned
     assert _fwd(lib, z=P(4100)) == binding.SSM_ERR_INVALID_ARG
     assert _fwd(lib, batch=0) == binding.SSM_OK                      # empty: nothing launched
@@ -114,7 +117,7 @@ def test_decode_argument_validation(lib):
         return lib.ssm_state_update(*a.values())
     assert call(state=None) == binding.SSM_ERR_INVALID_ARG
     assert call(state=P(4100)) == binding.SSM_ERR_INVALID_ARG
-    assert call(dstate=32) == binding.SSM_ERR_UNSUPPORTED
+    assert call(dstate=24) == binding.SSM_ERR_UNSUPPORTED
     assert call(io=3) == binding.SSM_ERR_INVALID_ARG
     assert call(batch=0) == binding.SSM_OK
     assert lib.ssm_state_update_ex(P(4096), P(4096), P(4096), P(4096), P(4096), P(4096), None, None, None, 1,
