@@ -51,6 +51,8 @@ def _load():
             lib.oracle_state_update_zoh_f64.restype = ci
             lib.oracle_selective_scan_bwd_f64.argtypes = [vp] * 8 + [ci] + [vp] * 12 + [i64, i64, i64, i64]
             lib.oracle_selective_scan_bwd_f64.restype = ci
+            lib.oracle_causal_conv_silu_f64.argtypes = [vp] * 6 + [i64, i64, i64, i64]
+            lib.oracle_causal_conv_silu_f64.restype = ci
             lib.oracle_num_threads.restype = ci
             lib.oracle_softplus_f64.argtypes = [ctypes.c_double]
             lib.oracle_softplus_f64.restype = ctypes.c_double
@@ -146,3 +148,20 @@ def selective_scan_bwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
     if rc != 0:
         raise ValueError("oracle_selective_scan_bwd_f64 rejected its arguments")
     return out
+
+
+def causal_conv_silu(x, w, bias=None, x_prev=None):
+    """u = silu(causal depthwise conv of x with w (dim, K) + bias), inputs before t = 0 taken
+    from x_prev (batch, dim, K-1) or zero.  Returns (u (b, d, L), x_next (b, d, K-1)): the
+    output and the last K-1 inputs (the state that continues the convolution)."""
+    x, w, bias, x_prev = map(_f64, (x, w, bias, x_prev))
+    b, d, L = x.shape
+    K = w.shape[1]
+    assert w.shape == (d, K) and (x_prev is None or x_prev.shape == (b, d, K - 1))
+    u = np.empty((b, d, L))
+    x_next = np.empty((b, d, max(K - 1, 0)))
+    rc = _load().oracle_causal_conv_silu_f64(_ptr(x), _ptr(w), _ptr(bias), _ptr(x_prev), _ptr(u),
+                                             _ptr(x_next) if K > 1 else None, b, d, L, K)
+    if rc != 0:
+        raise ValueError("oracle_causal_conv_silu_f64 rejected its arguments")
+    return u, x_next

@@ -368,6 +368,46 @@ int oracle_selective_scan_bwd_f64(const double* u, const double* delta, const do
     return fail ? -1 : 0;
 }
 
+/*
+ * Causal depthwise convolution of width K along t, then SiLU: the local-feature step before
+ * the scan in the Mamba block ([Hist] Mamba Block 数据流: x -> 1D conv -> SiLU -> S6;
+ * [Card] Mamba架构设计):
+ *   u[b,d,t] = silu( bias[d] + sum_{k=0}^{K-1} w[d,k] * x[b,d,t-(K-1)+k] )
+ * where inputs before t = 0 are x_prev[b,d,0..K-2] (oldest first) when given, else zero.
+ * x: (batch, dim, L); w: (dim, K); bias: (dim) or NULL; x_prev: (batch, dim, K-1) or NULL;
+ * u: (batch, dim, L) output.  When x_next is given it receives the last K-1 inputs seen
+ * (the state that continues the convolution).  Returns 0, or -1 on a bad argument.
+ */
+int oracle_causal_conv_silu_f64(const double* x, const double* w, const double* bias, const double* x_prev,
+                                double* u, double* x_next, int64_t batch, int64_t dim, int64_t L, int64_t K)
+{
+    if (batch < 0 || dim < 0 || L < 0 || K < 1 || K > 16 || !x || !w || !u) return -1;
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t d = 0; d < dim; ++d) {
+            const int64_t row = b * dim + d;
+            for (int64_t t = 0; t < L; ++t) {
+                double acc = bias ? bias[d] : 0.0;
+                for (int64_t k = 0; k < K; ++k) {
+                    const int64_t s = t - (K - 1) + k;  /* input index, may be negative */
+                    double xv = 0.0;
+                    if (s >= 0) xv = x[row * L + s];
+                    else if (x_prev) xv = x_prev[row * (K - 1) + (K - 1 + s)];
+                    acc += w[d * K + k] * xv;
+                }
+                u[row * L + t] = silu_f64(acc);
+            }
+            if (x_next)
+                for (int64_t j = 0; j < K - 1; ++j) {
+                    const int64_t s = L - (K - 1) + j;
+                    x_next[row * (K - 1) + j] =
+                        s >= 0 ? x[row * L + s] : (x_prev ? x_prev[row * (K - 1) + (K - 1 + s)] : 0.0);
+                }
+        }
+    }
+    return 0;
+}
+
 /* Number of OpenMP threads the oracle will use (reported beside CPU timings). */
 int oracle_num_threads(void)
 {

@@ -479,3 +479,40 @@ def test_zoh_decode_chain_equals_scan():
                                         delta_bias=case["delta_bias"], softplus=case["softplus"], zoh=True)
         np.testing.assert_allclose(yt, y[..., t], rtol=1e-12, atol=1e-13)
     np.testing.assert_allclose(state, last, rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------------------------
+# Causal depthwise conv1d + SiLU before the scan ([Hist] Mamba Block 数据流): against
+# numpy.convolve per channel and scipy's expit, with and without a carried-in state.
+# ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("K", [1, 2, 4])
+def test_causal_conv_matches_numpy_convolve(K):
+    from scipy.special import expit
+    rng = _rng(70 + K)
+    b, d, L = 2, 3, 11
+    x = rng.standard_normal((b, d, L))
+    w = rng.standard_normal((d, K))
+    bias = rng.standard_normal(d)
+    prev = rng.standard_normal((b, d, K - 1))
+    for with_prev in (False, True):
+        u, x_next = oracle.causal_conv_silu(x, w, bias, prev if with_prev else None)
+        for bi in range(b):
+            for di in range(d):
+                head = prev[bi, di] if with_prev else np.zeros(K - 1)
+                full = np.concatenate([head, x[bi, di]])
+                # causal: output t uses full[t .. t+K-1] with w in order (oldest first)
+                conv = np.convolve(full, w[di][::-1], mode="valid")
+                pre = conv + bias[di]
+                np.testing.assert_allclose(u[bi, di], pre * expit(pre), rtol=1e-13, atol=1e-14)
+                np.testing.assert_array_equal(x_next[bi, di], full[len(full) - (K - 1):] if K > 1 else [])
+
+
+def test_causal_conv_continuation():
+    # converting [0, L1) then [L1, L) with the carried-in inputs equals converting [0, L)
+    rng = _rng(75)
+    x = rng.standard_normal((2, 3, 13))
+    w = rng.standard_normal((3, 4))
+    u, _ = oracle.causal_conv_silu(x, w)
+    u1, s1 = oracle.causal_conv_silu(x[..., :5], w)
+    u2, _ = oracle.causal_conv_silu(x[..., 5:], w, x_prev=s1)
+    np.testing.assert_allclose(np.concatenate([u1, u2], axis=2), u, rtol=1e-14, atol=1e-15)
