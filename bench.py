@@ -366,6 +366,34 @@ def measure_zoh(ssm, stream, pk, steps=10):
             "unit": UNIT, "ms_per_step": ms}
 
 
+def measure_conv(ssm, stream, pk, steps=10):
+    """Headline workload scanned from x through the fused causal conv1d (width 4) + SiLU."""
+    w = workloads.WORKLOADS[workloads.HEADLINE]
+    _, g = forward_buffers(w, "cuda")
+    conv = {k: (v.cuda() if v is not None else None) for k, v in workloads.conv_inputs(w.batch, w.dim, 4, seed=5).items()}
+    ws = ssm.new_workspace(w.batch, w.dim, w.dstate, w.seqlen)
+
+    def call():
+        ssm.ssm_selective_scan_fwd_conv(g["u"], conv["conv_weight"], conv["conv_bias"], g["delta"], g["A"], g["B"],
+                                        g["C"], g["D"], g["z"], g["delta_bias"], True, g["y"], g["last"], ws,
+                                        stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(steps):
+            call()
+        ev1.record(stream)
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1) / steps
+    del g
+    return {"workload": w.name, "prologue": "causal conv1d width 4 + SiLU, fused", "value": w.elements / (ms / 1e3) / 1e9,
+            "unit": UNIT, "ms_per_step": ms}
+
+
 def measure_backward(ssm, stream, pk, steps=5):
     """Backward of the headline workload (gradients of every input for a seeded N(0, 1) dy),
     timed with CUDA events on the launching stream; inputs larger than L2."""
@@ -536,7 +564,8 @@ def run_gpu(args, world, rank, local):
         line["e2e"] = e2e_forward(ssm, w, inp, ws, e2e_steps, stream)
     if world == 1 and not args.skip_extra:
         line["also"] = {"long": measure_long(ssm, stream, pk), "decode": measure_decode(ssm, stream, pk),
-                        "backward": measure_backward(ssm, stream, pk), "zoh": measure_zoh(ssm, stream, pk)}
+                        "backward": measure_backward(ssm, stream, pk), "zoh": measure_zoh(ssm, stream, pk),
+                        "conv": measure_conv(ssm, stream, pk)}
     if rank == 0 and world == 1 and not args.skip_cpu:
         rate, secs, desc, cores = cpu_oracle_rate(w, args.cpu_budget)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}

@@ -170,6 +170,37 @@ ssm_status_t ssm_selective_scan_fwd_state(
     void* workspace, size_t workspace_bytes, const ssm_fwd_options_t* opts, ssm_stream_t stream);
 
 /*
+ * Causal depthwise conv1d + SiLU in front of the scan: the local-feature step of the Mamba
+ * block's x branch ([Hist] Mamba Block 数据流: x -> 1D conv -> SiLU -> S6; [Card] Mamba架构设计),
+ *   u[b,d,t] = silu( bias[d] + sum_{k<width} weight[d,k] * x[b,d,t-width+1+k] ),
+ * with the inputs before t = 0 taken from state_in (zeros if NULL).
+ */
+typedef struct {
+    const float* weight;    /* (dim, width) fp32, oldest tap first; required                       */
+    const float* bias;      /* (dim) fp32, or NULL (0)                                              */
+    int width;              /* 1 .. 4                                                               */
+    const float* state_in;  /* (batch, dim, width-1) fp32 inputs before t = 0, oldest first, or NULL */
+    float* state_out;       /* (batch, dim, width-1) fp32: the last width-1 inputs, or NULL; it may
+                               be the same buffer as state_in (each channel reads its state before
+                               writing it)                                                          */
+    void* u_out;            /* io_dtype (batch, dim, seqlen): u as fed to the scan, or NULL         */
+} ssm_conv_t;
+
+/*
+ * Forward scan of u = silu(conv(x)) computed on the fly from x (io_dtype, (batch, dim,
+ * seqlen), in place of u): the staged x tile is converted in shared memory, so u never makes
+ * a round trip through HBM unless u_out asks for it.  u is rounded to io_dtype before the
+ * scan (as a separate conv kernel storing u would).  Every other argument as
+ * ssm_selective_scan_fwd_state.  d_state 16 only; SSM_ALGO_CHUNKED returns SSM_ERR_UNSUPPORTED.
+ */
+ssm_status_t ssm_selective_scan_fwd_conv(
+    const void* x, const ssm_conv_t* conv, const void* delta, const float* A, const void* B, const void* C,
+    const float* D, const void* z, const float* delta_bias, int softplus,
+    const float* initial_state, void* y, float* last_state,
+    int batch, int dim, int dstate, int64_t seqlen, ssm_dtype_t io_dtype,
+    void* workspace, size_t workspace_bytes, const ssm_fwd_options_t* opts, ssm_stream_t stream);
+
+/*
  * Backward of the forward scan: the gradients of a loss L with respect to every input,
  * given dy = dL/dy and optionally dlast_state = dL/d last_state.  The forward is
  * recomputed rather than stored ([Tech] 四.1: keep little in the forward pass and
@@ -221,6 +252,19 @@ ssm_status_t ssm_state_update(
     float* state, const void* u, const void* delta, const float* A, const void* B, const void* C,
     const float* D, const void* z, const float* delta_bias, int softplus, void* y,
     int batch, int dim, int dstate, ssm_dtype_t io_dtype, ssm_stream_t stream);
+
+/*
+ * One decode step with the conv prologue: u = silu(conv_bias + sum_k conv_weight[d,k] *
+ * [conv_state, x]_k) (rounded to io_dtype), then the step of ssm_state_update_ex with u;
+ * conv_state (batch, dim, conv_width-1) fp32, oldest first, is shifted in place to end with x.
+ * conv_width 0 means no conv (x is u).  d_state 16 with a conv.
+ */
+ssm_status_t ssm_state_update_conv(
+    float* state, float* conv_state, const void* x, const float* conv_weight, const float* conv_bias,
+    int conv_width, const void* delta, const float* A, const void* B, const void* C,
+    const float* D, const void* z, const float* delta_bias, int softplus, void* y,
+    int batch, int dim, int dstate, ssm_dtype_t io_dtype, ssm_discretization_t discretization,
+    ssm_stream_t stream);
 
 /* ssm_state_update with an explicit discretisation (ssm_discretization_t). */
 ssm_status_t ssm_state_update_ex(

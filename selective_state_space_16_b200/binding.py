@@ -41,6 +41,12 @@ class FwdOptions(ctypes.Structure):
                 ("discretization", ctypes.c_int)]
 
 
+class ConvSpec(ctypes.Structure):
+    """ssm_conv_t: causal conv1d + SiLU in front of the scan."""
+    _fields_ = [("weight", ctypes.c_void_p), ("bias", ctypes.c_void_p), ("width", ctypes.c_int),
+                ("state_in", ctypes.c_void_p), ("state_out", ctypes.c_void_p), ("u_out", ctypes.c_void_p)]
+
+
 _lib = None
 _lock = threading.Lock()
 
@@ -78,6 +84,12 @@ def load() -> ctypes.CDLL:
             lib.ssm_state_update.restype = ci
             lib.ssm_state_update_ex.argtypes = [vp] * 9 + [ci, vp, ci, ci, ci, ci, ci, vp]
             lib.ssm_state_update_ex.restype = ci
+            lib.ssm_state_update_conv.argtypes = [vp] * 5 + [ci] + [vp] * 7 + [ci, vp, ci, ci, ci, ci, ci, vp]
+            lib.ssm_state_update_conv.restype = ci
+            lib.ssm_selective_scan_fwd_conv.argtypes = ([vp, ctypes.POINTER(ConvSpec)] + [vp] * 7 + [ci] +
+                                                        [vp] * 3 + [ci, ci, ci, i64, ci, vp, sz,
+                                                                    ctypes.POINTER(FwdOptions), vp])
+            lib.ssm_selective_scan_fwd_conv.restype = ci
             lib.ssm_read_status.argtypes = [vp, vp]
             lib.ssm_read_status.restype = ci
             _lib = lib
@@ -215,6 +227,40 @@ def selective_scan_bwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
                            initial_state=initial_state, dlast_state=dlast_state,
                            dinitial_state=out["dinitial_state"], stream=stream)
     return out
+
+
+def ssm_selective_scan_fwd_conv(x, conv_weight, conv_bias, delta, A, B, C, D, z, delta_bias, softplus, y, last_state,
+                                workspace, conv_state_in=None, conv_state_out=None, u_out=None, initial_state=None,
+                                stream=None, algo=None, lanes_per_channel=0, zoh=False, check=True):
+    """Marshal a forward scan of u = silu(causal conv(x)): x (b, d, L) in the I/O dtype;
+    conv_weight (d, K) fp32; conv_bias (d) fp32 or None; conv_state_in/out (b, d, K-1) fp32 or
+    None; u_out (b, d, L) I/O dtype or None."""
+    b, d, L = x.shape
+    n = A.shape[1]
+    spec = ConvSpec(_ptr(conv_weight), _ptr(conv_bias), int(conv_weight.shape[1]), _ptr(conv_state_in),
+                    _ptr(conv_state_out), _ptr(u_out))
+    a = ALGOS[algo] if isinstance(algo, str) else (algo or SSM_ALGO_AUTO)
+    opts = FwdOptions(a, lanes_per_channel, 0, -1, SSM_DISC_ZOH if zoh else SSM_DISC_SIMPLIFIED)
+    code = load().ssm_selective_scan_fwd_conv(
+        _ptr(x), ctypes.byref(spec), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+        int(bool(softplus)), _ptr(initial_state), _ptr(y), _ptr(last_state), b, d, n, L, _io(x), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), ctypes.byref(opts), _stream(stream))
+    if check:
+        _check(code, "ssm_selective_scan_fwd_conv")
+    return code
+
+
+def ssm_state_update_conv(state, conv_state, x, conv_weight, conv_bias, delta, A, B, C, D, z, delta_bias, softplus,
+                          y, zoh=False, stream=None, check=True):
+    """Marshal a decode step with the conv prologue: conv_state (b, d, K-1) fp32 in/out."""
+    b, d, n = state.shape
+    code = load().ssm_state_update_conv(
+        _ptr(state), _ptr(conv_state), _ptr(x), _ptr(conv_weight), _ptr(conv_bias), int(conv_weight.shape[1]),
+        _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias), int(bool(softplus)), _ptr(y),
+        b, d, n, _io(x), SSM_DISC_ZOH if zoh else SSM_DISC_SIMPLIFIED, _stream(stream))
+    if check:
+        _check(code, "ssm_state_update_conv")
+    return code
 
 
 def ssm_state_update(state, u, delta, A, B, C, D, z, delta_bias, softplus, y, stream=None, check=True, zoh=False):

@@ -59,6 +59,13 @@ struct DirectParams {
     long long L;
     int softplus;
     int zoh;  // zero-order-hold input weight instead of Delta*B
+    // causal conv1d + SiLU prologue (conv_k > 0): u = silu(conv(x)), x given in `u`
+    const float* conv_w;   // (dim, conv_k), oldest tap first
+    const float* conv_b;   // (dim) or null
+    const float* conv_in;  // (batch, dim, conv_k - 1) or null
+    float* conv_out;       // (batch, dim, conv_k - 1) or null
+    void* u_out;           // (batch, dim, L) IO or null
+    int conv_k;            // 0: no conv
 };
 
 template <typename IO, int G>
@@ -87,12 +94,30 @@ __global__ void __launch_bounds__(128) scan_fwd_direct_kernel(const DirectParams
     }
     const float Dd = (valid && p.D) ? p.D[d] : 0.f;
     const float bias = (valid && p.bias) ? p.bias[d] : 0.f;
+    // conv prologue: taps right-aligned in cw, the last three inputs in xh (oldest first)
+    const int K = p.conv_k;
+    float cw[4] = {0.f, 0.f, 0.f, 0.f}, xh[3] = {0.f, 0.f, 0.f};
+    const float cb = (K > 0 && valid && p.conv_b) ? p.conv_b[d] : 0.f;
+    if (K > 0 && valid) {
+        for (int k = 0; k < K; ++k) cw[4 - K + k] = p.conv_w[d * K + k];
+        if (p.conv_in)
+            for (int k = 0; k < K - 1; ++k) xh[3 - (K - 1) + k] = p.conv_in[ch * (K - 1) + k];
+    }
 
     for (long long t = 0; t < p.L; ++t) {
         float ut = 0.f, dt = 0.f;
         if (valid) {
             ut = IoTraits<IO>::to_f32(u[t]);
             dt = step_size(IoTraits<IO>::to_f32(dl[t]), bias, p.softplus != 0);
+            if (K > 0) {  // u = silu(conv(x)) rounded to the I/O type, as a separate conv kernel would store it
+                const float xt = ut;
+                const float pre = fmaf(cw[3], xt, fmaf(cw[2], xh[2], fmaf(cw[1], xh[1], fmaf(cw[0], xh[0], cb))));
+                xh[0] = xh[1];
+                xh[1] = xh[2];
+                xh[2] = xt;
+                ut = IoTraits<IO>::to_f32(IoTraits<IO>::from_f32(silu_f32(pre)));
+                if (p.u_out && nl == 0) static_cast<IO*>(p.u_out)[ch * p.L + t] = IoTraits<IO>::from_f32(ut);
+            }
         }
         const float w = dt * ut;
         const float* row = bcb + t * 32;
@@ -119,6 +144,8 @@ __global__ void __launch_bounds__(128) scan_fwd_direct_kernel(const DirectParams
 #pragma unroll
         for (int j = 0; j < NC; ++j) dst[j] = h[j];
     }
+    if (K > 1 && valid && p.conv_out && nl == 0)
+        for (int k = 0; k < K - 1; ++k) p.conv_out[ch * (K - 1) + k] = xh[3 - (K - 1) + k];
 }
 
 // ---------------------------------------------------------------------------------------
@@ -141,6 +168,12 @@ struct DecodeParams {
     int batch, dim;
     int softplus;
     int zoh;  // zero-order-hold input weight instead of Delta*B
+    // causal conv1d + SiLU (conv_k > 0): u = silu(conv([conv_state, x])), x given in `u`;
+    // conv_state (batch, dim, conv_k - 1) fp32, oldest first, shifted in place
+    const float* conv_w;
+    const float* conv_b;
+    float* conv_state;
+    int conv_k;
 };
 
 template <typename IO>
@@ -168,6 +201,13 @@ __global__ void __launch_bounds__(256) state_update_kernel(const DecodeParams p)
             Cq[j] = IoTraits<IO>::to_f32(Cp[j]);
         }
         ut = IoTraits<IO>::to_f32(static_cast<const IO*>(p.u)[rr]);
+        if (p.conv_k > 0) {  // u = silu(conv([conv_state, x])), rounded to the I/O type
+            const int K = p.conv_k;
+            float pre = p.conv_b ? p.conv_b[d] : 0.f;
+            for (int k = 0; k < K - 1; ++k) pre = fmaf(p.conv_w[d * K + k], p.conv_state[rr * (K - 1) + k], pre);
+            pre = fmaf(p.conv_w[d * K + K - 1], ut, pre);
+            ut = IoTraits<IO>::to_f32(IoTraits<IO>::from_f32(silu_f32(pre)));
+        }
         const float bias = p.bias ? p.bias[d] : 0.f;
         dt = step_size(IoTraits<IO>::to_f32(static_cast<const IO*>(p.delta)[rr]), bias, p.softplus != 0);
         if (p.z) zt = IoTraits<IO>::to_f32(static_cast<const IO*>(p.z)[rr]);
@@ -187,6 +227,15 @@ __global__ void __launch_bounds__(256) state_update_kernel(const DecodeParams p)
     }
     acc += __shfl_xor_sync(0xffffffffu, acc, 1, 32);
     acc += __shfl_xor_sync(0xffffffffu, acc, 2, 32);
+    if (p.conv_k > 1) {
+        __syncwarp();  // every thread of the channel has read conv_state
+        if (valid && q == 0) {
+            const int K = p.conv_k;
+            const float xt = IoTraits<IO>::to_f32(static_cast<const IO*>(p.u)[rr]);
+            for (int k = 0; k < K - 2; ++k) p.conv_state[rr * (K - 1) + k] = p.conv_state[rr * (K - 1) + k + 1];
+            p.conv_state[rr * (K - 1) + K - 2] = xt;
+        }
+    }
     if (valid) {
         *reinterpret_cast<float4*>(p.state + rr * 16 + q * 4) = make_float4(hs[0], hs[1], hs[2], hs[3]);
         if (q == 0) {

@@ -56,6 +56,14 @@ struct SeqParams {
     int softplus;
     int has_z;
     uint32_t wait_limit;
+    // causal conv1d + SiLU prologue (CONV kernels): the staged "u" tiles hold x
+    const void* x;             // (batch, dim, L) IO: the conv input
+    const float* conv_w;       // (dim, conv_k) fp32, oldest tap first
+    const float* conv_b;       // (dim) or null
+    const float* conv_in;      // (batch, dim, conv_k - 1) fp32 inputs before t = 0, or null (zero)
+    float* conv_out;           // (batch, dim, conv_k - 1) fp32: the last conv_k - 1 inputs, or null
+    void* u_out;               // (batch, dim, L) IO: the conv output, or null
+    int conv_k;                // 1 .. 4
 };
 
 __host__ __device__ constexpr int round_up_i(int v, int m) { return (v + m - 1) / m * m; }
@@ -113,7 +121,12 @@ __device__ __forceinline__ void load_run(const uint8_t* src, float (&out)[N]) {
 // Store N fp32 values as N consecutive IO elements at a naturally aligned address.
 template <typename IO, int N>
 __device__ __forceinline__ void store_run(IO* dst, const float (&v)[N]) {
-    if constexpr (sizeof(IO) == 2 && N == 4) {
+    if constexpr (sizeof(IO) == 2 && N == 8) {
+        *reinterpret_cast<uint4*>(dst) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                                    pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+    } else if constexpr (sizeof(IO) == 4 && N == 4) {
+        *reinterpret_cast<float4*>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+    } else if constexpr (sizeof(IO) == 2 && N == 4) {
         *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
     } else if constexpr (sizeof(IO) == 2 && N == 2) {
         *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(v[0], v[1]);
@@ -133,8 +146,8 @@ __device__ __forceinline__ void store_run(IO* dst, const float (&v)[N]) {
 // of a stage are unrolled (compile-time shared-memory offsets) with ping-pong step-size
 // buffers: the step sizes of group g+1 (for the last group: group 0 of the next stage,
 // after waiting for it) are computed while group g is scanned.
-template <typename IO, int G, int CPL, int S, bool HZ, bool ZOH>
-__device__ __forceinline__ void seq_consumer(const uint8_t* smem, uint64_t* full_bar, uint64_t* empty_bar,
+template <typename IO, int G, int CPL, int S, bool HZ, bool ZOH, bool CONV>
+__device__ __forceinline__ void seq_consumer(uint8_t* smem, uint64_t* full_bar, uint64_t* empty_bar,
                                              const int* abort_flag, const SeqParams& p, long long r_begin, int nt,
                                              int b_first, int stage_bytes, int nstages, int L32) {
     using Cfg = SeqCfg<IO, G, CPL>;
@@ -187,6 +200,81 @@ __device__ __forceinline__ void seq_consumer(const uint8_t* smem, uint64_t* full
     }
     const bool softplus = p.softplus != 0;
     const uint32_t wait_limit = p.wait_limit;
+
+    // Causal conv1d + SiLU of the staged x tile, in place ([Hist] Mamba Block 数据流: x -> 1D
+    // conv -> SiLU -> S6).  Lane (cg, nl) converts steps nl*SPL .. of its channel cg; the three
+    // inputs before its first step come from lane nl-1 by shuffle (lane 0: from the previous
+    // stage, carried in registers).  u is rounded to the I/O type, as a separate conv kernel
+    // writing u would round it; the scan below then reads u from the tile as usual.
+    constexpr int SPL = TC / G;  // steps per lane
+    static_assert(!CONV || (CPL == 1 && SPL % GS == 0 && SPL >= 3), "conv: one channel per lane");
+    float cw[4] = {0.f, 0.f, 0.f, 0.f}, cb = 0.f, carry[3] = {0.f, 0.f, 0.f};
+    if constexpr (CONV) {
+        const int K = p.conv_k;
+        if (valid[0]) {
+            for (int k = 0; k < K; ++k) cw[4 - K + k] = p.conv_w[static_cast<long long>(d[0]) * K + k];
+            cb = p.conv_b ? p.conv_b[d[0]] : 0.f;
+            if (p.conv_in && nl == 0)
+                for (int k = 0; k < K - 1; ++k)
+                    carry[3 - (K - 1) + k] = p.conv_in[(static_cast<long long>(b) * p.dim + d[0]) * (K - 1) + k];
+        }
+    }
+    auto conv_stage = [&](uint8_t* st, int tk) {
+        if constexpr (CONV) {
+            float xs[SPL];
+#pragma unroll
+            for (int m = 0; m < SPL / GS; ++m)
+                Group16<IO>::unpack(*reinterpret_cast<const uint4*>(st + (cbase[0] ^ ((nl * (SPL / GS) + m) << 4))),
+                                    *reinterpret_cast<float(*)[GS]>(xs + m * GS));
+            // inputs before this lane's first step: the previous lane's last three (lane 0:
+            // the carry); lane 0 keeps the last lane's last three for the next stage
+            float prev[3];
+            const int src = gbase | ((nl + G - 1) & (G - 1));
+#pragma unroll
+            for (int k = 0; k < 3; ++k) {
+                const float got = __shfl_sync(0xffffffffu, xs[SPL - 3 + k], src, 32);
+                prev[k] = nl == 0 ? carry[k] : got;
+                if (nl == 0) carry[k] = got;
+            }
+            float uo[SPL];
+#pragma unroll
+            for (int i = 0; i < SPL; ++i) {
+                float pre = cb;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int j = i - 3 + k;
+                    pre = fmaf(cw[k], j >= 0 ? xs[j] : prev[3 + j], pre);
+                }
+                uo[i] = IoTraits<IO>::to_f32(IoTraits<IO>::from_f32(silu_f32(pre)));
+            }
+#pragma unroll
+            for (int m = 0; m < SPL / GS; ++m) {
+                float v[GS];
+#pragma unroll
+                for (int e = 0; e < GS; ++e) v[e] = uo[m * GS + e];
+                uint8_t* dst = st + (cbase[0] ^ ((nl * (SPL / GS) + m) << 4));
+                store_run<IO, GS>(reinterpret_cast<IO*>(dst), v);
+            }
+            if (p.u_out && valid[0]) {
+                IO* urow = static_cast<IO*>(p.u_out) + (static_cast<long long>(b) * p.dim + d[0]) * p.L;
+                const int t0 = tk + nl * SPL;
+                if (t0 + SPL <= L32) {
+#pragma unroll
+                    for (int m = 0; m < SPL / GS; ++m) {
+                        float v[GS];
+#pragma unroll
+                        for (int e = 0; e < GS; ++e) v[e] = uo[m * GS + e];
+                        store_run<IO, GS>(urow + t0 + m * GS, v);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < SPL; ++i)
+                        if (t0 + i < L32) urow[t0 + i] = IoTraits<IO>::from_f32(uo[i]);
+                }
+            }
+            __syncwarp();
+        }
+    };
 
     // Bounded, warp-uniform wait for ring slot s (a timeout can never leave part of the
     // warp inside the full-mask shuffles).
@@ -305,7 +393,10 @@ __device__ __forceinline__ void seq_consumer(const uint8_t* smem, uint64_t* full
     int slot = 0;
     uint32_t parity = 0;
     bool alive = wait_full(0, 0, 0);
-    if (alive) prologue(st, 0, 0, spA);
+    if (alive) {
+        conv_stage(smem, 0);
+        prologue(st, 0, 0, spA);
+    }
 #pragma unroll 1
     for (int k = 0, tk = 0; alive && k < nstages; ++k, tk += TC) {
 #pragma unroll
@@ -317,7 +408,10 @@ __device__ __forceinline__ void seq_consumer(const uint8_t* smem, uint64_t* full
             } else if (k + 1 < nstages) {
                 const int sn = slot + 1 == S ? 0 : slot + 1;
                 alive = wait_full(sn, slot + 1 == S ? parity ^ 1u : parity, k + 1);
-                if (alive) prologue(smem + sn * stage_bytes, 0, tk + TC, spA);
+                if (alive) {
+                    conv_stage(smem + sn * stage_bytes, tk + TC);
+                    prologue(smem + sn * stage_bytes, 0, tk + TC, spA);
+                }
             }
             scan_group(st, g + 1, tk + (g + 1) * GS, spB);
         }
@@ -331,6 +425,20 @@ __device__ __forceinline__ void seq_consumer(const uint8_t* smem, uint64_t* full
         st = smem + slot * stage_bytes;
     }
 
+    if constexpr (CONV) {
+        // the last conv_k - 1 inputs (from x, or from conv_in when the sequence is shorter)
+        const int K = p.conv_k;
+        if (p.conv_out && valid[0] && nl == 0) {
+            const long long row = static_cast<long long>(b) * p.dim + d[0];
+            for (int k = 0; k < K - 1; ++k) {
+                const long long s2 = static_cast<long long>(L32) - (K - 1) + k;
+                float v = 0.f;
+                if (s2 >= 0) v = IoTraits<IO>::to_f32(static_cast<const IO*>(p.x)[row * p.L + s2]);
+                else if (p.conv_in) v = p.conv_in[row * (K - 1) + (K - 1 + s2)];
+                p.conv_out[row * (K - 1) + k] = v;
+            }
+        }
+    }
 #pragma unroll
     for (int c = 0; c < CPL; ++c)
         if (valid[c] && p.last_state) {
@@ -340,7 +448,7 @@ __device__ __forceinline__ void seq_consumer(const uint8_t* smem, uint64_t* full
         }
 }
 
-template <typename IO, int G, int CPL, int S, bool ZOH = false>
+template <typename IO, int G, int CPL, int S, bool ZOH = false, bool CONV = false>
 __global__ void __launch_bounds__((SeqCfg<IO, G, CPL>::kMaxWarps + 1) * 32, 1)
 scan_fwd_seq_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_dl,
                     const __grid_constant__ CUtensorMap map_z, const __grid_constant__ CUtensorMap map_bc,
@@ -424,11 +532,11 @@ scan_fwd_seq_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_cons
             }
         } else if (warp < nwarps) {
             if (p.has_z)
-                seq_consumer<IO, G, CPL, S, true, ZOH>(smem, full_bar, empty_bar, &abort_flag, p, r_begin, nt,
-                                                       b_first, stage_bytes, nstages, L32);
+                seq_consumer<IO, G, CPL, S, true, ZOH, CONV>(smem, full_bar, empty_bar, &abort_flag, p, r_begin, nt,
+                                                             b_first, stage_bytes, nstages, L32);
             else
-                seq_consumer<IO, G, CPL, S, false, ZOH>(smem, full_bar, empty_bar, &abort_flag, p, r_begin, nt,
-                                                        b_first, stage_bytes, nstages, L32);
+                seq_consumer<IO, G, CPL, S, false, ZOH, CONV>(smem, full_bar, empty_bar, &abort_flag, p, r_begin, nt,
+                                                              b_first, stage_bytes, nstages, L32);
         }
         // Every warp leaves the round before the barriers are re-initialised for the next.
         __syncthreads();

@@ -131,6 +131,14 @@ bool ensure_smem_attr(const void* kernel, int bytes) {
 }
 
 // ------------------------------------------------------------------ forward launches
+// Causal conv1d + SiLU prologue of a forward call (conv_k = 0: none; `u` then holds x).
+struct ConvArgs {
+    const float *w = nullptr, *b = nullptr, *in = nullptr;
+    float* out = nullptr;
+    void* u_out = nullptr;
+    int k = 0;
+};
+
 struct FwdArgs {
     const void *u, *delta, *B, *C, *z;
     const float *A, *D, *bias;
@@ -145,14 +153,15 @@ struct FwdArgs {
     uint8_t* ws;
     cudaStream_t stream;
     int sm_count;
+    ConvArgs conv;
 };
 
-template <typename IO, int G, int CPL, bool ZOH>
+template <typename IO, int G, int CPL, bool ZOH, bool CONV = false>
 const void* seq_kernel_ptr(int stages) {
     switch (stages) {
-        case 2: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 2, ZOH>);
-        case 3: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 3, ZOH>);
-        default: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 4, ZOH>);
+        case 2: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 2, ZOH, CONV>);
+        case 3: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 3, ZOH, CONV>);
+        default: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 4, ZOH, CONV>);
     }
 }
 
@@ -165,7 +174,7 @@ struct SeqPlan {
     bool ok = false;
 };
 
-template <typename IO, int G, int CPL, bool ZOH = false>
+template <typename IO, int G, int CPL, bool ZOH = false, bool CONV = false>
 SeqPlan plan_seq(const FwdArgs& a) {
     using Cfg = ssm::SeqCfg<IO, G, CPL>;
     SeqPlan pl;
@@ -188,7 +197,7 @@ SeqPlan plan_seq(const FwdArgs& a) {
         if (stages < 2) continue;
         const int threads = (Cfg::warps_for(mt) + 1) * 32;
         const int smem = Cfg::smem_bytes(mt, stages);
-        const void* kern = seq_kernel_ptr<IO, G, CPL, ZOH>(stages);
+        const void* kern = seq_kernel_ptr<IO, G, CPL, ZOH, CONV>(stages);
         int occ = 0;
         if (!ensure_smem_attr(kern, smem) ||
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, smem) != cudaSuccess || occ < per_sm)
@@ -220,7 +229,7 @@ double predict_seq(const FwdArgs& a, const SeqPlan& pl) {
     return tiles * cost / hide;
 }
 
-template <typename IO, int G, int CPL, bool ZOH = false>
+template <typename IO, int G, int CPL, bool ZOH = false, bool CONV = false>
 ssm_status_t launch_seq(const FwdArgs& a, const SeqPlan& pl) {
     using Cfg = ssm::SeqCfg<IO, G, CPL>;
     if (!pl.ok) return SSM_ERR_UNSUPPORTED;
@@ -254,11 +263,18 @@ ssm_status_t launch_seq(const FwdArgs& a, const SeqPlan& pl) {
     p.softplus = a.softplus;
     p.has_z = a.z != nullptr;
     p.wait_limit = kDefaultWaitLimit;
+    p.x = a.u;
+    p.conv_w = a.conv.w;
+    p.conv_b = a.conv.b;
+    p.conv_in = a.conv.in;
+    p.conv_out = a.conv.out;
+    p.u_out = a.conv.u_out;
+    p.conv_k = a.conv.k;
     if (a.L >= (1LL << 31) - 1024) return SSM_ERR_UNSUPPORTED;
     switch (pl.stages) {
-        case 2: ssm::scan_fwd_seq_kernel<IO, G, CPL, 2, ZOH><<<pl.grid, pl.threads, pl.smem, a.stream>>>(mu, mdl, mz, mbc, p); break;
-        case 3: ssm::scan_fwd_seq_kernel<IO, G, CPL, 3, ZOH><<<pl.grid, pl.threads, pl.smem, a.stream>>>(mu, mdl, mz, mbc, p); break;
-        default: ssm::scan_fwd_seq_kernel<IO, G, CPL, 4, ZOH><<<pl.grid, pl.threads, pl.smem, a.stream>>>(mu, mdl, mz, mbc, p); break;
+        case 2: ssm::scan_fwd_seq_kernel<IO, G, CPL, 2, ZOH, CONV><<<pl.grid, pl.threads, pl.smem, a.stream>>>(mu, mdl, mz, mbc, p); break;
+        case 3: ssm::scan_fwd_seq_kernel<IO, G, CPL, 3, ZOH, CONV><<<pl.grid, pl.threads, pl.smem, a.stream>>>(mu, mdl, mz, mbc, p); break;
+        default: ssm::scan_fwd_seq_kernel<IO, G, CPL, 4, ZOH, CONV><<<pl.grid, pl.threads, pl.smem, a.stream>>>(mu, mdl, mz, mbc, p); break;
     }
     return launch_status();
 }
@@ -334,12 +350,31 @@ ssm_status_t launch_direct(const FwdArgs& a) {
     p.L = a.L;
     p.softplus = a.softplus;
     p.zoh = a.zoh;
+    p.conv_w = a.conv.w;
+    p.conv_b = a.conv.b;
+    p.conv_in = a.conv.in;
+    p.conv_out = a.conv.out;
+    p.u_out = a.conv.u_out;
+    p.conv_k = a.conv.k;
     constexpr int G = 2;
     const long long threads = static_cast<long long>(a.batch) * a.dim * G;
     const long long grid = (threads + 127) / 128;
     if (grid > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
     ssm::scan_fwd_direct_kernel<IO, G><<<static_cast<unsigned>(grid), 128, 0, a.stream>>>(p);
     return launch_status();
+}
+
+// The zero-order-hold and conv-prologue kernels exist for 4 and 8 lanes per channel.
+template <typename IO, bool ZOH, bool CONV>
+ssm_status_t launch_flagged(const FwdArgs& a, const ssm_fwd_options_t& o) {
+    const SeqPlan p4 = plan_seq<IO, 4, 1, ZOH, CONV>(a);
+    if constexpr (sizeof(IO) == 2) {
+        const SeqPlan p8 = plan_seq<IO, 8, 1, ZOH, CONV>(a);
+        const bool use8 = o.lanes_per_channel == 8 ||
+                          (o.lanes_per_channel == 0 && predict_seq<IO, 8, 1>(a, p8) < predict_seq<IO, 4, 1>(a, p4));
+        if (use8) return launch_seq<IO, 8, 1, ZOH, CONV>(a, p8);
+    }
+    return launch_seq<IO, 4, 1, ZOH, CONV>(a, p4);
 }
 
 template <typename IO>
@@ -360,8 +395,8 @@ ssm_status_t launch_forward(const FwdArgs& a, const ssm_fwd_options_t& o) {
     int algo = o.algo;
     if (!tma_ok) algo = SSM_ALGO_DIRECT;
     if (algo == SSM_ALGO_DIRECT) return launch_direct<IO>(a);
-    if (a.zoh && algo == SSM_ALGO_CHUNKED) return SSM_ERR_UNSUPPORTED;  // simplified discretisation only
-    if (algo == SSM_ALGO_AUTO && a.zoh) algo = SSM_ALGO_SEQUENTIAL;
+    if ((a.zoh || a.conv.k > 0) && algo == SSM_ALGO_CHUNKED) return SSM_ERR_UNSUPPORTED;  // plain scan only
+    if (algo == SSM_ALGO_AUTO && (a.zoh || a.conv.k > 0)) algo = SSM_ALGO_SEQUENTIAL;
     if (algo == SSM_ALGO_AUTO) {
         // The sequential kernel is faster whenever the channels alone give each SM a few
         // warps (measured on B200: at 5120 channels x 32768 steps it runs at ~1.8x the
@@ -375,15 +410,10 @@ ssm_status_t launch_forward(const FwdArgs& a, const ssm_fwd_options_t& o) {
     // Variants: (lanes per channel G, channels per lane CPL).  lanes_per_channel selects
     // G explicitly (CPL = 1), or G = 4 with CPL = 2 when given as 42.  The zero-order-hold
     // weight is built into the 4- and 8-lane variants only.
-    if (a.zoh) {
-        const SeqPlan z4 = plan_seq<IO, 4, 1, true>(a);
-        if constexpr (sizeof(IO) == 2) {
-            const SeqPlan z8 = plan_seq<IO, 8, 1, true>(a);
-            const bool use8 = o.lanes_per_channel == 8 ||
-                              (o.lanes_per_channel == 0 && predict_seq<IO, 8, 1>(a, z8) < predict_seq<IO, 4, 1>(a, z4));
-            if (use8) return launch_seq<IO, 8, 1, true>(a, z8);
-        }
-        return launch_seq<IO, 4, 1, true>(a, z4);
+    if (a.zoh || a.conv.k > 0) {
+        if (a.zoh && a.conv.k > 0) return launch_flagged<IO, true, true>(a, o);
+        if (a.zoh) return launch_flagged<IO, true, false>(a, o);
+        return launch_flagged<IO, false, true>(a, o);
     }
     const SeqPlan p2 = plan_seq<IO, 2, 1>(a), p4 = plan_seq<IO, 4, 1>(a), p42 = plan_seq<IO, 4, 2>(a);
     SeqPlan p8;
@@ -610,12 +640,14 @@ ssm_status_t ssm_workspace_init(void* workspace, size_t workspace_bytes, ssm_str
                : SSM_ERR_LAUNCH;
 }
 
-ssm_status_t ssm_selective_scan_fwd_state(const void* u, const void* delta, const float* A, const void* B,
-                                          const void* C, const float* D, const void* z, const float* delta_bias,
-                                          int softplus, const float* initial_state, void* y, float* last_state,
-                                          int batch, int dim, int dstate, int64_t seqlen, ssm_dtype_t io_dtype,
-                                          void* workspace, size_t workspace_bytes, const ssm_fwd_options_t* opts,
-                                          ssm_stream_t stream) {
+}  // extern "C"
+
+namespace {
+ssm_status_t forward_entry(const void* u, const void* delta, const float* A, const void* B, const void* C,
+                           const float* D, const void* z, const float* delta_bias, int softplus,
+                           const float* initial_state, void* y, float* last_state, int batch, int dim, int dstate,
+                           int64_t seqlen, ssm_dtype_t io_dtype, void* workspace, size_t workspace_bytes,
+                           const ssm_fwd_options_t* opts, ssm_stream_t stream, const ConvArgs& conv) {
     if (batch < 0 || dim < 0 || seqlen < 0) return SSM_ERR_INVALID_ARG;
     // Tensors with elements must have a pointer; zero-element tensors may be NULL.
     const bool seq_elems = batch > 0 && dim > 0 && seqlen > 0;
@@ -657,12 +689,58 @@ ssm_status_t ssm_selective_scan_fwd_state(const void* u, const void* delta, cons
         return SSM_OK;
     }
     FwdArgs a{u, delta, B, C, z, A, D, delta_bias, softplus, initial_state, o.discretization == SSM_DISC_ZOH, y,
-              last_state, batch, dim, seqlen, io_dtype, static_cast<uint8_t*>(workspace), s, sm_count};
+              last_state, batch, dim, seqlen, io_dtype, static_cast<uint8_t*>(workspace), s, sm_count, conv};
     if (dstate != 16) {
-        if (o.algo == SSM_ALGO_CHUNKED) return SSM_ERR_UNSUPPORTED;  // d_state 16 only
+        if (o.algo == SSM_ALGO_CHUNKED || conv.k > 0) return SSM_ERR_UNSUPPORTED;  // d_state 16 only
         return io_dtype == SSM_BF16 ? launch_wide<__nv_bfloat16>(a, dstate) : launch_wide<float>(a, dstate);
     }
     return io_dtype == SSM_BF16 ? launch_forward<__nv_bfloat16>(a, o) : launch_forward<float>(a, o);
+}
+}  // namespace
+
+extern "C" {
+
+ssm_status_t ssm_selective_scan_fwd_state(const void* u, const void* delta, const float* A, const void* B,
+                                          const void* C, const float* D, const void* z, const float* delta_bias,
+                                          int softplus, const float* initial_state, void* y, float* last_state,
+                                          int batch, int dim, int dstate, int64_t seqlen, ssm_dtype_t io_dtype,
+                                          void* workspace, size_t workspace_bytes, const ssm_fwd_options_t* opts,
+                                          ssm_stream_t stream) {
+    return forward_entry(u, delta, A, B, C, D, z, delta_bias, softplus, initial_state, y, last_state, batch, dim,
+                         dstate, seqlen, io_dtype, workspace, workspace_bytes, opts, stream, ConvArgs{});
+}
+
+ssm_status_t ssm_selective_scan_fwd_conv(const void* x, const ssm_conv_t* conv, const void* delta, const float* A,
+                                         const void* B, const void* C, const float* D, const void* z,
+                                         const float* delta_bias, int softplus, const float* initial_state, void* y,
+                                         float* last_state, int batch, int dim, int dstate, int64_t seqlen,
+                                         ssm_dtype_t io_dtype, void* workspace, size_t workspace_bytes,
+                                         const ssm_fwd_options_t* opts, ssm_stream_t stream) {
+    if (!conv || conv->width < 1 || conv->width > 4) return SSM_ERR_INVALID_ARG;
+    if (dim > 0 && !conv->weight) return SSM_ERR_INVALID_ARG;
+    if (batch > 0 && dim > 0 && seqlen > 0 && conv->u_out && !aligned16(conv->u_out)) return SSM_ERR_INVALID_ARG;
+    if (dstate != 16) return SSM_ERR_UNSUPPORTED;
+    ConvArgs c;
+    c.w = conv->weight;
+    c.b = conv->bias;
+    c.in = conv->width > 1 ? conv->state_in : nullptr;
+    c.out = conv->width > 1 ? conv->state_out : nullptr;
+    c.u_out = conv->u_out;
+    c.k = conv->width;
+    if (seqlen == 0 && c.out && batch > 0 && dim > 0) {  // nothing to scan: the conv state passes through
+        ssm_status_t st = forward_entry(x, delta, A, B, C, D, z, delta_bias, softplus, initial_state, y, last_state,
+                                        batch, dim, dstate, seqlen, io_dtype, workspace, workspace_bytes, opts,
+                                        stream, c);
+        if (st != SSM_OK) return st;
+        const size_t bytes = static_cast<size_t>(batch) * dim * (c.k - 1) * sizeof(float);
+        cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+        cudaError_t e = cudaSuccess;
+        if (!c.in) e = cudaMemsetAsync(c.out, 0, bytes, s);
+        else if (c.in != c.out) e = cudaMemcpyAsync(c.out, c.in, bytes, cudaMemcpyDeviceToDevice, s);
+        return e == cudaSuccess ? SSM_OK : SSM_ERR_LAUNCH;
+    }
+    return forward_entry(x, delta, A, B, C, D, z, delta_bias, softplus, initial_state, y, last_state, batch, dim,
+                         dstate, seqlen, io_dtype, workspace, workspace_bytes, opts, stream, c);
 }
 
 ssm_status_t ssm_selective_scan_fwd_ex(const void* u, const void* delta, const float* A, const void* B,
@@ -694,6 +772,20 @@ ssm_status_t ssm_state_update_ex(float* state, const void* u, const void* delta,
                                  const void* C, const float* D, const void* z, const float* delta_bias, int softplus,
                                  void* y, int batch, int dim, int dstate, ssm_dtype_t io_dtype,
                                  ssm_discretization_t discretization, ssm_stream_t stream) {
+    return ssm_state_update_conv(state, nullptr, u, nullptr, nullptr, 0, delta, A, B, C, D, z, delta_bias, softplus, y,
+                                 batch, dim, dstate, io_dtype, discretization, stream);
+}
+
+ssm_status_t ssm_state_update_conv(float* state, float* conv_state, const void* x, const float* conv_weight,
+                                   const float* conv_bias, int conv_width, const void* delta, const float* A,
+                                   const void* B, const void* C, const float* D, const void* z,
+                                   const float* delta_bias, int softplus, void* y, int batch, int dim, int dstate,
+                                   ssm_dtype_t io_dtype, ssm_discretization_t discretization, ssm_stream_t stream) {
+    const void* u = x;
+    if (conv_width < 0 || conv_width > 4) return SSM_ERR_INVALID_ARG;
+    if (conv_width > 0 && batch > 0 && dim > 0 && (!conv_weight || (conv_width > 1 && !conv_state)))
+        return SSM_ERR_INVALID_ARG;
+    if (conv_width > 0 && dstate != 16) return SSM_ERR_UNSUPPORTED;
     if (batch < 0 || dim < 0) return SSM_ERR_INVALID_ARG;
     if (discretization != SSM_DISC_SIMPLIFIED && discretization != SSM_DISC_ZOH) return SSM_ERR_INVALID_ARG;
     if (batch > 0 && dim > 0 && (!state || !u || !delta || !A || !B || !C || !y)) return SSM_ERR_INVALID_ARG;
@@ -727,7 +819,7 @@ ssm_status_t ssm_state_update_ex(float* state, const void* u, const void* delta,
         return launch_status();
     }
     ssm::DecodeParams p{state, u, delta, A, B, C, D, z, delta_bias, y, batch, dim, softplus,
-                        discretization == SSM_DISC_ZOH};
+                        discretization == SSM_DISC_ZOH, conv_weight, conv_bias, conv_state, conv_width};
     const long long threads = static_cast<long long>(batch) * dim * 4;
     const long long grid = (threads + 255) / 256;
     if (grid > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;

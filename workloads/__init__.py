@@ -15,6 +15,8 @@ Recipe (per workload):
   delta_bias[d]  = inverse softplus of dt, dt log-uniform in [dt_min, dt_max]
                    (computed in fp64, stored fp32)
   softplus on.
+The causal-conv prologue draws weight ~ N(0, 1)/sqrt(width), bias ~ 0.1 N(0, 1) and a
+carried-in conv state ~ N(0, 1), fp32.
 Scans that continue from a given state (initial_state) draw it ~ N(0, 1), fp32,
 shape (batch, dim, dstate), from their own seed.
 Decode workloads additionally draw an initial state ~ N(0, 1) of shape
@@ -82,6 +84,16 @@ def initial_state(batch, dim, dstate=16, seed=0, scale=1.0):
     continue from a given state."""
     g = torch.Generator().manual_seed(seed)
     return _randn(g, (batch, dim, dstate), scale).contiguous()
+
+
+def conv_inputs(batch, dim, width=4, seed=0, with_bias=True, with_state=False):
+    """Seeded causal-conv parameters: weight (dim, width) ~ N(0, 1) / sqrt(width), bias (dim)
+    ~ 0.1 N(0, 1), and optionally a carried-in state (batch, dim, width-1) ~ N(0, 1), all fp32."""
+    g = torch.Generator().manual_seed(seed)
+    w = _randn(g, (dim, width), 1.0 / math.sqrt(width)).contiguous()
+    b = _randn(g, (dim,), 0.1) if with_bias else None
+    st = _randn(g, (batch, dim, width - 1)).contiguous() if with_state else None
+    return dict(conv_weight=w, conv_bias=b, conv_state_in=st)
 
 
 def scan_inputs(batch, dim, seqlen, dstate=16, io="bf16", dt_min=1e-3, dt_max=1e-1, seed=0,
