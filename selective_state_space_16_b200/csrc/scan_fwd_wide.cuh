@@ -8,15 +8,15 @@
 //
 // The step is the one of the d_state = 16 kernels (simplified or zero-order-hold weight,
 // [Card] 离散化变换 / [Eng] §2.2).  With N exponentials per element these shapes are bound by
-// the special-function unit (N/16 times the work of N = 16 per element), so the kernel is
-// plain (no staging): G = N/4 lanes per channel (N/8 for N = 256), each lane holding 4 (8)
-// chains of the channel in registers for the whole sequence in f32x2 pairs, 32/G channels per
-// warp.  Steps go in batches of G: lane nl of a channel loads and evaluates the step size of
-// step nl (coalesced loads), the lanes walk the G steps with the step size and input
-// broadcast by shuffles, each lane reading its chains' B and C values from the packed fp32
-// rows (one row of 2N floats per step, shared by all channels of the batch row through L1),
-// and the G lanes' partial sums of C.h are reduce-scattered so that lane nl finishes (D skip,
-// gate, rounding, store) step nl.
+// the special-function unit (N/16 times the work of N = 16 per element).  G = N/4 lanes per
+// channel (N/8 for N = 256), each lane holding 4 (8) chains of the channel in registers for
+// the whole sequence in f32x2 pairs, 32/G channels per warp, 8 warps per block, all on one
+// batch row.  The block stages the packed fp32 B/C rows (2N floats per step) of 64 (32) steps
+// at a time through a double-buffered cp.async ring in shared memory.  Steps go in batches of
+// G: lane nl of a channel loads (one batch ahead) and evaluates the step size of step nl, the
+// lanes walk the G steps with the step size and input broadcast by shuffles, and the G lanes'
+// partial sums of C.h are reduce-scattered so that lane nl finishes (D skip, gate, rounding,
+// store) step nl.
 #pragma once
 
 #include "common.cuh"
@@ -41,101 +41,143 @@ struct WideCfg {
     static constexpr int kG = N / kNC;             // lanes per channel: 8, 16, 32, 32
     static constexpr int kCPW = 32 / kG;           // channels per warp: 4, 2, 1, 1
     static constexpr int kT = kG;                  // steps per batch (one step per lane of a channel)
+    // warps per block (one batch row per block); N = 256 stages 128 KB per block, so its
+    // blocks are twice as large to keep 16 warps per SM
+    static constexpr int kWarps = N == 256 ? 16 : 8;
+    static constexpr int kCPB = kWarps * kCPW;     // channels per block
+    static constexpr int kST = N <= 64 ? 64 : 32;  // steps per staged stage of B/C rows
+    static constexpr int kStageFloats = kST * 2 * N;
+    static constexpr int kSmem = 2 * kStageFloats * 4;  // double-buffered stages
 };
 
 template <typename IO, int N>
-__global__ void __launch_bounds__(256) scan_fwd_wide_kernel(const WideParams p) {
+__global__ void __launch_bounds__(WideCfg<N>::kWarps * 32, N == 256 ? 1 : 2) scan_fwd_wide_kernel(const WideParams p) {
     using Cfg = WideCfg<N>;
-    constexpr int NC = Cfg::kNC, G = Cfg::kG, CPW = Cfg::kCPW, T = Cfg::kT;
+    constexpr int NC = Cfg::kNC, G = Cfg::kG, CPW = Cfg::kCPW, T = Cfg::kT, ST = Cfg::kST;
     static_assert(N == 32 || N == 64 || N == 128 || N == 256, "N in {32, 64, 128, 256}");
-    const int lane = threadIdx.x & 31;
+    static_assert(ST % T == 0, "whole batches per stage");
+    extern __shared__ float4 wide_smem[];
+    float* ring = reinterpret_cast<float*>(wide_smem);  // [2][ST][2N]
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int cg = lane / G, nl = lane % G, gbase = lane & ~(G - 1);
-    const long long nch = static_cast<long long>(p.batch) * p.dim;
-    const long long ch0 = (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * CPW;
-    if (ch0 >= nch) return;  // whole warps leave together
-    const long long ch = ch0 + cg;  // flat (b, d) of this lane's channel
-    const bool valid = ch < nch;
-    const long long cc = valid ? ch : ch0;
-    const int b = static_cast<int>(cc / p.dim), d = static_cast<int>(cc % p.dim);
+    const int b = blockIdx.y;
+    const int d = blockIdx.x * Cfg::kCPB + warp * CPW + cg;
+    const bool valid = d < p.dim;
+    const int dd = valid ? d : 0;
     const long long L = p.L;
-    const IO* u = static_cast<const IO*>(p.u) + cc * L;
-    const IO* dl = static_cast<const IO*>(p.delta) + cc * L;
-    const IO* z = p.z ? static_cast<const IO*>(p.z) + cc * L : nullptr;
-    IO* y = static_cast<IO*>(p.y) + cc * L;
-    const float* bcb = p.bc + static_cast<long long>(b) * L * (2 * N) + nl * NC;
+    const long long ch = static_cast<long long>(b) * p.dim + dd;
+    const IO* u = static_cast<const IO*>(p.u) + ch * L;
+    const IO* dl = static_cast<const IO*>(p.delta) + ch * L;
+    const IO* z = p.z ? static_cast<const IO*>(p.z) + ch * L : nullptr;
+    IO* y = static_cast<IO*>(p.y) + ch * L;
+    const float* bcrow = p.bc + static_cast<long long>(b) * L * (2 * N);
 
     float2 A2[NC / 2], invA[NC / 2], h[NC / 2];
 #pragma unroll
     for (int j = 0; j < NC / 2; ++j) {
-        const float a0 = p.A[static_cast<long long>(d) * N + nl * NC + 2 * j];
-        const float a1 = p.A[static_cast<long long>(d) * N + nl * NC + 2 * j + 1];
+        const float a0 = p.A[static_cast<long long>(dd) * N + nl * NC + 2 * j];
+        const float a1 = p.A[static_cast<long long>(dd) * N + nl * NC + 2 * j + 1];
         A2[j] = make_float2(a0 * kLog2e, a1 * kLog2e);
         invA[j] = make_float2(1.f / a0, 1.f / a1);
-        h[j] = (p.h0 && valid) ? *reinterpret_cast<const float2*>(p.h0 + cc * N + nl * NC + 2 * j)
+        h[j] = (p.h0 && valid) ? *reinterpret_cast<const float2*>(p.h0 + ch * N + nl * NC + 2 * j)
                                : make_float2(0.f, 0.f);
     }
-    const float Dd = p.D ? p.D[d] : 0.f;
-    const float bias = p.bias ? p.bias[d] : 0.f;
+    const float Dd = (valid && p.D) ? p.D[dd] : 0.f;
+    const float bias = (valid && p.bias) ? p.bias[dd] : 0.f;
     const bool softplus = p.softplus != 0, zoh = p.zoh != 0;
 
-    for (long long t0 = 0; t0 < L; t0 += T) {
-        // lane nl of the channel loads and finishes step t0 + nl
-        const long long t = t0 + nl;
+    // B/C rows of stage k into ring slot k & 1 (zero past L), one cp.async group per stage.
+    const long long nstages = (L + ST - 1) / ST;
+    auto issue = [&](long long k) {
+        if (k < nstages) {
+            float* dst = ring + (k & 1) * Cfg::kStageFloats;
+            for (int c = threadIdx.x; c < Cfg::kStageFloats / 4; c += blockDim.x) {
+                const int i = c / (2 * N / 4), part = c % (2 * N / 4);
+                const long long t = k * ST + i;
+                const bool in = t < L;
+                cp_async_16(dst + i * 2 * N + part * 4, in ? bcrow + t * 2 * N + part * 4 : bcrow, in ? 16u : 0u);
+            }
+        }
+        cp_async_commit();
+    };
+    // Inputs of the lane's own step of a batch (0 past L), loaded one batch ahead.
+    auto load_own = [&](long long t, float& ul, float& xl, float& zl) {
         const bool in = valid && t < L;
-        const float ul = in ? IoTraits<IO>::to_f32(u[t]) : 0.f;
-        const float dtl = in ? step_size(IoTraits<IO>::to_f32(dl[t]), bias, softplus) : 0.f;  // 0 past L
-        const float zl = (in && z) ? IoTraits<IO>::to_f32(z[t]) : 0.f;
-        float yp[T];
+        ul = in ? IoTraits<IO>::to_f32(u[t]) : 0.f;
+        xl = in ? IoTraits<IO>::to_f32(dl[t]) : 0.f;
+        zl = (in && z) ? IoTraits<IO>::to_f32(z[t]) : 0.f;
+    };
+
+    issue(0);
+    float un, xn, zn;
+    load_own(nl, un, xn, zn);
+    for (long long k = 0; k < nstages; ++k) {
+        issue(k + 1);
+        cp_async_wait<1>();
+        __syncthreads();  // stage k visible to every warp
+        const float* stage = ring + (k & 1) * Cfg::kStageFloats + nl * NC;
+#pragma unroll 1
+        for (int bt = 0; bt < ST; bt += T) {
+            const long long t0 = k * ST + bt;
+            const long long t = t0 + nl;
+            const float ul = un, zl = zn;
+            const float dtl = (valid && t < L) ? step_size(xn, bias, softplus) : 0.f;  // 0 past L
+            load_own(t + T, un, xn, zn);  // next batch (the next stage's first for the last batch)
+            float yp[T];
 #pragma unroll
-        for (int i = 0; i < T; ++i) {
-            const float dti = __shfl_sync(0xffffffffu, dtl, gbase | i);
-            const float ui = __shfl_sync(0xffffffffu, ul, gbase | i);
-            // rows past L repeat row L-1; their step size is 0, so the state does not move
-            const float* row = bcb + min(t0 + i, L - 1) * (2 * N);
-            float2 Bv[NC / 2], Cv[NC / 2];
+            for (int i = 0; i < T; ++i) {
+                const float dti = __shfl_sync(0xffffffffu, dtl, gbase | i);
+                const float ui = __shfl_sync(0xffffffffu, ul, gbase | i);
+                const float* row = stage + (bt + i) * 2 * N;
+                float2 Bv[NC / 2], Cv[NC / 2];
 #pragma unroll
-            for (int j = 0; j < NC / 2; j += 2) {
-                const float4 bq = *reinterpret_cast<const float4*>(row + 2 * j);
-                const float4 cq = *reinterpret_cast<const float4*>(row + N + 2 * j);
-                Bv[j] = make_float2(bq.x, bq.y);
-                Bv[j + 1] = make_float2(bq.z, bq.w);
-                Cv[j] = make_float2(cq.x, cq.y);
-                Cv[j + 1] = make_float2(cq.z, cq.w);
+                for (int j = 0; j < NC / 2; j += 2) {
+                    const float4 bq = *reinterpret_cast<const float4*>(row + 2 * j);
+                    const float4 cq = *reinterpret_cast<const float4*>(row + N + 2 * j);
+                    Bv[j] = make_float2(bq.x, bq.y);
+                    Bv[j + 1] = make_float2(bq.z, bq.w);
+                    Cv[j] = make_float2(cq.x, cq.y);
+                    Cv[j + 1] = make_float2(cq.z, cq.w);
+                }
+                const float2 dd2 = make_float2(dti, dti), ww = make_float2(dti * ui, dti * ui);
+                float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int j = 0; j < NC / 2; ++j) {
+                    const float2 arg = __fmul2_rn(dd2, A2[j]);
+                    const float2 a = make_float2(ex2_mufu(arg.x), ex2_mufu(arg.y));
+                    float2 beta = __fmul2_rn(ww, Bv[j]);
+                    if (zoh)
+                        beta = zoh_beta2(arg, a, beta, __fmul2_rn(__fmul2_rn(make_float2(ui, ui), Bv[j]), invA[j]));
+                    h[j] = __ffma2_rn(a, h[j], beta);
+                    acc = __ffma2_rn(Cv[j], h[j], acc);
+                }
+                yp[i] = acc.x + acc.y;
             }
-            const float2 dd = make_float2(dti, dti), ww = make_float2(dti * ui, dti * ui);
-            float2 acc = make_float2(0.f, 0.f);
+            // Reduce-scatter the T partial sums over the G lanes of the channel (upper lane
+            // bit first): lane nl ends with the full sum of step t0 + nl in yp[0].
 #pragma unroll
-            for (int j = 0; j < NC / 2; ++j) {
-                const float2 arg = __fmul2_rn(dd, A2[j]);
-                const float2 a = make_float2(ex2_mufu(arg.x), ex2_mufu(arg.y));
-                float2 beta = __fmul2_rn(ww, Bv[j]);
-                if (zoh) beta = zoh_beta2(arg, a, beta, __fmul2_rn(__fmul2_rn(make_float2(ui, ui), Bv[j]), invA[j]));
-                h[j] = __ffma2_rn(a, h[j], beta);
-                acc = __ffma2_rn(Cv[j], h[j], acc);
+            for (int m = G / 2; m >= 1; m >>= 1) {
+                const bool upper = (nl & m) != 0;
+#pragma unroll
+                for (int i = 0; i < m; ++i) {
+                    const float send = upper ? yp[i] : yp[i + m];
+                    const float keep = upper ? yp[i + m] : yp[i];
+                    yp[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+                }
             }
-            yp[i] = acc.x + acc.y;
-        }
-        // Reduce-scatter the T partial sums over the G lanes of the channel (upper lane bit
-        // first): lane nl ends with the full sum of step t0 + nl in yp[0].
-#pragma unroll
-        for (int m = G / 2; m >= 1; m >>= 1) {
-            const bool upper = (nl & m) != 0;
-#pragma unroll
-            for (int i = 0; i < m; ++i) {
-                const float send = upper ? yp[i] : yp[i + m];
-                const float keep = upper ? yp[i + m] : yp[i];
-                yp[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+            if (valid && t < L) {
+                float v = fmaf(Dd, ul, yp[0]);
+                if (z) v *= silu_f32(zl);
+                y[t] = IoTraits<IO>::from_f32(v);
             }
         }
-        if (in) {
-            float v = fmaf(Dd, ul, yp[0]);
-            if (z) v *= silu_f32(zl);
-            y[t] = IoTraits<IO>::from_f32(v);
-        }
+        __syncthreads();  // every warp is done with slot k & 1 before it is refilled
     }
+    cp_async_wait<0>();
     if (p.last_state && valid)
 #pragma unroll
-        for (int j = 0; j < NC / 2; ++j) *reinterpret_cast<float2*>(p.last_state + cc * N + nl * NC + 2 * j) = h[j];
+        for (int j = 0; j < NC / 2; ++j) *reinterpret_cast<float2*>(p.last_state + ch * N + nl * NC + 2 * j) = h[j];
 }
 
 // B, C (batch, N, L) -> fp32 rows [batch][L][2N] (B then C): 32 x 32 tiles through shared

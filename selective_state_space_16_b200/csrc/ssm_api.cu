@@ -460,10 +460,11 @@ ssm_status_t launch_wide_n(const FwdArgs& a) {
     p.L = a.L;
     p.softplus = a.softplus;
     p.zoh = a.zoh;
-    constexpr int cpb = 8 * ssm::WideCfg<N>::kCPW;  // channels per block of 8 warps
-    const long long grid = (static_cast<long long>(a.batch) * a.dim + cpb - 1) / cpb;
-    if (grid > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
-    ssm::scan_fwd_wide_kernel<IO, N><<<static_cast<unsigned>(grid), 256, 0, a.stream>>>(p);
+    using Cfg = ssm::WideCfg<N>;
+    auto kern = ssm::scan_fwd_wide_kernel<IO, N>;
+    if (!ensure_smem_attr(reinterpret_cast<const void*>(kern), Cfg::kSmem)) return SSM_ERR_LAUNCH;
+    const dim3 grid(static_cast<unsigned>((a.dim + Cfg::kCPB - 1) / Cfg::kCPB), static_cast<unsigned>(a.batch));
+    kern<<<grid, Cfg::kWarps * 32, Cfg::kSmem, a.stream>>>(p);
     return launch_status();
 }
 
