@@ -27,9 +27,10 @@
 // kernels), with the chain arithmetic in f32x2 pairs.  Each warp first runs the forward
 // over the whole sequence and stores the state at the start of every 8-step segment
 // (checkpoints, in the workspace).  Then it walks the segments from the last to the
-// first: it re-runs the segment from its checkpoint, keeping h_{t-1} and exp(Delta A) of
-// the 8 steps in shared memory, forms v_t, dz_t and dv_t, and runs the gradient
-// recurrence backwards through the segment.
+// first: it re-runs the segment from its checkpoint, keeping h_{t-1} of the 8 steps in
+// shared memory, forms v_t, dz_t and dv_t, and runs the gradient recurrence backwards
+// through the segment (recomputing exp(Delta A): the shared-memory data path, not the
+// exponential unit, bounds this kernel).
 //   - Sums over the 16 chains (du, dDelta, v) are reduce-scattered over the 4 lanes of a
 //     channel, so that lane nl finishes steps 2nl, 2nl+1 of the segment.
 //   - Sums over channels (dB, dC) are reduce-scattered over the 8 channels of a warp,
@@ -51,7 +52,7 @@ constexpr int kBwdWarps = 4;     // warps per CTA (5 CTAs per SM: every CTA resi
 constexpr int kBwdChannels = kBwdWarps * 8;
 constexpr int kBwdRing = 4;      // segments of B/C rows in flight (cp.async ring)
 // dynamic shared memory of scan_bwd_kernel: h and decay stages, dB/dC stage, B/C ring
-constexpr int kBwdSmem = kBwdWarps * kBwdSeg * 32 * (16 + 16 + 4) + kBwdRing * kBwdSeg * 32 * 4;
+constexpr int kBwdSmem = kBwdWarps * kBwdSeg * 32 * (16 + 4) + kBwdRing * kBwdSeg * 32 * 4;
 
 struct BwdParams {
     const void *u, *delta, *z, *dy;  // (batch, dim, L) IO
@@ -81,11 +82,10 @@ template <typename IO>
 __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdParams p) {
     constexpr int T = kBwdSeg, G = 4, PER = T / G, R = kBwdRing;
     extern __shared__ float4 bwd_smem[];
-    // h_{t-1} and exp(Delta_t A) of the segment's steps: [warp][step][lane] (16 bytes each)
+    // h_{t-1} of the segment's steps: [warp][step][lane] (16 bytes each)
     float4* hstage = bwd_smem;
-    float4* astage = bwd_smem + kBwdWarps * T * 32;
     // per-warp dB/dC partials of the segment's steps: [warp][step][32 columns]
-    float* cstage = reinterpret_cast<float*>(bwd_smem + 2 * kBwdWarps * T * 32);
+    float* cstage = reinterpret_cast<float*>(bwd_smem + kBwdWarps * T * 32);
     // ring of R segments of packed B/C rows (shared by the CTA: one batch row): [slot][step][32]
     float* bcring = cstage + kBwdWarps * T * 32;
 
@@ -212,7 +212,6 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
     }
     float dD_acc = 0.f, dbias_acc = 0.f;
     float4* hst = hstage + warp * T * 32;
-    float4* ast = astage + warp * T * 32;
     float* cst = cstage + warp * T * 32;
     const int col = (cg >> 2) * 16 + nl * 4 + (cg & 3);  // dB/dC column this lane ends with
 
@@ -246,7 +245,6 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
             const float4 Bq = ld4(bcs + i * 32), Cq = ld4(bcs + i * 32 + 16);
             const float2 a0 = decay(dti, 0), a1 = decay(dti, 1);
             hst[i * 32 + lane] = make_float4(hs[0].x, hs[0].y, hs[1].x, hs[1].y);
-            ast[i * 32 + lane] = make_float4(a0.x, a0.y, a1.x, a1.y);
             const float2 ww = f2(dti * ui, dti * ui);
             hs[0] = __ffma2_rn(a0, hs[0], __fmul2_rn(ww, lo(Bq)));
             hs[1] = __ffma2_rn(a1, hs[1], __fmul2_rn(ww, hi(Bq)));
@@ -291,9 +289,10 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
             const float ui = __shfl_sync(0xffffffffu, cur.u[i % PER], srcl[i / PER]);
             const float dvi = __shfl_sync(0xffffffffu, dv[i % PER], srcl[i / PER]);
             const float4 Bq = ld4(bcs + i * 32), Cq = ld4(bcs + i * 32 + 16);
-            const float4 hq = hst[i * 32 + lane], aq = ast[i * 32 + lane];
+            const float4 hq = hst[i * 32 + lane];
             const float2 Bv[2] = {lo(Bq), hi(Bq)}, Cv[2] = {lo(Cq), hi(Cq)};
-            const float2 hp[2] = {lo(hq), hi(hq)}, av[2] = {lo(aq), hi(aq)};
+            // exp(Delta A) again (the exponential unit has room; the shared-memory path does not)
+            const float2 hp[2] = {lo(hq), hi(hq)}, av[2] = {decay(dti, 0), decay(dti, 1)};
             const float2 dv2 = f2(dvi, dvi), dt2 = f2(dti, dti), u2 = f2(ui, ui);
             const float2 w2 = f2(dti * ui, dti * ui);
             float2 sdt = f2(0.f, 0.f), sdu = f2(0.f, 0.f), dB[2], dC[2];
