@@ -137,16 +137,21 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- distributed plumbing
-def dist_setup(n_gpus: int):
+def dist_setup(n_gpus: int, backend: str | None = None):
+    """One process per GPU (torchrun's RANK / LOCAL_RANK / WORLD_SIZE / MASTER_*): NCCL over
+    NVLink on GPUs; gloo when no GPU is visible (the CPU tests of this plumbing)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        backend = backend or ("nccl" if torch.cuda.is_available() else "gloo")
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     return world, rank, local
 
 
@@ -157,12 +162,20 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The job's time is the slowest rank's (every rank calls this, in the same order)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(elements_per_rank: int, world: int, steps: int, t_max: float) -> float:
+    """Whole-job G elements/s: every rank scans its own full workload (weak scaling: one
+    independent batch per GPU, no data-path collective), timed by the slowest rank."""
+    return elements_per_rank * world * steps / t_max / 1e9
 
 
 # ----------------------------------------------------------------------------- measurements
@@ -556,7 +569,7 @@ def run_gpu(args, world, rank, local):
     t = time_forward(ssm, g, ws, args.steps, args.warmup, world, stream, clocks)
     t = max_over_ranks(t, world)
     per_call = t / args.steps
-    value = w.elements * world * args.steps / t / 1e9
+    value = job_throughput(w.elements, world, args.steps, t)
     assert ssm.ssm_read_status(ws) == 0
 
     sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
