@@ -42,7 +42,7 @@
  * B, C: (batch, dstate, L); A: (dim, dstate); D, delta_bias: (dim);
  * h0 / last_state / decode state: (batch, dim, dstate).
  *
- * Readings taken where the pages are silent (listed with reasons in the design doc):
+ * Readings taken where the pages are silent:
  *   - D is a per-channel scalar, NULL means 0; z NULL means no gate; delta_bias
  *     NULL means 0.
  *   - softplus is evaluated in the overflow-free form max(x,0) + log1p(exp(-|x|)).
