@@ -176,7 +176,11 @@ struct DecodeParams {
     int conv_k;
 };
 
-template <typename IO>
+// Four threads per (b, d) channel, each one 16-byte quarter of the state; a full grid, one
+// quarter per thread (a lean kernel keeps ~60 warps per SM resident, which is what hides
+// the memory latency of this step).  ZOH and CONV are template flags so that the plain step
+// carries none of their registers.
+template <typename IO, bool ZOH, bool CONV>
 __global__ void __launch_bounds__(256) state_update_kernel(const DecodeParams p) {
     const long long gid = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
     const long long row = gid >> 2;  // flat (b, d)
@@ -189,7 +193,7 @@ __global__ void __launch_bounds__(256) state_update_kernel(const DecodeParams p)
     float4 hv = make_float4(0.f, 0.f, 0.f, 0.f);
     float4 av = make_float4(0.f, 0.f, 0.f, 0.f);
     float Bq[4] = {0.f, 0.f, 0.f, 0.f}, Cq[4] = {0.f, 0.f, 0.f, 0.f};
-    float ut = 0.f, dt = 0.f, zt = 0.f, Dd = 0.f;
+    float ut = 0.f, dt = 0.f, zt = 0.f, Dd = 0.f, xt = 0.f;
     if (valid) {
         hv = *reinterpret_cast<const float4*>(p.state + rr * 16 + q * 4);
         av = *reinterpret_cast<const float4*>(p.A + d * 16 + q * 4);
@@ -201,11 +205,12 @@ __global__ void __launch_bounds__(256) state_update_kernel(const DecodeParams p)
             Cq[j] = IoTraits<IO>::to_f32(Cp[j]);
         }
         ut = IoTraits<IO>::to_f32(static_cast<const IO*>(p.u)[rr]);
-        if (p.conv_k > 0) {  // u = silu(conv([conv_state, x])), rounded to the I/O type
+        if constexpr (CONV) {  // u = silu(conv([conv_state, x])), rounded to the I/O type
             const int K = p.conv_k;
+            xt = ut;
             float pre = p.conv_b ? p.conv_b[d] : 0.f;
             for (int k = 0; k < K - 1; ++k) pre = fmaf(p.conv_w[d * K + k], p.conv_state[rr * (K - 1) + k], pre);
-            pre = fmaf(p.conv_w[d * K + K - 1], ut, pre);
+            pre = fmaf(p.conv_w[d * K + K - 1], xt, pre);
             ut = IoTraits<IO>::to_f32(IoTraits<IO>::from_f32(silu_f32(pre)));
         }
         const float bias = p.bias ? p.bias[d] : 0.f;
@@ -221,19 +226,21 @@ __global__ void __launch_bounds__(256) state_update_kernel(const DecodeParams p)
     for (int j = 0; j < 4; ++j) {
         const float y = dt * as[j] * kLog2e;
         const float a = ex2_mufu(y);
-        const float beta = p.zoh ? zoh_beta(y, a, w * Bq[j], ut * Bq[j] / as[j]) : w * Bq[j];
+        float beta = w * Bq[j];
+        if constexpr (ZOH) beta = zoh_beta(y, a, beta, ut * Bq[j] / as[j]);
         hs[j] = fmaf(a, hs[j], beta);
         acc = fmaf(Cq[j], hs[j], acc);
     }
     acc += __shfl_xor_sync(0xffffffffu, acc, 1, 32);
     acc += __shfl_xor_sync(0xffffffffu, acc, 2, 32);
-    if (p.conv_k > 1) {
-        __syncwarp();  // every thread of the channel has read conv_state
-        if (valid && q == 0) {
-            const int K = p.conv_k;
-            const float xt = IoTraits<IO>::to_f32(static_cast<const IO*>(p.u)[rr]);
-            for (int k = 0; k < K - 2; ++k) p.conv_state[rr * (K - 1) + k] = p.conv_state[rr * (K - 1) + k + 1];
-            p.conv_state[rr * (K - 1) + K - 2] = xt;
+    if constexpr (CONV) {
+        if (p.conv_k > 1) {
+            __syncwarp();  // every thread of the channel has read conv_state
+            if (valid && q == 0) {
+                const int K = p.conv_k;
+                for (int k = 0; k < K - 2; ++k) p.conv_state[rr * (K - 1) + k] = p.conv_state[rr * (K - 1) + k + 1];
+                p.conv_state[rr * (K - 1) + K - 2] = xt;
+            }
         }
     }
     if (valid) {

@@ -825,10 +825,19 @@ ssm_status_t ssm_state_update_conv(float* state, float* conv_state, const void* 
     const long long grid = (threads + 255) / 256;
     if (grid > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (io_dtype == SSM_BF16)
-        ssm::state_update_kernel<__nv_bfloat16><<<static_cast<unsigned>(grid), 256, 0, s>>>(p);
-    else
-        ssm::state_update_kernel<float><<<static_cast<unsigned>(grid), 256, 0, s>>>(p);
+    const unsigned g = static_cast<unsigned>(grid);
+    const bool zoh = discretization == SSM_DISC_ZOH, conv = conv_width > 0;
+#define SSM_DECODE(IO_T)                                                                              \
+    if (zoh && conv) ssm::state_update_kernel<IO_T, true, true><<<g, 256, 0, s>>>(p);                 \
+    else if (zoh) ssm::state_update_kernel<IO_T, true, false><<<g, 256, 0, s>>>(p);                   \
+    else if (conv) ssm::state_update_kernel<IO_T, false, true><<<g, 256, 0, s>>>(p);                  \
+    else ssm::state_update_kernel<IO_T, false, false><<<g, 256, 0, s>>>(p);
+    if (io_dtype == SSM_BF16) {
+        SSM_DECODE(__nv_bfloat16)
+    } else {
+        SSM_DECODE(float)
+    }
+#undef SSM_DECODE
     return launch_status();
 }
 
