@@ -1,6 +1,8 @@
 // aux_kernels.cuh -- the kernels around the main forward scans:
 //   pack_bc_kernel      B, C (batch, 16, L) -> fp32 [batch][L][32] rows (B then C), so a
 //                       step's 16 B and 16 C values are one 128-byte row for broadcast reads;
+//   pack_bc_pairs_kernel bf16 B, C -> bf16 rows ordered by state pairs (the backward's
+//                       shared-memory ring: half the bytes per step);
 //   scan_fwd_direct     forward scan with direct global loads, for any seqlen / alignment;
 //   state_update_kernel the one-token decode step, fp32 state read-modified-written in place.
 //
@@ -35,6 +37,33 @@ __global__ void __launch_bounds__(256) pack_bc_kernel(const IO* __restrict__ B, 
         const int c = idx >> 5, r = idx & 31;
         const long long t = t0 + c;
         if (t < L) bc[(static_cast<long long>(b) * L + t) * 32 + r] = tile[r][c];
+    }
+}
+
+// The same transpose for bf16 inputs, kept in bf16 (exact) and ordered by state pairs:
+// [batch][L][16] 32-bit words, word 2j = (B_2j, B_2j+1), word 2j+1 = (C_2j, C_2j+1) (low
+// half the even state), so the B and C values of a lane's chains at one step are one
+// contiguous vector and a step's row is 64 bytes.  grid = (ceil(L/64), batch), 256 threads.
+__global__ void __launch_bounds__(256) pack_bc_pairs_kernel(const uint16_t* __restrict__ B,
+                                                            const uint16_t* __restrict__ C,
+                                                            uint32_t* __restrict__ bc, long long L) {
+    __shared__ uint16_t tile[32][66];
+    const int b = blockIdx.y;
+    const long long t0 = static_cast<long long>(blockIdx.x) * 64;
+    for (int idx = threadIdx.x; idx < 32 * 64; idx += 256) {
+        const int r = idx >> 6, c = idx & 63;
+        const long long t = t0 + c;
+        const uint16_t* src = (r < 16) ? B : C;
+        tile[r][c] = (t < L) ? src[(static_cast<long long>(b) * 16 + (r & 15)) * L + t] : uint16_t(0);
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < 16 * 64; idx += 256) {
+        const int c = idx >> 4, k = idx & 15;
+        const long long t = t0 + c;
+        const int r = (k & 1) * 16 + (k >> 1) * 2;  // first row of the word's pair
+        if (t < L)
+            bc[(static_cast<long long>(b) * L + t) * 16 + k] =
+                static_cast<uint32_t>(tile[r][c]) | (static_cast<uint32_t>(tile[r + 1][c]) << 16);
     }
 }
 

@@ -51,12 +51,14 @@ constexpr int kBwdSeg = 8;       // steps per segment (checkpoint interval)
 constexpr int kBwdWarps = 4;     // warps per CTA (5 CTAs per SM: every CTA resident at once)
 constexpr int kBwdChannels = kBwdWarps * 8;
 constexpr int kBwdRing = 4;      // segments of B/C rows in flight (cp.async ring)
-// dynamic shared memory of scan_bwd_kernel: h and decay stages, dB/dC stage, B/C ring
+// dynamic shared memory of scan_bwd_kernel: h stage, dB/dC stage, B/C ring (sized for
+// fp32 rows; bf16 rows use half of it)
 constexpr int kBwdSmem = kBwdWarps * kBwdSeg * 32 * (16 + 4) + kBwdRing * kBwdSeg * 32 * 4;
 
 struct BwdParams {
     const void *u, *delta, *z, *dy;  // (batch, dim, L) IO
-    const float* bc;                 // packed B/C rows, fp32 [batch][L][32]
+    const void* bc;                  // packed B/C rows: fp32 [batch][L][32] (B then C), or for
+                                     // bf16 inputs bf16 state pairs (pack_bc_pairs_kernel)
     const float *A, *D, *bias, *h0, *dlast;
     void *du, *ddelta, *dz;          // (batch, dim, L) IO outputs (dz only with z)
     float* dh0;                      // (batch, dim, 16) or null
@@ -70,6 +72,11 @@ struct BwdParams {
     int nseg, ncta;
     int softplus;
 };
+
+// Two bf16 values packed in a 32-bit word (low half first) as fp32 (exact).
+__device__ __forceinline__ float2 bf16_pair(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
 
 __device__ __forceinline__ float sigmoid_f32(float x) { return __fdividef(1.f, 1.f + ex2_mufu(-x * kLog2e)); }
 
@@ -86,8 +93,10 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
     float4* hstage = bwd_smem;
     // per-warp dB/dC partials of the segment's steps: [warp][step][32 columns]
     float* cstage = reinterpret_cast<float*>(bwd_smem + kBwdWarps * T * 32);
-    // ring of R segments of packed B/C rows (shared by the CTA: one batch row): [slot][step][32]
-    float* bcring = cstage + kBwdWarps * T * 32;
+    // ring of R segments of packed B/C rows (shared by the CTA: one batch row): [slot][step][RB bytes]
+    constexpr int RB = sizeof(IO) == 2 ? 64 : 128;  // bytes of one step's row
+    constexpr int CPR = RB / 16;                    // 16-byte chunks per row
+    uint8_t* bcring = reinterpret_cast<uint8_t*>(cstage + kBwdWarps * T * 32);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cg = lane >> 2, nl = lane & 3, gbase = lane & ~3;
@@ -104,7 +113,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
     IO* du_row = static_cast<IO*>(p.du) + row;
     IO* ddelta_row = static_cast<IO*>(p.ddelta) + row;
     IO* dz_row = p.dz ? static_cast<IO*>(p.dz) + row : nullptr;
-    const float* bcrow = p.bc + static_cast<long long>(b) * p.L * 32;
+    const uint8_t* bcrow = static_cast<const uint8_t*>(p.bc) + static_cast<long long>(b) * p.L * RB;
     float* ckrow = p.ckpt + (static_cast<long long>(b) * p.nseg * p.dim + dd) * 16 + nl * 4;  // segment stride dim*16
     const long long ckstride = static_cast<long long>(p.dim) * 16;
     int srcl[4];  // lanes of this channel, by step owner
@@ -132,15 +141,35 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
         return f2(ex2_mufu(arg.x), ex2_mufu(arg.y));
     };
     auto ckpt_at = [&](int s) { return ckrow + s * ckstride; };
+    // B and C of the lane's 4 chains at one step, from the lane's place in a ring row
+    // (byte 16 nl: fp32 B there and C 64 bytes on; bf16 pairs (B, C, B, C) there).
+    auto load_bc = [&](const uint8_t* r, float2 (&Bv)[2], float2 (&Cv)[2]) {
+        if constexpr (sizeof(IO) == 2) {
+            const uint4 w = *reinterpret_cast<const uint4*>(r);
+            Bv[0] = bf16_pair(w.x); Cv[0] = bf16_pair(w.y); Bv[1] = bf16_pair(w.z); Cv[1] = bf16_pair(w.w);
+        } else {
+            const float4 Bq = ld4(reinterpret_cast<const float*>(r)), Cq = ld4(reinterpret_cast<const float*>(r + 64));
+            Bv[0] = lo(Bq); Bv[1] = hi(Bq); Cv[0] = lo(Cq); Cv[1] = hi(Cq);
+        }
+    };
+    auto load_b = [&](const uint8_t* r, float2 (&Bv)[2]) {
+        if constexpr (sizeof(IO) == 2) {
+            const uint4 w = *reinterpret_cast<const uint4*>(r);
+            Bv[0] = bf16_pair(w.x); Bv[1] = bf16_pair(w.z);
+        } else {
+            const float4 Bq = ld4(reinterpret_cast<const float*>(r));
+            Bv[0] = lo(Bq); Bv[1] = hi(Bq);
+        }
+    };
 
     // B/C rows of segment `seg` into ring slot `slot` (threads 0..63, 16 bytes each; zero
     // past L); every thread commits a group, so that group counts agree across threads.
     auto issue_bc = [&](int seg, int slot) {
-        if (threadIdx.x < T * 8 && seg >= 0 && seg < p.nseg) {
-            const int i = threadIdx.x >> 3, part = threadIdx.x & 7;
+        if (threadIdx.x < T * CPR && seg >= 0 && seg < p.nseg) {
+            const int i = threadIdx.x / CPR, part = threadIdx.x % CPR;
             const int t = seg * T + i;
             const bool in = t < L;
-            cp_async_16(bcring + (slot * T + i) * 32 + part * 4, in ? bcrow + static_cast<long long>(t) * 32 + part * 4 : bcrow,
+            cp_async_16(bcring + (slot * T + i) * RB + part * 16, in ? bcrow + static_cast<long long>(t) * RB + part * 16 : bcrow,
                         in ? 16u : 0u);
         }
         cp_async_commit();
@@ -189,15 +218,16 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
         if (valid) *reinterpret_cast<float4*>(ckpt_at(s)) = make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
         float dt[PER];
         step_sizes(s, cur, dt);
-        const float* bcs = bcring + (s % R) * T * 32 + nl * 4;
+        const uint8_t* bcs = bcring + (s % R) * T * RB + nl * 16;
 #pragma unroll
         for (int i = 0; i < T; ++i) {
             const float dti = __shfl_sync(0xffffffffu, dt[i % PER], srcl[i / PER]);
             const float ui = __shfl_sync(0xffffffffu, cur.u[i % PER], srcl[i / PER]);
-            const float4 Bq = ld4(bcs + i * 32);
+            float2 Bv[2];
+            load_b(bcs + i * RB, Bv);
             const float2 ww = f2(dti * ui, dti * ui);
-            h[0] = __ffma2_rn(decay(dti, 0), h[0], __fmul2_rn(ww, lo(Bq)));
-            h[1] = __ffma2_rn(decay(dti, 1), h[1], __fmul2_rn(ww, hi(Bq)));
+            h[0] = __ffma2_rn(decay(dti, 0), h[0], __fmul2_rn(ww, Bv[0]));
+            h[1] = __ffma2_rn(decay(dti, 1), h[1], __fmul2_rn(ww, Bv[1]));
         }
     }
     cp_async_wait<0>();
@@ -230,7 +260,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
         issue_bc(s - (R - 1), (k + R - 1) % R);
         cp_async_wait<R - 1>();
         __syncthreads();
-        const float* bcs = bcring + (k % R) * T * 32 + nl * 4;
+        const uint8_t* bcs = bcring + (k % R) * T * RB + nl * 16;
         float dt[PER];
         step_sizes(s, cur, dt);
 
@@ -242,13 +272,14 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
         for (int i = 0; i < T; ++i) {
             const float dti = __shfl_sync(0xffffffffu, dt[i % PER], srcl[i / PER]);
             const float ui = __shfl_sync(0xffffffffu, cur.u[i % PER], srcl[i / PER]);
-            const float4 Bq = ld4(bcs + i * 32), Cq = ld4(bcs + i * 32 + 16);
+            float2 Bv[2], Cv[2];
+            load_bc(bcs + i * RB, Bv, Cv);
             const float2 a0 = decay(dti, 0), a1 = decay(dti, 1);
             hst[i * 32 + lane] = make_float4(hs[0].x, hs[0].y, hs[1].x, hs[1].y);
             const float2 ww = f2(dti * ui, dti * ui);
-            hs[0] = __ffma2_rn(a0, hs[0], __fmul2_rn(ww, lo(Bq)));
-            hs[1] = __ffma2_rn(a1, hs[1], __fmul2_rn(ww, hi(Bq)));
-            const float2 acc = __ffma2_rn(hi(Cq), hs[1], __fmul2_rn(lo(Cq), hs[0]));
+            hs[0] = __ffma2_rn(a0, hs[0], __fmul2_rn(ww, Bv[0]));
+            hs[1] = __ffma2_rn(a1, hs[1], __fmul2_rn(ww, Bv[1]));
+            const float2 acc = __ffma2_rn(Cv[1], hs[1], __fmul2_rn(Cv[0], hs[0]));
             vp[i] = acc.x + acc.y;
         }
         // Reduce-scatter over the 4 lanes (upper lane bit first): lane nl ends with the
@@ -288,9 +319,9 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
             const float dti = __shfl_sync(0xffffffffu, dt[i % PER], srcl[i / PER]);
             const float ui = __shfl_sync(0xffffffffu, cur.u[i % PER], srcl[i / PER]);
             const float dvi = __shfl_sync(0xffffffffu, dv[i % PER], srcl[i / PER]);
-            const float4 Bq = ld4(bcs + i * 32), Cq = ld4(bcs + i * 32 + 16);
+            float2 Bv[2], Cv[2];
+            load_bc(bcs + i * RB, Bv, Cv);
             const float4 hq = hst[i * 32 + lane];
-            const float2 Bv[2] = {lo(Bq), hi(Bq)}, Cv[2] = {lo(Cq), hi(Cq)};
             // exp(Delta A) again (the exponential unit has room; the shared-memory path does not)
             const float2 hp[2] = {lo(hq), hi(hq)}, av[2] = {decay(dti, 0), decay(dti, 1)};
             const float2 dv2 = f2(dvi, dvi), dt2 = f2(dti, dti), u2 = f2(ui, ui);

@@ -527,11 +527,18 @@ struct BwdArgs {
 template <typename IO>
 ssm_status_t launch_backward(const BwdArgs& a) {
     const BwdLayout wl = bwd_layout(a.batch, a.dim, a.L);
-    float* bc = reinterpret_cast<float*>(a.ws + wl.bc_off);
+    uint8_t* bc = a.ws + wl.bc_off;
     {
+        // B/C rows for the kernel's ring: bf16 inputs stay bf16 (state pairs), fp32 as rows
         const dim3 grid(static_cast<unsigned>((a.L + 63) / 64), static_cast<unsigned>(a.batch));
-        ssm::pack_bc_kernel<IO><<<grid, 256, 0, a.stream>>>(static_cast<const IO*>(a.B), static_cast<const IO*>(a.C),
-                                                           bc, a.L);
+        if constexpr (sizeof(IO) == 2)
+            ssm::pack_bc_pairs_kernel<<<grid, 256, 0, a.stream>>>(static_cast<const uint16_t*>(a.B),
+                                                                  static_cast<const uint16_t*>(a.C),
+                                                                  reinterpret_cast<uint32_t*>(bc), a.L);
+        else
+            ssm::pack_bc_kernel<IO><<<grid, 256, 0, a.stream>>>(static_cast<const IO*>(a.B),
+                                                               static_cast<const IO*>(a.C),
+                                                               reinterpret_cast<float*>(bc), a.L);
         if (cudaGetLastError() != cudaSuccess) return SSM_ERR_LAUNCH;
     }
     ssm::BwdParams p{};
