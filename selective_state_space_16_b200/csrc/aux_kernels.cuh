@@ -180,8 +180,9 @@ __global__ void __launch_bounds__(128) scan_fwd_direct_kernel(const DirectParams
 // ---------------------------------------------------------------------------------------
 // One-token decode ([Card] 线性扫描算法: one fixed-size state update per token;
 // [Eng] §6.3: the states of a batch laid out on contiguous threads).
-// Four threads per (b, d), each owning 4 of the 16 fp32 state values (one 16-byte
-// vector), so a warp reads and writes 512 contiguous bytes of state.
+// TPC = 16 / NS threads per (b, d) channel, each owning NS consecutive fp32 state values
+// (NS / 4 16-byte vectors), so a warp reads and writes contiguous state.  grid.y is the
+// batch row (B and C are the same for the whole CTA), grid.x covers dim.
 // ---------------------------------------------------------------------------------------
 struct DecodeParams {
     float* state;
@@ -196,7 +197,8 @@ struct DecodeParams {
     void* y;
     int batch, dim;
     int softplus;
-    int zoh;  // zero-order-hold input weight instead of Delta*B
+    int zoh;     // zero-order-hold input weight instead of Delta*B
+    int bc_vec;  // B and C 16-byte aligned: vector loads
     // causal conv1d + SiLU (conv_k > 0): u = silu(conv([conv_state, x])), x given in `u`;
     // conv_state (batch, dim, conv_k - 1) fp32, oldest first, shifted in place
     const float* conv_w;
@@ -205,63 +207,93 @@ struct DecodeParams {
     int conv_k;
 };
 
-// Four threads per (b, d) channel, each one 16-byte quarter of the state; a full grid, one
-// quarter per thread (a lean kernel keeps ~60 warps per SM resident, which is what hides
-// the memory latency of this step).  ZOH and CONV are template flags so that the plain step
-// carries none of their registers.
-template <typename IO, bool ZOH, bool CONV>
-__global__ void __launch_bounds__(256) state_update_kernel(const DecodeParams p) {
-    const long long gid = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
-    const long long row = gid >> 2;  // flat (b, d)
-    const int q = static_cast<int>(gid & 3);
-    const bool valid = row < static_cast<long long>(p.batch) * p.dim;
-    const long long rr = valid ? row : 0;
-    const int b = static_cast<int>(rr / p.dim);
-    const int d = static_cast<int>(rr % p.dim);
-
-    float4 hv = make_float4(0.f, 0.f, 0.f, 0.f);
-    float4 av = make_float4(0.f, 0.f, 0.f, 0.f);
-    float Bq[4] = {0.f, 0.f, 0.f, 0.f}, Cq[4] = {0.f, 0.f, 0.f, 0.f};
-    float ut = 0.f, dt = 0.f, zt = 0.f, Dd = 0.f, xt = 0.f;
-    if (valid) {
-        hv = *reinterpret_cast<const float4*>(p.state + rr * 16 + q * 4);
-        av = *reinterpret_cast<const float4*>(p.A + d * 16 + q * 4);
-        const IO* Bp = static_cast<const IO*>(p.B) + b * 16 + q * 4;
-        const IO* Cp = static_cast<const IO*>(p.C) + b * 16 + q * 4;
+// NS consecutive IO values at src (index in elements) as fp32; `vec`: src is 2*NS- (bf16)
+// or 4*NS-byte aligned (NS = 4, 8 or 16), else element loads.
+template <typename IO, int NS>
+__device__ __forceinline__ void decode_load(const IO* src, bool vec, float (&out)[NS]) {
+    if (vec) {
+        if constexpr (sizeof(IO) == 2) {
+            uint32_t w[NS / 2];
+            if constexpr (NS == 4) {
+                const uint2 v = *reinterpret_cast<const uint2*>(src);
+                w[0] = v.x; w[1] = v.y;
+            } else {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            Bq[j] = IoTraits<IO>::to_f32(Bp[j]);
-            Cq[j] = IoTraits<IO>::to_f32(Cp[j]);
+                for (int k = 0; k < NS / 8; ++k) {
+                    const uint4 v = reinterpret_cast<const uint4*>(src)[k];
+                    w[4 * k] = v.x; w[4 * k + 1] = v.y; w[4 * k + 2] = v.z; w[4 * k + 3] = v.w;
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < NS / 2; ++k) {
+                out[2 * k] = __uint_as_float(w[k] << 16);
+                out[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < NS / 4; ++k) {
+                const float4 v = reinterpret_cast<const float4*>(src)[k];
+                out[4 * k] = v.x; out[4 * k + 1] = v.y; out[4 * k + 2] = v.z; out[4 * k + 3] = v.w;
+            }
         }
-        ut = IoTraits<IO>::to_f32(static_cast<const IO*>(p.u)[rr]);
-        if constexpr (CONV) {  // u = silu(conv([conv_state, x])), rounded to the I/O type
-            const int K = p.conv_k;
-            xt = ut;
-            float pre = p.conv_b ? p.conv_b[d] : 0.f;
-            for (int k = 0; k < K - 1; ++k) pre = fmaf(p.conv_w[d * K + k], p.conv_state[rr * (K - 1) + k], pre);
-            pre = fmaf(p.conv_w[d * K + K - 1], xt, pre);
-            ut = IoTraits<IO>::to_f32(IoTraits<IO>::from_f32(silu_f32(pre)));
-        }
-        const float bias = p.bias ? p.bias[d] : 0.f;
-        dt = step_size(IoTraits<IO>::to_f32(static_cast<const IO*>(p.delta)[rr]), bias, p.softplus != 0);
-        if (p.z) zt = IoTraits<IO>::to_f32(static_cast<const IO*>(p.z)[rr]);
-        Dd = p.D ? p.D[d] : 0.f;
+    } else {
+#pragma unroll
+        for (int k = 0; k < NS; ++k) out[k] = IoTraits<IO>::to_f32(src[k]);
     }
+}
+
+// ZOH and CONV are template flags so that the plain step carries none of their registers.
+template <typename IO, bool ZOH, bool CONV, int NS>
+__global__ void __launch_bounds__(256) state_update_kernel(const DecodeParams p) {
+    constexpr int TPC = 16 / NS;
+    const int b = blockIdx.y;
+    const int tl = blockIdx.x * 256 + threadIdx.x;
+    const int d = tl / TPC, q = tl % TPC;
+    const bool valid = d < p.dim;
+    const int dd = valid ? d : p.dim - 1;
+    const long long rr = static_cast<long long>(b) * p.dim + dd;  // flat (b, d)
+
+    // every load first (state from HBM, the rest mostly from L2), then the arithmetic
+    float hs[NS], as[NS], Bq[NS], Cq[NS];
+#pragma unroll
+    for (int k = 0; k < NS / 4; ++k) {
+        const float4 h4 = reinterpret_cast<const float4*>(p.state + rr * 16 + q * NS)[k];
+        const float4 a4 = reinterpret_cast<const float4*>(p.A + dd * 16 + q * NS)[k];
+        hs[4 * k] = h4.x; hs[4 * k + 1] = h4.y; hs[4 * k + 2] = h4.z; hs[4 * k + 3] = h4.w;
+        as[4 * k] = a4.x; as[4 * k + 1] = a4.y; as[4 * k + 2] = a4.z; as[4 * k + 3] = a4.w;
+    }
+    const bool vec = p.bc_vec != 0;
+    decode_load<IO, NS>(static_cast<const IO*>(p.B) + b * 16 + q * NS, vec, Bq);
+    decode_load<IO, NS>(static_cast<const IO*>(p.C) + b * 16 + q * NS, vec, Cq);
+    float ut = IoTraits<IO>::to_f32(static_cast<const IO*>(p.u)[rr]);
+    const float raw = IoTraits<IO>::to_f32(static_cast<const IO*>(p.delta)[rr]);
+    const float zt = p.z ? IoTraits<IO>::to_f32(static_cast<const IO*>(p.z)[rr]) : 0.f;
+    const float bias = p.bias ? p.bias[dd] : 0.f;
+    const float Dd = p.D ? p.D[dd] : 0.f;
+    float xt = 0.f;
+    if constexpr (CONV) {  // u = silu(conv([conv_state, x])), rounded to the I/O type
+        const int K = p.conv_k;
+        xt = ut;
+        float pre = p.conv_b ? p.conv_b[dd] : 0.f;
+        for (int k = 0; k < K - 1; ++k) pre = fmaf(p.conv_w[dd * K + k], p.conv_state[rr * (K - 1) + k], pre);
+        pre = fmaf(p.conv_w[dd * K + K - 1], xt, pre);
+        ut = IoTraits<IO>::to_f32(IoTraits<IO>::from_f32(silu_f32(pre)));
+    }
+    const float dt = step_size(raw, bias, p.softplus != 0);
     const float w = dt * ut;
-    float hs[4] = {hv.x, hv.y, hv.z, hv.w};
-    const float as[4] = {av.x, av.y, av.z, av.w};
+    const float dl = dt * kLog2e;
     float acc = 0.f;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const float y = dt * as[j] * kLog2e;
+    for (int j = 0; j < NS; ++j) {
+        const float y = dl * as[j];
         const float a = ex2_mufu(y);
         float beta = w * Bq[j];
         if constexpr (ZOH) beta = zoh_beta(y, a, beta, ut * Bq[j] / as[j]);
         hs[j] = fmaf(a, hs[j], beta);
         acc = fmaf(Cq[j], hs[j], acc);
     }
-    acc += __shfl_xor_sync(0xffffffffu, acc, 1, 32);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 2, 32);
+#pragma unroll
+    for (int m = 1; m < TPC; m <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m, 32);
     if constexpr (CONV) {
         if (p.conv_k > 1) {
             __syncwarp();  // every thread of the channel has read conv_state
@@ -273,7 +305,10 @@ __global__ void __launch_bounds__(256) state_update_kernel(const DecodeParams p)
         }
     }
     if (valid) {
-        *reinterpret_cast<float4*>(p.state + rr * 16 + q * 4) = make_float4(hs[0], hs[1], hs[2], hs[3]);
+#pragma unroll
+        for (int k = 0; k < NS / 4; ++k)
+            reinterpret_cast<float4*>(p.state + rr * 16 + q * NS)[k] =
+                make_float4(hs[4 * k], hs[4 * k + 1], hs[4 * k + 2], hs[4 * k + 3]);
         if (q == 0) {
             float v = fmaf(Dd, ut, acc);
             if (p.z) v *= silu_f32(zt);

@@ -26,6 +26,8 @@ using ssm::WorkspaceHeader;
 
 constexpr int kAbiVersion = 2;
 constexpr uint32_t kDefaultWaitLimit = 1u << 22;
+// d_state-16 decode: fp32 state values per thread (4, 8 or 16; 16 / that many threads per channel)
+constexpr int kDecodeStatesPerThread = 8;
 constexpr uint32_t kDefaultSpinLimit = 1u << 21;  // look-back polls (~64 ns sleep each)
 
 size_t round_up(size_t v, size_t m) { return (v + m - 1) / m * m; }
@@ -827,18 +829,19 @@ ssm_status_t ssm_state_update_conv(float* state, float* conv_state, const void* 
         return launch_status();
     }
     ssm::DecodeParams p{state, u, delta, A, B, C, D, z, delta_bias, y, batch, dim, softplus,
-                        discretization == SSM_DISC_ZOH, conv_weight, conv_bias, conv_state, conv_width};
-    const long long threads = static_cast<long long>(batch) * dim * 4;
-    const long long grid = (threads + 255) / 256;
-    if (grid > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
+                        discretization == SSM_DISC_ZOH, aligned16(B) && aligned16(C),
+                        conv_weight, conv_bias, conv_state, conv_width};
+    constexpr int NS = kDecodeStatesPerThread;
+    if (batch > 65535) return SSM_ERR_UNSUPPORTED;
+    const dim3 g(static_cast<unsigned>((static_cast<long long>(dim) * (16 / NS) + 255) / 256),
+                 static_cast<unsigned>(batch));
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const unsigned g = static_cast<unsigned>(grid);
     const bool zoh = discretization == SSM_DISC_ZOH, conv = conv_width > 0;
 #define SSM_DECODE(IO_T)                                                                              \
-    if (zoh && conv) ssm::state_update_kernel<IO_T, true, true><<<g, 256, 0, s>>>(p);                 \
-    else if (zoh) ssm::state_update_kernel<IO_T, true, false><<<g, 256, 0, s>>>(p);                   \
-    else if (conv) ssm::state_update_kernel<IO_T, false, true><<<g, 256, 0, s>>>(p);                  \
-    else ssm::state_update_kernel<IO_T, false, false><<<g, 256, 0, s>>>(p);
+    if (zoh && conv) ssm::state_update_kernel<IO_T, true, true, NS><<<g, 256, 0, s>>>(p);             \
+    else if (zoh) ssm::state_update_kernel<IO_T, true, false, NS><<<g, 256, 0, s>>>(p);               \
+    else if (conv) ssm::state_update_kernel<IO_T, false, true, NS><<<g, 256, 0, s>>>(p);              \
+    else ssm::state_update_kernel<IO_T, false, false, NS><<<g, 256, 0, s>>>(p);
     if (io_dtype == SSM_BF16) {
         SSM_DECODE(__nv_bfloat16)
     } else {

@@ -163,6 +163,28 @@ def test_decode_small_chain(cuda_device, io):
         assert_close(state, st_ref, io, f"decode state step {step}")
 
 
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_decode_unaligned_bc(cuda_device, io):
+    # B and C one element past a 16-byte boundary: the step reads them element by element
+    dec = workloads.decode_inputs(2, 37, io=io, seed=23, pool=1)
+    s = dec["sets"][0]
+    sg = {k: v.cuda() for k, v in s.items()}
+    for k in ("B", "C"):
+        buf = torch.zeros(sg[k].numel() + 1, dtype=sg[k].dtype, device="cuda")
+        buf[1:] = sg[k].reshape(-1)
+        sg[k] = buf[1:].view(sg[k].shape)
+        assert sg[k].data_ptr() % 16 != 0
+    g = dict(A=dec["A"].cuda(), D=dec["D"].cuda(), delta_bias=dec["delta_bias"].cuda())
+    state = dec["state0"].cuda()
+    y = torch.empty_like(sg["u"])
+    _decode_gpu_step(state, sg, g, y)
+    y_ref, st_ref = oracle.state_update(dec["state0"], s["u"], s["delta"], dec["A"], s["B"], s["C"], D=dec["D"],
+                                        z=s["z"], delta_bias=dec["delta_bias"])
+    torch.cuda.synchronize()
+    assert_close(y, y_ref, io, "decode y, unaligned B/C")
+    assert_close(state, st_ref, io, "decode state, unaligned B/C")
+
+
 def test_decode_chain_equals_forward(cuda_device):
     inp = workloads.scan_inputs(2, 40, 64, io="f32", seed=22)
     y_fwd, last_fwd = gpu_forward(inp)
