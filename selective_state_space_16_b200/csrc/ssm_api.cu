@@ -833,15 +833,16 @@ ssm_status_t ssm_state_update_conv(float* state, float* conv_state, const void* 
                         conv_weight, conv_bias, conv_state, conv_width};
     constexpr int NS = kDecodeStatesPerThread;
     if (batch > 65535) return SSM_ERR_UNSUPPORTED;
-    const dim3 g(static_cast<unsigned>((static_cast<long long>(dim) * (16 / NS) + 255) / 256),
+    constexpr int TH = ssm::kDecodeThreads;
+    const dim3 g(static_cast<unsigned>((static_cast<long long>(dim) * (16 / NS) + TH - 1) / TH),
                  static_cast<unsigned>(batch));
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool zoh = discretization == SSM_DISC_ZOH, conv = conv_width > 0;
 #define SSM_DECODE(IO_T)                                                                              \
-    if (zoh && conv) ssm::state_update_kernel<IO_T, true, true, NS><<<g, 256, 0, s>>>(p);             \
-    else if (zoh) ssm::state_update_kernel<IO_T, true, false, NS><<<g, 256, 0, s>>>(p);               \
-    else if (conv) ssm::state_update_kernel<IO_T, false, true, NS><<<g, 256, 0, s>>>(p);              \
-    else ssm::state_update_kernel<IO_T, false, false, NS><<<g, 256, 0, s>>>(p);
+    if (zoh && conv) ssm::state_update_kernel<IO_T, true, true, NS><<<g, TH, 0, s>>>(p);             \
+    else if (zoh) ssm::state_update_kernel<IO_T, true, false, NS><<<g, TH, 0, s>>>(p);               \
+    else if (conv) ssm::state_update_kernel<IO_T, false, true, NS><<<g, TH, 0, s>>>(p);              \
+    else ssm::state_update_kernel<IO_T, false, false, NS><<<g, TH, 0, s>>>(p);
     if (io_dtype == SSM_BF16) {
         SSM_DECODE(__nv_bfloat16)
     } else {
