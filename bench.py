@@ -94,6 +94,8 @@ class ClockSampler:
             else:
                 self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._sample()  # the first queries of a process are slow: make them before timing
+            self.samples, self.reasons = [], set()
         except Exception:
             self._h = None
 
