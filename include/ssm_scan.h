@@ -244,9 +244,11 @@ ssm_status_t ssm_selective_scan_bwd(
  * [Eng] §6.2).  For every (b, d):  h[n] <- exp(Delta*A[d,n]) h[n] + Delta*B[b,n]*u[b,d],
  * y[b,d] = (sum_n C[b,n] h[n] + D[d] u[b,d]) * silu(z[b,d]), with the fp32 state
  * read, modified and written IN PLACE.
- *   state       fp32 (batch, dim, dstate), in/out.
- *   u, delta, z, y: io_dtype (batch, dim);  B, C: io_dtype (batch, dstate).
+ *   state       fp32 (batch, dim, dstate), in/out; state and A 16-byte aligned.
+ *   u, delta, z, y: io_dtype (batch, dim);  B, C: io_dtype (batch, dstate), any alignment
+ *   (read as 16-byte vectors when both are 16-byte aligned).
  *   D, delta_bias, z optional as above.  No workspace.
+ *   d_state 16: batch <= 65535, else SSM_ERR_UNSUPPORTED.
  */
 ssm_status_t ssm_state_update(
     float* state, const void* u, const void* delta, const float* A, const void* B, const void* C,

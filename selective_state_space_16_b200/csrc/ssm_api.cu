@@ -803,6 +803,7 @@ ssm_status_t ssm_state_update_conv(float* state, float* conv_state, const void* 
     if (!dstate_supported(dstate)) return SSM_ERR_UNSUPPORTED;
     if (!aligned16(state) || !aligned16(A)) return SSM_ERR_INVALID_ARG;
     if (batch == 0 || dim == 0) return SSM_OK;
+    if (dstate == 16 && batch > 65535) return SSM_ERR_UNSUPPORTED;  // the batch row is a grid y index
     ssm_status_t st = check_device(nullptr);
     if (st != SSM_OK) return st;
     if (dstate != 16) {
@@ -832,7 +833,6 @@ ssm_status_t ssm_state_update_conv(float* state, float* conv_state, const void* 
                         discretization == SSM_DISC_ZOH, aligned16(B) && aligned16(C),
                         conv_weight, conv_bias, conv_state, conv_width};
     constexpr int NS = kDecodeStatesPerThread;
-    if (batch > 65535) return SSM_ERR_UNSUPPORTED;
     constexpr int TH = ssm::kDecodeThreads;
     const dim3 g(static_cast<unsigned>((static_cast<long long>(dim) * (16 / NS) + TH - 1) / TH),
                  static_cast<unsigned>(batch));

@@ -120,6 +120,7 @@ def test_decode_argument_validation(lib):
     assert call(dstate=24) == binding.SSM_ERR_UNSUPPORTED
     assert call(io=3) == binding.SSM_ERR_INVALID_ARG
     assert call(batch=0) == binding.SSM_OK
+    assert call(batch=65536) == binding.SSM_ERR_UNSUPPORTED  # the batch row is the grid's y index
     assert lib.ssm_state_update_ex(P(4096), P(4096), P(4096), P(4096), P(4096), P(4096), None, None, None, 1,
                                    P(4096), 2, 3, 16, binding.SSM_F32, 5, None) == binding.SSM_ERR_INVALID_ARG
 
