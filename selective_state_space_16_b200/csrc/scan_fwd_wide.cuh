@@ -50,8 +50,14 @@ struct WideCfg {
     static constexpr int kSmem = 2 * kStageFloats * 4;  // double-buffered stages
 };
 
+// Blocks per SM in the launch bound: measured on B200 (batch 4, d_inner 2048, L 2048), 3 blocks
+// (80 registers) take N = 128 from 1.081 to 0.948 ms but spill at N = 32, 64 (0.31 -> 0.33 ms,
+// 0.535 -> 0.547 ms); N = 256 holds 128 KB of B/C stages (one block).
+template <int N>
+constexpr int wide_min_blocks() { return N == 256 ? 1 : N == 128 ? 3 : 2; }
+
 template <typename IO, int N>
-__global__ void __launch_bounds__(WideCfg<N>::kWarps * 32, N == 256 ? 1 : 2) scan_fwd_wide_kernel(const WideParams p) {
+__global__ void __launch_bounds__(WideCfg<N>::kWarps * 32, wide_min_blocks<N>()) scan_fwd_wide_kernel(const WideParams p) {
     using Cfg = WideCfg<N>;
     constexpr int NC = Cfg::kNC, G = Cfg::kG, CPW = Cfg::kCPW, T = Cfg::kT, ST = Cfg::kST;
     static_assert(N == 32 || N == 64 || N == 128 || N == 256, "N in {32, 64, 128, 256}");
