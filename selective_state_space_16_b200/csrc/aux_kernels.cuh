@@ -243,13 +243,13 @@ __device__ __forceinline__ void decode_load(const IO* src, bool vec, float (&out
 }
 
 // ZOH and CONV are template flags so that the plain step carries none of their registers.
-// 128-thread CTAs, at most 40 registers for the plain step (12 CTAs = 48 warps per SM):
-// measured on B200 (b256 d5120, 1000 chained steps) 34.1 us per step, against 35.0 with
-// 256-thread CTAs at the same bound, 37.5 with 256 threads and 42 registers (40 warps) and
-// 41.0 with 32 registers (spills).
-constexpr int kDecodeThreads = 128;
+// 64-thread CTAs, at most 40 registers for the plain step (24 CTAs = 48 warps per SM):
+// measured on B200 (b256 d5120, 1000 chained steps) 33.6 us per step, against 34.4 with
+// 128-thread CTAs and 35.0 with 256 at the same bound, 37.5 with 256 threads and 42
+// registers (40 warps) and 41.0 with 32 registers (spills).
+constexpr int kDecodeThreads = 64;
 template <typename IO, bool ZOH, bool CONV, int NS>
-__global__ void __launch_bounds__(kDecodeThreads, (ZOH || CONV) ? 8 : 12) state_update_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kDecodeThreads, (ZOH || CONV) ? 16 : 24) state_update_kernel(const DecodeParams p) {
     constexpr int TPC = 16 / NS;
     const int b = blockIdx.y;
     const int tl = blockIdx.x * kDecodeThreads + threadIdx.x;
