@@ -291,7 +291,9 @@ ssm_status_t ssm_state_update_ex(
  * more return SSM_ERR_SCRATCH_LIMIT before anything is launched.
  *   - The first call on each device looks up the array's device address (once per
  *     device, with that device current); make that first call before any stream
- *     capture begins.
+ *     capture begins.  The address is kept for the life of the process: after a
+ *     cudaDeviceReset (or any reset of the device's primary context) this entry point
+ *     must not be called again on that device.
  *   - All calls share the one array: calls whose kernels can overlap on the GPU
  *     (different streams, or different host threads) race on it.  Order them on one
  *     stream or synchronise between them.

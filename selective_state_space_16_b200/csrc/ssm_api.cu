@@ -867,8 +867,9 @@ ssm_status_t ssm_selective_scan_fwd_noalloc(const void* u, const void* delta, co
         if (q && !aligned16(q)) return SSM_ERR_INVALID_ARG;
     if (batch == 0 || dim == 0) return SSM_OK;
     if (batch > 65535) return SSM_ERR_UNSUPPORTED;
-    if (ssm_selective_scan_workspace_size(batch, dim, dstate, seqlen) > SSM_NOALLOC_SCRATCH_BYTES)
-        return SSM_ERR_SCRATCH_LIMIT;
+    // The kernels this entry point runs (sequential or direct) use only the header and the
+    // B/C rows, i.e. the workspace up to the look-back region: 256 + round_up(batch*L*128, 256).
+    if (ws_layout(batch, dim, seqlen).flags_off > SSM_NOALLOC_SCRATCH_BYTES) return SSM_ERR_SCRATCH_LIMIT;
     int sm_count = 0;
     ssm_status_t st = check_device(&sm_count);
     if (st != SSM_OK) return st;

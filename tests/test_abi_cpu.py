@@ -163,3 +163,21 @@ def test_backward_argument_validation(lib):
     f = binding.ssm_selective_scan_bwd_workspace_size
     assert f(4, 5120, 16, 2048) % 256 == 0 and f(4, 5120, 16, 2048) > 4 * 2048 * 128
     assert f(1, 1, 8, 1) == 0
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(),
+                    reason="fake pointers: an accepted call would launch kernels on a real device")
+def test_noalloc_scratch_limit_follows_its_formula(lib):
+    """ssm_selective_scan_fwd_noalloc accepts every problem whose header + transposed B/C rows
+    (256 + round_up(batch * seqlen * 128, 256) bytes) fit its 8 MiB scratch, whatever dim is.
+    Without a device an accepted call stops at the device check (SSM_ERR_LAUNCH); a rejected
+    one returns SSM_ERR_SCRATCH_LIMIT before that."""
+    def call(batch, dim, L):
+        return lib.ssm_selective_scan_fwd_noalloc(P(4096), P(4096), P(4096), P(4096), P(4096), None, None, None, 1,
+                                                  P(4096), None, batch, dim, 16, L, binding.SSM_BF16, None)
+    accepted = [(1, 5120, 2048), (4, 5120, 256), (8, 1536, 2048), (4, 5120, 2048), (1, 5120, 65534),
+                (2, 5120, 32767)]
+    for shape in accepted:
+        assert call(*shape) == binding.SSM_ERR_LAUNCH, shape
+    for shape in [(1, 64, 65536), (1, 5120, 65535), (4, 8, 1 << 15), (3, 5120, 21845)]:
+        assert call(*shape) == binding.SSM_ERR_SCRATCH_LIMIT, shape
