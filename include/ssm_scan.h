@@ -59,8 +59,21 @@ typedef enum {
     SSM_ERR_LAUNCH = 3,        /* a CUDA call or kernel launch failed                           */
     SSM_ERR_TIMEOUT = 4,       /* device: a bounded wait in the kernel gave up (see read_status) */
     SSM_ERR_WORKSPACE = 5,     /* workspace missing or smaller than ssm_selective_scan_workspace_size */
-    SSM_ERR_SCRATCH_LIMIT = 6  /* the problem needs more than the fixed scratch of ssm_selective_scan_fwd_noalloc */
+    SSM_ERR_SCRATCH_LIMIT = 6, /* the problem needs more than the fixed scratch of ssm_selective_scan_fwd_noalloc */
+    SSM_ERR_BOUNDS = 7         /* device, debug library only: an index range check failed (see below) */
 } ssm_status_t;
+
+/*
+ * Debug library.  libssm_scan_debug.so is the same library compiled with -DSSM_DEBUG_CHECKS:
+ * the kernels range-check their shared-memory offsets, TMA coordinates and global indices,
+ * and a failed check records SSM_ERR_BOUNDS in the workspace status word (read back with
+ * ssm_read_status) and skips the access instead of touching memory.  It stands in for a
+ * memory checker; the release library compiles every check away.
+ *
+ * Fault injection.  With the environment variable SSM_FAKE_LAUNCH_FAILURE set (to any value),
+ * every call that would launch a kernel returns SSM_ERR_LAUNCH before launching anything, as
+ * if the launch had failed; it lets callers test their error handling without a GPU fault.
+ */
 
 typedef enum { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype_t;
 

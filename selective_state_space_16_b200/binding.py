@@ -8,6 +8,7 @@ fallback.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import threading
@@ -16,9 +17,10 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libssm_scan.so")
+DEBUG_LIB_PATH = os.path.join(_HERE, "libssm_scan_debug.so")
 
 (SSM_OK, SSM_ERR_INVALID_ARG, SSM_ERR_UNSUPPORTED, SSM_ERR_LAUNCH, SSM_ERR_TIMEOUT, SSM_ERR_WORKSPACE,
- SSM_ERR_SCRATCH_LIMIT) = range(7)
+ SSM_ERR_SCRATCH_LIMIT, SSM_ERR_BOUNDS) = range(8)
 NOALLOC_SCRATCH_BYTES = 8 << 20
 SSM_F32, SSM_BF16 = 0, 1
 SSM_ALGO_AUTO, SSM_ALGO_SEQUENTIAL, SSM_ALGO_CHUNKED, SSM_ALGO_DIRECT = range(4)
@@ -51,6 +53,44 @@ _lib = None
 _lock = threading.Lock()
 
 
+def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
+    """Declare the argument and result types of every entry point of a loaded library."""
+    vp, ci, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    lib.ssm_abi_version.restype = ci
+    lib.ssm_status_string.argtypes = [ci]
+    lib.ssm_status_string.restype = ctypes.c_char_p
+    lib.ssm_selective_scan_workspace_size.argtypes = [ci, ci, ci, i64]
+    lib.ssm_selective_scan_workspace_size.restype = sz
+    lib.ssm_workspace_init.argtypes = [vp, sz, vp]
+    lib.ssm_workspace_init.restype = ci
+    fwd = [vp, vp, vp, vp, vp, vp, vp, vp, ci, vp, vp, ci, ci, ci, i64, ci, vp, sz]
+    lib.ssm_selective_scan_fwd.argtypes = fwd + [vp]
+    lib.ssm_selective_scan_fwd.restype = ci
+    lib.ssm_selective_scan_fwd_ex.argtypes = fwd + [ctypes.POINTER(FwdOptions), vp]
+    lib.ssm_selective_scan_fwd_ex.restype = ci
+    lib.ssm_selective_scan_fwd_state.argtypes = fwd[:9] + [vp] + fwd[9:] + [ctypes.POINTER(FwdOptions), vp]
+    lib.ssm_selective_scan_fwd_state.restype = ci
+    lib.ssm_selective_scan_fwd_noalloc.argtypes = fwd[:16] + [vp]
+    lib.ssm_selective_scan_fwd_noalloc.restype = ci
+    lib.ssm_selective_scan_bwd_workspace_size.argtypes = [ci, ci, ci, i64]
+    lib.ssm_selective_scan_bwd_workspace_size.restype = sz
+    lib.ssm_selective_scan_bwd.argtypes = [vp] * 8 + [ci] + [vp] * 12 + [ci, ci, ci, i64, ci, vp, sz, vp]
+    lib.ssm_selective_scan_bwd.restype = ci
+    lib.ssm_state_update.argtypes = [vp] * 9 + [ci, vp, ci, ci, ci, ci, vp]
+    lib.ssm_state_update.restype = ci
+    lib.ssm_state_update_ex.argtypes = [vp] * 9 + [ci, vp, ci, ci, ci, ci, ci, vp]
+    lib.ssm_state_update_ex.restype = ci
+    lib.ssm_state_update_conv.argtypes = [vp] * 5 + [ci] + [vp] * 7 + [ci, vp, ci, ci, ci, ci, ci, vp]
+    lib.ssm_state_update_conv.restype = ci
+    lib.ssm_selective_scan_fwd_conv.argtypes = ([vp, ctypes.POINTER(ConvSpec)] + [vp] * 7 + [ci] +
+                                                [vp] * 3 + [ci, ci, ci, i64, ci, vp, sz,
+                                                            ctypes.POINTER(FwdOptions), vp])
+    lib.ssm_selective_scan_fwd_conv.restype = ci
+    lib.ssm_read_status.argtypes = [vp, vp]
+    lib.ssm_read_status.restype = ci
+    return lib
+
+
 def load() -> ctypes.CDLL:
     """Load libssm_scan.so (raises if it was not built: run __graft_entry__.build())."""
     global _lib
@@ -58,42 +98,26 @@ def load() -> ctypes.CDLL:
         if _lib is None:
             if not os.path.exists(LIB_PATH):
                 raise ImportError(f"{LIB_PATH} is missing; build it with selective_state_space_16_b200/build.py")
-            lib = ctypes.CDLL(LIB_PATH)
-            vp, ci, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
-            lib.ssm_abi_version.restype = ci
-            lib.ssm_status_string.argtypes = [ci]
-            lib.ssm_status_string.restype = ctypes.c_char_p
-            lib.ssm_selective_scan_workspace_size.argtypes = [ci, ci, ci, i64]
-            lib.ssm_selective_scan_workspace_size.restype = sz
-            lib.ssm_workspace_init.argtypes = [vp, sz, vp]
-            lib.ssm_workspace_init.restype = ci
-            fwd = [vp, vp, vp, vp, vp, vp, vp, vp, ci, vp, vp, ci, ci, ci, i64, ci, vp, sz]
-            lib.ssm_selective_scan_fwd.argtypes = fwd + [vp]
-            lib.ssm_selective_scan_fwd.restype = ci
-            lib.ssm_selective_scan_fwd_ex.argtypes = fwd + [ctypes.POINTER(FwdOptions), vp]
-            lib.ssm_selective_scan_fwd_ex.restype = ci
-            lib.ssm_selective_scan_fwd_state.argtypes = fwd[:9] + [vp] + fwd[9:] + [ctypes.POINTER(FwdOptions), vp]
-            lib.ssm_selective_scan_fwd_state.restype = ci
-            lib.ssm_selective_scan_fwd_noalloc.argtypes = fwd[:16] + [vp]
-            lib.ssm_selective_scan_fwd_noalloc.restype = ci
-            lib.ssm_selective_scan_bwd_workspace_size.argtypes = [ci, ci, ci, i64]
-            lib.ssm_selective_scan_bwd_workspace_size.restype = sz
-            lib.ssm_selective_scan_bwd.argtypes = [vp] * 8 + [ci] + [vp] * 12 + [ci, ci, ci, i64, ci, vp, sz, vp]
-            lib.ssm_selective_scan_bwd.restype = ci
-            lib.ssm_state_update.argtypes = [vp] * 9 + [ci, vp, ci, ci, ci, ci, vp]
-            lib.ssm_state_update.restype = ci
-            lib.ssm_state_update_ex.argtypes = [vp] * 9 + [ci, vp, ci, ci, ci, ci, ci, vp]
-            lib.ssm_state_update_ex.restype = ci
-            lib.ssm_state_update_conv.argtypes = [vp] * 5 + [ci] + [vp] * 7 + [ci, vp, ci, ci, ci, ci, ci, vp]
-            lib.ssm_state_update_conv.restype = ci
-            lib.ssm_selective_scan_fwd_conv.argtypes = ([vp, ctypes.POINTER(ConvSpec)] + [vp] * 7 + [ci] +
-                                                        [vp] * 3 + [ci, ci, ci, i64, ci, vp, sz,
-                                                                    ctypes.POINTER(FwdOptions), vp])
-            lib.ssm_selective_scan_fwd_conv.restype = ci
-            lib.ssm_read_status.argtypes = [vp, vp]
-            lib.ssm_read_status.restype = ci
-            _lib = lib
+            _lib = _declare(ctypes.CDLL(LIB_PATH))
     return _lib
+
+
+@contextlib.contextmanager
+def use_debug_library():
+    """Route every call of this module through libssm_scan_debug.so (the range-checked
+    build) inside the `with` block."""
+    global _lib
+    if not os.path.exists(DEBUG_LIB_PATH):
+        raise ImportError(f"{DEBUG_LIB_PATH} is missing; build it with build.py --debug")
+    debug = _declare(ctypes.CDLL(DEBUG_LIB_PATH))
+    with _lock:
+        saved = load() if _lib is None else _lib
+        _lib = debug
+    try:
+        yield debug
+    finally:
+        with _lock:
+            _lib = saved
 
 
 def status_string(code: int) -> str:

@@ -7,6 +7,10 @@ looked up at run time, so the .so loads on machines without a GPU driver.
 Each kernel family is its own translation unit (csrc/*.cu); they are compiled to
 objects in parallel (csrc/_build/) and linked into one library.  An object is
 rebuilt when its source or any header it includes (transitively) is newer.
+
+build(debug=True) makes libssm_scan_debug.so (objects in csrc/_build_debug/): the
+same sources with -DSSM_DEBUG_CHECKS, whose kernels range-check their indices and
+report SSM_ERR_BOUNDS through the workspace status word instead of faulting.
 """
 from __future__ import annotations
 
@@ -22,6 +26,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 OBJ = os.path.join(CSRC, "_build")
 LIB = os.path.join(HERE, "libssm_scan.so")
+OBJ_DEBUG = os.path.join(CSRC, "_build_debug")
+LIB_DEBUG = os.path.join(HERE, "libssm_scan_debug.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -55,8 +61,8 @@ def sources():
     return sorted(out)
 
 
-def _obj(unit):
-    return os.path.join(OBJ, os.path.basename(unit)[:-3] + ".o")
+def _obj(unit, debug=False):
+    return os.path.join(OBJ_DEBUG if debug else OBJ, os.path.basename(unit)[:-3] + ".o")
 
 
 def _stale(target, deps):
@@ -66,14 +72,15 @@ def _stale(target, deps):
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def stale() -> bool:
-    return _stale(LIB, sources())
+def stale(debug: bool = False) -> bool:
+    return _stale(LIB_DEBUG if debug else LIB, sources())
 
 
-def _compile(unit, extra, verbose):
-    obj = _obj(unit)
+def _compile(unit, extra, verbose, debug=False):
+    obj = _obj(unit, debug)
     tmp = obj + f".tmp{os.getpid()}"
-    cmd = [NVCC, *COMPILE_FLAGS, *extra, "-I", os.path.join(ROOT, "include"), "-c", unit, "-o", tmp]
+    cmd = [NVCC, *COMPILE_FLAGS, *(["-DSSM_DEBUG_CHECKS"] if debug else []), *extra, "-I",
+           os.path.join(ROOT, "include"), "-c", unit, "-o", tmp]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -85,24 +92,24 @@ def _compile(unit, extra, verbose):
     return obj
 
 
-def build(force: bool = False, verbose: bool = False, extra=(), jobs: int | None = None) -> str:
-    if not force and not stale():
-        return LIB
-    os.makedirs(OBJ, exist_ok=True)
-    todo = [u for u in units() if force or _stale(_obj(u), _deps(u))]
+def build(force: bool = False, verbose: bool = False, extra=(), jobs: int | None = None, debug: bool = False) -> str:
+    lib = LIB_DEBUG if debug else LIB
+    if not force and not stale(debug):
+        return lib
+    os.makedirs(OBJ_DEBUG if debug else OBJ, exist_ok=True)
+    todo = [u for u in units() if force or _stale(_obj(u, debug), _deps(u))]
     jobs = jobs or max(1, min(len(todo), os.cpu_count() or 1))
     with ThreadPoolExecutor(max_workers=jobs) as ex:
-        list(ex.map(lambda u: _compile(u, list(extra), verbose), todo))
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [NVCC, *LINK_FLAGS, "-o", tmp, *[_obj(u) for u in units()]]
+        list(ex.map(lambda u: _compile(u, list(extra), verbose, debug), todo))
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = [NVCC, *LINK_FLAGS, "-o", tmp, *[_obj(u, debug) for u in units()]]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True,
-          extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else [])
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose=True, debug="--debug" in sys.argv,
+                extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else []))

@@ -87,6 +87,7 @@ const char* ssm_status_string(ssm_status_t s) {
         case SSM_ERR_TIMEOUT: return "device wait timed out";
         case SSM_ERR_WORKSPACE: return "workspace missing or too small";
         case SSM_ERR_SCRATCH_LIMIT: return "problem larger than the fixed scratch of the no-allocation entry point";
+        case SSM_ERR_BOUNDS: return "device index out of range (debug library check)";
     }
     return "unknown status";
 }

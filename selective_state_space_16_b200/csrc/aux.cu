@@ -13,7 +13,8 @@ ssm_status_t launch_pack(const FwdArgs& a) {
     const dim3 grid(static_cast<unsigned>((a.L + 63) / 64), static_cast<unsigned>(a.batch));
     ssm::pack_bc_kernel<IO><<<grid, 256, 0, a.stream>>>(
         static_cast<const IO*>(a.B), static_cast<const IO*>(a.C),
-        reinterpret_cast<float*>(a.ws + ws_layout(a.batch, a.dim, a.L).bc_off), a.L);
+        reinterpret_cast<float*>(a.ws + ws_layout(a.batch, a.dim, a.L).bc_off), a.L,
+        reinterpret_cast<WorkspaceHeader*>(a.ws));
     return launch_status();
 }
 
@@ -41,6 +42,7 @@ ssm_status_t launch_direct(const FwdArgs& a) {
     p.conv_out = a.conv.out;
     p.u_out = a.conv.u_out;
     p.conv_k = a.conv.k;
+    p.hdr = reinterpret_cast<WorkspaceHeader*>(a.ws);
     constexpr int G = 2;
     const long long threads = static_cast<long long>(a.batch) * a.dim * G;
     const long long grid = (threads + 127) / 128;
@@ -60,7 +62,8 @@ ssm_status_t launch_pack_bwd(const BwdArgs& a, uint8_t* bc) {
                                                               reinterpret_cast<uint32_t*>(bc), a.L);
     else
         ssm::pack_bc_kernel<IO><<<grid, 256, 0, a.stream>>>(static_cast<const IO*>(a.B), static_cast<const IO*>(a.C),
-                                                           reinterpret_cast<float*>(bc), a.L);
+                                                           reinterpret_cast<float*>(bc), a.L,
+                                                           reinterpret_cast<WorkspaceHeader*>(a.ws));
     return launch_status();
 }
 

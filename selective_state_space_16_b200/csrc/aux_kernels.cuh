@@ -22,7 +22,7 @@ namespace ssm {
 // ---------------------------------------------------------------------------------------
 template <typename IO>
 __global__ void __launch_bounds__(256) pack_bc_kernel(const IO* __restrict__ B, const IO* __restrict__ C,
-                                                      float* __restrict__ bc, long long L) {
+                                                      float* __restrict__ bc, long long L, WorkspaceHeader* hdr) {
     __shared__ float tile[32][65];
     const int b = blockIdx.y;
     const long long t0 = static_cast<long long>(blockIdx.x) * 64;
@@ -36,7 +36,9 @@ __global__ void __launch_bounds__(256) pack_bc_kernel(const IO* __restrict__ B, 
     for (int idx = threadIdx.x; idx < 32 * 64; idx += 256) {
         const int c = idx >> 5, r = idx & 31;
         const long long t = t0 + c;
-        if (t < L) bc[(static_cast<long long>(b) * L + t) * 32 + r] = tile[r][c];
+        if (t < L && dcheck(hdr, (static_cast<long long>(b) * L + t) * 32 + r < static_cast<long long>(gridDim.y) * L * 32,
+                            kSitePack, t))
+            bc[(static_cast<long long>(b) * L + t) * 32 + r] = tile[r][c];
     }
 }
 
@@ -95,6 +97,7 @@ struct DirectParams {
     float* conv_out;       // (batch, dim, conv_k - 1) or null
     void* u_out;           // (batch, dim, L) IO or null
     int conv_k;            // 0: no conv
+    WorkspaceHeader* hdr;  // status word (debug range checks)
 };
 
 template <typename IO, int G>
@@ -149,7 +152,10 @@ __global__ void __launch_bounds__(128) scan_fwd_direct_kernel(const DirectParams
             }
         }
         const float w = dt * ut;
-        const float* row = bcb + t * 32;
+        const float* row = dcheck(p.hdr, (static_cast<long long>(b) * p.L + t) * 32 + 32 <= static_cast<long long>(p.batch) * p.L * 32,
+                                  kSiteDirect, t)
+                               ? bcb + t * 32
+                               : p.bc;
         float acc = 0.f;
 #pragma unroll
         for (int j = 0; j < NC; ++j) {
@@ -162,13 +168,14 @@ __global__ void __launch_bounds__(128) scan_fwd_direct_kernel(const DirectParams
         }
 #pragma unroll
         for (int m = G / 2; m >= 1; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m, 32);
-        if (valid && nl == 0) {
+        if (valid && nl == 0 && dcheck(p.hdr, ch * p.L + t < static_cast<long long>(p.batch) * p.dim * p.L, kSiteDirect, t)) {
             float v = fmaf(Dd, ut, acc);
             if (z) v *= silu_f32(IoTraits<IO>::to_f32(z[t]));
             y[t] = IoTraits<IO>::from_f32(v);
         }
     }
-    if (valid && p.last_state) {
+    if (valid && p.last_state &&
+        dcheck(p.hdr, ch * 16 + nl * NC + NC <= static_cast<long long>(p.batch) * p.dim * 16, kSiteDirect, ch)) {
         float* dst = p.last_state + ch * 16 + nl * NC;
 #pragma unroll
         for (int j = 0; j < NC; ++j) dst[j] = h[j];

@@ -53,6 +53,7 @@ ssm_status_t launch_backward(const BwdArgs& a) {
     p.nseg = wl.nseg;
     p.ncta = wl.ncta;
     p.softplus = a.softplus;
+    p.hdr = reinterpret_cast<WorkspaceHeader*>(a.ws);
     constexpr int smem = ssm::kBwdSmem;
     auto kern = ssm::scan_bwd_kernel<IO>;
     if (!ensure_smem_attr(reinterpret_cast<const void*>(kern), smem)) return SSM_ERR_LAUNCH;

@@ -181,6 +181,36 @@ __device__ __forceinline__ void report_status(WorkspaceHeader* hdr, uint32_t cod
     }
 }
 
+// Range checks of the debug build (-DSSM_DEBUG_CHECKS).  dcheck(hdr, ok, site, value)
+// returns ok; when ok is false it records kDevBounds in the workspace header with
+// where = {site, block, thread, value}, and the caller skips the guarded access, so a bad
+// index is reported instead of touching memory.  Release builds compile every check away
+// (dcheck is constant true and its arguments are never evaluated for effect).
+constexpr uint32_t kDevBounds = 7u;
+enum DcheckSite : uint32_t {
+    kSiteSeqTile = 1,       // sequential kernel: tile / batch-row slot of a consumer lane in the round
+    kSiteSeqTma = 2,        // sequential kernel: TMA destination or coordinate of a stage copy
+    kSiteSeqY = 3,          // sequential kernel: y element index
+    kSiteSeqState = 4,      // sequential kernel: last_state index
+    kSiteChunkKey = 5,      // chunked kernel: look-back key (flags / payload)
+    kSiteChunkSmem = 6,     // chunked kernel: shared aggregate / speculative carry index
+    kSiteChunkY = 7,        // chunked kernel: y element or last_state index
+    kSiteDirect = 8,        // direct kernel: B/C row, y or last_state index
+    kSitePack = 9,          // B/C transpose: workspace row index
+    kSiteBwdCkpt = 10,      // backward: checkpoint index
+    kSiteBwdPart = 11,      // backward: per-CTA dB/dC partial index
+    kSiteBwdOut = 12,       // backward: gradient element index
+    kSiteBwdSmem = 13,      // backward: shared ring / per-warp buffer offset
+};
+#ifdef SSM_DEBUG_CHECKS
+__device__ __forceinline__ bool dcheck(WorkspaceHeader* hdr, bool ok, uint32_t site, long long value) {
+    if (!ok) report_status(hdr, kDevBounds, site, blockIdx.x, threadIdx.x, static_cast<uint32_t>(value));
+    return ok;
+}
+#else
+__device__ __forceinline__ constexpr bool dcheck(WorkspaceHeader*, bool, uint32_t, long long) { return true; }
+#endif
+
 // ---------------------------------------------------------------------------------------
 // Element types
 // ---------------------------------------------------------------------------------------

@@ -1,4 +1,5 @@
 // host_common.cu -- definitions of the shared host helpers declared in host_common.h.
+#include <cstdlib>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -61,6 +62,9 @@ bool ensure_smem_attr(const void* kernel, int bytes) {
 }
 
 ssm_status_t check_device(int* sm_count) {
+    // Host-side fault injection (documented in ssm_scan.h): report a failed launch before
+    // anything is launched.
+    if (std::getenv("SSM_FAKE_LAUNCH_FAILURE") != nullptr) return SSM_ERR_LAUNCH;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return SSM_ERR_LAUNCH;
     int major = 0;

@@ -58,7 +58,8 @@ bool make_map_3d(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* 
 bool ensure_smem_attr(const void* kernel, int bytes);
 
 // SSM_OK on an sm_100 device (and its SM count), SSM_ERR_UNSUPPORTED on another
-// architecture, SSM_ERR_LAUNCH when no device can be queried.
+// architecture, SSM_ERR_LAUNCH when no device can be queried (or when the fault-injection
+// variable SSM_FAKE_LAUNCH_FAILURE is set).
 ssm_status_t check_device(int* sm_count);
 
 inline ssm_status_t launch_status() {

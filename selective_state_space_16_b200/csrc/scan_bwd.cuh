@@ -71,6 +71,7 @@ struct BwdParams {
     long long L;
     int nseg, ncta;
     int softplus;
+    WorkspaceHeader* hdr;            // status word (debug range checks)
 };
 
 // Two bf16 values packed in a 32-bit word (low half first) as fp32 (exact).
@@ -215,7 +216,8 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
         issue_bc(s + R - 1, (s + R - 1) % R);
         cp_async_wait<R - 1>();
         __syncthreads();              // segment s's B/C rows are visible to every warp
-        if (valid) *reinterpret_cast<float4*>(ckpt_at(s)) = make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
+        if (valid && dcheck(p.hdr, s < p.nseg, kSiteBwdCkpt, s))
+            *reinterpret_cast<float4*>(ckpt_at(s)) = make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
         float dt[PER];
         step_sizes(s, cur, dt);
         const uint8_t* bcs = bcring + (s % R) * T * RB + nl * 16;
@@ -372,7 +374,8 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
 #pragma unroll
         for (int r = 0; r < PER; ++r) {
             const int t = t0 + nl * PER + r;
-            if (valid && t < L) {
+            if (valid && t < L &&
+                dcheck(p.hdr, row + t < static_cast<long long>(p.batch) * p.dim * L, kSiteBwdOut, t)) {
                 const float dx = softplus ? ddt[r] * sigmoid_f32(cur.x[r] + bias) : ddt[r];
                 dbias_acc += dx;
                 ddelta_row[t] = IoTraits<IO>::from_f32(dx);
@@ -389,7 +392,8 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
             float sum = 0.f;
 #pragma unroll
             for (int w = 0; w < kBwdWarps; ++w) sum += cstage[(w * T + i) * 32 + c];
-            if (t < L) p.dbc_part[((static_cast<long long>(b) * p.ncta + blockIdx.x) * p.L + t) * 32 + c] = sum;
+            if (t < L && dcheck(p.hdr, blockIdx.x < static_cast<unsigned>(p.ncta) && b < p.batch, kSiteBwdPart, t))
+                p.dbc_part[((static_cast<long long>(b) * p.ncta + blockIdx.x) * p.L + t) * 32 + c] = sum;
         }
     }
     cp_async_wait<0>();

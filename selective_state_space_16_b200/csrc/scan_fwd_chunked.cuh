@@ -165,7 +165,8 @@ scan_fwd_chunked_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_
             }
             // lane = wc * 16 + cg * 4 + nl: column wc, channel cg, chains nl*4 .. nl*4+3
             int okc = 0;
-            if (k > 0) {
+            const long long nkeys = p.total_tiles * 2 * p.nchunks;
+            if (k > 0 && dcheck(p.hdr, ((tile * 2 + (lane >> 4)) * p.nchunks + k - 1) < nkeys, kSiteChunkKey, tk)) {
                 const int wc = lane >> 4;
                 const long long key = (tile * 2 + wc) * p.nchunks + (k - 1);
                 const uint32_t f = ld_acquire_gpu(p.flags + key);
@@ -286,7 +287,9 @@ scan_fwd_chunked_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_
 
             // Decoupled look-back (the last time-warp of each column; slice-1 lanes carry
             // the payload for their 4 chains, lane 0 polls the flags).
-            if (lookback_warp) {
+            if (lookback_warp &&
+                dcheck(p.hdr, (tile * 2 + wc) * p.nchunks + k < p.total_tiles * 2 * p.nchunks && k < p.nchunks,
+                       kSiteChunkKey, tk)) {
                 const long long key = (tile * 2 + wc) * p.nchunks + k;
                 // unit aggregate: fold the time-warps' pairs in order
                 float hu[4], pu[4];
@@ -452,7 +455,9 @@ scan_fwd_chunked_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_
                     yo[r] = v;
                 }
                 const int t0 = k * TC + g * GS + nl * PER;
-                if (valid) {
+                if (valid && dcheck(p.hdr, t0 >= p.L || (static_cast<long long>(b) * p.dim + d) * p.L + t0 <
+                                                              static_cast<long long>(p.batch) * p.dim * p.L,
+                                    kSiteChunkY, t0)) {
                     IO* yrow = static_cast<IO*>(p.y) + (static_cast<long long>(b) * p.dim + d) * p.L;
                     if (t0 + PER <= p.L) {
                         store_run<IO, PER>(yrow + t0, yo);
@@ -464,7 +469,9 @@ scan_fwd_chunked_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_
                 }
             }
             // The state after the last step of the sequence (steps past L are identities).
-            if (valid && p.last_state && k == p.nchunks - 1 && wt == NWT - 1 && s == 1) {
+            if (valid && p.last_state && k == p.nchunks - 1 && wt == NWT - 1 && s == 1 &&
+                dcheck(p.hdr, (static_cast<long long>(b) * p.dim + d) * 16 + 16 <= static_cast<long long>(p.batch) * p.dim * 16,
+                       kSiteChunkY, d)) {
                 float* dst = p.last_state + (static_cast<long long>(b) * p.dim + d) * 16 + nl * 4;
                 *reinterpret_cast<float4*>(dst) = make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
             }

@@ -173,7 +173,12 @@ __device__ __forceinline__ void seq_consumer(uint8_t* smem, uint64_t* full_bar, 
         // Byte offset of the lane's 16-byte chunk of group g inside a u/delta/z tile block:
         // cbase ^ (g << 4) (the 128-byte swizzle XORs the chunk index with the row).
         cbase[c] = j * Cfg::kTileBytes + row * 128 + (row << 4);
+        if (!dcheck(p.hdr, j < p.max_tiles && tile < p.total_tiles, kSiteSeqTile, j)) {
+            valid[c] = false;
+            cbase[c] = row * 128 + (row << 4);
+        }
     }
+    if (!dcheck(p.hdr, b >= b_first && b - b_first < Cfg::kMaxBatchRows, kSiteSeqTile, b - b_first)) b = b_first;
     const int dl_off = p.max_tiles * Cfg::kTileBytes;
     const int z_off = 2 * p.max_tiles * Cfg::kTileBytes;
     const int bc_off = 3 * p.max_tiles * Cfg::kTileBytes + (b - b_first) * Cfg::kBC + nl * NC * 4;
@@ -376,7 +381,11 @@ __device__ __forceinline__ void seq_consumer(uint8_t* smem, uint64_t* full_bar, 
                 if constexpr (HZ) v *= gate_silu<IO>(ze[r]);
                 yo[r] = v;
             }
-            if (valid[c]) {
+            // (steps at or past L store nothing)
+            if (valid[c] &&
+                dcheck(p.hdr, t0 >= L32 || (static_cast<long long>(b) * p.dim + d[c]) * p.L + t0 <
+                                               static_cast<long long>(p.batch) * p.dim * p.L,
+                       kSiteSeqY, t0)) {
                 if (t0 + PER <= L32) {
                     store_run<IO, PER>(yrow[c] + t0, yo);
                 } else {
@@ -441,7 +450,9 @@ __device__ __forceinline__ void seq_consumer(uint8_t* smem, uint64_t* full_bar, 
     }
 #pragma unroll
     for (int c = 0; c < CPL; ++c)
-        if (valid[c] && p.last_state) {
+        if (valid[c] && p.last_state &&
+            dcheck(p.hdr, (static_cast<long long>(b) * p.dim + d[c]) * 16 + nl * NC + NC <= static_cast<long long>(p.batch) * p.dim * 16,
+                   kSiteSeqState, d[c])) {
             float* dst = p.last_state + (static_cast<long long>(b) * p.dim + d[c]) * 16 + nl * NC;
 #pragma unroll
             for (int jj = 0; jj < NC / 2; ++jj) *reinterpret_cast<float2*>(dst + 2 * jj) = h[c][jj];
@@ -513,9 +524,16 @@ scan_fwd_seq_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_cons
                         break;
                     }
                     uint8_t* st = smem + s * stage_bytes;
+                    const int t0 = k * TC;
+                    // the TMA x coordinate must be 16-byte aligned; every copy lands inside the slot
+                    if (!dcheck(p.hdr, (t0 % TC) == 0 && nt <= p.max_tiles && nb <= Cfg::kMaxBatchRows &&
+                                           b_first + nb <= p.batch,
+                                kSiteSeqTma, t0)) {
+                        atomicExch(&abort_flag, 1);
+                        break;
+                    }
                     fence_proxy_async_smem();
                     mbar_arrive_expect_tx(&full_bar[s], bytes);
-                    const int t0 = k * TC;
                     for (int j = 0; j < nt; ++j) {
                         const long long tile = r_begin + j;
                         const int b = static_cast<int>(tile / p.tiles_per_batch);

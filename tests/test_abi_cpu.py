@@ -45,9 +45,21 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in range(7):
-        assert binding.status_string(code)
+    for code in range(8):
+        assert binding.status_string(code) != "unknown status"
     assert "workspace" in binding.status_string(binding.SSM_ERR_WORKSPACE)
+    assert "range" in binding.status_string(binding.SSM_ERR_BOUNDS)
+
+
+def test_debug_library_builds_and_exports_every_declared_symbol():
+    """The range-checked build (-DSSM_DEBUG_CHECKS) compiles and offers the same C ABI."""
+    from selective_state_space_16_b200 import build as b
+    path = b.build(debug=True)
+    import ctypes as ct
+    dbg = ct.CDLL(path)
+    missing = [n for n in _declared_functions() if not hasattr(dbg, n)]
+    assert not missing, missing
+    assert dbg.ssm_abi_version() == 2
 
 
 def test_workspace_size(lib):
