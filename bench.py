@@ -78,7 +78,7 @@ class ClockSampler:
                0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
-    def __init__(self, device_index: int, period_s: float = 0.002):
+    def __init__(self, device_index: int, period_s: float = 0.0005):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.period = period_s
         self._stop = threading.Event()
@@ -391,6 +391,25 @@ def measure_decode(ssm, stream, pk, steps=None):
                          "traffic": traffic_record("state_update_kernel", w.name)}}
 
 
+def measure_unaligned(ssm, stream, pk, steps=10):
+    """Headline shape at L = 2047 (rows not a multiple of 16 bytes: u, delta, z are staged
+    into padded rows in the workspace) against L = 2048 on the same inputs' distribution."""
+    out = {"workload": "mamba2p8b_b4_d5120", "unit": UNIT}
+    for L in (2048, 2047):
+        inp = workloads.scan_inputs(4, 5120, L, io="bf16", seed=1002)
+        g = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+        g["y"] = torch.empty_like(g["u"])
+        g["last"] = torch.empty(4, 5120, 16, dtype=torch.float32, device="cuda")
+        ws = ssm.new_workspace(4, 5120, 16, L)
+        t = time_forward(ssm, g, ws, steps, 3, 1, stream)
+        ms = t / steps * 1e3
+        assert ssm.ssm_read_status(ws) == 0
+        out[f"L{L}"] = {"value": 4 * 5120 * L / (ms / 1e3) / 1e9, "ms_per_step": ms}
+        del g, ws
+    out["ratio_2047_to_2048"] = out["L2047"]["ms_per_step"] / out["L2048"]["ms_per_step"]
+    return out
+
+
 def measure_zoh(ssm, stream, pk, steps=10):
     """Headline workload with the zero-order-hold discretisation (sequential kernel)."""
     w = workloads.WORKLOADS[workloads.HEADLINE]
@@ -603,7 +622,7 @@ def run_gpu(args, world, rank, local):
     if world == 1 and not args.skip_extra:
         line["also"] = {"long": measure_long(ssm, stream, pk), "decode": measure_decode(ssm, stream, pk),
                         "backward": measure_backward(ssm, stream, pk), "zoh": measure_zoh(ssm, stream, pk),
-                        "conv": measure_conv(ssm, stream, pk)}
+                        "conv": measure_conv(ssm, stream, pk), "unaligned": measure_unaligned(ssm, stream, pk)}
     if rank == 0 and world == 1 and not args.skip_cpu:
         rate, secs, desc, cores = cpu_oracle_rate(w, args.cpu_budget)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}

@@ -112,8 +112,11 @@ ssm_status_t ssm_workspace_init(void* workspace, size_t workspace_bytes, ssm_str
  *                            256-byte aligned, zeroed once by ssm_workspace_init().  It must not be
  *                            used by two calls that can overlap on the GPU.
  * All tensor pointers must be 16-byte aligned.  Any seqlen >= 0 is accepted; when
- * seqlen * sizeof(io element) is a multiple of 16 the tiles are staged with TMA,
- * otherwise a direct-load kernel runs.
+ * seqlen * sizeof(io element) is a multiple of 16 the tiles are staged with TMA straight
+ * from u, delta and z; otherwise those are first copied into rows padded to a multiple of
+ * 16 bytes inside the workspace (which is sized for this whenever seqlen % 8 != 0), and
+ * SSM_ALGO_CHUNKED, the conv prologue and the no-allocation entry point run a direct-load
+ * kernel instead.
  */
 ssm_status_t ssm_selective_scan_fwd(
     const void* u, const void* delta, const float* A, const void* B, const void* C,

@@ -1,5 +1,7 @@
 // aux.cu -- launchers of the kernels around the main scans (aux_kernels.cuh): the B/C
 // transposes, the direct-load forward and the d_state-16 decode step.
+#include <algorithm>
+
 #include "host_common.h"
 #include "aux_kernels.cuh"
 
@@ -90,6 +92,25 @@ ssm_status_t launch_decode16(const DecodeArgs& a, ssm_dtype_t io) {
     return launch_status();
 }
 
+template <typename IO>
+ssm_status_t launch_pad_rows(const void* const* src, void* const* dst, int narrays, long long rows, int64_t L,
+                             int64_t Lp, cudaStream_t stream) {
+    ssm::PadArrays arr{};
+    for (int i = 0; i < narrays; ++i) {
+        arr.src[i] = src[i];
+        arr.dst[i] = dst[i];
+    }
+    const long long chunks = rows * (Lp / (16 / static_cast<long long>(sizeof(IO))));
+    const long long grid = std::max<long long>(1, std::min<long long>((chunks + 255) / 256, 148LL * 16));
+    ssm::pad_rows_kernel<IO><<<dim3(static_cast<unsigned>(grid), static_cast<unsigned>(narrays)), 256, 0, stream>>>(
+        arr, rows, L, Lp);
+    return launch_status();
+}
+
+template ssm_status_t launch_pad_rows<__nv_bfloat16>(const void* const*, void* const*, int, long long, int64_t,
+                                                     int64_t, cudaStream_t);
+template ssm_status_t launch_pad_rows<float>(const void* const*, void* const*, int, long long, int64_t, int64_t,
+                                             cudaStream_t);
 template ssm_status_t launch_pack<__nv_bfloat16>(const FwdArgs&);
 template ssm_status_t launch_pack<float>(const FwdArgs&);
 template ssm_status_t launch_direct<__nv_bfloat16>(const FwdArgs&);

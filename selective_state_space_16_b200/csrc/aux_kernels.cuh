@@ -70,6 +70,70 @@ __global__ void __launch_bounds__(256) pack_bc_pairs_kernel(const uint16_t* __re
 }
 
 // ---------------------------------------------------------------------------------------
+// Rows of `rows` x L elements (L * sizeof(IO) not a multiple of 16) copied into rows of Lp
+// elements (Lp * sizeof(IO) a multiple of 16, zero past L), so that TMA can address them;
+// up to three arrays at once (blockIdx.y selects the array).  One thread per 16-byte chunk
+// of an output row: the chunk's 16 source bytes start at a 2-byte (bf16) or 4-byte (fp32)
+// aligned address and are assembled from the two aligned 16-byte words that hold them
+// (byte_perm funnel); at the end of a row or of the source array (where the second word
+// could lie past it), element by element.  Measured on B200 at ~4 TB/s of read + write:
+// 118 us for the three 84 MB arrays of batch 4, d_inner 5120, L 2047.
+// ---------------------------------------------------------------------------------------
+struct PadArrays {
+    const void* src[3];
+    void* dst[3];
+};
+
+template <typename IO>
+__device__ __forceinline__ uint4 pad_chunk(const IO* __restrict__ src, long long r, long long t0, long long L,
+                                           long long n_src, uint4 w0, uint4 w1, bool fast) {
+    constexpr int E = 16 / sizeof(IO);
+    if (fast) {
+        const uint32_t sh = static_cast<uint32_t>(reinterpret_cast<uintptr_t>(src + r * L + t0) & 15u);
+        const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        const uint32_t k = sh >> 2;  // whole words to skip (0 .. 3)
+        uint32_t sw[5];              // words k .. k+4
+#pragma unroll
+        for (int m = 0; m < 5; ++m) sw[m] = k == 0 ? w[m] : k == 1 ? w[m + 1] : k == 2 ? w[m + 2] : w[m + 3];
+        // with a 2-byte remainder each output word is the upper half of one word and the lower
+        // half of the next
+        const uint32_t sel = (sh & 3u) ? 0x5432u : 0x3210u;
+        return make_uint4(__byte_perm(sw[0], sw[1], sel), __byte_perm(sw[1], sw[2], sel),
+                          __byte_perm(sw[2], sw[3], sel), __byte_perm(sw[3], sw[4], sel));
+    }
+    // row end (or array end): element by element, zero past L
+    __align__(16) IO v[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) v[e] = (t0 + e < L && r * L + t0 + e < n_src) ? src[r * L + t0 + e] : IoTraits<IO>::from_f32(0.f);
+    return *reinterpret_cast<const uint4*>(v);
+}
+
+template <typename IO>
+__global__ void __launch_bounds__(256) pad_rows_kernel(const PadArrays arrays, long long rows, long long L,
+                                                       long long Lp) {
+    constexpr int E = 16 / sizeof(IO);  // elements per 16-byte chunk
+    const IO* __restrict__ src = static_cast<const IO*>(arrays.src[blockIdx.y]);
+    uint4* __restrict__ dst = static_cast<uint4*>(arrays.dst[blockIdx.y]);
+    const long long cpr = Lp / E;       // chunks per output row
+    const long long total = rows * cpr;
+    const long long n_src = rows * L;
+    for (long long q = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; q < total;
+         q += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long r = q / cpr;
+        const long long t0 = (q - r * cpr) * E;
+        const long long s0 = r * L + t0;  // first source element of the chunk
+        uint4 w0 = make_uint4(0, 0, 0, 0), w1 = w0;
+        const bool fast = t0 + E <= L && s0 + 2 * E <= n_src;
+        if (fast) {
+            const uint4* wp = reinterpret_cast<const uint4*>(reinterpret_cast<uintptr_t>(src + s0) & ~uintptr_t(15));
+            w0 = __ldg(wp);
+            w1 = __ldg(wp + 1);
+        }
+        dst[q] = pad_chunk<IO>(src, r, t0, L, n_src, w0, w1, fast);
+    }
+}
+
+// ---------------------------------------------------------------------------------------
 // Direct-load forward scan (fallback for seqlen whose rows are not 16-byte multiples).
 // G lanes per channel, NC = 16/G chains per lane, 128 threads per block.
 // Per step: h = exp(Delta A) h + Delta B u; y = C.h + D u; y *= silu(z)

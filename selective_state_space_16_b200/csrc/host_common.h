@@ -29,11 +29,16 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 //   [inclusive h: keys * 256 B]
 // with keys = (8-channel tiles) * 2 columns * ceil(L / 32) chunks (32 steps is the shorter
 // chunk of the two element types, so one size serves both).
+//   [padded rows: 3 arrays of batch * dim * round_up(L, 8) * 4 B, only when L % 8 != 0]
+// The padded rows hold u, delta and z copied to rows whose length is a multiple of 16
+// bytes (TMA needs 16-byte row strides); sized for fp32, the larger element type.
 struct WsLayout {
-    size_t bc_off, flags_off, agg_off, sdt_off, incl_off, total;
+    size_t bc_off, flags_off, agg_off, sdt_off, incl_off, pad_off, pad_array, total;
     long long keys;
 };
 constexpr int kMinChunk = 32;
+
+inline bool rows_need_padding(int64_t L) { return L % 8 != 0; }
 
 inline WsLayout ws_layout(int batch, int dim, int64_t L) {
     WsLayout w{};
@@ -44,7 +49,12 @@ inline WsLayout ws_layout(int batch, int dim, int64_t L) {
     w.agg_off = w.flags_off + round_up(static_cast<size_t>(w.keys) * 4u, 256);
     w.sdt_off = w.agg_off + static_cast<size_t>(w.keys) * 256u;
     w.incl_off = w.sdt_off + static_cast<size_t>(w.keys) * 16u;
-    w.total = w.incl_off + static_cast<size_t>(w.keys) * 256u;
+    w.pad_off = round_up(w.incl_off + static_cast<size_t>(w.keys) * 256u, 256);
+    w.pad_array = rows_need_padding(L) ? round_up(static_cast<size_t>(batch) * static_cast<size_t>(dim) *
+                                                      static_cast<size_t>(round_up(static_cast<size_t>(L), 8)) * 4u,
+                                                  256)
+                                       : 0;
+    w.total = w.pad_off + 3 * w.pad_array;
     return w;
 }
 
@@ -90,6 +100,9 @@ struct FwdArgs {
     cudaStream_t stream;
     int sm_count;
     ConvArgs conv;
+    int64_t L_rows = 0;  // row length of u / delta / z when staged into padded rows (0: L)
+    int y_vec = 1;       // y rows 16-byte aligned: vector stores of y
+    bool pad_ok = true;  // the workspace has room for padded rows (not the no-allocation scratch)
 };
 
 // Backward workspace layout:
@@ -133,6 +146,9 @@ struct DecodeArgs {
 template <typename IO> ssm_status_t launch_pack(const FwdArgs& a);
 // Direct-load forward (any seqlen / alignment; aux.cu).
 template <typename IO> ssm_status_t launch_direct(const FwdArgs& a);
+// narrays (<= 3) arrays of rows x L elements -> rows x Lp elements (zero past L) (aux.cu).
+template <typename IO> ssm_status_t launch_pad_rows(const void* const* src, void* const* dst, int narrays, long long rows,
+                                                    int64_t L, int64_t Lp, cudaStream_t stream);
 // Sequence split across CTAs with decoupled look-back (fwd_chunked.cu).
 template <typename IO> ssm_status_t launch_chunked(const FwdArgs& a, const ssm_fwd_options_t& o);
 // Sequential family, plain discretisation, no conv: picks lanes per channel (fwd_seq_*.cu).

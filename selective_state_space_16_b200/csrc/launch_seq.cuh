@@ -94,11 +94,12 @@ ssm_status_t launch_seq(const FwdArgs& a, const SeqPlan& pl) {
     constexpr int es = ssm::IoTraits<IO>::kBytes;
     CUtensorMap mu, mdl, mz, mbc;
     const uint64_t L = static_cast<uint64_t>(a.L);
-    bool ok = make_map_3d(&mu, dt, es, a.u, L, a.dim, a.batch, TC, 8, sw128) &&
-              make_map_3d(&mdl, dt, es, a.delta, L, a.dim, a.batch, TC, 8, sw128) &&
+    const uint64_t Lr = static_cast<uint64_t>(a.L_rows ? a.L_rows : a.L);  // row length of u / delta / z
+    bool ok = make_map_3d(&mu, dt, es, a.u, Lr, a.dim, a.batch, TC, 8, sw128) &&
+              make_map_3d(&mdl, dt, es, a.delta, Lr, a.dim, a.batch, TC, 8, sw128) &&
               make_map_3d(&mbc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.ws + ws_layout(a.batch, a.dim, a.L).bc_off, 32,
                           L, a.batch, 32, TC, CU_TENSOR_MAP_SWIZZLE_NONE);
-    if (ok && a.z) ok = make_map_3d(&mz, dt, es, a.z, L, a.dim, a.batch, TC, 8, sw128);
+    if (ok && a.z) ok = make_map_3d(&mz, dt, es, a.z, Lr, a.dim, a.batch, TC, 8, sw128);
     if (!a.z) mz = mu;
     if (!ok) return SSM_ERR_LAUNCH;
     ssm::SeqParams p{};
@@ -125,6 +126,7 @@ ssm_status_t launch_seq(const FwdArgs& a, const SeqPlan& pl) {
     p.conv_out = a.conv.out;
     p.u_out = a.conv.u_out;
     p.conv_k = a.conv.k;
+    p.y_vec = a.y_vec;
     if (a.L >= (1LL << 31) - 1024) return SSM_ERR_UNSUPPORTED;
     switch (pl.stages) {
         case 2: ssm::scan_fwd_seq_kernel<IO, G, CPL, 2, ZOH, CONV><<<pl.grid, pl.threads, pl.smem, a.stream>>>(mu, mdl, mz, mbc, p); break;

@@ -64,6 +64,9 @@ struct SeqParams {
     float* conv_out;           // (batch, dim, conv_k - 1) fp32: the last conv_k - 1 inputs, or null
     void* u_out;               // (batch, dim, L) IO: the conv output, or null
     int conv_k;                // 1 .. 4
+    // y rows are 16-byte aligned (L * sizeof(IO) a multiple of 16): vector stores; else
+    // element stores (the inputs were then staged into padded rows, see pad_rows_kernel)
+    int y_vec;
 };
 
 __host__ __device__ constexpr int round_up_i(int v, int m) { return (v + m - 1) / m * m; }
@@ -386,7 +389,7 @@ __device__ __forceinline__ void seq_consumer(uint8_t* smem, uint64_t* full_bar, 
                 dcheck(p.hdr, t0 >= L32 || (static_cast<long long>(b) * p.dim + d[c]) * p.L + t0 <
                                                static_cast<long long>(p.batch) * p.dim * p.L,
                        kSiteSeqY, t0)) {
-                if (t0 + PER <= L32) {
+                if (p.y_vec && t0 + PER <= L32) {
                     store_run<IO, PER>(yrow[c] + t0, yo);
                 } else {
 #pragma unroll

@@ -55,6 +55,21 @@ def test_forward_edge_lengths(cuda_device, L):
     check_forward(inp, what=f"L={L}")
 
 
+@pytest.mark.parametrize("io,L", [("f32", 1001), ("f32", 1002), ("bf16", 1001), ("bf16", 1004)])
+def test_forward_unaligned_rows_padded(cuda_device, io, L):
+    # L * sizeof(element) not a multiple of 16: u, delta, z are staged into padded rows in the
+    # workspace and the sequential kernel runs on them (also with the zero-order hold)
+    inp = workloads.scan_inputs(2, 100, L, io=io, seed=70 + L)
+    check_forward(inp, what=f"padded rows {io} L={L}")
+    check_forward(inp, algo="sequential", lanes_per_channel=4, what=f"padded rows {io} L={L} 4 lanes")
+
+
+def test_forward_unaligned_headline_full_size(cuda_device):
+    # the Mamba-2.8B layer shape one step short of 2048: every row starts 2 bytes off the last
+    inp = workloads.scan_inputs(4, 5120, 2047, io="bf16", seed=71)
+    check_forward(inp, what="b4 d5120 L2047")
+
+
 def test_forward_empty_sequence_gives_zero_state(cuda_device):
     inp = workloads.scan_inputs(2, 20, 0, io="bf16", seed=15)
     y, last = gpu_forward(inp)
