@@ -51,6 +51,10 @@ def _load():
             lib.oracle_state_update_zoh_f64.restype = ci
             lib.oracle_selective_scan_bwd_f64.argtypes = [vp] * 8 + [ci] + [vp] * 12 + [i64, i64, i64, i64]
             lib.oracle_selective_scan_bwd_f64.restype = ci
+            lib.oracle_selective_scan_bwd_zoh_f64.argtypes = [vp] * 8 + [ci] + [vp] * 12 + [i64, i64, i64, i64, ci]
+            lib.oracle_selective_scan_bwd_zoh_f64.restype = ci
+            lib.oracle_causal_conv_silu_bwd_f64.argtypes = [vp] * 10 + [i64, i64, i64, i64]
+            lib.oracle_causal_conv_silu_bwd_f64.restype = ci
             lib.oracle_causal_conv_silu_f64.argtypes = [vp] * 6 + [i64, i64, i64, i64]
             lib.oracle_causal_conv_silu_f64.restype = ci
             lib.oracle_num_threads.restype = ci
@@ -127,11 +131,12 @@ def state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, soft
 
 
 def selective_scan_bwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True, h0=None, dy=None,
-                       dlast=None):
+                       dlast=None, zoh=False):
     """Gradients of L = sum(dy * y) + sum(dlast * last_state) for the forward scan with these
-    inputs.  Returns a dict of float64 arrays: du, ddelta (b, d, L); dA (d, N); dB, dC (b, N, L);
-    dD, ddelta_bias (d) (always, as if D / delta_bias were given); dz (b, d, L) or None;
-    dh0 (b, d, N) (the gradient with respect to the initial state, zero or h0)."""
+    inputs (zoh: of the zero-order-hold scan).  Returns a dict of float64 arrays: du, ddelta
+    (b, d, L); dA (d, N); dB, dC (b, N, L); dD, ddelta_bias (d) (always, as if D / delta_bias
+    were given); dz (b, d, L) or None; dh0 (b, d, N) (the gradient with respect to the initial
+    state, zero or h0)."""
     u, delta, A, B, C = map(_f64, (u, delta, A, B, C))
     D, z, delta_bias, h0, dy, dlast = map(_f64, (D, z, delta_bias, h0, dy, dlast))
     b, d, L = u.shape
@@ -141,10 +146,11 @@ def selective_scan_bwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
     out = dict(du=np.empty((b, d, L)), ddelta=np.empty((b, d, L)), dA=np.empty((d, n)),
                dB=np.empty((b, n, L)), dC=np.empty((b, n, L)), dD=np.empty(d), ddelta_bias=np.empty(d),
                dz=np.empty((b, d, L)) if z is not None else None, dh0=np.empty((b, d, n)))
-    rc = _load().oracle_selective_scan_bwd_f64(
+    rc = _load().oracle_selective_scan_bwd_zoh_f64(
         _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias), int(bool(softplus)),
         _ptr(h0), _ptr(dy), _ptr(dlast), _ptr(out["du"]), _ptr(out["ddelta"]), _ptr(out["dA"]), _ptr(out["dB"]),
-        _ptr(out["dC"]), _ptr(out["dD"]), _ptr(out["dz"]), _ptr(out["ddelta_bias"]), _ptr(out["dh0"]), b, d, n, L)
+        _ptr(out["dC"]), _ptr(out["dD"]), _ptr(out["dz"]), _ptr(out["ddelta_bias"]), _ptr(out["dh0"]), b, d, n, L,
+        int(bool(zoh)))
     if rc != 0:
         raise ValueError("oracle_selective_scan_bwd_f64 rejected its arguments")
     return out
@@ -165,3 +171,23 @@ def causal_conv_silu(x, w, bias=None, x_prev=None):
     if rc != 0:
         raise ValueError("oracle_causal_conv_silu_f64 rejected its arguments")
     return u, x_next
+
+
+def causal_conv_silu_bwd(x, w, du, bias=None, x_prev=None, dx_next=None):
+    """Gradients through causal_conv_silu, given du = dL/du (b, d, L) and optionally dx_next =
+    dL/d x_next (b, d, K-1).  Returns a dict of float64 arrays: dx (b, d, L), dw (d, K),
+    dbias (d) (always, as if bias were given), dx_prev (b, d, K-1)."""
+    x, w, du, bias, x_prev, dx_next = map(_f64, (x, w, du, bias, x_prev, dx_next))
+    b, d, L = x.shape
+    K = w.shape[1]
+    assert w.shape == (d, K) and du.shape == x.shape
+    assert x_prev is None or x_prev.shape == (b, d, K - 1)
+    assert dx_next is None or dx_next.shape == (b, d, K - 1)
+    out = dict(dx=np.empty((b, d, L)), dw=np.empty((d, K)), dbias=np.empty(d), dx_prev=np.empty((b, d, K - 1)))
+    rc = _load().oracle_causal_conv_silu_bwd_f64(_ptr(x), _ptr(w), _ptr(bias), _ptr(x_prev), _ptr(du),
+                                                 _ptr(dx_next), _ptr(out["dx"]), _ptr(out["dw"]),
+                                                 _ptr(out["dbias"]), _ptr(out["dx_prev"]) if K > 1 else None,
+                                                 b, d, L, K)
+    if rc != 0:
+        raise ValueError("oracle_causal_conv_silu_bwd_f64 rejected its arguments")
+    return out

@@ -36,7 +36,10 @@
  * gradients of L = sum dy*y + sum dlast*last_state: the same forward loop, keeping
  * every state, then the chain rule applied to each step in reverse order (the
  * recompute-in-backward scheme of [Tech] 四.1 and [S4M] 3.3, here with everything
- * kept).  It is pinned by finite differences of the forward scan.
+ * kept).  oracle_selective_scan_bwd_zoh_f64 does the same for either discretisation,
+ * and oracle_causal_conv_silu_bwd_f64 is the chain rule through the conv prologue
+ * (u = silu(conv(x))), given the gradient reaching u.  All three are pinned by finite
+ * differences of the forward functions.
  *
  * Layouts (all contiguous, row-major): u, delta, z, y: (batch, dim, L);
  * B, C: (batch, dstate, L); A: (dim, dstate); D, delta_bias: (dim);
@@ -216,6 +219,29 @@ static double sigmoid_f64(double x)
 }
 
 /*
+ * Derivatives of the input weight per unit B, phi(dt, a) = dt (simplified) or expm1(dt a) / a
+ * (zero-order hold, [Eng] §2.2; dt at a = 0):
+ *   d phi / d dt = 1 (simplified);  exp(dt a) (ZOH: the derivative of expm1 is exp).
+ *   d phi / d a  = 0 (simplified);  (dt a exp(dt a) - expm1(dt a)) / a^2 (ZOH).
+ * The ZOH form in a loses digits to cancellation when x = dt a is small, so there it takes the
+ * Taylor series of the same function, dt^2 (1/2 + x/3 + x^2/8 + x^3/30 + ...): the k-th term
+ * of (x e^x - (e^x - 1)) / x^2 is x^k / (k! (k + 2)), summed to x^3 (the next term,
+ * x^4/144, is below 1e-14 relative for |x| < 1e-3).
+ */
+static double input_weight_ddt(double dt, double a, int zoh)
+{
+    return zoh ? exp(dt * a) : 1.0;
+}
+
+static double input_weight_dA(double dt, double a, int zoh)
+{
+    if (!zoh) return 0.0;
+    const double x = dt * a;
+    if (fabs(x) < 1e-3) return dt * dt * (0.5 + x * (1.0 / 3.0 + x * (1.0 / 8.0 + x * (1.0 / 30.0))));
+    return (x * exp(x) - expm1(x)) / (a * a);
+}
+
+/*
  * Backward of one channel (b, d): the forward loop again, keeping every state, then
  * the chain rule applied to it step by step in reverse order.  Per-channel outputs are
  * written; the sums over channels (dB, dC) and over batch rows (dA, dD, ddelta_bias)
@@ -228,7 +254,7 @@ static void channel_bwd(int64_t b, int64_t d, const double* u, const double* del
                         const double* delta_bias, int softplus, const double* h0, const double* dy,
                         const double* dlast, double* du, double* ddelta, double* dz, double* dh0,
                         double* accB, double* accC, double* accA, double* accD, double* accBias,
-                        int64_t dim, int64_t N, int64_t L, double* H, double* Dt)
+                        int64_t dim, int64_t N, int64_t L, double* H, double* Dt, int zoh)
 {
     const int64_t row = b * dim + d;
     const double Dd = D ? D[d] : 0.0;
@@ -237,7 +263,8 @@ static void channel_bwd(int64_t b, int64_t d, const double* u, const double* del
         const double ut = u[row * L + t];
         Dt[t] = step_size(delta[row * L + t], delta_bias, d, softplus);
         for (int64_t n = 0; n < N; ++n)
-            H[(t + 1) * N + n] = exp(Dt[t] * A[d * N + n]) * H[t * N + n] + Dt[t] * B[(b * N + n) * L + t] * ut;
+            H[(t + 1) * N + n] = exp(Dt[t] * A[d * N + n]) * H[t * N + n] +
+                                 input_weight(Dt[t], A[d * N + n], B[(b * N + n) * L + t], zoh) * ut;
     }
     /* g[n] = dL/dh: the gradient reaching the state, starting from dL/d last_state. */
     double g[256];
@@ -256,15 +283,16 @@ static void channel_bwd(int64_t b, int64_t d, const double* u, const double* del
         accD[d] += dv * ut;
         double dut = Dd * dv, ddt = 0.0;
         for (int64_t n = 0; n < N; ++n) {
-            const double Bn = B[(b * N + n) * L + t], Cn = C[(b * N + n) * L + t];
-            const double hprev = H[t * N + n], abar = exp(dt * A[d * N + n]);
+            const double Bn = B[(b * N + n) * L + t], Cn = C[(b * N + n) * L + t], An = A[d * N + n];
+            const double hprev = H[t * N + n], abar = exp(dt * An);
+            /* h_t = abar * h_{t-1} + phi * B * u, phi the input weight per unit B */
+            const double phi = input_weight(dt, An, 1.0, zoh);
             accC[n * L + t] += dv * H[(t + 1) * N + n];
             g[n] += dv * Cn;                          /* dL/dh_t complete */
-            /* h_t = abar * h_{t-1} + dt * B * u */
-            ddt += g[n] * (A[d * N + n] * abar * hprev + Bn * ut);
-            accB[n * L + t] += g[n] * dt * ut;
-            dut += g[n] * dt * Bn;
-            accA[d * N + n] += g[n] * dt * abar * hprev;
+            ddt += g[n] * (An * abar * hprev + input_weight_ddt(dt, An, zoh) * Bn * ut);
+            accB[n * L + t] += g[n] * phi * ut;
+            dut += g[n] * phi * Bn;
+            accA[d * N + n] += g[n] * (dt * abar * hprev + input_weight_dA(dt, An, zoh) * Bn * ut);
             g[n] *= abar;                             /* dL/dh_{t-1} through this step */
         }
         du[row * L + t] = dut;
@@ -286,6 +314,14 @@ static void channel_bwd(int64_t b, int64_t d, const double* u, const double* del
  * batch rows are formed per thread and added in thread order, so a run is reproducible
  * for a given thread count.  Returns 0, or -1 on a bad argument or allocation failure.
  */
+int oracle_selective_scan_bwd_zoh_f64(const double* u, const double* delta, const double* A,
+                                      const double* B, const double* C, const double* D,
+                                      const double* z, const double* delta_bias, int softplus,
+                                      const double* h0, const double* dy, const double* dlast,
+                                      double* du, double* ddelta, double* dA, double* dB, double* dC,
+                                      double* dD, double* dz, double* ddelta_bias, double* dh0,
+                                      int64_t batch, int64_t dim, int64_t dstate, int64_t L, int zoh);
+
 int oracle_selective_scan_bwd_f64(const double* u, const double* delta, const double* A,
                                   const double* B, const double* C, const double* D,
                                   const double* z, const double* delta_bias, int softplus,
@@ -293,6 +329,20 @@ int oracle_selective_scan_bwd_f64(const double* u, const double* delta, const do
                                   double* du, double* ddelta, double* dA, double* dB, double* dC,
                                   double* dD, double* dz, double* ddelta_bias, double* dh0,
                                   int64_t batch, int64_t dim, int64_t dstate, int64_t L)
+{
+    return oracle_selective_scan_bwd_zoh_f64(u, delta, A, B, C, D, z, delta_bias, softplus, h0, dy, dlast, du,
+                                             ddelta, dA, dB, dC, dD, dz, ddelta_bias, dh0, batch, dim, dstate, L, 0);
+}
+
+/* As oracle_selective_scan_bwd_f64, for the zero-order-hold input weight when zoh != 0
+ * (the gradients of oracle_selective_scan_zoh_f64). */
+int oracle_selective_scan_bwd_zoh_f64(const double* u, const double* delta, const double* A,
+                                      const double* B, const double* C, const double* D,
+                                      const double* z, const double* delta_bias, int softplus,
+                                      const double* h0, const double* dy, const double* dlast,
+                                      double* du, double* ddelta, double* dA, double* dB, double* dC,
+                                      double* dD, double* dz, double* ddelta_bias, double* dh0,
+                                      int64_t batch, int64_t dim, int64_t dstate, int64_t L, int zoh)
 {
     if (batch < 0 || dim < 0 || dstate < 1 || dstate > 256 || L < 0) return -1;
     if (!u || !delta || !A || !B || !C || !dy || !du || !ddelta || !dA || !dB || !dC || !dD ||
@@ -332,7 +382,7 @@ int oracle_selective_scan_bwd_f64(const double* u, const double* delta, const do
                 if (H && Dt)
                     channel_bwd(b, d, u, delta, A, B, C, D, z, delta_bias, softplus, h0, dy, dlast, du, ddelta,
                                 dz, dh0, accB + tid * nl, accC + tid * nl, accA + tid * dn, accD + tid * dim,
-                                accBias + tid * dim, dim, N, L, H, Dt);
+                                accBias + tid * dim, dim, N, L, H, Dt, zoh);
             free(H);
             free(Dt);
         }
@@ -406,6 +456,65 @@ int oracle_causal_conv_silu_f64(const double* x, const double* w, const double* 
         }
     }
     return 0;
+}
+
+/*
+ * Backward of oracle_causal_conv_silu_f64: given du = dL/du (batch, dim, L) and optionally
+ * dx_next = dL/d x_next (batch, dim, K-1), the gradients of the conv's inputs.  With
+ * p[t] = bias + sum_k w[k] xin[t-(K-1)+k] (xin: x_prev before t = 0, then x) and u = silu(p):
+ *   dp[t]      = du[t] * silu'(p[t])
+ *   dxin[s]   += w[k] * dp[t]          for every (t, k) with s = t-(K-1)+k
+ *   dxin[s]   += dx_next[j]            for s = L-(K-1)+j (x_next copies those inputs)
+ *   dw[d,k]   += dp[t] * xin[t-(K-1)+k]  (summed over batch rows and t)
+ *   dbias[d]  += dp[t]                  (summed over batch rows and t)
+ * dx (batch, dim, L) receives dxin[0..L), dx_prev (batch, dim, K-1; optional) dxin[-(K-1)..0).
+ * dw (dim, K) and dbias (dim; optional) are written, not accumulated.  The sums over batch
+ * rows are formed per channel in batch order.  Returns 0, or -1 on a bad argument.
+ */
+int oracle_causal_conv_silu_bwd_f64(const double* x, const double* w, const double* bias, const double* x_prev,
+                                    const double* du, const double* dx_next, double* dx, double* dw,
+                                    double* dbias, double* dx_prev, int64_t batch, int64_t dim, int64_t L,
+                                    int64_t K)
+{
+    if (batch < 0 || dim < 0 || L < 0 || K < 1 || K > 16 || !x || !w || !du || !dx || !dw) return -1;
+    int fail = 0;
+    #pragma omp parallel for schedule(static)
+    for (int64_t d = 0; d < dim; ++d) {
+        double gw[16] = {0.0}, gb = 0.0;
+        double* dxin = malloc(((size_t)L + (size_t)K) * sizeof(double));  /* index s + (K-1) */
+        if (!dxin) {
+            #pragma omp atomic write
+            fail = 1;
+        }
+        for (int64_t b = 0; b < batch && dxin; ++b) {
+            const int64_t row = b * dim + d;
+            for (int64_t i = 0; i < L + K - 1; ++i) dxin[i] = 0.0;
+            for (int64_t t = 0; t < L; ++t) {
+                double p = bias ? bias[d] : 0.0;
+                double xin[16];
+                for (int64_t k = 0; k < K; ++k) {
+                    const int64_t s = t - (K - 1) + k;
+                    xin[k] = s >= 0 ? x[row * L + s] : (x_prev ? x_prev[row * (K - 1) + (K - 1 + s)] : 0.0);
+                    p += w[d * K + k] * xin[k];
+                }
+                const double dp = du[row * L + t] * silu_grad_f64(p);
+                gb += dp;
+                for (int64_t k = 0; k < K; ++k) {
+                    gw[k] += dp * xin[k];
+                    dxin[t + k] += w[d * K + k] * dp;       /* s + (K-1) = t + k */
+                }
+            }
+            if (dx_next)
+                for (int64_t j = 0; j < K - 1; ++j) dxin[L + j] += dx_next[row * (K - 1) + j];
+            for (int64_t s = 0; s < L; ++s) dx[row * L + s] = dxin[s + K - 1];
+            if (dx_prev)
+                for (int64_t j = 0; j < K - 1; ++j) dx_prev[row * (K - 1) + j] = dxin[j];
+        }
+        for (int64_t k = 0; k < K; ++k) dw[d * K + k] = gw[k];
+        if (dbias) dbias[d] = gb;
+        free(dxin);
+    }
+    return fail ? -1 : 0;
 }
 
 /* Number of OpenMP threads the oracle will use (reported beside CPU timings). */

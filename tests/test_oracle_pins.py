@@ -516,3 +516,127 @@ def test_causal_conv_continuation():
     u1, s1 = oracle.causal_conv_silu(x[..., :5], w)
     u2, _ = oracle.causal_conv_silu(x[..., 5:], w, x_prev=s1)
     np.testing.assert_allclose(np.concatenate([u1, u2], axis=2), u, rtol=1e-14, atol=1e-15)
+
+
+# ---------------------------------------------------------------------------------------------
+# Backward of the zero-order-hold scan and of the conv prologue, against central finite
+# differences of the forward functions pinned above (the RK4-pinned ZOH scan and the
+# numpy.convolve-pinned conv).  A dropped or mis-signed term in any gradient fails here.
+# ---------------------------------------------------------------------------------------------
+def _central_fd(loss, base, eps=1e-6):
+    fd = np.zeros_like(base)
+    for idx in np.ndindex(base.shape):
+        hi, lo = base.copy(), base.copy()
+        hi[idx] += eps
+        lo[idx] -= eps
+        fd[idx] = (loss(hi) - loss(lo)) / (2 * eps)
+    return fd
+
+
+def _assert_fd(got, fd, what):
+    np.testing.assert_allclose(got, fd, rtol=1e-6, atol=1e-7 * (1 + np.abs(fd).max()), err_msg=what)
+
+
+@pytest.mark.parametrize("flags", [dict(), dict(softplus=False), dict(with_z=False, with_D=False, with_bias=False)],
+                         ids=["full", "softplus_off", "bare"])
+def test_backward_zoh_matches_finite_differences(flags):
+    rng = _rng(81)
+    case = _selective_case(rng, b=2, d=3, n=4, L=9, **flags)
+    if not case["softplus"]:
+        case["delta"] = np.abs(case["delta"]) + 0.05
+        case["delta_bias"] = rng.uniform(0.0, 0.05, case["delta_bias"].shape)
+    # both regimes of the ZOH weight's A-derivative: |Delta A| < 1e-3 (series) and A = 0
+    case["A"][0, 1] = -2e-5
+    case["A"][1, 2] = 0.0
+    case["A"][2, 0] = 3e-4
+    b, d, L = case["u"].shape
+    n = case["A"].shape[1]
+    h0 = rng.standard_normal((b, d, n))
+    dy = rng.standard_normal((b, d, L))
+    dlast = rng.standard_normal((b, d, n))
+    grads = oracle.selective_scan_bwd(**case, h0=h0, dy=dy, dlast=dlast, zoh=True)
+    plain = oracle.selective_scan_bwd(**case, h0=h0, dy=dy, dlast=dlast)
+    assert np.abs(grads["dA"] - plain["dA"]).max() > 1e-3   # the ZOH weight does depend on A
+
+    def loss_of(name):
+        def loss(value):
+            c = dict(case, h0=h0)
+            c[name] = value
+            y, last = oracle.selective_scan(**c, zoh=True)
+            return float((dy * y).sum() + (dlast * last).sum())
+        return loss
+
+    names = [("u", "du"), ("delta", "ddelta"), ("A", "dA"), ("B", "dB"), ("C", "dC"), ("h0", "dh0")]
+    names += [(k, "d" + k) for k in ("D", "z", "delta_bias") if case[k] is not None]
+    for name, key in names:
+        base = h0 if name == "h0" else case[name]
+        _assert_fd(grads[key], _central_fd(loss_of(name), base), f"zoh {name}")
+
+
+def test_backward_zoh_tends_to_simplified_for_small_steps():
+    # For Delta A -> 0 the ZOH weight expm1(Delta A)/A B approaches Delta B, and so do the
+    # gradients (to first order in Delta A).
+    rng = _rng(82)
+    case = _selective_case(rng, b=1, d=2, n=3, L=6, softplus=False)
+    case["delta"] = np.full_like(case["delta"], 1e-7)
+    case["delta_bias"] = np.zeros(2)
+    dy = rng.standard_normal(case["u"].shape)
+    gz = oracle.selective_scan_bwd(**case, dy=dy, zoh=True)
+    gs = oracle.selective_scan_bwd(**case, dy=dy)
+    for k in ("du", "ddelta", "dB", "dC", "dD", "dz"):
+        np.testing.assert_allclose(gz[k], gs[k], rtol=1e-5, atol=1e-12, err_msg=k)
+
+
+@pytest.mark.parametrize("K,L,with_prev,with_bias", [(1, 7, False, True), (2, 7, True, False), (4, 9, True, True),
+                                                     (4, 2, True, True), (4, 9, False, False), (3, 1, True, True)],
+                         ids=["K1", "K2_prev", "K4_prev", "K4_shortL", "K4_bare", "K3_L1"])
+def test_conv_backward_matches_finite_differences(K, L, with_prev, with_bias):
+    rng = _rng(90 + 7 * K + L)
+    b, d = 2, 3
+    x = rng.standard_normal((b, d, L))
+    w = rng.standard_normal((d, K))
+    bias = rng.standard_normal(d) if with_bias else None
+    prev = rng.standard_normal((b, d, K - 1)) if with_prev else None
+    du = rng.standard_normal((b, d, L))
+    dxn = rng.standard_normal((b, d, K - 1))
+    g = oracle.causal_conv_silu_bwd(x, w, du, bias, prev, dx_next=dxn)
+
+    def loss(xx=x, ww=w, bb=bias, pp=prev):
+        u, x_next = oracle.causal_conv_silu(xx, ww, bb, pp)
+        return float((du * u).sum() + (dxn * x_next).sum())
+
+    _assert_fd(g["dx"], _central_fd(lambda v: loss(xx=v), x), "conv dx")
+    _assert_fd(g["dw"], _central_fd(lambda v: loss(ww=v), w), "conv dw")
+    _assert_fd(g["dbias"], _central_fd(lambda v: loss(bb=v), bias if with_bias else np.zeros(d)), "conv dbias")
+    if K > 1:
+        _assert_fd(g["dx_prev"], _central_fd(lambda v: loss(pp=v), prev if with_prev else np.zeros((b, d, K - 1))),
+                   "conv dx_prev")
+    # without dx_next the state output carries no gradient
+    g0 = oracle.causal_conv_silu_bwd(x, w, du, bias, prev)
+    _assert_fd(g0["dx"], _central_fd(lambda v: float((du * oracle.causal_conv_silu(v, w, bias, prev)[0]).sum()), x),
+               "conv dx (no dx_next)")
+
+
+@pytest.mark.parametrize("zoh", [False, True], ids=["simplified", "zoh"])
+def test_conv_scan_chain_matches_finite_differences(zoh):
+    # the whole Mamba x branch: u = silu(conv(x)), then the scan; gradients with respect to
+    # x and the conv weight through both backward functions
+    rng = _rng(95)
+    b, d, n, L, K = 2, 3, 4, 8, 4
+    case = _selective_case(rng, b=b, d=d, n=n, L=L)
+    x = rng.standard_normal((b, d, L))
+    w = 0.5 * rng.standard_normal((d, K))
+    cb = rng.standard_normal(d)
+    prev = rng.standard_normal((b, d, K - 1))
+    dy = rng.standard_normal((b, d, L))
+    u, _ = oracle.causal_conv_silu(x, w, cb, prev)
+    gs = oracle.selective_scan_bwd(**dict(case, u=u), dy=dy, zoh=zoh)
+    gc = oracle.causal_conv_silu_bwd(x, w, gs["du"], cb, prev)
+
+    def loss(xx=x, ww=w):
+        uu, _ = oracle.causal_conv_silu(xx, ww, cb, prev)
+        y, _ = oracle.selective_scan(**dict(case, u=uu), zoh=zoh)
+        return float((dy * y).sum())
+
+    _assert_fd(gc["dx"], _central_fd(lambda v: loss(xx=v), x), "chain dx")
+    _assert_fd(gc["dw"], _central_fd(lambda v: loss(ww=v), w), "chain dw")
