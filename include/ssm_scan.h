@@ -137,8 +137,8 @@ typedef enum {
  * Discretisation of the continuous system ([Eng] §2.2).  SIMPLIFIED (the default): Abar = exp(Delta A),
  * Bbar = Delta B ([Card] 离散化变换).  ZOH: the zero-order hold, Bbar = (Delta A)^-1 (exp(Delta A) - 1)
  * Delta B = expm1(Delta A)/A * B for the diagonal A (Delta B when A = 0).  ZOH is supported by the
- * sequential and direct forward kernels and by decode; SSM_ALGO_CHUNKED and the backward return
- * SSM_ERR_UNSUPPORTED for it.
+ * sequential and direct forward kernels, by decode and by ssm_selective_scan_bwd_ex;
+ * SSM_ALGO_CHUNKED returns SSM_ERR_UNSUPPORTED for it.
  */
 typedef enum { SSM_DISC_SIMPLIFIED = 0, SSM_DISC_ZOH = 1 } ssm_discretization_t;
 
@@ -254,6 +254,46 @@ ssm_status_t ssm_selective_scan_bwd(
     float* ddelta_bias, float* dinitial_state,
     int batch, int dim, int dstate, int64_t seqlen, ssm_dtype_t io_dtype,
     void* workspace, size_t workspace_bytes, ssm_stream_t stream);
+
+/* Options of ssm_selective_scan_bwd_ex.  Zero-initialise the whole struct: all zero (or opts
+ * NULL) is ssm_selective_scan_bwd. */
+typedef struct {
+    int discretization;            /* ssm_discretization_t of the forward; 0 = SSM_DISC_SIMPLIFIED        */
+    const ssm_conv_t* conv;        /* the forward's conv prologue, or NULL.  weight, bias, width and
+                                      state_in are read; state_out and u_out are ignored.                */
+    float* dconv_weight;           /* (dim, width) fp32 output; required with conv                       */
+    float* dconv_bias;             /* (dim) fp32 output, or NULL                                          */
+    float* dconv_state_in;         /* (batch, dim, width-1) fp32 output: gradient of conv->state_in, or NULL */
+    const float* dconv_state_out;  /* (batch, dim, width-1) fp32: gradient reaching conv->state_out (the
+                                      carried-out inputs), or NULL (zero)                                 */
+} ssm_bwd_options_t;
+
+/*
+ * Backward of the zero-order-hold scan and / or of ssm_selective_scan_fwd_conv.  Arguments,
+ * workspace (ssm_selective_scan_bwd_workspace_size) and errors as ssm_selective_scan_bwd, and:
+ *   discretization = SSM_DISC_ZOH: the gradients of the ZOH scan, where the input weight is
+ *     phi B with phi = expm1(Delta A) / A ([Eng] §2.2): dB_t += g phi u_t,
+ *     du_t = sum_n g phi B_t + D dv_t, dDelta_t = sum_n g a_t (A h_{t-1} + B_t u_t),
+ *     dA += g (Delta_t a_t h_{t-1} + dphi/dA B_t u_t), dphi/dA = (Delta a_t - phi) / A
+ *     (its Taylor series where |Delta A| < 1/16).
+ *   conv != NULL: `u` is the conv input x (io_dtype (batch, dim, seqlen)) and `du` receives dx.
+ *     u = silu(p), p_t = bias + sum_k weight[k] x_{t-width+1+k}, is recomputed from x (rounded to
+ *     io_dtype as the forward rounds it) and never stored; with du_t the gradient reaching u
+ *     (taken through the rounding unchanged) and dp_t = du_t silu'(p_t):
+ *       dx_s = sum_k weight[k] dp_{s+width-1-k} (+ dconv_state_out for the last width-1 inputs),
+ *       dconv_weight[d,k] = sum over batch rows and t of dp_t x_{t-width+1+k},
+ *       dconv_bias[d] = sum dp_t,  dconv_state_in = dx_s for s = -(width-1) .. -1.
+ *     d_state 16.  The conv arrays need no alignment beyond their element type.
+ * seqlen == 0: dconv_weight and dconv_bias are zero and dconv_state_in is dconv_state_out.
+ */
+ssm_status_t ssm_selective_scan_bwd_ex(
+    const void* u, const void* delta, const float* A, const void* B, const void* C,
+    const float* D, const void* z, const float* delta_bias, int softplus,
+    const float* initial_state, const void* dy, const float* dlast_state,
+    void* du, void* ddelta, float* dA, float* dB, float* dC, float* dD, void* dz,
+    float* ddelta_bias, float* dinitial_state,
+    int batch, int dim, int dstate, int64_t seqlen, ssm_dtype_t io_dtype,
+    void* workspace, size_t workspace_bytes, const ssm_bwd_options_t* opts, ssm_stream_t stream);
 
 /*
  * One-token decode ([Card] 线性扫描算法: a fixed-size state update per token;

@@ -10,6 +10,7 @@ from .binding import (  # noqa: F401
     selective_scan_fwd,
     ssm_read_status,
     ssm_selective_scan_bwd,
+    ssm_selective_scan_bwd_ex,
     ssm_selective_scan_bwd_workspace_size,
     ssm_selective_scan_fwd,
     ssm_selective_scan_fwd_conv,

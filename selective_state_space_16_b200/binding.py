@@ -49,6 +49,13 @@ class ConvSpec(ctypes.Structure):
                 ("state_in", ctypes.c_void_p), ("state_out", ctypes.c_void_p), ("u_out", ctypes.c_void_p)]
 
 
+class BwdOptions(ctypes.Structure):
+    """ssm_bwd_options_t: discretisation and conv prologue of a backward call."""
+    _fields_ = [("discretization", ctypes.c_int), ("conv", ctypes.POINTER(ConvSpec)),
+                ("dconv_weight", ctypes.c_void_p), ("dconv_bias", ctypes.c_void_p),
+                ("dconv_state_in", ctypes.c_void_p), ("dconv_state_out", ctypes.c_void_p)]
+
+
 _lib = None
 _lock = threading.Lock()
 
@@ -76,6 +83,9 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.ssm_selective_scan_bwd_workspace_size.restype = sz
     lib.ssm_selective_scan_bwd.argtypes = [vp] * 8 + [ci] + [vp] * 12 + [ci, ci, ci, i64, ci, vp, sz, vp]
     lib.ssm_selective_scan_bwd.restype = ci
+    lib.ssm_selective_scan_bwd_ex.argtypes = ([vp] * 8 + [ci] + [vp] * 12 + [ci, ci, ci, i64, ci, vp, sz,
+                                                                         ctypes.POINTER(BwdOptions), vp])
+    lib.ssm_selective_scan_bwd_ex.restype = ci
     lib.ssm_state_update.argtypes = [vp] * 9 + [ci, vp, ci, ci, ci, ci, vp]
     lib.ssm_state_update.restype = ci
     lib.ssm_state_update_ex.argtypes = [vp] * 9 + [ci, vp, ci, ci, ci, ci, ci, vp]
@@ -231,11 +241,40 @@ def ssm_selective_scan_bwd(u, delta, A, B, C, D, z, delta_bias, softplus, dy, du
     return code
 
 
+def ssm_selective_scan_bwd_ex(u, delta, A, B, C, D, z, delta_bias, softplus, dy, du, ddelta, dA, dB, dC, dD, dz,
+                              ddelta_bias, workspace, initial_state=None, dlast_state=None, dinitial_state=None,
+                              zoh=False, conv_weight=None, conv_bias=None, conv_state_in=None, dconv_weight=None,
+                              dconv_bias=None, dconv_state_in=None, dconv_state_out=None, stream=None, check=True):
+    """Marshal ssm_selective_scan_bwd_ex: as ssm_selective_scan_bwd, plus zoh and, when
+    conv_weight (d, K) fp32 is given, the conv prologue: u is then x and du receives dx;
+    dconv_weight (d, K), dconv_bias (d), dconv_state_in / dconv_state_out (b, d, K-1) fp32."""
+    b, d, L = u.shape
+    n = A.shape[1]
+    spec = None
+    if conv_weight is not None:
+        spec = ConvSpec(_ptr(conv_weight), _ptr(conv_bias), int(conv_weight.shape[1]), _ptr(conv_state_in), None,
+                        None)
+    opts = BwdOptions(SSM_DISC_ZOH if zoh else SSM_DISC_SIMPLIFIED,
+                      ctypes.pointer(spec) if spec is not None else None, _ptr(dconv_weight), _ptr(dconv_bias),
+                      _ptr(dconv_state_in), _ptr(dconv_state_out))
+    code = load().ssm_selective_scan_bwd_ex(
+        _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias), int(bool(softplus)),
+        _ptr(initial_state), _ptr(dy), _ptr(dlast_state), _ptr(du), _ptr(ddelta), _ptr(dA), _ptr(dB), _ptr(dC),
+        _ptr(dD), _ptr(dz), _ptr(ddelta_bias), _ptr(dinitial_state), b, d, n, L, _io(u), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), ctypes.byref(opts), _stream(stream))
+    if check:
+        _check(code, "ssm_selective_scan_bwd_ex")
+    return code
+
+
 def selective_scan_bwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True, dy=None,
-                       initial_state=None, dlast_state=None, workspace=None, stream=None):
+                       initial_state=None, dlast_state=None, workspace=None, stream=None, zoh=False,
+                       conv_weight=None, conv_bias=None, conv_state_in=None, dconv_state_out=None):
     """Convenience wrapper: allocates every gradient and, if not given, a workspace, then
-    calls ssm_selective_scan_bwd.  Returns a dict du, ddelta, dz (or None), dA, dB, dC, dD,
-    ddelta_bias, dinitial_state."""
+    calls ssm_selective_scan_bwd (ssm_selective_scan_bwd_ex with zoh or a conv).  Returns a dict
+    du, ddelta, dz (or None), dA, dB, dC, dD, ddelta_bias, dinitial_state; with conv_weight
+    (u is then the conv input x) also dx (in place of du, which is then None), dconv_weight,
+    dconv_bias and dconv_state_in (None for width 1)."""
     b, d, L = u.shape
     n = A.shape[1]
     f32 = dict(dtype=torch.float32, device=u.device)
@@ -246,10 +285,28 @@ def selective_scan_bwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
     if workspace is None:
         workspace = torch.empty(max(ssm_selective_scan_bwd_workspace_size(b, d, n, L), 256), dtype=torch.uint8,
                                 device=u.device)
-    ssm_selective_scan_bwd(u, delta, A, B, C, D, z, delta_bias, softplus, dy, out["du"], out["ddelta"], out["dA"],
-                           out["dB"], out["dC"], out["dD"], out["dz"], out["ddelta_bias"], workspace,
-                           initial_state=initial_state, dlast_state=dlast_state,
-                           dinitial_state=out["dinitial_state"], stream=stream)
+    if not zoh and conv_weight is None:
+        ssm_selective_scan_bwd(u, delta, A, B, C, D, z, delta_bias, softplus, dy, out["du"], out["ddelta"],
+                               out["dA"], out["dB"], out["dC"], out["dD"], out["dz"], out["ddelta_bias"], workspace,
+                               initial_state=initial_state, dlast_state=dlast_state,
+                               dinitial_state=out["dinitial_state"], stream=stream)
+        return out
+    if conv_weight is not None:
+        K = int(conv_weight.shape[1])
+        out["dx"] = out.pop("du")
+        out["du"] = None
+        out["dconv_weight"] = torch.empty((d, K), **f32)
+        out["dconv_bias"] = torch.empty(d, **f32)
+        out["dconv_state_in"] = torch.empty((b, d, K - 1), **f32) if K > 1 else None
+    ssm_selective_scan_bwd_ex(u, delta, A, B, C, D, z, delta_bias, softplus, dy,
+                              out["dx"] if conv_weight is not None else out["du"], out["ddelta"], out["dA"],
+                              out["dB"], out["dC"], out["dD"], out["dz"], out["ddelta_bias"], workspace,
+                              initial_state=initial_state, dlast_state=dlast_state,
+                              dinitial_state=out["dinitial_state"], zoh=zoh, conv_weight=conv_weight,
+                              conv_bias=conv_bias, conv_state_in=conv_state_in,
+                              dconv_weight=out.get("dconv_weight"), dconv_bias=out.get("dconv_bias"),
+                              dconv_state_in=out.get("dconv_state_in"), dconv_state_out=dconv_state_out,
+                              stream=stream)
     return out
 
 

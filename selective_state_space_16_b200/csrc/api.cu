@@ -337,14 +337,31 @@ size_t ssm_selective_scan_bwd_workspace_size(int batch, int dim, int dstate, int
     return round_up(bwd_layout(batch, dim, seqlen).total, 256);
 }
 
-ssm_status_t ssm_selective_scan_bwd(const void* u, const void* delta, const float* A, const void* B, const void* C,
-                                    const float* D, const void* z, const float* delta_bias, int softplus,
-                                    const float* initial_state, const void* dy, const float* dlast_state, void* du,
-                                    void* ddelta, float* dA, float* dB, float* dC, float* dD, void* dz,
-                                    float* ddelta_bias, float* dinitial_state, int batch, int dim, int dstate,
-                                    int64_t seqlen, ssm_dtype_t io_dtype, void* workspace, size_t workspace_bytes,
-                                    ssm_stream_t stream) {
+ssm_status_t ssm_selective_scan_bwd_ex(const void* u, const void* delta, const float* A, const void* B,
+                                       const void* C, const float* D, const void* z, const float* delta_bias,
+                                       int softplus, const float* initial_state, const void* dy,
+                                       const float* dlast_state, void* du, void* ddelta, float* dA, float* dB,
+                                       float* dC, float* dD, void* dz, float* ddelta_bias, float* dinitial_state,
+                                       int batch, int dim, int dstate, int64_t seqlen, ssm_dtype_t io_dtype,
+                                       void* workspace, size_t workspace_bytes, const ssm_bwd_options_t* opts,
+                                       ssm_stream_t stream) {
     if (batch < 0 || dim < 0 || seqlen < 0) return SSM_ERR_INVALID_ARG;
+    ssm_bwd_options_t o{};
+    if (opts) o = *opts;
+    if (o.discretization != SSM_DISC_SIMPLIFIED && o.discretization != SSM_DISC_ZOH) return SSM_ERR_INVALID_ARG;
+    ConvBwdArgs conv;
+    if (o.conv) {
+        if (o.conv->width < 1 || o.conv->width > 4) return SSM_ERR_INVALID_ARG;
+        if (dim > 0 && (!o.conv->weight || !o.dconv_weight)) return SSM_ERR_INVALID_ARG;
+        conv.k = o.conv->width;
+        conv.w = o.conv->weight;
+        conv.b = o.conv->bias;
+        conv.in = conv.k > 1 ? o.conv->state_in : nullptr;
+        conv.dout = conv.k > 1 ? o.dconv_state_out : nullptr;
+        conv.dw = o.dconv_weight;
+        conv.db = o.dconv_bias;
+        conv.din = conv.k > 1 ? o.dconv_state_in : nullptr;
+    }
     const bool seq_elems = batch > 0 && dim > 0 && seqlen > 0;
     if (seq_elems && (!u || !delta || !B || !C || !dy || !du || !ddelta || !dB || !dC || (z && !dz)))
         return SSM_ERR_INVALID_ARG;
@@ -364,7 +381,7 @@ ssm_status_t ssm_selective_scan_bwd(const void* u, const void* delta, const floa
     ssm_status_t st = check_device(nullptr);
     if (st != SSM_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (seqlen == 0) {  // no steps: only the state passes through
+    if (seqlen == 0) {  // no steps: only the state (and the conv's carried inputs) pass through
         const size_t state_bytes = static_cast<size_t>(batch) * dim * 16 * sizeof(float);
         cudaError_t e = cudaMemsetAsync(dA, 0, static_cast<size_t>(dim) * 16 * sizeof(float), s);
         if (e == cudaSuccess && dD) e = cudaMemsetAsync(dD, 0, static_cast<size_t>(dim) * sizeof(float), s);
@@ -373,11 +390,32 @@ ssm_status_t ssm_selective_scan_bwd(const void* u, const void* delta, const floa
         if (e == cudaSuccess && dinitial_state)
             e = dlast_state ? cudaMemcpyAsync(dinitial_state, dlast_state, state_bytes, cudaMemcpyDeviceToDevice, s)
                             : cudaMemsetAsync(dinitial_state, 0, state_bytes, s);
+        if (conv.k > 0) {
+            const size_t cs_bytes = static_cast<size_t>(batch) * dim * (conv.k - 1) * sizeof(float);
+            if (e == cudaSuccess) e = cudaMemsetAsync(conv.dw, 0, static_cast<size_t>(dim) * conv.k * sizeof(float), s);
+            if (e == cudaSuccess && conv.db) e = cudaMemsetAsync(conv.db, 0, static_cast<size_t>(dim) * sizeof(float), s);
+            if (e == cudaSuccess && conv.din && cs_bytes > 0)
+                e = conv.dout ? cudaMemcpyAsync(conv.din, conv.dout, cs_bytes, cudaMemcpyDeviceToDevice, s)
+                              : cudaMemsetAsync(conv.din, 0, cs_bytes, s);
+        }
         return e == cudaSuccess ? SSM_OK : SSM_ERR_LAUNCH;
     }
     BwdArgs a{u, delta, B, C, z, dy, A, D, delta_bias, initial_state, dlast_state, softplus, du, ddelta, dz, dA, dB,
-              dC, dD, ddelta_bias, dinitial_state, batch, dim, seqlen, static_cast<uint8_t*>(workspace), s};
+              dC, dD, ddelta_bias, dinitial_state, batch, dim, seqlen, static_cast<uint8_t*>(workspace), s,
+              o.discretization == SSM_DISC_ZOH, conv};
     return io_dtype == SSM_BF16 ? launch_backward<__nv_bfloat16>(a) : launch_backward<float>(a);
+}
+
+ssm_status_t ssm_selective_scan_bwd(const void* u, const void* delta, const float* A, const void* B, const void* C,
+                                    const float* D, const void* z, const float* delta_bias, int softplus,
+                                    const float* initial_state, const void* dy, const float* dlast_state, void* du,
+                                    void* ddelta, float* dA, float* dB, float* dC, float* dD, void* dz,
+                                    float* ddelta_bias, float* dinitial_state, int batch, int dim, int dstate,
+                                    int64_t seqlen, ssm_dtype_t io_dtype, void* workspace, size_t workspace_bytes,
+                                    ssm_stream_t stream) {
+    return ssm_selective_scan_bwd_ex(u, delta, A, B, C, D, z, delta_bias, softplus, initial_state, dy, dlast_state,
+                                     du, ddelta, dA, dB, dC, dD, dz, ddelta_bias, dinitial_state, batch, dim, dstate,
+                                     seqlen, io_dtype, workspace, workspace_bytes, nullptr, stream);
 }
 
 ssm_status_t ssm_read_status(void* workspace, ssm_stream_t stream) {

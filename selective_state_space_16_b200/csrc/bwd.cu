@@ -15,9 +15,22 @@ BwdLayout bwd_layout(int batch, int dim, int64_t L) {
     w.dA_off = w.dbc_off + round_up(B * static_cast<size_t>(w.ncta) * Ls * 128u, 256);
     w.dD_off = w.dA_off + round_up(B * D * 64u, 256);
     w.dbias_off = w.dD_off + round_up(B * D * 4u, 256);
-    w.total = w.dbias_off + round_up(B * D * 4u, 256);
+    w.dcw_off = w.dbias_off + round_up(B * D * 4u, 256);
+    w.dcb_off = w.dcw_off + round_up(B * D * 16u, 256);
+    w.total = w.dcb_off + round_up(B * D * 4u, 256);
     return w;
 }
+
+namespace {
+template <typename IO>
+using BwdKernel = void (*)(const ssm::BwdParams);
+
+template <typename IO>
+BwdKernel<IO> bwd_kernel(bool zoh, bool conv) {
+    if (conv) return zoh ? ssm::scan_bwd_kernel<IO, true, true> : ssm::scan_bwd_kernel<IO, false, true>;
+    return zoh ? ssm::scan_bwd_kernel<IO, true, false> : ssm::scan_bwd_kernel<IO, false, false>;
+}
+}  // namespace
 
 template <typename IO>
 ssm_status_t launch_backward(const BwdArgs& a) {
@@ -54,8 +67,16 @@ ssm_status_t launch_backward(const BwdArgs& a) {
     p.ncta = wl.ncta;
     p.softplus = a.softplus;
     p.hdr = reinterpret_cast<WorkspaceHeader*>(a.ws);
+    p.conv_w = a.conv.w;
+    p.conv_b = a.conv.b;
+    p.conv_in = a.conv.in;
+    p.dconv_out = a.conv.dout;
+    p.dconv_in = a.conv.din;
+    p.dcw_part = reinterpret_cast<float*>(a.ws + wl.dcw_off);
+    p.dcb_part = reinterpret_cast<float*>(a.ws + wl.dcb_off);
+    p.conv_k = a.conv.k;
     constexpr int smem = ssm::kBwdSmem;
-    auto kern = ssm::scan_bwd_kernel<IO>;
+    auto kern = bwd_kernel<IO>(a.zoh != 0, a.conv.k > 0);
     if (!ensure_smem_attr(reinterpret_cast<const void*>(kern), smem)) return SSM_ERR_LAUNCH;
     kern<<<dim3(static_cast<unsigned>(wl.ncta), static_cast<unsigned>(a.batch)), ssm::kBwdWarps * 32, smem,
            a.stream>>>(p);
@@ -70,6 +91,11 @@ ssm_status_t launch_backward(const BwdArgs& a) {
     f.dA = a.dA;
     f.dD = a.dD;
     f.dbias = a.dbias;
+    f.dcw_part = p.dcw_part;
+    f.dcb_part = p.dcb_part;
+    f.dconv_w = a.conv.dw;
+    f.dconv_b = a.conv.db;
+    f.conv_k = a.conv.k;
     f.batch = a.batch;
     f.dim = a.dim;
     f.ncta = wl.ncta;

@@ -109,11 +109,19 @@ struct FwdArgs {
 //   [header 256 B][B/C rows: batch * L * 128 B][checkpoints: batch * nseg * dim * 64 B]
 //   [dB/dC per CTA: batch * ncta * L * 128 B][dA per batch row: batch * dim * 64 B]
 //   [dD per batch row: batch * dim * 4 B][ddelta_bias per batch row: batch * dim * 4 B]
+//   [conv weight per batch row: batch * dim * 16 B][conv bias per batch row: batch * dim * 4 B]
 struct BwdLayout {
-    size_t bc_off, ckpt_off, dbc_off, dA_off, dD_off, dbias_off, total;
+    size_t bc_off, ckpt_off, dbc_off, dA_off, dD_off, dbias_off, dcw_off, dcb_off, total;
     int nseg, ncta;
 };
 BwdLayout bwd_layout(int batch, int dim, int64_t L);
+
+// Conv prologue of a backward call (k = 0: none; `u` then holds x and `du` receives dx).
+struct ConvBwdArgs {
+    const float *w = nullptr, *b = nullptr, *in = nullptr, *dout = nullptr;
+    float *dw = nullptr, *db = nullptr, *din = nullptr;
+    int k = 0;
+};
 
 struct BwdArgs {
     const void *u, *delta, *B, *C, *z, *dy;
@@ -125,6 +133,8 @@ struct BwdArgs {
     int64_t L;
     uint8_t* ws;
     cudaStream_t stream;
+    int zoh = 0;
+    ConvBwdArgs conv;
 };
 
 struct DecodeArgs {

@@ -39,6 +39,20 @@
 //     does not depend on scheduling).
 //   - dA, dD and ddelta_bias are summed over time in registers, written per batch row and
 //     added over batch rows by the second kernel.
+//
+// Zero-order hold (ZOH, [Eng] §2.2): the input weight Delta B becomes phi B with
+// phi = expm1(Delta A) / A, so that dB_t += g phi u_t, du_t = sum_n g phi B_t + D dv_t,
+// dDelta_t = sum_n g (A a_t h_{t-1} + a_t B_t u_t) (dphi/dDelta = a_t) and
+// dA_n += g (Delta_t a_t h_{t-1} + dphi/dA B_t u_t) (zoh_dphi_dA2).
+//
+// Conv prologue (CONV, [Hist] Mamba Block 数据流: x -> conv1d -> SiLU -> S6): the kernel reads x
+// and forms u = silu(p), p_t = cb + sum_k w_k x_{t-3+k} (taps right-aligned, rounded to the I/O
+// type as the forward rounds it) from a 5-step window of x per lane.  The conv's backward is
+// folded into the reverse walk: dp_t = du_t silu'(p_t), and dx_t = sum_k w_k dp_{t+3-k} needs
+// dp of steps t .. t+3 -- the lane's own two steps, the next lanes' and, across the segment
+// boundary, the first steps of the later segment, which the walk has already finished and
+// carries in registers.  dw_k and the conv bias are summed like dD; after step 0 the carried
+// dp gives the gradient of the conv's carried-in inputs.  du itself never reaches HBM.
 #pragma once
 
 #include "common.cuh"
@@ -67,6 +81,14 @@ struct BwdParams {
     float* dA_part;                  // workspace: [batch][dim][16]
     float* dD_part;                  // workspace: [batch][dim]
     float* dbias_part;               // workspace: [batch][dim]
+    // conv prologue (CONV kernels): u holds x
+    const float *conv_w, *conv_b;    // (dim, conv_k) oldest tap first; (dim) or null
+    const float* conv_in;            // (batch, dim, conv_k - 1): inputs before t = 0, or null (zero)
+    const float* dconv_out;          // (batch, dim, conv_k - 1): gradient reaching the carried-out inputs, or null
+    float* dconv_in;                 // (batch, dim, conv_k - 1) output, or null
+    float* dcw_part;                 // workspace: [batch][dim][4] (taps right-aligned)
+    float* dcb_part;                 // workspace: [batch][dim]
+    int conv_k;
     int batch, dim;
     long long L;
     int nseg, ncta;
@@ -86,8 +108,8 @@ __device__ __forceinline__ float load_io(const void* base, long long i) {
     return IoTraits<IO>::to_f32(static_cast<const IO*>(base)[i]);
 }
 
-template <typename IO>
-__global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdParams p) {
+template <typename IO, bool ZOH, bool CONV>
+__global__ void __launch_bounds__(kBwdWarps * 32, CONV ? 4 : 5) scan_bwd_kernel(const BwdParams p) {
     constexpr int T = kBwdSeg, G = 4, PER = T / G, R = kBwdRing;
     extern __shared__ float4 bwd_smem[];
     // h_{t-1} of the segment's steps: [warp][step][lane] (16 bytes each)
@@ -123,13 +145,17 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
     const bool softplus = p.softplus != 0;
     const bool has_z = p.z != nullptr;
 
-    float2 An[2], A2[2];  // A of the lane's 4 chains as pairs; A2 = A log2(e)
+    float2 An[2], A2[2], invA[2];  // A of the lane's 4 chains as pairs; A2 = A log2(e); 1 / A (ZOH)
     {
         const float4 a = valid ? *reinterpret_cast<const float4*>(p.A + dd * 16 + nl * 4) : make_float4(0, 0, 0, 0);
         An[0] = f2(a.x, a.y);
         An[1] = f2(a.z, a.w);
         A2[0] = f2(a.x * kLog2e, a.y * kLog2e);
         A2[1] = f2(a.z * kLog2e, a.w * kLog2e);
+        if constexpr (ZOH) {
+            invA[0] = f2(1.f / a.x, 1.f / a.y);
+            invA[1] = f2(1.f / a.z, 1.f / a.w);
+        }
     }
     const float Dd = (valid && p.D) ? p.D[dd] : 0.f;
     const float bias = (valid && p.bias) ? p.bias[dd] : 0.f;
@@ -141,6 +167,27 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
         const float2 arg = __fmul2_rn(f2(dti, dti), A2[j]);
         return f2(ex2_mufu(arg.x), ex2_mufu(arg.y));
     };
+    // input weight times u of chain pair j (per unit B): Delta u, or phi u with the ZOH weight
+    // phi formed from a = decay(Delta, j)
+    auto weight_u = [&](float dti, float ui, int j, float2 a) {
+        if constexpr (ZOH)
+            return __fmul2_rn(zoh_beta2(__fmul2_rn(f2(dti, dti), A2[j]), a, f2(dti, dti), invA[j]), f2(ui, ui));
+        else return f2(dti * ui, dti * ui);
+    };
+    // conv taps (right-aligned: tap k of a width-K conv at 4 - K + k) and bias
+    float cw[4] = {0.f, 0.f, 0.f, 0.f}, cb = 0.f;
+    const int K = CONV ? p.conv_k : 1;
+    const long long crow = (static_cast<long long>(b) * p.dim + dd) * (K - 1);  // conv state row
+    if constexpr (CONV) {
+        if (valid) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int k = j - (4 - K);
+                cw[j] = k >= 0 ? p.conv_w[static_cast<long long>(dd) * K + k] : 0.f;
+            }
+            cb = p.conv_b ? p.conv_b[dd] : 0.f;
+        }
+    }
     auto ckpt_at = [&](int s) { return ckrow + s * ckstride; };
     // B and C of the lane's 4 chains at one step, from the lane's place in a ring row
     // (byte 16 nl: fp32 B there and C 64 bytes on; bf16 pairs (B, C, B, C) there).
@@ -176,9 +223,12 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
         cp_async_commit();
     };
 
-    // Raw inputs of the lane's own steps 2nl, 2nl+1 of segment seg: delta, u, dy, z.
+    // Raw inputs of the lane's own steps 2nl, 2nl+1 of segment seg: delta, u, dy, z.  With the
+    // conv, xw holds the conv inputs of steps 2nl-3 .. 2nl+1 (x, the carried-in state before
+    // t = 0) and conv_u() forms p and u from them once the loads have landed.
+    constexpr int W = CONV ? PER + 3 : 1;
     struct Raw {
-        float x[PER], u[PER], dy[PER], z[PER];
+        float x[PER], u[PER], dy[PER], z[PER], xw[W], pre[CONV ? PER : 1];
     };
     auto load_raw = [&](int seg, bool with_grad, Raw& r) {
 #pragma unroll
@@ -186,9 +236,34 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
             const int t = seg * T + nl * PER + k;
             const bool in = valid && seg >= 0 && t < L;
             r.x[k] = in ? IoTraits<IO>::to_f32(x_row[t]) : 0.f;
-            r.u[k] = in ? IoTraits<IO>::to_f32(u_row[t]) : 0.f;
+            if constexpr (!CONV) r.u[k] = in ? IoTraits<IO>::to_f32(u_row[t]) : 0.f;
             r.dy[k] = (in && with_grad) ? IoTraits<IO>::to_f32(dy_row[t]) : 0.f;
             r.z[k] = (in && with_grad && has_z) ? IoTraits<IO>::to_f32(z_row[t]) : 0.f;
+        }
+        if constexpr (CONV) {
+#pragma unroll
+            for (int i = 0; i < W; ++i) {
+                const int t = seg * T + nl * PER - 3 + i;
+                float v = 0.f;
+                if (valid && seg >= 0 && t < L) {
+                    if (t >= 0) v = IoTraits<IO>::to_f32(u_row[t]);
+                    else if (p.conv_in && t >= -(K - 1)) v = p.conv_in[crow + (K - 1) + t];
+                }
+                r.xw[i] = v;
+            }
+        }
+    };
+    auto conv_u = [&](int seg, Raw& r) {
+        if constexpr (CONV) {
+#pragma unroll
+            for (int k = 0; k < PER; ++k) {
+                float pre = cb;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) pre = fmaf(cw[j], r.xw[k + j], pre);
+                const int t = seg * T + nl * PER + k;
+                r.pre[k] = pre;
+                r.u[k] = (valid && t < L) ? IoTraits<IO>::to_f32(IoTraits<IO>::from_f32(silu_f32(pre))) : 0.f;
+            }
         }
     };
     auto step_sizes = [&](int seg, const Raw& r, float (&dt)[PER]) {
@@ -210,7 +285,8 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
     Raw nxt;
     load_raw(0, false, nxt);
     for (int s = 0; s < p.nseg; ++s) {
-        const Raw cur = nxt;
+        Raw cur = nxt;
+        conv_u(s, cur);
         load_raw(s + 1, false, nxt);  // next segment's inputs, in flight during this one
         __syncthreads();              // every warp is done with the slot refilled below
         issue_bc(s + R - 1, (s + R - 1) % R);
@@ -227,9 +303,11 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
             const float ui = __shfl_sync(0xffffffffu, cur.u[i % PER], srcl[i / PER]);
             float2 Bv[2];
             load_b(bcs + i * RB, Bv);
-            const float2 ww = f2(dti * ui, dti * ui);
-            h[0] = __ffma2_rn(decay(dti, 0), h[0], __fmul2_rn(ww, Bv[0]));
-            h[1] = __ffma2_rn(decay(dti, 1), h[1], __fmul2_rn(ww, Bv[1]));
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const float2 a = decay(dti, j);
+                h[j] = __ffma2_rn(a, h[j], __fmul2_rn(weight_u(dti, ui, j, a), Bv[j]));
+            }
         }
     }
     cp_async_wait<0>();
@@ -251,10 +329,13 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
     for (int r = 0; r < R - 1; ++r) issue_bc(p.nseg - 1 - r, r);
     load_raw(p.nseg - 1, true, nxt);
     float4 ck_nxt = valid ? ld4(ckpt_at(p.nseg - 1)) : make_float4(0, 0, 0, 0);
+    float dpc[PER] = {0.f, 0.f};                       // conv: dp of the lane's steps in the later segment
+    float dcw[4] = {0.f, 0.f, 0.f, 0.f}, dcb = 0.f;    // conv: weight and bias gradients (time sums)
     for (int k = 0; k < p.nseg; ++k) {
         const int s = p.nseg - 1 - k;
         const int t0 = s * T;
-        const Raw cur = nxt;
+        Raw cur = nxt;
+        conv_u(s, cur);
         const float4 ck = ck_nxt;
         load_raw(s - 1, true, nxt);
         if (valid && s > 0) ck_nxt = ld4(ckpt_at(s - 1));
@@ -278,9 +359,8 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
             load_bc(bcs + i * RB, Bv, Cv);
             const float2 a0 = decay(dti, 0), a1 = decay(dti, 1);
             hst[i * 32 + lane] = make_float4(hs[0].x, hs[0].y, hs[1].x, hs[1].y);
-            const float2 ww = f2(dti * ui, dti * ui);
-            hs[0] = __ffma2_rn(a0, hs[0], __fmul2_rn(ww, Bv[0]));
-            hs[1] = __ffma2_rn(a1, hs[1], __fmul2_rn(ww, Bv[1]));
+            hs[0] = __ffma2_rn(a0, hs[0], __fmul2_rn(weight_u(dti, ui, 0, a0), Bv[0]));
+            hs[1] = __ffma2_rn(a1, hs[1], __fmul2_rn(weight_u(dti, ui, 1, a1), Bv[1]));
             const float2 acc = __ffma2_rn(Cv[1], hs[1], __fmul2_rn(Cv[0], hs[0]));
             vp[i] = acc.x + acc.y;
         }
@@ -334,15 +414,26 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
                 g[j] = __ffma2_rn(dv2, Cv[j], g[j]);
                 dC[j] = __fmul2_rn(dv2, hn[j]);
                 const float2 ah = __fmul2_rn(av[j], hp[j]);
-                dA_acc[j] = __ffma2_rn(__fmul2_rn(g[j], dt2), ah, dA_acc[j]);
-                sdt = __ffma2_rn(g[j], __ffma2_rn(An[j], ah, __fmul2_rn(Bv[j], u2)), sdt);
-                sdu = __ffma2_rn(g[j], Bv[j], sdu);
-                dB[j] = __fmul2_rn(g[j], w2);
+                if constexpr (ZOH) {
+                    const float2 y = __fmul2_rn(dt2, A2[j]);
+                    const float2 phi = zoh_beta2(y, av[j], dt2, invA[j]);
+                    const float2 bu = __fmul2_rn(Bv[j], u2);
+                    const float2 dphi = zoh_dphi_dA2(y, av[j], dt2, phi, invA[j]);
+                    dA_acc[j] = __ffma2_rn(g[j], __ffma2_rn(dt2, ah, __fmul2_rn(dphi, bu)), dA_acc[j]);
+                    sdt = __ffma2_rn(g[j], __ffma2_rn(An[j], ah, __fmul2_rn(av[j], bu)), sdt);
+                    sdu = __ffma2_rn(g[j], __fmul2_rn(phi, Bv[j]), sdu);
+                    dB[j] = __fmul2_rn(g[j], __fmul2_rn(phi, u2));
+                } else {
+                    dA_acc[j] = __ffma2_rn(__fmul2_rn(g[j], dt2), ah, dA_acc[j]);
+                    sdt = __ffma2_rn(g[j], __ffma2_rn(An[j], ah, __fmul2_rn(Bv[j], u2)), sdt);
+                    sdu = __ffma2_rn(g[j], Bv[j], sdu);
+                    dB[j] = __fmul2_rn(g[j], w2);
+                }
                 g[j] = __fmul2_rn(g[j], av[j]);
                 hn[j] = hp[j];
             }
             ddt[i] = sdt.x + sdt.y;
-            dup[i] = (sdu.x + sdu.y) * dti;
+            dup[i] = ZOH ? sdu.x + sdu.y : (sdu.x + sdu.y) * dti;
             // dB/dC: reduce-scatter the 8 values over the warp's 8 channels (lane bits 4, 3, 2).
             float vals[8] = {dB[0].x, dB[0].y, dB[1].x, dB[1].y, dC[0].x, dC[0].y, dC[1].x, dC[1].y};
 #pragma unroll
@@ -371,6 +462,38 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
                 dup[i] = k2 + __shfl_xor_sync(0xffffffffu, s2, m);
             }
         }
+        // Conv: dp = du silu'(p) of the lane's steps, then dx_t = sum_j cw_j dp_{t+3-j} from the
+        // window dp_t .. dp_{t+4}: own steps, the next lane's, the first of the lane after
+        // (lanes past the segment's end: their steps of the later segment, carried in dpc).
+        float dxv[PER] = {0.f, 0.f};
+        if constexpr (CONV) {
+            float dp[PER];
+#pragma unroll
+            for (int r = 0; r < PER; ++r) {
+                const int t = t0 + nl * PER + r;
+                const float pre = cur.pre[r];
+                const float sg = sigmoid_f32(pre);
+                dp[r] = (valid && t < L) ? fmaf(Dd, dv[r], dup[r]) * sg * fmaf(pre, 1.f - sg, 1.f) : 0.f;
+                dcb += dp[r];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) dcw[j] = fmaf(dp[r], cur.xw[r + j], dcw[j]);
+            }
+            const int l1 = gbase | ((nl + 1) & 3), l2 = gbase | ((nl + 2) & 3);
+            const float a0 = __shfl_sync(0xffffffffu, dp[0], l1), a1 = __shfl_sync(0xffffffffu, dp[1], l1);
+            const float b0 = __shfl_sync(0xffffffffu, dp[0], l2);
+            const float c0 = __shfl_sync(0xffffffffu, dpc[0], l1), c1 = __shfl_sync(0xffffffffu, dpc[1], l1);
+            const float e0 = __shfl_sync(0xffffffffu, dpc[0], l2);
+            const float win[PER + 3] = {dp[0], dp[1], nl + 1 < 4 ? a0 : c0, nl + 1 < 4 ? a1 : c1, nl + 2 < 4 ? b0 : e0};
+#pragma unroll
+            for (int r = 0; r < PER; ++r) {
+                float acc = 0.f;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc = fmaf(cw[j], win[r + 3 - j], acc);
+                dxv[r] = acc;
+            }
+            dpc[0] = dp[0];
+            dpc[1] = dp[1];
+        }
 #pragma unroll
         for (int r = 0; r < PER; ++r) {
             const int t = t0 + nl * PER + r;
@@ -379,7 +502,13 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
                 const float dx = softplus ? ddt[r] * sigmoid_f32(cur.x[r] + bias) : ddt[r];
                 dbias_acc += dx;
                 ddelta_row[t] = IoTraits<IO>::from_f32(dx);
-                du_row[t] = IoTraits<IO>::from_f32(fmaf(Dd, dv[r], dup[r]));
+                if constexpr (CONV) {
+                    float v = dxv[r];
+                    if (p.dconv_out && t >= L - (K - 1)) v += p.dconv_out[crow + t - (L - (K - 1))];
+                    du_row[t] = IoTraits<IO>::from_f32(v);  // du holds dx with the conv
+                } else {
+                    du_row[t] = IoTraits<IO>::from_f32(fmaf(Dd, dv[r], dup[r]));
+                }
                 if (has_z) dz_row[t] = IoTraits<IO>::from_f32(dzv[r]);
             }
         }
@@ -412,6 +541,35 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
         p.dD_part[static_cast<long long>(b) * p.dim + dd] = dD_acc;
         p.dbias_part[static_cast<long long>(b) * p.dim + dd] = dbias_acc;
     }
+    if constexpr (CONV) {
+        // Conv carried-in inputs x_s, s = -3 .. -1: d x_s = sum_j cw_j dp_{s+3-j} over dp_0 .. dp_2
+        // (lane nl 0 holds steps 0, 1 and lane 1 step 2 of segment 0 in dpc).
+        const float q0 = __shfl_sync(0xffffffffu, dpc[0], gbase), q1 = __shfl_sync(0xffffffffu, dpc[1], gbase);
+        const float q2 = __shfl_sync(0xffffffffu, dpc[0], gbase | 1);
+#pragma unroll
+        for (int m = 1; m <= 2; m <<= 1) {
+            dcb += __shfl_xor_sync(0xffffffffu, dcb, m);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) dcw[j] += __shfl_xor_sync(0xffffffffu, dcw[j], m);
+        }
+        if (valid && nl == 0) {
+            const long long prow = static_cast<long long>(b) * p.dim + dd;
+            *reinterpret_cast<float4*>(p.dcw_part + prow * 4) = make_float4(dcw[0], dcw[1], dcw[2], dcw[3]);
+            p.dcb_part[prow] = dcb;
+            if (p.dconv_in) {
+                const float dxs[3] = {cw[0] * q0, fmaf(cw[0], q1, cw[1] * q0), fmaf(cw[0], q2, fmaf(cw[1], q1, cw[2] * q0))};
+#pragma unroll
+                for (int i = 0; i < 3; ++i) {   // input index s = i - 3
+                    const int j = i - (4 - K);  // its place in the carried-in state
+                    if (j >= 0) {
+                        float v = dxs[i];
+                        if (p.dconv_out && i - 3 >= L - (K - 1)) v += p.dconv_out[crow + i - 3 - (L - (K - 1))];
+                        p.dconv_in[crow + j] = v;
+                    }
+                }
+            }
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------------------
@@ -423,6 +581,9 @@ struct BwdFinalParams {
     const float* dbc_part;
     const float *dA_part, *dD_part, *dbias_part;
     float *dB, *dC, *dA, *dD, *dbias;
+    const float *dcw_part, *dcb_part;  // conv prologue (conv_k > 0)
+    float *dconv_w, *dconv_b;
+    int conv_k;
     int batch, dim, ncta;
     long long L;
 };
@@ -467,6 +628,16 @@ __global__ void __launch_bounds__(256) scan_bwd_reduce_params_kernel(const BwdFi
         }
         if (p.dD) p.dD[i] = sd;
         if (p.dbias) p.dbias[i] = sb;
+        if (p.conv_k > 0) {
+            float w[4] = {0.f, 0.f, 0.f, 0.f}, cb = 0.f;
+            for (int b = 0; b < p.batch; ++b) {
+                const long long r = static_cast<long long>(b) * p.dim + i;
+                for (int k = 0; k < 4; ++k) w[k] += p.dcw_part[r * 4 + k];
+                cb += p.dcb_part[r];
+            }
+            for (int k = 0; k < p.conv_k; ++k) p.dconv_w[i * p.conv_k + k] = w[4 - p.conv_k + k];
+            if (p.dconv_b) p.dconv_b[i] = cb;
+        }
     }
 }
 

@@ -67,6 +67,25 @@ __device__ __forceinline__ float2 zoh_beta2(float2 y, float2 a, float2 wB, float
     return make_float2(fabsf(y.x) < kZohSmall ? small.x : big.x, fabsf(y.y) < kZohSmall ? small.y : big.y);
 }
 
+// Derivative of the zero-order-hold weight per unit input, phi(Delta, A) = expm1(Delta A) / A,
+// with respect to A, for a pair of chains (the backward of the ZOH scan):
+//   dphi/dA = (Delta a - phi) / A                             for |y| >= kZohSmall,
+//           = Delta^2 (1/2 + x/3 + x^2/8 + x^3/30)              for |y| <  kZohSmall (x = y ln 2),
+// the second the Taylor series of the first (the k-th coefficient of (x e^x - e^x + 1) / x^2 is
+// 1 / (k! (k + 2)); the first term left out, x^4 / 144, is 2.1e-7 of the sum at |x| = 1/16), which avoids the
+// cancellation of Delta a - phi for small Delta A.  phi is the weight (zoh_beta2 with wB = Delta,
+// uB_over_A = 1 / A); the derivative with respect to Delta is a itself.
+constexpr float kZohQ1 = kLn2 / 3.f, kZohQ2 = kLn2 * kLn2 / 8.f, kZohQ3 = kLn2 * kLn2 * kLn2 / 30.f;
+
+__device__ __forceinline__ float2 zoh_dphi_dA2(float2 y, float2 a, float2 dt, float2 phi, float2 invA) {
+    const float2 q = __ffma2_rn(__ffma2_rn(__ffma2_rn(make_float2(kZohQ3, kZohQ3), y, make_float2(kZohQ2, kZohQ2)), y,
+                                           make_float2(kZohQ1, kZohQ1)),
+                                y, make_float2(0.5f, 0.5f));
+    const float2 small = __fmul2_rn(__fmul2_rn(dt, dt), q);
+    const float2 big = __fmul2_rn(__ffma2_rn(dt, a, make_float2(-phi.x, -phi.y)), invA);
+    return make_float2(fabsf(y.x) < kZohSmall ? small.x : big.x, fabsf(y.y) < kZohSmall ? small.y : big.y);
+}
+
 // silu(z) = z / (1 + e^-z), the SiLU gate of the Mamba block ([Hist] Mamba Block 数据流).
 // For z -> -inf the denominator overflows to +inf and the result is 0.
 __device__ __forceinline__ float silu_f32(float z) {

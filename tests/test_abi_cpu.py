@@ -177,6 +177,25 @@ def test_backward_argument_validation(lib):
     assert f(1, 1, 8, 1) == 0
 
 
+def test_backward_ex_argument_validation(lib):
+    """ssm_selective_scan_bwd_ex rejects bad options before touching the device."""
+    w = P(4096)
+    def call(disc=binding.SSM_DISC_SIMPLIFIED, width=None, weight=w, dweight=P(4096), batch=2):
+        spec = None if width is None else binding.ConvSpec(weight, None, width, None, None, None)
+        opts = binding.BwdOptions(disc, ctypes.pointer(spec) if spec is not None else None, dweight, None, None, None)
+        return lib.ssm_selective_scan_bwd_ex(P(4096), P(4096), P(4096), P(4096), P(4096), None, None, None, 1, None,
+                                             P(4096), None, P(4096), P(4096), P(4096), P(4096), P(4096), None, None,
+                                             None, None, batch, 3, 16, 8, binding.SSM_BF16, P(4096), 1 << 30,
+                                             ctypes.byref(opts), None)
+    assert call(disc=7) == binding.SSM_ERR_INVALID_ARG
+    assert call(width=0) == binding.SSM_ERR_INVALID_ARG
+    assert call(width=5) == binding.SSM_ERR_INVALID_ARG
+    assert call(width=4, weight=None) == binding.SSM_ERR_INVALID_ARG
+    assert call(width=4, dweight=None) == binding.SSM_ERR_INVALID_ARG
+    assert call(width=4, batch=0) == binding.SSM_OK
+    assert call(disc=binding.SSM_DISC_ZOH, batch=0) == binding.SSM_OK
+
+
 @pytest.mark.skipif(__import__("torch").cuda.is_available(),
                     reason="fake pointers: an accepted call would launch kernels on a real device")
 def test_noalloc_scratch_limit_follows_its_formula(lib):

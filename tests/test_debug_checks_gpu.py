@@ -111,3 +111,20 @@ def test_debug_status_reports_where(cuda_device, debug_lib):
     torch.cuda.synchronize()
     header = ws[:32].view(torch.int32).cpu().tolist()   # epoch, ticket, done, status, where[4]
     assert header[3] == 0 and header[4:8] == [0, 0, 0, 0], header
+
+
+@pytest.mark.parametrize("zoh", [False, True])
+def test_debug_backward_conv_clean(cuda_device, debug_lib, zoh):
+    """The conv + ZOH backward through the range-checked library: clean status word."""
+    b, d, L = 2, 40, 130
+    cpu = workloads.scan_inputs(b, d, L, io="bf16", seed=67)
+    conv = to_dev(workloads.conv_inputs(b, d, 4, seed=68, with_state=True), "cuda")
+    g = to_dev(cpu, "cuda")
+    dy = torch.randn(b, d, L, generator=torch.Generator().manual_seed(69)).to(torch.bfloat16).cuda()
+    ws = torch.zeros(max(ssm.ssm_selective_scan_bwd_workspace_size(b, d, 16, L), 256), dtype=torch.uint8,
+                     device="cuda")
+    out = ssm.selective_scan_bwd(**g, softplus=True, dy=dy, workspace=ws, zoh=zoh, conv_weight=conv["conv_weight"],
+                                 conv_bias=conv["conv_bias"], conv_state_in=conv["conv_state_in"],
+                                 dconv_state_out=torch.ones(b, d, 3, device="cuda"))
+    assert ssm.ssm_read_status(ws) == binding.SSM_OK
+    assert torch.isfinite(out["dx"].float()).all() and torch.isfinite(out["dconv_weight"]).all()
