@@ -451,6 +451,48 @@ def measure_conv(ssm, stream, pk, steps=10):
             "unit": UNIT, "ms_per_step": ms}
 
 
+WIDE_SHAPE = (4, 2048, 2048)   # batch, d_inner, L of the wider-state measurements (bf16 I/O)
+
+
+def measure_wide(ssm, stream, pk, steps=5, only=None):
+    """Forward scan with d_state 32, 64, 128 and 256 (batch 4, d_inner 2048, L 2048, bf16 I/O;
+    inputs above L2 except B/C), timed per call with CUDA events on the launching stream.  With
+    N exponentials per element the bound is the special-function unit: roofline Gelem/s =
+    ex2 peak / N."""
+    bsz, dim, L = WIDE_SHAPE
+    sm_count = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    ex2_peak = sm_count * MUFU_EX2_PER_CLK_PER_SM * pk["sm_max_mhz"] * 1e6 / 1e9
+    out = {"workload": f"b{bsz}_d{dim}_L{L}_bf16", "unit": UNIT, "ex2_peak_gex2s": ex2_peak}
+    for n in (only,) if only else (32, 64, 128, 256):
+        inp = workloads.scan_inputs(bsz, dim, L, dstate=n, io="bf16", seed=900 + n)
+        g = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+        y = torch.empty_like(g["u"])
+        last = torch.empty(bsz, dim, n, dtype=torch.float32, device="cuda")
+        ws = ssm.new_workspace(bsz, dim, n, L)
+
+        def call():
+            ssm.ssm_selective_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"],
+                                       True, y, last, ws, stream=stream)
+
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                call()
+            torch.cuda.synchronize()
+            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ev0.record(stream)
+            for _ in range(steps):
+                call()
+            ev1.record(stream)
+        torch.cuda.synchronize()
+        ms = ev0.elapsed_time(ev1) / steps
+        assert ssm.ssm_read_status(ws) == 0
+        rate = bsz * dim * L / (ms / 1e3) / 1e9
+        out[f"N{n}"] = {"ms_per_step": ms, "value": rate, "roofline_value": ex2_peak / n,
+                        "ex2_frac": rate * n / ex2_peak}
+        del g, y, last, ws
+    return out
+
+
 def measure_backward(ssm, stream, pk, steps=5):
     """Backward of the headline workload (gradients of every input for a seeded N(0, 1) dy),
     timed with CUDA events on the launching stream; inputs larger than L2."""
@@ -622,7 +664,8 @@ def run_gpu(args, world, rank, local):
     if world == 1 and not args.skip_extra:
         line["also"] = {"long": measure_long(ssm, stream, pk), "decode": measure_decode(ssm, stream, pk),
                         "backward": measure_backward(ssm, stream, pk), "zoh": measure_zoh(ssm, stream, pk),
-                        "conv": measure_conv(ssm, stream, pk), "unaligned": measure_unaligned(ssm, stream, pk)}
+                        "conv": measure_conv(ssm, stream, pk), "unaligned": measure_unaligned(ssm, stream, pk),
+                        "wide": measure_wide(ssm, stream, pk)}
     if rank == 0 and world == 1 and not args.skip_cpu:
         rate, secs, desc, cores = cpu_oracle_rate(w, args.cpu_budget)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
@@ -640,6 +683,8 @@ def run_profile_workload(args):
         out = measure_long(ssm, stream, pk, steps=args.steps)
     elif args.workload == "backward":
         out = measure_backward(ssm, stream, pk, steps=args.steps)
+    elif args.workload == "wide":
+        out = measure_wide(ssm, stream, pk, steps=args.steps, only=args.dstate)
     else:
         w = workloads.WORKLOADS[4]
         out = measure_decode(ssm, stream, pk, steps=args.steps)
@@ -656,8 +701,10 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-extra", action="store_true")
-    ap.add_argument("--workload", default="headline", choices=["headline", "long", "decode", "backward"],
-                    help="profiling runs: 'long' / 'decode' / 'backward' run only that workload a few times")
+    ap.add_argument("--workload", default="headline", choices=["headline", "long", "decode", "backward", "wide"],
+                    help="profiling runs: 'long' / 'decode' / 'backward' / 'wide' run only that workload a few times")
+    ap.add_argument("--dstate", type=int, default=None, choices=[32, 64, 128, 256],
+                    help="with --workload wide: that d_state only")
     args = ap.parse_args()
     world, rank, local = dist_setup(args.gpus) if args.impl == "native" else (
         int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)

@@ -8,15 +8,19 @@
 //
 // The step is the one of the d_state = 16 kernels (simplified or zero-order-hold weight,
 // [Card] 离散化变换 / [Eng] §2.2).  With N exponentials per element these shapes are bound by
-// the special-function unit (N/16 times the work of N = 16 per element).  G = N/4 lanes per
-// channel (N/8 for N = 256), each lane holding 4 (8) chains of the channel in registers for
-// the whole sequence in f32x2 pairs, 32/G channels per warp, 8 warps per block, all on one
-// batch row.  The block stages the packed fp32 B/C rows (2N floats per step) of 64 (32) steps
-// at a time through a double-buffered cp.async ring in shared memory.  Steps go in batches of
-// G: lane nl of a channel loads (one batch ahead) and evaluates the step size of step nl, the
-// lanes walk the G steps with the step size and input broadcast by shuffles, and the G lanes'
-// partial sums of C.h are reduce-scattered so that lane nl finishes (D skip, gate, rounding,
-// store) step nl.
+// the special-function unit (N/16 times the work of N = 16 per element) -- and, were every
+// lane to load its own B/C values, equally by the shared-memory data path: a lane's chains need
+// 2 floats of B/C per exponential, one 4-byte wavefront slot per float, so N/16 wavefronts per
+// element against the unit's N/16 clocks.  Each lane therefore holds the same NC chains of TWO
+// channels (CPL = 2; N = 32 keeps one), so that one load of B/C feeds both: G = N/NC lanes per
+// channel group (WideCfg), the chains in f32x2 pairs in registers for the whole sequence, all
+// warps of a block on one batch row.  The block stages the packed fp32 B/C rows (2N floats
+// per step) of 16 to 64 steps at a time through a double-buffered cp.async ring in shared
+// memory.  Steps go in batches of 8: lane nl loads (one batch ahead) and
+// evaluates the step size of step nl mod 8 of its channels (the G/8 copies redundantly), the
+// lanes walk the 8 steps with step size and input broadcast by shuffles, and the partial sums
+// of C.h are reduce-scattered over 8 lanes and added over the G/8 copies, so that each (step,
+// channel) is finished (D skip, gate, rounding, store) by one lane.
 #pragma once
 
 #include "common.cuh"
@@ -37,61 +41,69 @@ struct WideParams {
 
 template <int N>
 struct WideCfg {
-    static constexpr int kNC = N <= 128 ? 4 : 8;  // chains per lane
-    static constexpr int kG = N / kNC;             // lanes per channel: 8, 16, 32, 32
-    static constexpr int kCPW = 32 / kG;           // channels per warp: 4, 2, 1, 1
-    static constexpr int kT = kG;                  // steps per batch (one step per lane of a channel)
-    // warps per block (one batch row per block); N = 256 stages 128 KB per block, so its
-    // blocks are twice as large to keep 16 warps per SM
-    static constexpr int kWarps = N == 256 ? 16 : 8;
+    // chains per lane and channel, channels per lane (one load of B/C feeds them all), warps
+    // per block, steps per staged stage of B/C rows: the best of the configurations measured
+    // on B200 (batch 4, d_inner 2048, L 2048, bf16) -- N = 32 keeps one channel per lane
+    // (its 8192 channels would leave too few warps), N = 256 stages 16 steps so that two
+    // blocks fit.
+    static constexpr int kNC = N == 32 ? 4 : N == 64 ? 4 : 8;
+    static constexpr int kCPL = N == 32 ? 1 : 2;
+    static constexpr int kWarps = N == 32 ? 4 : 8;
+    static constexpr int kST = N == 32 ? 64 : N == 64 ? 64 : N == 128 ? 32 : 16;
+    static constexpr int kG = N / kNC;             // lanes per channel group: 8, 16, 16, 32
+    static constexpr int kGPW = 32 / kG;           // lane groups per warp
+    static constexpr int kCPW = kGPW * kCPL;       // channels per warp: 4, 4, 4, 2
+    static constexpr int kT = 8;                   // steps per batch
     static constexpr int kCPB = kWarps * kCPW;     // channels per block
-    static constexpr int kST = N <= 64 ? 64 : 32;  // steps per staged stage of B/C rows
     static constexpr int kStageFloats = kST * 2 * N;
     static constexpr int kSmem = 2 * kStageFloats * 4;  // double-buffered stages
 };
 
-// Blocks per SM in the launch bound: measured on B200 (batch 4, d_inner 2048, L 2048), 3 blocks
-// (80 registers) take N = 128 from 1.081 to 0.948 ms but spill at N = 32, 64 (0.31 -> 0.33 ms,
-// 0.535 -> 0.547 ms); N = 256 holds 128 KB of B/C stages (one block).
+// Blocks per SM in the launch bound (128 registers per thread at 16 warps per SM).
 template <int N>
-constexpr int wide_min_blocks() { return N == 256 ? 1 : N == 128 ? 3 : 2; }
+constexpr int wide_min_blocks() { return N == 32 ? 4 : 2; }
 
-template <typename IO, int N>
+template <typename IO, int N, bool ZOH>
 __global__ void __launch_bounds__(WideCfg<N>::kWarps * 32, wide_min_blocks<N>()) scan_fwd_wide_kernel(const WideParams p) {
     using Cfg = WideCfg<N>;
-    constexpr int NC = Cfg::kNC, G = Cfg::kG, CPW = Cfg::kCPW, T = Cfg::kT, ST = Cfg::kST;
+    constexpr int NC = Cfg::kNC, CPL = Cfg::kCPL, G = Cfg::kG, T = Cfg::kT, ST = Cfg::kST;
     static_assert(N == 32 || N == 64 || N == 128 || N == 256, "N in {32, 64, 128, 256}");
-    static_assert(ST % T == 0, "whole batches per stage");
+    static_assert(ST % T == 0 && G % T == 0 && NC % 4 == 0, "whole batches per stage, 16-byte B/C loads");
     extern __shared__ float4 wide_smem[];
     float* ring = reinterpret_cast<float*>(wide_smem);  // [2][ST][2N]
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int cg = lane / G, nl = lane % G, gbase = lane & ~(G - 1);
+    const int gi = lane / G, nl = lane % G, gbase = lane & ~(G - 1);
+    const int own = nl & (T - 1);  // the lane's step of each batch (all G / T copies hold it)
     const int b = blockIdx.y;
-    const int d = blockIdx.x * Cfg::kCPB + warp * CPW + cg;
-    const bool valid = d < p.dim;
-    const int dd = valid ? d : 0;
     const long long L = p.L;
-    const long long ch = static_cast<long long>(b) * p.dim + dd;
-    const IO* u = static_cast<const IO*>(p.u) + ch * L;
-    const IO* dl = static_cast<const IO*>(p.delta) + ch * L;
-    const IO* z = p.z ? static_cast<const IO*>(p.z) + ch * L : nullptr;
-    IO* y = static_cast<IO*>(p.y) + ch * L;
     const float* bcrow = p.bc + static_cast<long long>(b) * L * (2 * N);
 
-    float2 A2[NC / 2], invA[NC / 2], h[NC / 2];
+    int d[CPL];
+    bool valid[CPL];
+    long long ch[CPL];
+    float2 A2[CPL][NC / 2], invA[CPL][ZOH ? NC / 2 : 1], h[CPL][NC / 2];
+    float Dd[CPL], bias[CPL];
 #pragma unroll
-    for (int j = 0; j < NC / 2; ++j) {
-        const float a0 = p.A[static_cast<long long>(dd) * N + nl * NC + 2 * j];
-        const float a1 = p.A[static_cast<long long>(dd) * N + nl * NC + 2 * j + 1];
-        A2[j] = make_float2(a0 * kLog2e, a1 * kLog2e);
-        invA[j] = make_float2(1.f / a0, 1.f / a1);
-        h[j] = (p.h0 && valid) ? *reinterpret_cast<const float2*>(p.h0 + ch * N + nl * NC + 2 * j)
-                               : make_float2(0.f, 0.f);
+    for (int c = 0; c < CPL; ++c) {
+        d[c] = blockIdx.x * Cfg::kCPB + warp * Cfg::kCPW + gi * CPL + c;
+        valid[c] = d[c] < p.dim;
+        const int dd = valid[c] ? d[c] : 0;
+        ch[c] = static_cast<long long>(b) * p.dim + dd;
+#pragma unroll
+        for (int j = 0; j < NC / 2; ++j) {
+            const float a0 = p.A[static_cast<long long>(dd) * N + nl * NC + 2 * j];
+            const float a1 = p.A[static_cast<long long>(dd) * N + nl * NC + 2 * j + 1];
+            A2[c][j] = make_float2(a0 * kLog2e, a1 * kLog2e);
+            if constexpr (ZOH) invA[c][j] = make_float2(1.f / a0, 1.f / a1);
+            h[c][j] = (p.h0 && valid[c]) ? *reinterpret_cast<const float2*>(p.h0 + ch[c] * N + nl * NC + 2 * j)
+                                         : make_float2(0.f, 0.f);
+        }
+        Dd[c] = (valid[c] && p.D) ? p.D[dd] : 0.f;
+        bias[c] = (valid[c] && p.bias) ? p.bias[dd] : 0.f;
     }
-    const float Dd = (valid && p.D) ? p.D[dd] : 0.f;
-    const float bias = (valid && p.bias) ? p.bias[dd] : 0.f;
-    const bool softplus = p.softplus != 0, zoh = p.zoh != 0;
+    const bool softplus = p.softplus != 0;
+    const IO* zbase = static_cast<const IO*>(p.z);
 
     // B/C rows of stage k into ring slot k & 1 (zero past L), one cp.async group per stage.
     const long long nstages = (L + ST - 1) / ST;
@@ -107,17 +119,20 @@ __global__ void __launch_bounds__(WideCfg<N>::kWarps * 32, wide_min_blocks<N>())
         }
         cp_async_commit();
     };
-    // Inputs of the lane's own step of a batch (0 past L), loaded one batch ahead.
-    auto load_own = [&](long long t, float& ul, float& xl, float& zl) {
-        const bool in = valid && t < L;
-        ul = in ? IoTraits<IO>::to_f32(u[t]) : 0.f;
-        xl = in ? IoTraits<IO>::to_f32(dl[t]) : 0.f;
-        zl = (in && z) ? IoTraits<IO>::to_f32(z[t]) : 0.f;
+    // Inputs of the lane's own step of a batch for its channels (0 past L), loaded one batch ahead.
+    auto load_own = [&](long long t, float (&ul)[CPL], float (&xl)[CPL], float (&zl)[CPL]) {
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+            const bool in = valid[c] && t < L;
+            ul[c] = in ? IoTraits<IO>::to_f32(static_cast<const IO*>(p.u)[ch[c] * L + t]) : 0.f;
+            xl[c] = in ? IoTraits<IO>::to_f32(static_cast<const IO*>(p.delta)[ch[c] * L + t]) : 0.f;
+            zl[c] = (in && zbase) ? IoTraits<IO>::to_f32(zbase[ch[c] * L + t]) : 0.f;
+        }
     };
 
     issue(0);
-    float un, xn, zn;
-    load_own(nl, un, xn, zn);
+    float un[CPL], xn[CPL], zn[CPL];
+    load_own(own, un, xn, zn);
     for (long long k = 0; k < nstages; ++k) {
         issue(k + 1);
         cp_async_wait<1>();
@@ -125,16 +140,18 @@ __global__ void __launch_bounds__(WideCfg<N>::kWarps * 32, wide_min_blocks<N>())
         const float* stage = ring + (k & 1) * Cfg::kStageFloats + nl * NC;
 #pragma unroll 1
         for (int bt = 0; bt < ST; bt += T) {
-            const long long t0 = k * ST + bt;
-            const long long t = t0 + nl;
-            const float ul = un, zl = zn;
-            const float dtl = (valid && t < L) ? step_size(xn, bias, softplus) : 0.f;  // 0 past L
+            const long long t = k * ST + bt + own;
+            float ul[CPL], zl[CPL], dtl[CPL];
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) {
+                ul[c] = un[c];
+                zl[c] = zn[c];
+                dtl[c] = (valid[c] && t < L) ? step_size(xn[c], bias[c], softplus) : 0.f;  // 0 past L
+            }
             load_own(t + T, un, xn, zn);  // next batch (the next stage's first for the last batch)
-            float yp[T];
+            float yp[CPL][T];
 #pragma unroll
             for (int i = 0; i < T; ++i) {
-                const float dti = __shfl_sync(0xffffffffu, dtl, gbase | i);
-                const float ui = __shfl_sync(0xffffffffu, ul, gbase | i);
                 const float* row = stage + (bt + i) * 2 * N;
                 float2 Bv[NC / 2], Cv[NC / 2];
 #pragma unroll
@@ -146,44 +163,84 @@ __global__ void __launch_bounds__(WideCfg<N>::kWarps * 32, wide_min_blocks<N>())
                     Cv[j] = make_float2(cq.x, cq.y);
                     Cv[j + 1] = make_float2(cq.z, cq.w);
                 }
-                const float2 dd2 = make_float2(dti, dti), ww = make_float2(dti * ui, dti * ui);
-                float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int j = 0; j < NC / 2; ++j) {
-                    const float2 arg = __fmul2_rn(dd2, A2[j]);
-                    const float2 a = make_float2(ex2_mufu(arg.x), ex2_mufu(arg.y));
-                    float2 beta = __fmul2_rn(ww, Bv[j]);
-                    if (zoh)
-                        beta = zoh_beta2(arg, a, beta, __fmul2_rn(__fmul2_rn(make_float2(ui, ui), Bv[j]), invA[j]));
-                    h[j] = __ffma2_rn(a, h[j], beta);
-                    acc = __ffma2_rn(Cv[j], h[j], acc);
+                for (int c = 0; c < CPL; ++c) {
+                    const float dti = __shfl_sync(0xffffffffu, dtl[c], gbase | i);
+                    const float ui = __shfl_sync(0xffffffffu, ul[c], gbase | i);
+                    const float2 dd2 = make_float2(dti, dti), ww = make_float2(dti * ui, dti * ui);
+                    float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int j = 0; j < NC / 2; ++j) {
+                        const float2 arg = __fmul2_rn(dd2, A2[c][j]);
+                        const float2 a = make_float2(ex2_mufu(arg.x), ex2_mufu(arg.y));
+                        float2 beta = __fmul2_rn(ww, Bv[j]);
+                        if constexpr (ZOH)
+                            beta = zoh_beta2(arg, a, beta, __fmul2_rn(__fmul2_rn(make_float2(ui, ui), Bv[j]), invA[c][j]));
+                        h[c][j] = __ffma2_rn(a, h[c][j], beta);
+                        acc = __ffma2_rn(Cv[j], h[c][j], acc);
+                    }
+                    yp[c][i] = acc.x + acc.y;
                 }
-                yp[i] = acc.x + acc.y;
             }
-            // Reduce-scatter the T partial sums over the G lanes of the channel (upper lane
-            // bit first): lane nl ends with the full sum of step t0 + nl in yp[0].
+            // Reduce-scatter the T partial sums of each channel over lane bits 2, 1, 0 (upper
+            // bit first): lane nl ends with its 8-lane subgroup's sum of step `own` in yp[c][0];
+            // then the G / 8 subgroups are added by xor shuffles over the higher lane bits.
 #pragma unroll
-            for (int m = G / 2; m >= 1; m >>= 1) {
+            for (int m = T / 2; m >= 1; m >>= 1) {
                 const bool upper = (nl & m) != 0;
 #pragma unroll
-                for (int i = 0; i < m; ++i) {
-                    const float send = upper ? yp[i] : yp[i + m];
-                    const float keep = upper ? yp[i + m] : yp[i];
-                    yp[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-                }
+                for (int c = 0; c < CPL; ++c)
+#pragma unroll
+                    for (int i = 0; i < m; ++i) {
+                        const float send = upper ? yp[c][i] : yp[c][i + m];
+                        const float keep = upper ? yp[c][i + m] : yp[c][i];
+                        yp[c][i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+                    }
             }
-            if (valid && t < L) {
-                float v = fmaf(Dd, ul, yp[0]);
-                if (z) v *= silu_f32(zl);
-                y[t] = IoTraits<IO>::from_f32(v);
+#pragma unroll
+            for (int m = T; m < G; m <<= 1)
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) yp[c][0] += __shfl_xor_sync(0xffffffffu, yp[c][0], m);
+            // Epilogue ([Eng] §2.2 D skip; [Hist] SiLU gate): copy q = nl / 8 of step `own`
+            // finishes channel q (G >= 16; copies past the channels idle), or the only copy
+            // finishes both (G = 8).  (The channel is picked by selects, not by an index.)
+            auto finish = [&](float yv, float uv, float zv, float Dv, long long cv) {
+                float v = fmaf(Dv, uv, yv);
+                if (zbase) v *= silu_f32(zv);
+                static_cast<IO*>(p.y)[cv * L + t] = IoTraits<IO>::from_f32(v);
+            };
+            if constexpr (G / T >= CPL) {
+                const int q = nl / T;
+                float yv = 0.f, uv = 0.f, zv = 0.f, Dv = 0.f;
+                long long cv = 0;
+                bool ok = false;
+#pragma unroll
+                for (int c = 0; c < CPL; ++c)
+                    if (c == q) {
+                        yv = yp[c][0];
+                        uv = ul[c];
+                        zv = zl[c];
+                        Dv = Dd[c];
+                        cv = ch[c];
+                        ok = valid[c];
+                    }
+                if (ok && t < L) finish(yv, uv, zv, Dv, cv);
+            } else {
+#pragma unroll
+                for (int c = 0; c < CPL; ++c)
+                    if (valid[c] && t < L) finish(yp[c][0], ul[c], zl[c], Dd[c], ch[c]);
             }
         }
         __syncthreads();  // every warp is done with slot k & 1 before it is refilled
     }
     cp_async_wait<0>();
-    if (p.last_state && valid)
+    if (p.last_state)
 #pragma unroll
-        for (int j = 0; j < NC / 2; ++j) *reinterpret_cast<float2*>(p.last_state + ch * N + nl * NC + 2 * j) = h[j];
+        for (int c = 0; c < CPL; ++c)
+            if (valid[c])
+#pragma unroll
+                for (int j = 0; j < NC / 2; ++j)
+                    *reinterpret_cast<float2*>(p.last_state + ch[c] * N + nl * NC + 2 * j) = h[c][j];
 }
 
 // B, C (batch, N, L) -> fp32 rows [batch][L][2N] (B then C): 32 x 32 tiles through shared

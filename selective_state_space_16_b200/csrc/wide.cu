@@ -30,7 +30,7 @@ ssm_status_t launch_wide_n(const FwdArgs& a) {
     p.softplus = a.softplus;
     p.zoh = a.zoh;
     using Cfg = ssm::WideCfg<N>;
-    auto kern = ssm::scan_fwd_wide_kernel<IO, N>;
+    auto kern = a.zoh ? ssm::scan_fwd_wide_kernel<IO, N, true> : ssm::scan_fwd_wide_kernel<IO, N, false>;
     if (!ensure_smem_attr(reinterpret_cast<const void*>(kern), Cfg::kSmem)) return SSM_ERR_LAUNCH;
     const dim3 grid(static_cast<unsigned>((a.dim + Cfg::kCPB - 1) / Cfg::kCPB), static_cast<unsigned>(a.batch));
     kern<<<grid, Cfg::kWarps * 32, Cfg::kSmem, a.stream>>>(p);

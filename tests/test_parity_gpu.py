@@ -112,6 +112,16 @@ def test_chunked_headline_full_size(cuda_device):
     check_forward(workloads.workload_inputs(w), algo="chunked", what=w.name + " chunked")
 
 
+def test_chunked_long_sequence_sampled(cuda_device):
+    # the long workload (L 32768, decay persisting across chunks) through the look-back
+    # kernel, every output of 384 sampled channels against the oracle
+    w = workloads.WORKLOADS[3]
+    inp = workloads.workload_inputs(w)
+    rng = np.random.default_rng(33)
+    channels = np.sort(rng.choice(w.batch * w.dim, size=384, replace=False))
+    check_forward(inp, channels=channels, algo="chunked", what=w.name + " chunked (sampled channels)")
+
+
 @pytest.mark.parametrize("io", ["f32", "bf16"])
 def test_chunked_many_chunks_few_channels(cuda_device, io):
     # one tile, 70+ chunks: the look-back chain is long and the ragged last chunk is partial
