@@ -189,6 +189,7 @@ KERNEL_SOURCES = {
                                 "scan_fwd_chunked.cuh"],
     "state_update_kernel": ["common.cuh", "scan_math.cuh", "poly_coeffs.cuh", "aux_kernels.cuh"],
     "scan_bwd_kernel": ["common.cuh", "scan_math.cuh", "poly_coeffs.cuh", "scan_fwd_seq.cuh", "scan_bwd.cuh"],
+    "scan_fwd_wide_kernel": ["common.cuh", "scan_math.cuh", "poly_coeffs.cuh", "scan_fwd_wide.cuh"],
 }
 
 
@@ -488,7 +489,8 @@ def measure_wide(ssm, stream, pk, steps=5, only=None):
         assert ssm.ssm_read_status(ws) == 0
         rate = bsz * dim * L / (ms / 1e3) / 1e9
         out[f"N{n}"] = {"ms_per_step": ms, "value": rate, "roofline_value": ex2_peak / n,
-                        "ex2_frac": rate * n / ex2_peak}
+                        "ex2_frac": rate * n / ex2_peak,
+                        "traffic": traffic_record("scan_fwd_wide_kernel", f"N{n}_b{bsz}_d{dim}_L{L}")}
         del g, y, last, ws
     return out
 
@@ -554,11 +556,14 @@ def _plan_oracle_sample(inp, w, budget_s):
     """Pick a sample of about `budget_s` seconds of oracle work: the whole workload repeated
     `reps` times, or (when one pass is longer) its first `channels` rows once."""
     import oracle
-    probe = _oracle_sample(inp, w, 32)
+    n_probe = min(w.batch * w.dim, 1024)  # enough rows to keep every oracle thread busy
+    probe = _oracle_sample(inp, w, n_probe)
+    for c in probe:  # untimed first call: thread-pool start-up and first-touch page faults
+        oracle.selective_scan(**c)
     t0 = time.perf_counter()
     for c in probe:
         oracle.selective_scan(**c)
-    per_row = (time.perf_counter() - t0) / 32
+    per_row = (time.perf_counter() - t0) / n_probe
     rows = w.batch * w.dim
     if per_row * rows <= budget_s:
         return rows, max(1, int(budget_s / (per_row * rows)))
