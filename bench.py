@@ -258,7 +258,7 @@ def forward_buffers(w, dev):
     return inp, g
 
 
-def e2e_forward(ssm, w, inp, y_ref, steps, stream, nstreams=4, chunks_per_row=2):
+def e2e_forward(ssm, w, inp, y_ref, steps, stream, nstreams=4, chunks_per_row=1):
     """Same metric through the public C-ABI call with HOST (pinned) buffers: every step
     copies all inputs host->device, runs the scan and copies y and the final state back.
     A step is cut into batch * chunks_per_row independent channel chunks; chunk c always
