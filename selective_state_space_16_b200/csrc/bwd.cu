@@ -100,7 +100,7 @@ ssm_status_t launch_backward(const BwdArgs& a) {
     f.dim = a.dim;
     f.ncta = wl.ncta;
     f.L = a.L;
-    ssm::scan_bwd_reduce_bc_kernel<<<dim3(static_cast<unsigned>((a.L + 31) / 32), static_cast<unsigned>(a.batch)), 256,
+    ssm::scan_bwd_reduce_bc_kernel<<<dim3(static_cast<unsigned>((a.L + 7) / 8), static_cast<unsigned>(a.batch)), 256,
                                      0, a.stream>>>(f);
     const long long n = static_cast<long long>(a.dim) * 16;
     ssm::scan_bwd_reduce_params_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, a.stream>>>(f);

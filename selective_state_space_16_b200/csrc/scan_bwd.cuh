@@ -574,7 +574,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, CONV ? 4 : 5) scan_bwd_kernel(
 
 // ---------------------------------------------------------------------------------------
 // Second pass: the sums over the CTAs of a batch row (dB, dC, transposed to (b, N, L);
-// grid (ceil(L / 32), batch)) and over batch rows (dA, dD, ddelta_bias; one thread per
+// grid (ceil(L / 8), batch)) and over batch rows (dA, dD, ddelta_bias; one thread per
 // output), each in a fixed order.
 // ---------------------------------------------------------------------------------------
 struct BwdFinalParams {
@@ -588,29 +588,21 @@ struct BwdFinalParams {
     long long L;
 };
 
+// One output per thread: thread (i, c) of block (x, b) sums the CTAs' rows of step 8x + i,
+// column c, in CTA order (independent loads, unrolled, so many are in flight), and writes
+// dB[b][c][t] (c < 16) or dC[b][c - 16][t].  grid (ceil(L / 8), batch), 256 threads.
 __global__ void __launch_bounds__(256) scan_bwd_reduce_bc_kernel(const BwdFinalParams p) {
-    __shared__ float tile[32][33];
     const int b = blockIdx.y;
-    const long long t0 = static_cast<long long>(blockIdx.x) * 32;
-    // threads: (t local, column) with column fastest for coalesced partial reads
-    for (int k = threadIdx.x; k < 32 * 32; k += blockDim.x) {
-        const int tl = k >> 5, c = k & 31;
-        const long long t = t0 + tl;
-        float s = 0.f;
-        if (t < p.L)
-            for (int j = 0; j < p.ncta; ++j) s += p.dbc_part[((static_cast<long long>(b) * p.ncta + j) * p.L + t) * 32 + c];
-        tile[c][tl] = s;
-    }
-    __syncthreads();
-    // write rows of 32 steps: dB[b][n][t0..] (c < 16) and dC[b][n][t0..] (c >= 16)
-    for (int k = threadIdx.x; k < 32 * 32; k += blockDim.x) {
-        const int c = k >> 5, tl = k & 31;
-        const long long t = t0 + tl;
-        if (t < p.L) {
-            float* dst = c < 16 ? p.dB : p.dC;
-            dst[(static_cast<long long>(b) * 16 + (c & 15)) * p.L + t] = tile[c][tl];
-        }
-    }
+    const int i = threadIdx.x >> 5, c = threadIdx.x & 31;
+    const long long t = static_cast<long long>(blockIdx.x) * 8 + i;
+    if (t >= p.L) return;
+    const float* src = p.dbc_part + (static_cast<long long>(b) * p.ncta * p.L + t) * 32 + c;
+    const long long stride = p.L * 32;  // floats between the rows of consecutive CTAs
+    float s = 0.f;
+#pragma unroll 8
+    for (int j = 0; j < p.ncta; ++j) s += src[j * stride];
+    float* dst = c < 16 ? p.dB : p.dC;
+    dst[(static_cast<long long>(b) * 16 + (c & 15)) * p.L + t] = s;
 }
 
 __global__ void __launch_bounds__(256) scan_bwd_reduce_params_kernel(const BwdFinalParams p) {
