@@ -21,6 +21,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import sys
 import threading
@@ -193,12 +194,16 @@ KERNEL_SOURCES = {
 }
 
 
+_COMMENT = re.compile(r"//[^\n]*|/\*.*?\*/", re.S)
+
+
 def kernel_source_hash(kernel: str) -> str:
+    """Hash of the code (comments stripped) of the device sources a kernel family is built from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "selective_state_space_16_b200", "csrc")
     for f in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(f.encode() + fh.read())
+        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+            h.update(f.encode() + _COMMENT.sub("", fh.read()).encode())
     return h.hexdigest()[:16]
 
 

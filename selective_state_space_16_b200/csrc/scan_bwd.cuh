@@ -62,7 +62,7 @@
 namespace ssm {
 
 constexpr int kBwdSeg = 8;       // steps per segment (checkpoint interval)
-constexpr int kBwdWarps = 4;     // warps per CTA (5 CTAs per SM: every CTA resident at once)
+constexpr int kBwdWarps = 4;     // warps per CTA (5 CTAs per SM, 4 with the conv prologue)
 constexpr int kBwdChannels = kBwdWarps * 8;
 constexpr int kBwdRing = 4;      // segments of B/C rows in flight (cp.async ring)
 // dynamic shared memory of scan_bwd_kernel: h stage, dB/dC stage, B/C ring (sized for
