@@ -71,8 +71,10 @@ ssm_status_t launch_forward(const FwdArgs& a, const ssm_fwd_options_t& o) {
         algo = (warps_per_sm < 4.0 && chunks >= 64) ? SSM_ALGO_CHUNKED : SSM_ALGO_SEQUENTIAL;
     }
     if (algo == SSM_ALGO_CHUNKED) return launch_chunked<IO>(a, o);
-    if (a.zoh || a.conv.k > 0) return launch_seq_flagged<IO>(a, o);
-    return launch_seq_plain<IO>(a, o);
+    FwdArgs b = a;
+    b.pdl = true;  // launched right after the B/C pack
+    if (a.zoh || a.conv.k > 0) return launch_seq_flagged<IO>(b, o);
+    return launch_seq_plain<IO>(b, o);
 }
 
 // Fixed scratch of ssm_selective_scan_fwd_noalloc (header + transposed B/C rows).  In

@@ -23,6 +23,7 @@ namespace ssm {
 template <typename IO>
 __global__ void __launch_bounds__(256) pack_bc_kernel(const IO* __restrict__ B, const IO* __restrict__ C,
                                                       float* __restrict__ bc, long long L, WorkspaceHeader* hdr) {
+    pdl_launch_dependents();  // the scan may start its prologue; it waits for these rows before loading them
     __shared__ float tile[32][65];
     const int b = blockIdx.y;
     const long long t0 = static_cast<long long>(blockIdx.x) * 64;

@@ -157,6 +157,13 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
 // Order this thread's earlier memory accesses before its later ones, GPU scope.
 __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
+// Programmatic dependent launch: pdl_launch_dependents lets the next kernel of the stream (if
+// launched with programmatic serialization) start before this one ends; pdl_wait_primary waits
+// until the previous kernel has completed and its writes are visible (a no-op when this kernel
+// was launched normally).
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }

@@ -103,6 +103,8 @@ struct FwdArgs {
     int64_t L_rows = 0;  // row length of u / delta / z when staged into padded rows (0: L)
     int y_vec = 1;       // y rows 16-byte aligned: vector stores of y
     bool pad_ok = true;  // the workspace has room for padded rows (not the no-allocation scratch)
+    bool pdl = false;    // the previous launch is the B/C pack: the scan may start early (it waits
+                         // for the pack before reading the B/C rows, and reads nothing else it writes)
 };
 
 // Backward workspace layout:

@@ -128,10 +128,27 @@ ssm_status_t launch_seq(const FwdArgs& a, const SeqPlan& pl) {
     p.conv_k = a.conv.k;
     p.y_vec = a.y_vec;
     if (a.L >= (1LL << 31) - 1024) return SSM_ERR_UNSUPPORTED;
+    // With a.pdl the kernel may start while the B/C pack before it is still running (programmatic
+    // dependent launch): its prologue and first input copies overlap the pack's tail.
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
+    cfg.blockDim = dim3(static_cast<unsigned>(pl.threads));
+    cfg.dynamicSmemBytes = static_cast<size_t>(pl.smem);
+    cfg.stream = a.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = a.pdl ? 1 : 0;
+    cudaError_t e;
     switch (pl.stages) {
-        case 2: ssm::scan_fwd_seq_kernel<IO, G, CPL, 2, ZOH, CONV><<<pl.grid, pl.threads, pl.smem, a.stream>>>(mu, mdl, mz, mbc, p); break;
-        case 3: ssm::scan_fwd_seq_kernel<IO, G, CPL, 3, ZOH, CONV><<<pl.grid, pl.threads, pl.smem, a.stream>>>(mu, mdl, mz, mbc, p); break;
-        default: ssm::scan_fwd_seq_kernel<IO, G, CPL, 4, ZOH, CONV><<<pl.grid, pl.threads, pl.smem, a.stream>>>(mu, mdl, mz, mbc, p); break;
+        case 2: e = cudaLaunchKernelEx(&cfg, ssm::scan_fwd_seq_kernel<IO, G, CPL, 2, ZOH, CONV>, mu, mdl, mz, mbc, p); break;
+        case 3: e = cudaLaunchKernelEx(&cfg, ssm::scan_fwd_seq_kernel<IO, G, CPL, 3, ZOH, CONV>, mu, mdl, mz, mbc, p); break;
+        default: e = cudaLaunchKernelEx(&cfg, ssm::scan_fwd_seq_kernel<IO, G, CPL, 4, ZOH, CONV>, mu, mdl, mz, mbc, p); break;
+    }
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return SSM_ERR_LAUNCH;
     }
     return launch_status();
 }

@@ -546,6 +546,9 @@ scan_fwd_seq_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_cons
                         if (p.has_z)
                             tma_load_3d(st + (2 * p.max_tiles + j) * Cfg::kTileBytes, &map_z, &full_bar[s], t0, dd, b);
                     }
+                    // The B/C rows come from the kernel launched just before this one (which may
+                    // still be running when this one starts): wait for it before the first copy.
+                    if (k == 0 && r_begin == t_begin) pdl_wait_primary();
                     for (int bb = 0; bb < nb; ++bb)
                         tma_load_3d(st + 3 * p.max_tiles * Cfg::kTileBytes + bb * Cfg::kBC, &map_bc, &full_bar[s], 0,
                                     t0, b_first + bb);
