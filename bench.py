@@ -518,23 +518,43 @@ def measure_backward(ssm, stream, pk, steps=5):
         ssm.ssm_selective_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"], True,
                                    dy, du, ddelta, dA, dB, dC, dD, dz, dbias, ws, stream=stream)
 
-    with torch.cuda.stream(stream):
-        for _ in range(2):
-            call()
+    def timed(fn):
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                fn()
+            torch.cuda.synchronize()
+            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ev0.record(stream)
+            for _ in range(steps):
+                fn()
+            ev1.record(stream)
         torch.cuda.synchronize()
-        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        ev0.record(stream)
-        for _ in range(steps):
-            call()
-        ev1.record(stream)
-    torch.cuda.synchronize()
-    ms = ev0.elapsed_time(ev1) / steps
+        return ev0.elapsed_time(ev1) / steps
+
+    ms = timed(call)
+    # the same with the zero-order hold and the conv prologue (width 4, carried-in state):
+    # u is then the conv input x and du receives dx
+    conv = {k: (v.cuda() if v is not None else None)
+            for k, v in workloads.conv_inputs(w.batch, w.dim, 4, seed=5, with_state=True).items()}
+    dcw, dcb = torch.empty(w.dim, 4, **f32), torch.empty(w.dim, **f32)
+    dcs = torch.empty(w.batch, w.dim, 3, **f32)
+
+    def call_ex():
+        ssm.ssm_selective_scan_bwd_ex(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"],
+                                      True, dy, du, ddelta, dA, dB, dC, dD, dz, dbias, ws, zoh=True,
+                                      conv_weight=conv["conv_weight"], conv_bias=conv["conv_bias"],
+                                      conv_state_in=conv["conv_state_in"], dconv_weight=dcw, dconv_bias=dcb,
+                                      dconv_state_in=dcs, stream=stream)
+
+    ms_ex = timed(call_ex)
     # algorithmic bytes: u, delta, z, dy read and du, ddelta, dz written (2 B each), B/C read,
     # dB/dC written (fp32), A/D/bias and their gradients
     nbytes = w.elements * 14 + w.batch * w.dstate * w.seqlen * (2 * 2 + 2 * 4) + w.dim * (w.dstate + 2) * 8
     gbs = nbytes / (ms / 1e3) / 1e9
     del g
     return {"workload": w.name, "value": w.elements / (ms / 1e3) / 1e9, "unit": UNIT, "ms_per_step": ms,
+            "zoh_conv": {"value": w.elements / (ms_ex / 1e3) / 1e9, "ms_per_step": ms_ex,
+                         "what": "ssm_selective_scan_bwd_ex: zero-order hold + conv1d width 4 (dx, conv gradients)"},
             "gradients": "du, ddelta, dz, dA, dB, dC, dD, ddelta_bias", "launches_per_step": 4,
             "hbm": {"achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
                     "algorithmic_bytes_per_step": nbytes,
