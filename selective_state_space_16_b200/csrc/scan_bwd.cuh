@@ -62,7 +62,8 @@
 namespace ssm {
 
 constexpr int kBwdSeg = 8;       // steps per segment (checkpoint interval)
-constexpr int kBwdWarps = 4;     // warps per CTA (5 CTAs per SM, 4 with the conv prologue)
+constexpr int kBwdWarps = 4;     // warps per CTA (5 CTAs per SM: the headline's CTAs in one wave;
+                                 // the conv variants spill a little to stay at 96 registers)
 constexpr int kBwdChannels = kBwdWarps * 8;
 constexpr int kBwdRing = 4;      // segments of B/C rows in flight (cp.async ring)
 // dynamic shared memory of scan_bwd_kernel: h stage, dB/dC stage, B/C ring (sized for
@@ -109,7 +110,7 @@ __device__ __forceinline__ float load_io(const void* base, long long i) {
 }
 
 template <typename IO, bool ZOH, bool CONV>
-__global__ void __launch_bounds__(kBwdWarps * 32, CONV ? 4 : 5) scan_bwd_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdParams p) {
     constexpr int T = kBwdSeg, G = 4, PER = T / G, R = kBwdRing;
     extern __shared__ float4 bwd_smem[];
     // h_{t-1} of the segment's steps: [warp][step][lane] (16 bytes each)
