@@ -547,6 +547,22 @@ def measure_backward(ssm, stream, pk, steps=5):
                                       dconv_state_in=dcs, stream=stream)
 
     ms_ex = timed(call_ex)
+    # the forward storing its 8-step checkpoints, and the backward reading them instead of
+    # recomputing them (a training step's pair of calls)
+    ck = torch.empty(w.batch, (w.seqlen + 7) // 8, w.dim, w.dstate, **f32)
+    fws = ssm.new_workspace(w.batch, w.dim, w.dstate, w.seqlen)
+
+    def fwd_ck():
+        ssm.ssm_selective_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"], True,
+                                   g["y"], g["last"], fws, stream=stream, checkpoints=ck)
+
+    def bwd_ck():
+        ssm.ssm_selective_scan_bwd_ex(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"],
+                                      True, dy, du, ddelta, dA, dB, dC, dD, dz, dbias, ws, checkpoints=ck,
+                                      stream=stream)
+
+    ms_fwd_ck = timed(fwd_ck)
+    ms_bwd_ck = timed(bwd_ck)
     # algorithmic bytes: u, delta, z, dy read and du, ddelta, dz written (2 B each), B/C read,
     # dB/dC written (fp32), A/D/bias and their gradients
     nbytes = w.elements * 14 + w.batch * w.dstate * w.seqlen * (2 * 2 + 2 * 4) + w.dim * (w.dstate + 2) * 8
@@ -555,6 +571,10 @@ def measure_backward(ssm, stream, pk, steps=5):
     return {"workload": w.name, "value": w.elements / (ms / 1e3) / 1e9, "unit": UNIT, "ms_per_step": ms,
             "zoh_conv": {"value": w.elements / (ms_ex / 1e3) / 1e9, "ms_per_step": ms_ex,
                          "what": "ssm_selective_scan_bwd_ex: zero-order hold + conv1d width 4 (dx, conv gradients)"},
+            "with_forward_checkpoints": {"value": w.elements / (ms_bwd_ck / 1e3) / 1e9, "ms_per_step": ms_bwd_ck,
+                                         "forward_ms_with_checkpoints": ms_fwd_ck,
+                                         "what": "backward reading the forward's 8-step checkpoints (no forward "
+                                                 "sweep); the forward call that stores them"},
             "gradients": "du, ddelta, dz, dA, dB, dC, dD, ddelta_bias", "launches_per_step": 4,
             "hbm": {"achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
                     "algorithmic_bytes_per_step": nbytes,

@@ -143,7 +143,8 @@ typedef enum {
 typedef enum { SSM_DISC_SIMPLIFIED = 0, SSM_DISC_ZOH = 1 } ssm_discretization_t;
 
 /* Options of the forward entry points.  Zero-initialise the whole struct: zero means the
- * default for every field (changed in ABI version 2: the discretization field was added). */
+ * default for every field (changed in ABI version 2: the discretization field was added; in
+ * version 3: the checkpoints field). */
 typedef struct {
     int algo;                  /* ssm_algo_t                                                      */
     int lanes_per_channel;     /* SEQUENTIAL: lanes sharing one channel: 2, 4 or 8 (8: bf16 only), or 42 =
@@ -151,6 +152,15 @@ typedef struct {
     uint32_t spin_limit;       /* CHUNKED: polls before a look-back wait gives up; 0 = default    */
     int debug_skip_publish;    /* CHUNKED, tests only: chunk index whose CTAs never publish; -1 = off */
     int discretization;        /* ssm_discretization_t; 0 = SSM_DISC_SIMPLIFIED                   */
+    float* checkpoints;        /* NULL, or fp32 (batch, ceil(seqlen/8), dim, dstate) output: the state
+                                  at the start of every 8-step segment (h before step 8s; segment 0:
+                                  the initial state), for ssm_selective_scan_bwd_ex, which then skips
+                                  its own forward sweep ([Tech] 四.1: keep a little in the forward
+                                  pass).  16-byte aligned.  Written by the sequential kernel only
+                                  (4 or 8 lanes per channel): d_state 16; SSM_ALGO_AUTO then runs
+                                  the sequential kernel, and SSM_ALGO_CHUNKED / SSM_ALGO_DIRECT (or
+                                  a direct-load fallback) and lanes_per_channel 2 or 42 return
+                                  SSM_ERR_UNSUPPORTED.                                            */
 } ssm_fwd_options_t;
 
 /* ssm_selective_scan_fwd with an explicit kernel choice (tuning and tests).  opts may be NULL. */
@@ -266,6 +276,9 @@ typedef struct {
     float* dconv_state_in;         /* (batch, dim, width-1) fp32 output: gradient of conv->state_in, or NULL */
     const float* dconv_state_out;  /* (batch, dim, width-1) fp32: gradient reaching conv->state_out (the
                                       carried-out inputs), or NULL (zero)                                 */
+    const float* checkpoints;      /* NULL, or the checkpoints a forward call with the same inputs (and
+                                      initial state) stored (ssm_fwd_options_t.checkpoints): the
+                                      backward then reads them instead of recomputing them          */
 } ssm_bwd_options_t;
 
 /*

@@ -40,7 +40,7 @@ SSM_DISC_SIMPLIFIED, SSM_DISC_ZOH = 0, 1
 class FwdOptions(ctypes.Structure):
     _fields_ = [("algo", ctypes.c_int), ("lanes_per_channel", ctypes.c_int),
                 ("spin_limit", ctypes.c_uint32), ("debug_skip_publish", ctypes.c_int),
-                ("discretization", ctypes.c_int)]
+                ("discretization", ctypes.c_int), ("checkpoints", ctypes.c_void_p)]
 
 
 class ConvSpec(ctypes.Structure):
@@ -53,7 +53,8 @@ class BwdOptions(ctypes.Structure):
     """ssm_bwd_options_t: discretisation and conv prologue of a backward call."""
     _fields_ = [("discretization", ctypes.c_int), ("conv", ctypes.POINTER(ConvSpec)),
                 ("dconv_weight", ctypes.c_void_p), ("dconv_bias", ctypes.c_void_p),
-                ("dconv_state_in", ctypes.c_void_p), ("dconv_state_out", ctypes.c_void_p)]
+                ("dconv_state_in", ctypes.c_void_p), ("dconv_state_out", ctypes.c_void_p),
+                ("checkpoints", ctypes.c_void_p)]
 
 
 _lib = None
@@ -176,11 +177,12 @@ def new_workspace(batch, dim, dstate, seqlen, device="cuda", stream=None):
 
 def ssm_selective_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus, y, last_state, workspace,
                            stream=None, algo=None, lanes_per_channel=0, spin_limit=0, debug_skip_publish=-1,
-                           check=True, initial_state=None, zoh=False):
+                           check=True, initial_state=None, zoh=False, checkpoints=None):
     """Marshal a forward-scan call.  u/delta/z/y: (b, d, L); B/C: (b, N, L); A: (d, N) fp32;
     D/delta_bias: (d) fp32 or None; last_state: (b, d, N) fp32 or None; workspace: uint8;
     initial_state: (b, d, N) fp32 or None (zero), through ssm_selective_scan_fwd_state;
-    zoh: zero-order-hold discretisation instead of the simplified one."""
+    zoh: zero-order-hold discretisation instead of the simplified one; checkpoints:
+    (b, ceil(L/8), d, N) fp32 output for the backward, or None."""
     lib = load()
     b, d, L = u.shape
     n = A.shape[1]
@@ -189,13 +191,13 @@ def ssm_selective_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus, y, las
     tail = [_ptr(y), _ptr(last_state), b, d, n, L, _io(u), _ptr(workspace),
             workspace.numel() * workspace.element_size()]
     default_opts = (algo is None and lanes_per_channel == 0 and spin_limit == 0 and debug_skip_publish < 0
-                    and not zoh)
+                    and not zoh and checkpoints is None)
     if default_opts and initial_state is None:
         code = lib.ssm_selective_scan_fwd(*head, *tail, _stream(stream))
     else:
         a = ALGOS[algo] if isinstance(algo, str) else (algo or SSM_ALGO_AUTO)
         opts = FwdOptions(a, lanes_per_channel, spin_limit, debug_skip_publish,
-                          SSM_DISC_ZOH if zoh else SSM_DISC_SIMPLIFIED)
+                          SSM_DISC_ZOH if zoh else SSM_DISC_SIMPLIFIED, _ptr(checkpoints))
         if initial_state is None:
             code = lib.ssm_selective_scan_fwd_ex(*head, *tail, ctypes.byref(opts), _stream(stream))
         else:
@@ -244,10 +246,12 @@ def ssm_selective_scan_bwd(u, delta, A, B, C, D, z, delta_bias, softplus, dy, du
 def ssm_selective_scan_bwd_ex(u, delta, A, B, C, D, z, delta_bias, softplus, dy, du, ddelta, dA, dB, dC, dD, dz,
                               ddelta_bias, workspace, initial_state=None, dlast_state=None, dinitial_state=None,
                               zoh=False, conv_weight=None, conv_bias=None, conv_state_in=None, dconv_weight=None,
-                              dconv_bias=None, dconv_state_in=None, dconv_state_out=None, stream=None, check=True):
+                              dconv_bias=None, dconv_state_in=None, dconv_state_out=None, checkpoints=None,
+                              stream=None, check=True):
     """Marshal ssm_selective_scan_bwd_ex: as ssm_selective_scan_bwd, plus zoh and, when
     conv_weight (d, K) fp32 is given, the conv prologue: u is then x and du receives dx;
-    dconv_weight (d, K), dconv_bias (d), dconv_state_in / dconv_state_out (b, d, K-1) fp32."""
+    dconv_weight (d, K), dconv_bias (d), dconv_state_in / dconv_state_out (b, d, K-1) fp32;
+    checkpoints: the forward's (b, ceil(L/8), d, N) fp32, or None."""
     b, d, L = u.shape
     n = A.shape[1]
     spec = None
@@ -256,7 +260,7 @@ def ssm_selective_scan_bwd_ex(u, delta, A, B, C, D, z, delta_bias, softplus, dy,
                         None)
     opts = BwdOptions(SSM_DISC_ZOH if zoh else SSM_DISC_SIMPLIFIED,
                       ctypes.pointer(spec) if spec is not None else None, _ptr(dconv_weight), _ptr(dconv_bias),
-                      _ptr(dconv_state_in), _ptr(dconv_state_out))
+                      _ptr(dconv_state_in), _ptr(dconv_state_out), _ptr(checkpoints))
     code = load().ssm_selective_scan_bwd_ex(
         _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias), int(bool(softplus)),
         _ptr(initial_state), _ptr(dy), _ptr(dlast_state), _ptr(du), _ptr(ddelta), _ptr(dA), _ptr(dB), _ptr(dC),
@@ -269,7 +273,8 @@ def ssm_selective_scan_bwd_ex(u, delta, A, B, C, D, z, delta_bias, softplus, dy,
 
 def selective_scan_bwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True, dy=None,
                        initial_state=None, dlast_state=None, workspace=None, stream=None, zoh=False,
-                       conv_weight=None, conv_bias=None, conv_state_in=None, dconv_state_out=None):
+                       conv_weight=None, conv_bias=None, conv_state_in=None, dconv_state_out=None,
+                       checkpoints=None):
     """Convenience wrapper: allocates every gradient and, if not given, a workspace, then
     calls ssm_selective_scan_bwd (ssm_selective_scan_bwd_ex with zoh or a conv).  Returns a dict
     du, ddelta, dz (or None), dA, dB, dC, dD, ddelta_bias, dinitial_state; with conv_weight
@@ -285,7 +290,7 @@ def selective_scan_bwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
     if workspace is None:
         workspace = torch.empty(max(ssm_selective_scan_bwd_workspace_size(b, d, n, L), 256), dtype=torch.uint8,
                                 device=u.device)
-    if not zoh and conv_weight is None:
+    if not zoh and conv_weight is None and checkpoints is None:
         ssm_selective_scan_bwd(u, delta, A, B, C, D, z, delta_bias, softplus, dy, out["du"], out["ddelta"],
                                out["dA"], out["dB"], out["dC"], out["dD"], out["dz"], out["ddelta_bias"], workspace,
                                initial_state=initial_state, dlast_state=dlast_state,
@@ -306,22 +311,23 @@ def selective_scan_bwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
                               conv_bias=conv_bias, conv_state_in=conv_state_in,
                               dconv_weight=out.get("dconv_weight"), dconv_bias=out.get("dconv_bias"),
                               dconv_state_in=out.get("dconv_state_in"), dconv_state_out=dconv_state_out,
-                              stream=stream)
+                              checkpoints=checkpoints, stream=stream)
     return out
 
 
 def ssm_selective_scan_fwd_conv(x, conv_weight, conv_bias, delta, A, B, C, D, z, delta_bias, softplus, y, last_state,
                                 workspace, conv_state_in=None, conv_state_out=None, u_out=None, initial_state=None,
-                                stream=None, algo=None, lanes_per_channel=0, zoh=False, check=True):
+                                stream=None, algo=None, lanes_per_channel=0, zoh=False, check=True,
+                                checkpoints=None):
     """Marshal a forward scan of u = silu(causal conv(x)): x (b, d, L) in the I/O dtype;
     conv_weight (d, K) fp32; conv_bias (d) fp32 or None; conv_state_in/out (b, d, K-1) fp32 or
-    None; u_out (b, d, L) I/O dtype or None."""
+    None; u_out (b, d, L) I/O dtype or None; checkpoints as ssm_selective_scan_fwd."""
     b, d, L = x.shape
     n = A.shape[1]
     spec = ConvSpec(_ptr(conv_weight), _ptr(conv_bias), int(conv_weight.shape[1]), _ptr(conv_state_in),
                     _ptr(conv_state_out), _ptr(u_out))
     a = ALGOS[algo] if isinstance(algo, str) else (algo or SSM_ALGO_AUTO)
-    opts = FwdOptions(a, lanes_per_channel, 0, -1, SSM_DISC_ZOH if zoh else SSM_DISC_SIMPLIFIED)
+    opts = FwdOptions(a, lanes_per_channel, 0, -1, SSM_DISC_ZOH if zoh else SSM_DISC_SIMPLIFIED, _ptr(checkpoints))
     code = load().ssm_selective_scan_fwd_conv(
         _ptr(x), ctypes.byref(spec), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
         int(bool(softplus)), _ptr(initial_state), _ptr(y), _ptr(last_state), b, d, n, L, _io(x), _ptr(workspace),

@@ -17,7 +17,7 @@ using namespace ssmh;
 
 namespace {
 
-constexpr int kAbiVersion = 2;
+constexpr int kAbiVersion = 3;
 
 // d_state values of the forward scan and decode: 16 (the tuned kernels) and the wider states
 // of scan_fwd_wide.cuh.
@@ -58,6 +58,8 @@ ssm_status_t launch_forward(const FwdArgs& a, const ssm_fwd_options_t& o) {
     if (!tma_ok && a.pad_ok && a.conv.k == 0 && (algo == SSM_ALGO_AUTO || algo == SSM_ALGO_SEQUENTIAL))
         return launch_forward_padded<IO>(a, o);
     if (!tma_ok) algo = SSM_ALGO_DIRECT;
+    if (a.ckpt && algo == SSM_ALGO_DIRECT) return SSM_ERR_UNSUPPORTED;  // checkpoints: sequential kernel only
+    if (a.ckpt && algo == SSM_ALGO_AUTO) algo = SSM_ALGO_SEQUENTIAL;
     if (algo == SSM_ALGO_DIRECT) return launch_direct<IO>(a);
     if ((a.zoh || a.conv.k > 0) && algo == SSM_ALGO_CHUNKED) return SSM_ERR_UNSUPPORTED;  // plain scan only
     if (algo == SSM_ALGO_AUTO && (a.zoh || a.conv.k > 0)) algo = SSM_ALGO_SEQUENTIAL;
@@ -157,9 +159,12 @@ ssm_status_t forward_entry(const void* u, const void* delta, const float* A, con
         const uintptr_t a0 = reinterpret_cast<uintptr_t>(initial_state), a1 = reinterpret_cast<uintptr_t>(last_state);
         if ((a0 <= a1 ? a1 - a0 : a0 - a1) < state_bytes) return SSM_ERR_INVALID_ARG;
     }
-    ssm_fwd_options_t o{SSM_ALGO_AUTO, 0, 0, -1, SSM_DISC_SIMPLIFIED};
+    ssm_fwd_options_t o{SSM_ALGO_AUTO, 0, 0, -1, SSM_DISC_SIMPLIFIED, nullptr};
     if (opts) o = *opts;
     if (o.algo < SSM_ALGO_AUTO || o.algo > SSM_ALGO_DIRECT) return SSM_ERR_INVALID_ARG;
+    if (o.checkpoints && !aligned16(o.checkpoints)) return SSM_ERR_INVALID_ARG;
+    // checkpoints come from the sequential kernel only
+    if (o.checkpoints && (o.algo == SSM_ALGO_CHUNKED || o.algo == SSM_ALGO_DIRECT)) return SSM_ERR_UNSUPPORTED;
     if (o.discretization != SSM_DISC_SIMPLIFIED && o.discretization != SSM_DISC_ZOH) return SSM_ERR_INVALID_ARG;
     if (batch == 0 || dim == 0) return SSM_OK;
     if (batch > 65535) return SSM_ERR_UNSUPPORTED;  // batch is a grid y-dimension of the B/C pack
@@ -182,8 +187,9 @@ ssm_status_t forward_entry(const void* u, const void* delta, const float* A, con
     }
     FwdArgs a{u, delta, B, C, z, A, D, delta_bias, softplus, initial_state, o.discretization == SSM_DISC_ZOH, y,
               last_state, batch, dim, seqlen, io_dtype, static_cast<uint8_t*>(workspace), s, sm_count, conv};
+    a.ckpt = o.checkpoints;
     if (dstate != 16) {
-        if (o.algo == SSM_ALGO_CHUNKED || conv.k > 0) return SSM_ERR_UNSUPPORTED;  // d_state 16 only
+        if (o.algo == SSM_ALGO_CHUNKED || conv.k > 0 || o.checkpoints) return SSM_ERR_UNSUPPORTED;  // d_state 16 only
         return io_dtype == SSM_BF16 ? launch_wide<__nv_bfloat16>(a, dstate) : launch_wide<float>(a, dstate);
     }
     return io_dtype == SSM_BF16 ? launch_forward<__nv_bfloat16>(a, o) : launch_forward<float>(a, o);
@@ -351,6 +357,7 @@ ssm_status_t ssm_selective_scan_bwd_ex(const void* u, const void* delta, const f
     ssm_bwd_options_t o{};
     if (opts) o = *opts;
     if (o.discretization != SSM_DISC_SIMPLIFIED && o.discretization != SSM_DISC_ZOH) return SSM_ERR_INVALID_ARG;
+    if (o.checkpoints && !aligned16(o.checkpoints)) return SSM_ERR_INVALID_ARG;
     ConvBwdArgs conv;
     if (o.conv) {
         if (o.conv->width < 1 || o.conv->width > 4) return SSM_ERR_INVALID_ARG;
@@ -404,7 +411,7 @@ ssm_status_t ssm_selective_scan_bwd_ex(const void* u, const void* delta, const f
     }
     BwdArgs a{u, delta, B, C, z, dy, A, D, delta_bias, initial_state, dlast_state, softplus, du, ddelta, dz, dA, dB,
               dC, dD, ddelta_bias, dinitial_state, batch, dim, seqlen, static_cast<uint8_t*>(workspace), s,
-              o.discretization == SSM_DISC_ZOH, conv};
+              o.discretization == SSM_DISC_ZOH, conv, o.checkpoints};
     return io_dtype == SSM_BF16 ? launch_backward<__nv_bfloat16>(a) : launch_backward<float>(a);
 }
 

@@ -55,7 +55,8 @@ ssm_status_t launch_backward(const BwdArgs& a) {
     p.ddelta = a.ddelta;
     p.dz = a.dz;
     p.dh0 = a.dh0;
-    p.ckpt = reinterpret_cast<float*>(a.ws + wl.ckpt_off);
+    p.ckpt = a.ckpt ? const_cast<float*>(a.ckpt) : reinterpret_cast<float*>(a.ws + wl.ckpt_off);
+    p.ckpt_given = a.ckpt != nullptr;
     p.dbc_part = reinterpret_cast<float*>(a.ws + wl.dbc_off);
     p.dA_part = reinterpret_cast<float*>(a.ws + wl.dA_off);
     p.dD_part = reinterpret_cast<float*>(a.ws + wl.dD_off);

@@ -105,6 +105,7 @@ struct FwdArgs {
     bool pad_ok = true;  // the workspace has room for padded rows (not the no-allocation scratch)
     bool pdl = false;    // the previous launch is the B/C pack: the scan may start early (it waits
                          // for the pack before reading the B/C rows, and reads nothing else it writes)
+    float* ckpt = nullptr;  // checkpoints for the backward (batch, ceil(L/8), dim, 16), or null
 };
 
 // Backward workspace layout:
@@ -137,6 +138,7 @@ struct BwdArgs {
     cudaStream_t stream;
     int zoh = 0;
     ConvBwdArgs conv;
+    const float* ckpt = nullptr;  // the forward's checkpoints (no forward sweep), or null
 };
 
 struct DecodeArgs {
@@ -167,6 +169,8 @@ template <typename IO> ssm_status_t launch_chunked(const FwdArgs& a, const ssm_f
 template <typename IO> ssm_status_t launch_seq_plain(const FwdArgs& a, const ssm_fwd_options_t& o);
 // Sequential family with the zero-order hold and / or the conv prologue (fwd_seq_flag_*.cu).
 template <typename IO> ssm_status_t launch_seq_flagged(const FwdArgs& a, const ssm_fwd_options_t& o);
+// Sequential family storing checkpoints for the backward, every variant (fwd_seq_ckpt_*.cu).
+template <typename IO> ssm_status_t launch_seq_ckpt(const FwdArgs& a, const ssm_fwd_options_t& o);
 // d_state 32 .. 256 forward (wide.cu).
 template <typename IO> ssm_status_t launch_wide(const FwdArgs& a, int n);
 // Backward (bwd.cu).

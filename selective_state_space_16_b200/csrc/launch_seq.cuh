@@ -11,12 +11,12 @@
 
 namespace ssmh {
 
-template <typename IO, int G, int CPL, bool ZOH, bool CONV = false>
+template <typename IO, int G, int CPL, bool ZOH, bool CONV = false, bool CK = false>
 const void* seq_kernel_ptr(int stages) {
     switch (stages) {
-        case 2: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 2, ZOH, CONV>);
-        case 3: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 3, ZOH, CONV>);
-        default: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 4, ZOH, CONV>);
+        case 2: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 2, ZOH, CONV, CK>);
+        case 3: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 3, ZOH, CONV, CK>);
+        default: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 4, ZOH, CONV, CK>);
     }
 }
 
@@ -29,7 +29,7 @@ struct SeqPlan {
     bool ok = false;
 };
 
-template <typename IO, int G, int CPL, bool ZOH = false, bool CONV = false>
+template <typename IO, int G, int CPL, bool ZOH = false, bool CONV = false, bool CK = false>
 SeqPlan plan_seq(const FwdArgs& a) {
     using Cfg = ssm::SeqCfg<IO, G, CPL>;
     SeqPlan pl;
@@ -52,7 +52,7 @@ SeqPlan plan_seq(const FwdArgs& a) {
         if (stages < 2) continue;
         const int threads = (Cfg::warps_for(mt) + 1) * 32;
         const int smem = Cfg::smem_bytes(mt, stages);
-        const void* kern = seq_kernel_ptr<IO, G, CPL, ZOH, CONV>(stages);
+        const void* kern = seq_kernel_ptr<IO, G, CPL, ZOH, CONV, CK>(stages);
         int occ = 0;
         if (!ensure_smem_attr(kern, smem) ||
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, smem) != cudaSuccess || occ < per_sm)
@@ -84,7 +84,7 @@ double predict_seq(const FwdArgs& a, const SeqPlan& pl) {
     return tiles * cost / hide;
 }
 
-template <typename IO, int G, int CPL, bool ZOH = false, bool CONV = false>
+template <typename IO, int G, int CPL, bool ZOH = false, bool CONV = false, bool CK = false>
 ssm_status_t launch_seq(const FwdArgs& a, const SeqPlan& pl) {
     using Cfg = ssm::SeqCfg<IO, G, CPL>;
     if (!pl.ok) return SSM_ERR_UNSUPPORTED;
@@ -127,6 +127,8 @@ ssm_status_t launch_seq(const FwdArgs& a, const SeqPlan& pl) {
     p.u_out = a.conv.u_out;
     p.conv_k = a.conv.k;
     p.y_vec = a.y_vec;
+    p.ckpt = a.ckpt;
+    p.nseg = static_cast<int>((a.L + 7) / 8);
     if (a.L >= (1LL << 31) - 1024) return SSM_ERR_UNSUPPORTED;
     // With a.pdl the kernel may start while the B/C pack before it is still running (programmatic
     // dependent launch): its prologue and first input copies overlap the pack's tail.
@@ -142,9 +144,9 @@ ssm_status_t launch_seq(const FwdArgs& a, const SeqPlan& pl) {
     cfg.numAttrs = a.pdl ? 1 : 0;
     cudaError_t e;
     switch (pl.stages) {
-        case 2: e = cudaLaunchKernelEx(&cfg, ssm::scan_fwd_seq_kernel<IO, G, CPL, 2, ZOH, CONV>, mu, mdl, mz, mbc, p); break;
-        case 3: e = cudaLaunchKernelEx(&cfg, ssm::scan_fwd_seq_kernel<IO, G, CPL, 3, ZOH, CONV>, mu, mdl, mz, mbc, p); break;
-        default: e = cudaLaunchKernelEx(&cfg, ssm::scan_fwd_seq_kernel<IO, G, CPL, 4, ZOH, CONV>, mu, mdl, mz, mbc, p); break;
+        case 2: e = cudaLaunchKernelEx(&cfg, ssm::scan_fwd_seq_kernel<IO, G, CPL, 2, ZOH, CONV, CK>, mu, mdl, mz, mbc, p); break;
+        case 3: e = cudaLaunchKernelEx(&cfg, ssm::scan_fwd_seq_kernel<IO, G, CPL, 3, ZOH, CONV, CK>, mu, mdl, mz, mbc, p); break;
+        default: e = cudaLaunchKernelEx(&cfg, ssm::scan_fwd_seq_kernel<IO, G, CPL, 4, ZOH, CONV, CK>, mu, mdl, mz, mbc, p); break;
     }
     if (e != cudaSuccess) {
         (void)cudaGetLastError();
@@ -153,23 +155,25 @@ ssm_status_t launch_seq(const FwdArgs& a, const SeqPlan& pl) {
     return launch_status();
 }
 
-// The zero-order-hold and conv-prologue kernels exist for 4 and 8 lanes per channel.
-template <typename IO, bool ZOH, bool CONV>
+// The zero-order-hold and conv-prologue kernels exist for 4 and 8 lanes per channel, with and
+// without checkpoints (CK).
+template <typename IO, bool ZOH, bool CONV, bool CK = false>
 ssm_status_t launch_flagged_g(const FwdArgs& a, const ssm_fwd_options_t& o) {
-    const SeqPlan p4 = plan_seq<IO, 4, 1, ZOH, CONV>(a);
+    const SeqPlan p4 = plan_seq<IO, 4, 1, ZOH, CONV, CK>(a);
     if constexpr (sizeof(IO) == 2) {
-        const SeqPlan p8 = plan_seq<IO, 8, 1, ZOH, CONV>(a);
+        const SeqPlan p8 = plan_seq<IO, 8, 1, ZOH, CONV, CK>(a);
         const bool use8 = o.lanes_per_channel == 8 ||
                           (o.lanes_per_channel == 0 && predict_seq<IO, 8, 1>(a, p8) < predict_seq<IO, 4, 1>(a, p4));
-        if (use8) return launch_seq<IO, 8, 1, ZOH, CONV>(a, p8);
+        if (use8) return launch_seq<IO, 8, 1, ZOH, CONV, CK>(a, p8);
     }
-    return launch_seq<IO, 4, 1, ZOH, CONV>(a, p4);
+    return launch_seq<IO, 4, 1, ZOH, CONV, CK>(a, p4);
 }
 
 // Plain discretisation without conv: variants (lanes per channel G, channels per lane CPL).
 // lanes_per_channel selects G explicitly (CPL = 1), or G = 4 with CPL = 2 when given as 42.
 template <typename IO>
 ssm_status_t launch_seq_plain(const FwdArgs& a, const ssm_fwd_options_t& o) {
+    if (a.ckpt) return launch_seq_ckpt<IO>(a, o);  // the checkpoint-storing kernels (fwd_seq_ckpt_*.cu)
     const SeqPlan p2 = plan_seq<IO, 2, 1>(a), p4 = plan_seq<IO, 4, 1>(a), p42 = plan_seq<IO, 4, 2>(a);
     SeqPlan p8;
     if constexpr (sizeof(IO) == 2) p8 = plan_seq<IO, 8, 1>(a);
@@ -194,9 +198,24 @@ ssm_status_t launch_seq_plain(const FwdArgs& a, const ssm_fwd_options_t& o) {
 // Zero-order hold and / or the conv prologue.
 template <typename IO>
 ssm_status_t launch_seq_flagged(const FwdArgs& a, const ssm_fwd_options_t& o) {
+    if (a.ckpt) return launch_seq_ckpt<IO>(a, o);  // the checkpoint-storing kernels (fwd_seq_ckpt_*.cu)
     if (a.zoh && a.conv.k > 0) return launch_flagged_g<IO, true, true>(a, o);
     if (a.zoh) return launch_flagged_g<IO, true, false>(a, o);
     return launch_flagged_g<IO, false, true>(a, o);
 }
+
+// Every discretisation / prologue combination with checkpoints for the backward (4 or 8 lanes
+// per channel).  Instantiated only in fwd_seq_ckpt_*.cu (extern below), so that the other
+// translation units do not compile these kernels.
+template <typename IO>
+ssm_status_t launch_seq_ckpt(const FwdArgs& a, const ssm_fwd_options_t& o) {
+    if (o.lanes_per_channel != 0 && o.lanes_per_channel != 4 && o.lanes_per_channel != 8) return SSM_ERR_UNSUPPORTED;
+    if (a.zoh && a.conv.k > 0) return launch_flagged_g<IO, true, true, true>(a, o);
+    if (a.zoh) return launch_flagged_g<IO, true, false, true>(a, o);
+    if (a.conv.k > 0) return launch_flagged_g<IO, false, true, true>(a, o);
+    return launch_flagged_g<IO, false, false, true>(a, o);
+}
+extern template ssm_status_t launch_seq_ckpt<__nv_bfloat16>(const FwdArgs&, const ssm_fwd_options_t&);
+extern template ssm_status_t launch_seq_ckpt<float>(const FwdArgs&, const ssm_fwd_options_t&);
 
 }  // namespace ssmh

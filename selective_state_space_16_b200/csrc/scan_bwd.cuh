@@ -77,7 +77,8 @@ struct BwdParams {
     const float *A, *D, *bias, *h0, *dlast;
     void *du, *ddelta, *dz;          // (batch, dim, L) IO outputs (dz only with z)
     float* dh0;                      // (batch, dim, 16) or null
-    float* ckpt;                     // workspace: [batch][nseg][dim][16]
+    float* ckpt;                     // workspace, or the forward's: [batch][nseg][dim][16]
+    int ckpt_given;                  // the checkpoints came from the forward: no forward sweep
     float* dbc_part;                 // workspace: [batch][ncta][L][32]  (dB n, then dC n)
     float* dA_part;                  // workspace: [batch][dim][16]
     float* dD_part;                  // workspace: [batch][dim]
@@ -276,43 +277,46 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
     };
 
     // ------------------------------------------------------------ forward sweep, checkpoints
-    float2 h[2];
-    {
-        const float4 h0 = (valid && p.h0) ? ld4(p.h0 + srow) : make_float4(0, 0, 0, 0);
-        h[0] = lo(h0);
-        h[1] = hi(h0);
-    }
-    for (int r = 0; r < R - 1; ++r) issue_bc(r, r);
+    // (skipped when the forward scan stored them: the checkpoints of ssm_fwd_options_t)
     Raw nxt;
-    load_raw(0, false, nxt);
-    for (int s = 0; s < p.nseg; ++s) {
-        Raw cur = nxt;
-        conv_u(s, cur);
-        load_raw(s + 1, false, nxt);  // next segment's inputs, in flight during this one
-        __syncthreads();              // every warp is done with the slot refilled below
-        issue_bc(s + R - 1, (s + R - 1) % R);
-        cp_async_wait<R - 1>();
-        __syncthreads();              // segment s's B/C rows are visible to every warp
-        if (valid && dcheck(p.hdr, s < p.nseg, kSiteBwdCkpt, s))
-            *reinterpret_cast<float4*>(ckpt_at(s)) = make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
-        float dt[PER];
-        step_sizes(s, cur, dt);
-        const uint8_t* bcs = bcring + (s % R) * T * RB + nl * 16;
+    if (!p.ckpt_given) {
+        float2 h[2];
+        {
+            const float4 h0 = (valid && p.h0) ? ld4(p.h0 + srow) : make_float4(0, 0, 0, 0);
+            h[0] = lo(h0);
+            h[1] = hi(h0);
+        }
+        for (int r = 0; r < R - 1; ++r) issue_bc(r, r);
+        load_raw(0, false, nxt);
+        for (int s = 0; s < p.nseg; ++s) {
+            Raw cur = nxt;
+            conv_u(s, cur);
+            load_raw(s + 1, false, nxt);  // next segment's inputs, in flight during this one
+            __syncthreads();              // every warp is done with the slot refilled below
+            issue_bc(s + R - 1, (s + R - 1) % R);
+            cp_async_wait<R - 1>();
+            __syncthreads();              // segment s's B/C rows are visible to every warp
+            if (valid && dcheck(p.hdr, s < p.nseg, kSiteBwdCkpt, s))
+                *reinterpret_cast<float4*>(ckpt_at(s)) = make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
+            float dt[PER];
+            step_sizes(s, cur, dt);
+            const uint8_t* bcs = bcring + (s % R) * T * RB + nl * 16;
 #pragma unroll
-        for (int i = 0; i < T; ++i) {
-            const float dti = __shfl_sync(0xffffffffu, dt[i % PER], srcl[i / PER]);
-            const float ui = __shfl_sync(0xffffffffu, cur.u[i % PER], srcl[i / PER]);
-            float2 Bv[2];
-            load_b(bcs + i * RB, Bv);
+            for (int i = 0; i < T; ++i) {
+                const float dti = __shfl_sync(0xffffffffu, dt[i % PER], srcl[i / PER]);
+                const float ui = __shfl_sync(0xffffffffu, cur.u[i % PER], srcl[i / PER]);
+                float2 Bv[2];
+                load_b(bcs + i * RB, Bv);
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const float2 a = decay(dti, j);
-                h[j] = __ffma2_rn(a, h[j], __fmul2_rn(weight_u(dti, ui, j, a), Bv[j]));
+                for (int j = 0; j < 2; ++j) {
+                    const float2 a = decay(dti, j);
+                    h[j] = __ffma2_rn(a, h[j], __fmul2_rn(weight_u(dti, ui, j, a), Bv[j]));
+                }
             }
         }
+        cp_async_wait<0>();
+        __syncthreads();
     }
-    cp_async_wait<0>();
-    __syncthreads();
 
     // ------------------------------------------------------------ reverse sweep
     float2 g[2], dA_acc[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};

@@ -67,6 +67,10 @@ struct SeqParams {
     // y rows are 16-byte aligned (L * sizeof(IO) a multiple of 16): vector stores; else
     // element stores (the inputs were then staged into padded rows, see pad_rows_kernel)
     int y_vec;
+    // checkpoints for the backward, or null: (batch, nseg, dim, 16) fp32, the state at the
+    // start of every 8-step segment (h before step 8s), nseg = ceil(L / 8)
+    float* ckpt;
+    int nseg;
 };
 
 __host__ __device__ constexpr int round_up_i(int v, int m) { return (v + m - 1) / m * m; }
@@ -149,7 +153,7 @@ __device__ __forceinline__ void store_run(IO* dst, const float (&v)[N]) {
 // of a stage are unrolled (compile-time shared-memory offsets) with ping-pong step-size
 // buffers: the step sizes of group g+1 (for the last group: group 0 of the next stage,
 // after waiting for it) are computed while group g is scanned.
-template <typename IO, int G, int CPL, int S, bool HZ, bool ZOH, bool CONV>
+template <typename IO, int G, int CPL, int S, bool HZ, bool ZOH, bool CONV, bool CK>
 __device__ __forceinline__ void seq_consumer(uint8_t* smem, uint64_t* full_bar, uint64_t* empty_bar,
                                              const int* abort_flag, const SeqParams& p, long long r_begin, int nt,
                                              int b_first, int stage_bytes, int nstages, int L32) {
@@ -208,6 +212,31 @@ __device__ __forceinline__ void seq_consumer(uint8_t* smem, uint64_t* full_bar, 
     }
     const bool softplus = p.softplus != 0;
     const uint32_t wait_limit = p.wait_limit;
+
+    // Checkpoints for the backward: after the group that ends at step t_end (a multiple of 8
+    // below L) the lane's chains hold h before step t_end, the start of segment t_end / 8.
+    // (A compile-time variant: the store between the groups would otherwise cost the kernels
+    // that write no checkpoints their cross-group scheduling.)
+    auto checkpoint = [&](int t_end) {
+        if (CK && (t_end & 7) == 0 && t_end < L32) {
+#pragma unroll
+            for (int c = 0; c < CPL; ++c)
+                if (valid[c] && dcheck(p.hdr, (t_end >> 3) < p.nseg, kSiteSeqState, t_end)) {
+                    float* dst = p.ckpt +
+                                 ((static_cast<long long>(b) * p.nseg + (t_end >> 3)) * p.dim + d[c]) * 16 + nl * NC;
+                    if constexpr (NC % 4 == 0) {  // 16-byte stores (nl * NC floats is a 16-byte offset)
+#pragma unroll
+                        for (int jj = 0; jj < NC / 2; jj += 2)
+                            *reinterpret_cast<float4*>(dst + 2 * jj) =
+                                make_float4(h[c][jj].x, h[c][jj].y, h[c][jj + 1].x, h[c][jj + 1].y);
+                    } else {
+#pragma unroll
+                        for (int jj = 0; jj < NC / 2; ++jj) *reinterpret_cast<float2*>(dst + 2 * jj) = h[c][jj];
+                    }
+                }
+        }
+    };
+    checkpoint(0);  // segment 0 starts from the initial state
 
     // Causal conv1d + SiLU of the staged x tile, in place ([Hist] Mamba Block 数据流: x -> 1D
     // conv -> SiLU -> S6).  Lane (cg, nl) converts steps nl*SPL .. of its channel cg; the three
@@ -425,7 +454,9 @@ __device__ __forceinline__ void seq_consumer(uint8_t* smem, uint64_t* full_bar, 
                     prologue(smem + sn * stage_bytes, 0, tk + TC, spA);
                 }
             }
+            checkpoint(tk + (g + 1) * GS);
             scan_group(st, g + 1, tk + (g + 1) * GS, spB);
+            checkpoint(tk + (g + 2) * GS);
         }
         // The stage is consumed: release it to the producer.
         __syncwarp();
@@ -462,7 +493,7 @@ __device__ __forceinline__ void seq_consumer(uint8_t* smem, uint64_t* full_bar, 
         }
 }
 
-template <typename IO, int G, int CPL, int S, bool ZOH = false, bool CONV = false>
+template <typename IO, int G, int CPL, int S, bool ZOH = false, bool CONV = false, bool CK = false>
 __global__ void __launch_bounds__((SeqCfg<IO, G, CPL>::kMaxWarps + 1) * 32, 1)
 scan_fwd_seq_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_dl,
                     const __grid_constant__ CUtensorMap map_z, const __grid_constant__ CUtensorMap map_bc,
@@ -556,10 +587,10 @@ scan_fwd_seq_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_cons
             }
         } else if (warp < nwarps) {
             if (p.has_z)
-                seq_consumer<IO, G, CPL, S, true, ZOH, CONV>(smem, full_bar, empty_bar, &abort_flag, p, r_begin, nt,
+                seq_consumer<IO, G, CPL, S, true, ZOH, CONV, CK>(smem, full_bar, empty_bar, &abort_flag, p, r_begin, nt,
                                                              b_first, stage_bytes, nstages, L32);
             else
-                seq_consumer<IO, G, CPL, S, false, ZOH, CONV>(smem, full_bar, empty_bar, &abort_flag, p, r_begin, nt,
+                seq_consumer<IO, G, CPL, S, false, ZOH, CONV, CK>(smem, full_bar, empty_bar, &abort_flag, p, r_begin, nt,
                                                               b_first, stage_bytes, nstages, L32);
         }
         // Every warp leaves the round before the barriers are re-initialised for the next.

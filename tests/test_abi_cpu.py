@@ -41,7 +41,7 @@ def test_header_declares_entry_points():
 def test_library_exports_every_declared_symbol(lib):
     missing = [n for n in _declared_functions() if not hasattr(lib, n)]
     assert not missing, missing
-    assert lib.ssm_abi_version() == 2
+    assert lib.ssm_abi_version() == 3
 
 
 def test_status_strings(lib):
@@ -59,7 +59,7 @@ def test_debug_library_builds_and_exports_every_declared_symbol():
     dbg = ct.CDLL(path)
     missing = [n for n in _declared_functions() if not hasattr(dbg, n)]
     assert not missing, missing
-    assert dbg.ssm_abi_version() == 2
+    assert dbg.ssm_abi_version() == 3
 
 
 def test_workspace_size(lib):
