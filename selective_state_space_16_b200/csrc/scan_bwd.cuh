@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
     // phi formed from a = decay(Delta, j)
     auto weight_u = [&](float dti, float ui, int j, float2 a) {
         if constexpr (ZOH)
-            return __fmul2_rn(zoh_beta2(__fmul2_rn(f2(dti, dti), A2[j]), a, f2(dti, dti), invA[j]), f2(ui, ui));
+            return __fmul2_rn(zoh_phi2(__fmul2_rn(f2(dti, dti), A2[j]), a, f2(dti, dti), invA[j]), f2(ui, ui));
         else return f2(dti * ui, dti * ui);
     };
     // conv taps (right-aligned: tap k of a width-K conv at 4 - K + k) and bias
@@ -421,7 +421,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdPa
                 const float2 ah = __fmul2_rn(av[j], hp[j]);
                 if constexpr (ZOH) {
                     const float2 y = __fmul2_rn(dt2, A2[j]);
-                    const float2 phi = zoh_beta2(y, av[j], dt2, invA[j]);
+                    const float2 phi = zoh_phi2(y, av[j], dt2, invA[j]);
                     const float2 bu = __fmul2_rn(Bv[j], u2);
                     const float2 dphi = zoh_dphi_dA2(y, av[j], dt2, phi, invA[j]);
                     dA_acc[j] = __ffma2_rn(g[j], __ffma2_rn(dt2, ah, __fmul2_rn(dphi, bu)), dA_acc[j]);

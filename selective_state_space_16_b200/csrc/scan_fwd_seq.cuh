@@ -20,7 +20,7 @@
 // data path is the scarce resource of this kernel).  Per step each lane computes
 //   a = 2^(Delta * A[d,n] * log2 e),  h = a*h + (Delta*u)*B[n],  y_partial += C[n]*h
 // (simplified discretisation Abar = exp(Delta A), Bbar = Delta B: [Card] 离散化变换; with ZOH the
-// zero-order-hold weight of [Eng] §2.2, see zoh_beta2),
+// zero-order-hold weight of [Eng] §2.2, see zoh_phi2),
 // and the G partial sums of y_t = sum_n C_t[n] h_t[n] are combined by a shuffle
 // reduce-scatter over each 16-byte group of GS steps, so that every lane finishes the
 // epilogue (D skip, silu gate, rounding, store) of GS/G steps and nothing is evaluated
@@ -373,10 +373,12 @@ __device__ __forceinline__ void seq_consumer(uint8_t* smem, uint64_t* full_bar, 
                 for (int jj = 0; jj < NC / 2; ++jj) {
                     const float2 arg = __fmul2_rn(dd, A2[c][jj]);
                     const float2 a = f2(ex2_mufu(arg.x), ex2_mufu(arg.y));
-                    float2 beta = __fmul2_rn(ww, Bv[jj]);
-                    if constexpr (ZOH)
-                        beta = zoh_beta2(arg, a, beta,
-                                         __fmul2_rn(__fmul2_rn(f2(uf[c][i], uf[c][i]), Bv[jj]), invA[c][jj]));
+                    float2 beta;
+                    if constexpr (ZOH)  // phi (u B), phi the hold weight per unit input
+                        beta = __fmul2_rn(zoh_phi2(arg, a, dd, invA[c][jj]),
+                                          __fmul2_rn(f2(uf[c][i], uf[c][i]), Bv[jj]));
+                    else
+                        beta = __fmul2_rn(ww, Bv[jj]);
                     h[c][jj] = __ffma2_rn(a, h[c][jj], beta);
                     acc = __ffma2_rn(Cv[jj], h[c][jj], acc);
                 }

@@ -173,9 +173,11 @@ __global__ void __launch_bounds__(WideCfg<N>::kWarps * 32, wide_min_blocks<N>())
                     for (int j = 0; j < NC / 2; ++j) {
                         const float2 arg = __fmul2_rn(dd2, A2[c][j]);
                         const float2 a = make_float2(ex2_mufu(arg.x), ex2_mufu(arg.y));
-                        float2 beta = __fmul2_rn(ww, Bv[j]);
-                        if constexpr (ZOH)
-                            beta = zoh_beta2(arg, a, beta, __fmul2_rn(__fmul2_rn(make_float2(ui, ui), Bv[j]), invA[c][j]));
+                        float2 beta;
+                        if constexpr (ZOH)  // phi (u B), phi the hold weight per unit input
+                            beta = __fmul2_rn(zoh_phi2(arg, a, dd2, invA[c][j]), __fmul2_rn(make_float2(ui, ui), Bv[j]));
+                        else
+                            beta = __fmul2_rn(ww, Bv[j]);
                         h[c][j] = __ffma2_rn(a, h[c][j], beta);
                         acc = __ffma2_rn(Cv[j], h[c][j], acc);
                     }

@@ -67,14 +67,28 @@ __device__ __forceinline__ float2 zoh_beta2(float2 y, float2 a, float2 wB, float
     return make_float2(fabsf(y.x) < kZohSmall ? small.x : big.x, fabsf(y.y) < kZohSmall ? small.y : big.y);
 }
 
+// The zero-order-hold weight per unit B u itself, phi = expm1(Delta A) / A, for a pair of chains,
+// from y = Delta A log2(e), a = 2^y, dt = Delta and invA = 1 / A:
+//   |y| >= kZohSmall:  (a - 1) / A = fma(a, invA, -invA)     (one rounding)
+//   |y| <  kZohSmall:  Delta (1 + x/2 + x^2/6 + x^3/24), x = y ln 2   (as zoh_beta2)
+// (the weight of zoh_beta2 without its factor u B, which the caller applies once).
+__device__ __forceinline__ float2 zoh_phi2(float2 y, float2 a, float2 dt, float2 invA) {
+    const float2 poly = __ffma2_rn(__ffma2_rn(__ffma2_rn(make_float2(kZohP3, kZohP3), y, make_float2(kZohP2, kZohP2)),
+                                              y, make_float2(kZohP1, kZohP1)),
+                                   y, make_float2(1.f, 1.f));
+    const float2 small = __fmul2_rn(dt, poly);
+    const float2 big = __ffma2_rn(a, invA, make_float2(-invA.x, -invA.y));
+    return make_float2(fabsf(y.x) < kZohSmall ? small.x : big.x, fabsf(y.y) < kZohSmall ? small.y : big.y);
+}
+
 // Derivative of the zero-order-hold weight per unit input, phi(Delta, A) = expm1(Delta A) / A,
 // with respect to A, for a pair of chains (the backward of the ZOH scan):
 //   dphi/dA = (Delta a - phi) / A                             for |y| >= kZohSmall,
 //           = Delta^2 (1/2 + x/3 + x^2/8 + x^3/30)              for |y| <  kZohSmall (x = y ln 2),
 // the second the Taylor series of the first (the k-th coefficient of (x e^x - e^x + 1) / x^2 is
 // 1 / (k! (k + 2)); the first term left out, x^4 / 144, is 2.1e-7 of the sum at |x| = 1/16), which avoids the
-// cancellation of Delta a - phi for small Delta A.  phi is the weight (zoh_beta2 with wB = Delta,
-// uB_over_A = 1 / A); the derivative with respect to Delta is a itself.
+// cancellation of Delta a - phi for small Delta A.  phi is the weight (zoh_phi2); the derivative
+// with respect to Delta is a itself.
 constexpr float kZohQ1 = kLn2 / 3.f, kZohQ2 = kLn2 * kLn2 / 8.f, kZohQ3 = kLn2 * kLn2 * kLn2 / 30.f;
 
 __device__ __forceinline__ float2 zoh_dphi_dA2(float2 y, float2 a, float2 dt, float2 phi, float2 invA) {
