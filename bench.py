@@ -198,12 +198,14 @@ _COMMENT = re.compile(r"//[^\n]*|/\*.*?\*/", re.S)
 
 
 def kernel_source_hash(kernel: str) -> str:
-    """Hash of the code (comments stripped) of the device sources a kernel family is built from."""
+    """Hash of the code (comments stripped, whitespace runs collapsed) of the device sources a
+    kernel family is built from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "selective_state_space_16_b200", "csrc")
     for f in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, f), encoding="utf-8") as fh:
-            h.update(f.encode() + _COMMENT.sub("", fh.read()).encode())
+            code = re.sub(r"\s+", " ", _COMMENT.sub("", fh.read())).strip()
+        h.update(f.encode() + code.encode())
     return h.hexdigest()[:16]
 
 

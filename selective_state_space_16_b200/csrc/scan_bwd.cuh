@@ -22,6 +22,9 @@
 //   g <- a_t g  (the gradient reaching h_{t-1}); after step 0 it is d initial_state
 //   ddelta_t = dDelta_t sigmoid(delta_t + bias)   (softplus' ; 1 without softplus)
 //
+// When the forward stored these checkpoints itself (ssm_fwd_options_t.checkpoints) the
+// forward sweep below is skipped and the walk reads them instead.
+//
 // Work split.  A CTA of 4 warps takes 32 consecutive channels of one batch row; a warp
 // takes 8 channels, 4 lanes per channel, each lane 4 of the 16 chains (as the forward
 // kernels), with the chain arithmetic in f32x2 pairs.  Each warp first runs the forward

@@ -32,7 +32,13 @@
 // the workspace to fp32 [t][32]; at most two batch rows per CTA) into shared memory
 // with TMA, through a ring of S stages signalled by mbarriers.  The 8-row u/delta/z
 // boxes use the 128-byte swizzle, so the per-lane 16-byte reads of one column hit
-// distinct banks; B/C are read as broadcasts.
+// distinct banks; B/C are read as broadcasts.  The kernel may be launched as a
+// programmatic dependent of the B/C transpose before it: the producer waits for that
+// grid only before its first B/C copy.
+//
+// Checkpoints (CK kernels, for the backward: [Tech] 四.1, keep a little in the forward
+// pass): after every group of steps that ends on a multiple of 8, each lane also stores
+// its chains, i.e. the state at the start of the next 8-step segment.
 #pragma once
 
 #include "common.cuh"
