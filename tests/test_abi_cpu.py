@@ -108,6 +108,26 @@ def test_forward_ex_rejects_unknown_algo(lib):
     assert rc == binding.SSM_ERR_INVALID_ARG
 
 
+def test_forward_checkpoint_options_are_validated(lib):
+    """Checkpoints (ABI 3) come from the sequential kernel only and must be 16-byte aligned;
+    both are checked before anything touches the device."""
+    def call(algo, ck, batch=1):
+        opts = binding.FwdOptions(algo, 0, 0, -1, 0, ck)
+        return lib.ssm_selective_scan_fwd_ex(P(4096), P(4096), P(4096), P(4096), P(4096), None, None, None, 1,
+                                             P(4096), None, batch, 1, 16, 8, binding.SSM_BF16, P(4096), 1 << 20,
+                                             ctypes.byref(opts), None)
+    assert call(binding.SSM_ALGO_CHUNKED, P(1 << 20)) == binding.SSM_ERR_UNSUPPORTED
+    assert call(binding.SSM_ALGO_DIRECT, P(1 << 20)) == binding.SSM_ERR_UNSUPPORTED
+    assert call(binding.SSM_ALGO_AUTO, P((1 << 20) + 8)) == binding.SSM_ERR_INVALID_ARG
+    assert call(binding.SSM_ALGO_AUTO, P(1 << 20), batch=0) == binding.SSM_OK
+    bopts = binding.BwdOptions(0, None, None, None, None, None, P((1 << 20) + 4))
+    rc = lib.ssm_selective_scan_bwd_ex(P(4096), P(4096), P(4096), P(4096), P(4096), None, None, None, 1, None,
+                                       P(4096), None, P(4096), P(4096), P(4096), P(4096), P(4096), None, None,
+                                       None, None, 2, 3, 16, 8, binding.SSM_BF16, P(4096), 1 << 30,
+                                       ctypes.byref(bopts), None)
+    assert rc == binding.SSM_ERR_INVALID_ARG
+
+
 def test_forward_state_argument_validation(lib):
     def call(h0, last, batch=2, dim=3):
         return lib.ssm_selective_scan_fwd_state(P(4096), P(4096), P(4096), P(4096), P(4096), None, None, None, 1,
