@@ -177,3 +177,23 @@ def test_checkpoints_unsupported_paths(cuda_device):
                                       ssm.new_workspace(b, d, 32, L), checkpoints=torch.zeros(b, 8, d, 32, device="cuda"),
                                       check=False)
     assert code == binding.SSM_ERR_UNSUPPORTED
+
+
+def test_backward_with_checkpoints_headline_shape(cuda_device):
+    # The Mamba-2.8B layer workload (batch 4, d_inner 5120, L 2048, bf16): the backward reading the
+    # forward's checkpoints agrees with the backward that recomputes them, every gradient, to the
+    # rounding of the fp32 states (the two forwards may split the chains over lanes differently).
+    w = workloads.WORKLOADS[2]
+    cpu = workloads.workload_inputs(w)
+    g = to_dev(cpu, "cuda")
+    dy = torch.randn(w.batch, w.dim, w.seqlen, generator=torch.Generator().manual_seed(460)).to(torch.bfloat16).cuda()
+    ck = _new_ckpt(w.batch, w.dim, w.seqlen)
+    ssm.selective_scan_fwd(**g, checkpoints=ck)
+    with_ck = ssm.selective_scan_bwd(**g, dy=dy, checkpoints=ck)
+    without = ssm.selective_scan_bwd(**g, dy=dy)
+    torch.cuda.synchronize()
+    assert torch.isfinite(ck).all()
+    for k in ["du", "ddelta", "dz", "dA", "dB", "dC", "dD", "ddelta_bias", "dinitial_state"]:
+        a, b = with_ck[k].double(), without[k].double()
+        err = float(((a - b).abs() / (1 + b.abs())).max())
+        assert err <= 2e-2, (k, err)
