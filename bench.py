@@ -413,8 +413,28 @@ def measure_unaligned(ssm, stream, pk, steps=10):
         ms = t / steps * 1e3
         assert ssm.ssm_read_status(ws) == 0
         out[f"L{L}"] = {"value": 4 * 5120 * L / (ms / 1e3) / 1e9, "ms_per_step": ms}
+        # the same from x through the fused conv1d (width 4) + SiLU
+        conv = {k: (v.cuda() if v is not None else None) for k, v in workloads.conv_inputs(4, 5120, 4, seed=5).items()}
+
+        def call():
+            ssm.ssm_selective_scan_fwd_conv(g["u"], conv["conv_weight"], conv["conv_bias"], g["delta"], g["A"], g["B"],
+                                            g["C"], g["D"], g["z"], g["delta_bias"], True, g["y"], g["last"], ws,
+                                            stream=stream)
+
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                call()
+            torch.cuda.synchronize()
+            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ev0.record(stream)
+            for _ in range(steps):
+                call()
+            ev1.record(stream)
+        torch.cuda.synchronize()
+        out[f"conv_L{L}"] = {"ms_per_step": ev0.elapsed_time(ev1) / steps}
         del g, ws
     out["ratio_2047_to_2048"] = out["L2047"]["ms_per_step"] / out["L2048"]["ms_per_step"]
+    out["conv_ratio_2047_to_2048"] = out["conv_L2047"]["ms_per_step"] / out["conv_L2048"]["ms_per_step"]
     return out
 
 

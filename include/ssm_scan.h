@@ -115,8 +115,8 @@ ssm_status_t ssm_workspace_init(void* workspace, size_t workspace_bytes, ssm_str
  * seqlen * sizeof(io element) is a multiple of 16 the tiles are staged with TMA straight
  * from u, delta and z; otherwise those are first copied into rows padded to a multiple of
  * 16 bytes inside the workspace (which is sized for this whenever seqlen % 8 != 0), and
- * SSM_ALGO_CHUNKED, the conv prologue and the no-allocation entry point run a direct-load
- * kernel instead.
+ * SSM_ALGO_CHUNKED, SSM_ALGO_DIRECT and the no-allocation entry point run a direct-load
+ * kernel instead (the conv prologue stages x in padded rows the same way).
  */
 ssm_status_t ssm_selective_scan_fwd(
     const void* u, const void* delta, const float* A, const void* B, const void* C,

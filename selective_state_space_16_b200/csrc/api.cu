@@ -27,9 +27,10 @@ bool dstate_supported(int n) { return n == 16 || n == 32 || n == 64 || n == 128 
 template <typename IO>
 constexpr int chunk_steps() { return 128 / static_cast<int>(sizeof(IO)); }
 
-// Rows of u / delta / z whose byte length is not a multiple of 16: TMA cannot address them,
-// so they are copied into padded rows in the workspace and the sequential kernel stages
-// those; y goes straight to the caller's rows with element stores.
+// Rows of u / delta / z (or x, with the conv prologue) whose byte length is not a multiple of
+// 16: TMA cannot address them, so they are copied into padded rows in the workspace and the
+// sequential kernel stages those; y (and u_out) go straight to the caller's rows with element
+// stores.
 template <typename IO>
 ssm_status_t launch_forward_padded(const FwdArgs& a, const ssm_fwd_options_t& o) {
     constexpr int64_t E = 16 / static_cast<int64_t>(sizeof(IO));
@@ -37,6 +38,7 @@ ssm_status_t launch_forward_padded(const FwdArgs& a, const ssm_fwd_options_t& o)
     FwdArgs pa = a;
     pa.L_rows = (a.L + E - 1) / E * E;
     pa.y_vec = 0;
+    pa.x_orig = a.u;  // with the conv prologue u holds x
     const long long rows = static_cast<long long>(a.batch) * a.dim;
     pa.u = a.ws + wl.pad_off;
     pa.delta = a.ws + wl.pad_off + wl.pad_array;
@@ -45,7 +47,7 @@ ssm_status_t launch_forward_padded(const FwdArgs& a, const ssm_fwd_options_t& o)
     void* const dst[3] = {const_cast<void*>(pa.u), const_cast<void*>(pa.delta), const_cast<void*>(pa.z)};
     const ssm_status_t st = launch_pad_rows<IO>(src, dst, a.z ? 3 : 2, rows, a.L, pa.L_rows, a.stream);
     if (st != SSM_OK) return st;
-    return a.zoh ? launch_seq_flagged<IO>(pa, o) : launch_seq_plain<IO>(pa, o);
+    return (a.zoh || a.conv.k > 0) ? launch_seq_flagged<IO>(pa, o) : launch_seq_plain<IO>(pa, o);
 }
 
 template <typename IO>
@@ -55,7 +57,7 @@ ssm_status_t launch_forward(const FwdArgs& a, const ssm_fwd_options_t& o) {
     const bool tma_ok = (static_cast<uint64_t>(a.L) * sizeof(IO)) % 16 == 0 && aligned16(a.u) &&
                         aligned16(a.delta) && aligned16(a.y) && (!a.z || aligned16(a.z));
     int algo = o.algo;
-    if (!tma_ok && a.pad_ok && a.conv.k == 0 && (algo == SSM_ALGO_AUTO || algo == SSM_ALGO_SEQUENTIAL))
+    if (!tma_ok && a.pad_ok && (algo == SSM_ALGO_AUTO || algo == SSM_ALGO_SEQUENTIAL))
         return launch_forward_padded<IO>(a, o);
     if (!tma_ok) algo = SSM_ALGO_DIRECT;
     if (a.ckpt && algo == SSM_ALGO_DIRECT) return SSM_ERR_UNSUPPORTED;  // checkpoints: sequential kernel only

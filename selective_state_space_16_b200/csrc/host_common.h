@@ -106,6 +106,7 @@ struct FwdArgs {
     bool pdl = false;    // the previous launch is the B/C pack: the scan may start early (it waits
                          // for the pack before reading the B/C rows, and reads nothing else it writes)
     float* ckpt = nullptr;  // checkpoints for the backward (batch, ceil(L/8), dim, 16), or null
+    const void* x_orig = nullptr;  // conv prologue on padded rows: the caller's x (rows of L)
 };
 
 // Backward workspace layout:

@@ -119,7 +119,7 @@ ssm_status_t launch_seq(const FwdArgs& a, const SeqPlan& pl) {
     p.softplus = a.softplus;
     p.has_z = a.z != nullptr;
     p.wait_limit = kDefaultWaitLimit;
-    p.x = a.u;
+    p.x = a.x_orig ? a.x_orig : a.u;  // the caller's x (the conv state-out reads its rows)
     p.conv_w = a.conv.w;
     p.conv_b = a.conv.b;
     p.conv_in = a.conv.in;

@@ -301,7 +301,7 @@ __device__ __forceinline__ void seq_consumer(uint8_t* smem, uint64_t* full_bar, 
             if (p.u_out && valid[0]) {
                 IO* urow = static_cast<IO*>(p.u_out) + (static_cast<long long>(b) * p.dim + d[0]) * p.L;
                 const int t0 = tk + nl * SPL;
-                if (t0 + SPL <= L32) {
+                if (p.y_vec && t0 + SPL <= L32) {  // (rows of u_out 16-byte aligned like those of y)
 #pragma unroll
                     for (int m = 0; m < SPL / GS; ++m) {
                         float v[GS];

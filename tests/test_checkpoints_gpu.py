@@ -76,8 +76,10 @@ def test_forward_checkpoints_zoh(cuda_device):
     assert_close(ck, _prefix_states(cpu, zoh=True), "f32", "zoh checkpoints")
 
 
-def test_forward_checkpoints_conv(cuda_device):
-    b, d, L = 2, 64, 160
+@pytest.mark.parametrize("L", [160, 157])
+def test_forward_checkpoints_conv(cuda_device, L):
+    # (L = 157: x staged in padded rows)
+    b, d = 2, 64
     cpu = workloads.scan_inputs(b, d, L, io="bf16", seed=430)
     conv = workloads.conv_inputs(b, d, 4, seed=431, with_state=True)
     g, c = to_dev(cpu, "cuda"), to_dev(conv, "cuda")
@@ -100,9 +102,7 @@ BWD_KEYS = ["ddelta", "dz", "dA", "dB", "dC", "dD", "ddelta_bias", "dinitial_sta
 @pytest.mark.parametrize("zoh,conv", [(False, False), (True, False), (False, True), (True, True)],
                          ids=["plain", "zoh", "conv", "zoh_conv"])
 def test_backward_with_forward_checkpoints(cuda_device, io, zoh, conv):
-    # the conv forward needs 16-byte rows for checkpoints (unaligned rows take the direct-load
-    # kernel, which stores none); the plain forward also stages ragged rows
-    b, d, L = 2, 70, (336 if conv else 333)
+    b, d, L = 2, 70, 333
     cpu = workloads.scan_inputs(b, d, L, io=io, seed=440)
     g = to_dev(cpu, "cuda")
     h0 = workloads.initial_state(b, d, seed=441)
@@ -162,14 +162,6 @@ def test_checkpoints_unsupported_paths(cuda_device):
                                           g["delta_bias"], True, y, last, ws, algo="sequential",
                                           lanes_per_channel=lanes, checkpoints=ck, check=False)
         assert code == binding.SSM_ERR_UNSUPPORTED, lanes
-    # conv with rows that are not 16-byte multiples runs the direct-load kernel
-    conv = to_dev(workloads.conv_inputs(b, d, 4, seed=452), "cuda")
-    odd = to_dev(workloads.scan_inputs(b, d, 63, io="bf16", seed=453), "cuda")
-    code = ssm.ssm_selective_scan_fwd_conv(odd["u"], conv["conv_weight"], conv["conv_bias"], odd["delta"], odd["A"],
-                                           odd["B"], odd["C"], odd["D"], odd["z"], odd["delta_bias"], True,
-                                           torch.empty_like(odd["u"]), last, ssm.new_workspace(b, d, 16, 63),
-                                           checkpoints=_new_ckpt(b, d, 63), check=False)
-    assert code == binding.SSM_ERR_UNSUPPORTED
     wide = workloads.scan_inputs(b, d, L, dstate=32, io="bf16", seed=451)
     gw = to_dev(wide, "cuda")
     code = ssm.ssm_selective_scan_fwd(gw["u"], gw["delta"], gw["A"], gw["B"], gw["C"], gw["D"], gw["z"],
