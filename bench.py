@@ -265,6 +265,22 @@ def forward_buffers(w, dev):
     return inp, g
 
 
+def time_calls(fn, stream, steps, warmup=3):
+    """Milliseconds per call of fn() (which launches on `stream`): `warmup` untimed calls, then
+    `steps` calls between two CUDA events recorded on that stream."""
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(steps):
+            fn()
+        ev1.record(stream)
+    torch.cuda.synchronize()
+    return ev0.elapsed_time(ev1) / steps
+
+
 def e2e_forward(ssm, w, inp, y_ref, steps, stream, nstreams=4, chunks_per_row=1):
     """Same metric through the public C-ABI call with HOST (pinned) buffers: every step
     copies all inputs host->device, runs the scan and copies y and the final state back.
@@ -380,16 +396,8 @@ def measure_decode(ssm, stream, pk, steps=None):
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
         chain(nsteps)
-    with torch.cuda.stream(stream):  # replay() launches on the current stream
-        graph.replay()
-        torch.cuda.synchronize()
-        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        ev0.record(stream)
-        graph.replay()
-        ev1.record(stream)
-    torch.cuda.synchronize()
-    t = ev0.elapsed_time(ev1) / 1e3
-    per_step = t / nsteps
+    # replay() launches on the current stream, which time_calls makes `stream`
+    per_step = time_calls(graph.replay, stream, 1, warmup=1) / 1e3 / nsteps
     gbs = decode_algorithmic_bytes(w) / per_step / 1e9
     del graph
     return {"workload": w.name, "value": w.batch * w.dim / per_step / 1e9, "unit": "Gelem/s (B*D per step)",
@@ -421,17 +429,7 @@ def measure_unaligned(ssm, stream, pk, steps=10):
                                             g["C"], g["D"], g["z"], g["delta_bias"], True, g["y"], g["last"], ws,
                                             stream=stream)
 
-        with torch.cuda.stream(stream):
-            for _ in range(3):
-                call()
-            torch.cuda.synchronize()
-            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            ev0.record(stream)
-            for _ in range(steps):
-                call()
-            ev1.record(stream)
-        torch.cuda.synchronize()
-        out[f"conv_L{L}"] = {"ms_per_step": ev0.elapsed_time(ev1) / steps}
+        out[f"conv_L{L}"] = {"ms_per_step": time_calls(call, stream, steps)}
         del g, ws
     out["ratio_2047_to_2048"] = out["L2047"]["ms_per_step"] / out["L2048"]["ms_per_step"]
     out["conv_ratio_2047_to_2048"] = out["conv_L2047"]["ms_per_step"] / out["conv_L2048"]["ms_per_step"]
@@ -463,17 +461,7 @@ def measure_conv(ssm, stream, pk, steps=10):
                                         g["C"], g["D"], g["z"], g["delta_bias"], True, g["y"], g["last"], ws,
                                         stream=stream)
 
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            call()
-        torch.cuda.synchronize()
-        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        ev0.record(stream)
-        for _ in range(steps):
-            call()
-        ev1.record(stream)
-    torch.cuda.synchronize()
-    ms = ev0.elapsed_time(ev1) / steps
+    ms = time_calls(call, stream, steps)
     del g
     return {"workload": w.name, "prologue": "causal conv1d width 4 + SiLU, fused", "value": w.elements / (ms / 1e3) / 1e9,
             "unit": UNIT, "ms_per_step": ms}
@@ -502,17 +490,7 @@ def measure_wide(ssm, stream, pk, steps=5, only=None):
             ssm.ssm_selective_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"],
                                        True, y, last, ws, stream=stream)
 
-        with torch.cuda.stream(stream):
-            for _ in range(3):
-                call()
-            torch.cuda.synchronize()
-            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            ev0.record(stream)
-            for _ in range(steps):
-                call()
-            ev1.record(stream)
-        torch.cuda.synchronize()
-        ms = ev0.elapsed_time(ev1) / steps
+        ms = time_calls(call, stream, steps)
         assert ssm.ssm_read_status(ws) == 0
         rate = bsz * dim * L / (ms / 1e3) / 1e9
         out[f"N{n}"] = {"ms_per_step": ms, "value": rate, "roofline_value": ex2_peak / n,
@@ -541,17 +519,7 @@ def measure_backward(ssm, stream, pk, steps=5):
                                    dy, du, ddelta, dA, dB, dC, dD, dz, dbias, ws, stream=stream)
 
     def timed(fn):
-        with torch.cuda.stream(stream):
-            for _ in range(2):
-                fn()
-            torch.cuda.synchronize()
-            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            ev0.record(stream)
-            for _ in range(steps):
-                fn()
-            ev1.record(stream)
-        torch.cuda.synchronize()
-        return ev0.elapsed_time(ev1) / steps
+        return time_calls(fn, stream, steps, warmup=2)
 
     ms = timed(call)
     # the same with the zero-order hold and the conv prologue (width 4, carried-in state):
