@@ -25,7 +25,7 @@
 // When the forward stored these checkpoints itself (ssm_fwd_options_t.checkpoints) the
 // forward sweep below is skipped and the walk reads them instead.
 //
-// Work split.  A CTA of 4 warps takes 32 consecutive channels of one batch row; a warp
+// Work split.  A CTA of 3 warps takes 24 consecutive channels of one batch row; a warp
 // takes 8 channels, 4 lanes per channel, each lane 4 of the 16 chains (as the forward
 // kernels), with the chain arithmetic in f32x2 pairs.  Each warp first runs the forward
 // over the whole sequence and stores the state at the start of every 8-step segment
@@ -65,8 +65,9 @@
 namespace ssm {
 
 constexpr int kBwdSeg = 8;       // steps per segment (checkpoint interval)
-constexpr int kBwdWarps = 4;     // warps per CTA (5 CTAs per SM: the headline's CTAs in one wave;
-                                 // the conv variants spill a little to stay at 96 registers)
+constexpr int kBwdWarps = 3;     // warps per CTA: 6 CTAs (18 warps) per SM at 96 registers, so a
+                                 // shape's CTAs spread evenly (the headline's 856 give every SM 5
+                                 // or 6; 4-warp CTAs gave 48 SMs 5 and 100 SMs 4, idling those)
 constexpr int kBwdChannels = kBwdWarps * 8;
 constexpr int kBwdRing = 4;      // segments of B/C rows in flight (cp.async ring)
 // dynamic shared memory of scan_bwd_kernel: h stage, dB/dC stage, B/C ring (sized for
@@ -114,7 +115,7 @@ __device__ __forceinline__ float load_io(const void* base, long long i) {
 }
 
 template <typename IO, bool ZOH, bool CONV>
-__global__ void __launch_bounds__(kBwdWarps * 32, 5) scan_bwd_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(kBwdWarps * 32, 6) scan_bwd_kernel(const BwdParams p) {
     constexpr int T = kBwdSeg, G = 4, PER = T / G, R = kBwdRing;
     extern __shared__ float4 bwd_smem[];
     // h_{t-1} of the segment's steps: [warp][step][lane] (16 bytes each)
