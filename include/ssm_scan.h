@@ -113,10 +113,14 @@ ssm_status_t ssm_workspace_init(void* workspace, size_t workspace_bytes, ssm_str
  *                            used by two calls that can overlap on the GPU.
  * All tensor pointers must be 16-byte aligned.  Any seqlen >= 0 is accepted; when
  * seqlen * sizeof(io element) is a multiple of 16 the tiles are staged with TMA straight
- * from u, delta and z; otherwise those are first copied into rows padded to a multiple of
- * 16 bytes inside the workspace (which is sized for this whenever seqlen % 8 != 0), and
- * SSM_ALGO_CHUNKED, SSM_ALGO_DIRECT and the no-allocation entry point run a direct-load
- * kernel instead (the conv prologue stages x in padded rows the same way).
+ * from u, delta and z (x with the conv prologue).  Otherwise TMA cannot address the rows:
+ * the sequential kernel's warps then copy their rows' 16-byte-aligned windows themselves
+ * and shift them into place (SSM_ALGO_SEQUENTIAL, the no-allocation entry point, and
+ * SSM_ALGO_AUTO on shapes with about 8 or more 8-channel tiles per SM), or u, delta and z
+ * are first copied into rows padded to a multiple of 16 bytes inside the workspace (which
+ * is sized for this whenever seqlen % 8 != 0: SSM_ALGO_AUTO on smaller shapes, with
+ * checkpoints, or with lanes_per_channel 2 or 42); SSM_ALGO_CHUNKED and SSM_ALGO_DIRECT run
+ * a direct-load kernel.
  */
 ssm_status_t ssm_selective_scan_fwd(
     const void* u, const void* delta, const float* A, const void* B, const void* C,

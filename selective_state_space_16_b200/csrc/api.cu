@@ -57,8 +57,27 @@ ssm_status_t launch_forward(const FwdArgs& a, const ssm_fwd_options_t& o) {
     const bool tma_ok = (static_cast<uint64_t>(a.L) * sizeof(IO)) % 16 == 0 && aligned16(a.u) &&
                         aligned16(a.delta) && aligned16(a.y) && (!a.z || aligned16(a.z));
     int algo = o.algo;
-    if (!tma_ok && a.pad_ok && (algo == SSM_ALGO_AUTO || algo == SSM_ALGO_SEQUENTIAL))
-        return launch_forward_padded<IO>(a, o);
+    if (!tma_ok && (algo == SSM_ALGO_AUTO || algo == SSM_ALGO_SEQUENTIAL)) {
+        // Unaligned rows: the sequential kernel either gathers them itself (GA kernels) or
+        // stages a padded copy.  Gathering costs the consumer warps ~20% (shared-memory traffic)
+        // but saves the copy; measured on B200 it wins when the shape gives every SM about 8 or
+        // more 8-channel tiles (b4 d5120 L2047: 0.376 against 0.429 ms) and loses with fewer
+        // (b1 d5120 L32767, 4.3 tiles per SM: 2.98 against 2.47 ms).  SEQUENTIAL, and callers
+        // without room for padded rows, always gather; checkpoints and 2 lanes per channel or
+        // two channels per lane (not built as GA kernels) come from the padded copy.
+        const double tiles_per_sm = static_cast<double>(a.batch) * ((a.dim + 7) / 8) / a.sm_count;
+        const bool ga_variant = o.lanes_per_channel != 2 && o.lanes_per_channel != 42;
+        const bool gather =
+            !a.ckpt && ga_variant && (algo == SSM_ALGO_SEQUENTIAL || !a.pad_ok || tiles_per_sm >= 8.0);
+        if (!gather) {
+            if (!a.pad_ok) return SSM_ERR_UNSUPPORTED;
+            return launch_forward_padded<IO>(a, o);
+        }
+        FwdArgs g = a;
+        g.y_vec = 0;
+        g.pdl = true;  // launched right after the B/C pack
+        return launch_seq_gather<IO>(g, o);
+    }
     if (!tma_ok) algo = SSM_ALGO_DIRECT;
     if (a.ckpt && algo == SSM_ALGO_DIRECT) return SSM_ERR_UNSUPPORTED;  // checkpoints: sequential kernel only
     if (a.ckpt && algo == SSM_ALGO_AUTO) algo = SSM_ALGO_SEQUENTIAL;
@@ -338,7 +357,7 @@ ssm_status_t ssm_selective_scan_fwd_noalloc(const void* u, const void* delta, co
     const ssm_fwd_options_t o{SSM_ALGO_SEQUENTIAL, 0, 0, -1, SSM_DISC_SIMPLIFIED};
     FwdArgs a{u, delta, B, C, z, A, D, delta_bias, softplus, nullptr, 0, y, last_state, batch, dim, seqlen,
               io_dtype, scratch, s, sm_count};
-    a.pad_ok = false;  // the fixed scratch has no room for padded rows: unaligned L runs the direct kernel
+    a.pad_ok = false;  // the fixed scratch has no room for padded rows: unaligned rows are gathered
     return io_dtype == SSM_BF16 ? launch_forward<__nv_bfloat16>(a, o) : launch_forward<float>(a, o);
 }
 

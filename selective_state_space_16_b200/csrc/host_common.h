@@ -172,6 +172,7 @@ template <typename IO> ssm_status_t launch_seq_plain(const FwdArgs& a, const ssm
 template <typename IO> ssm_status_t launch_seq_flagged(const FwdArgs& a, const ssm_fwd_options_t& o);
 // Sequential family storing checkpoints for the backward, every variant (fwd_seq_ckpt_*.cu).
 template <typename IO> ssm_status_t launch_seq_ckpt(const FwdArgs& a, const ssm_fwd_options_t& o);
+template <typename IO> ssm_status_t launch_seq_gather(const FwdArgs& a, const ssm_fwd_options_t& o);
 // d_state 32 .. 256 forward (wide.cu).
 template <typename IO> ssm_status_t launch_wide(const FwdArgs& a, int n);
 // Backward (bwd.cu).

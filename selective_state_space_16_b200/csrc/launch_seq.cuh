@@ -11,12 +11,17 @@
 
 namespace ssmh {
 
-template <typename IO, int G, int CPL, bool ZOH, bool CONV = false, bool CK = false>
+template <typename IO, int G, int CPL, bool ZOH, bool CONV = false, bool CK = false, bool GA = false>
 const void* seq_kernel_ptr(int stages) {
-    switch (stages) {
-        case 2: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 2, ZOH, CONV, CK>);
-        case 3: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 3, ZOH, CONV, CK>);
-        default: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 4, ZOH, CONV, CK>);
+    if constexpr (GA) {  // (gathered rows: rings of 3 or 4 stages)
+        if (stages == 3) return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 3, ZOH, CONV, CK, true>);
+        return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 4, ZOH, CONV, CK, true>);
+    } else {
+        switch (stages) {
+            case 2: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 2, ZOH, CONV, CK>);
+            case 3: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 3, ZOH, CONV, CK>);
+            default: return reinterpret_cast<const void*>(ssm::scan_fwd_seq_kernel<IO, G, CPL, 4, ZOH, CONV, CK>);
+        }
     }
 }
 
@@ -29,7 +34,7 @@ struct SeqPlan {
     bool ok = false;
 };
 
-template <typename IO, int G, int CPL, bool ZOH = false, bool CONV = false, bool CK = false>
+template <typename IO, int G, int CPL, bool ZOH = false, bool CONV = false, bool CK = false, bool GA = false>
 SeqPlan plan_seq(const FwdArgs& a) {
     using Cfg = ssm::SeqCfg<IO, G, CPL>;
     SeqPlan pl;
@@ -48,11 +53,12 @@ SeqPlan plan_seq(const FwdArgs& a) {
             mt = tiles_cap;  // several rounds per CTA
         }
         const int budget = (228 * 1024) / per_sm - 1024 - 256;  // per-CTA reserve and static barriers
-        const int stages = std::min(4, (budget - 1024) / Cfg::stage_bytes(mt));
-        if (stages < 2) continue;
+        const int info = GA ? Cfg::gather_info_bytes(mt) : 0;  // (gathered rows: one word per row)
+        const int stages = std::min(4, (budget - 1024 - info) / Cfg::stage_bytes(mt));
+        if (stages < (GA ? 3 : 2)) continue;
         const int threads = (Cfg::warps_for(mt) + 1) * 32;
-        const int smem = Cfg::smem_bytes(mt, stages);
-        const void* kern = seq_kernel_ptr<IO, G, CPL, ZOH, CONV, CK>(stages);
+        const int smem = Cfg::smem_bytes(mt, stages) + info;
+        const void* kern = seq_kernel_ptr<IO, G, CPL, ZOH, CONV, CK, GA>(stages);
         int occ = 0;
         if (!ensure_smem_attr(kern, smem) ||
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, smem) != cudaSuccess || occ < per_sm)
@@ -84,7 +90,7 @@ double predict_seq(const FwdArgs& a, const SeqPlan& pl) {
     return tiles * cost / hide;
 }
 
-template <typename IO, int G, int CPL, bool ZOH = false, bool CONV = false, bool CK = false>
+template <typename IO, int G, int CPL, bool ZOH = false, bool CONV = false, bool CK = false, bool GA = false>
 ssm_status_t launch_seq(const FwdArgs& a, const SeqPlan& pl) {
     using Cfg = ssm::SeqCfg<IO, G, CPL>;
     if (!pl.ok) return SSM_ERR_UNSUPPORTED;
@@ -95,12 +101,16 @@ ssm_status_t launch_seq(const FwdArgs& a, const SeqPlan& pl) {
     CUtensorMap mu, mdl, mz, mbc;
     const uint64_t L = static_cast<uint64_t>(a.L);
     const uint64_t Lr = static_cast<uint64_t>(a.L_rows ? a.L_rows : a.L);  // row length of u / delta / z
-    bool ok = make_map_3d(&mu, dt, es, a.u, Lr, a.dim, a.batch, TC, 8, sw128) &&
-              make_map_3d(&mdl, dt, es, a.delta, Lr, a.dim, a.batch, TC, 8, sw128) &&
-              make_map_3d(&mbc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.ws + ws_layout(a.batch, a.dim, a.L).bc_off, 32,
+    bool ok = make_map_3d(&mbc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.ws + ws_layout(a.batch, a.dim, a.L).bc_off, 32,
                           L, a.batch, 32, TC, CU_TENSOR_MAP_SWIZZLE_NONE);
-    if (ok && a.z) ok = make_map_3d(&mz, dt, es, a.z, Lr, a.dim, a.batch, TC, 8, sw128);
-    if (!a.z) mz = mu;
+    if (GA) {  // the kernel reads u / delta / z itself; the maps are placeholders
+        mu = mdl = mz = mbc;
+    } else {
+        ok = ok && make_map_3d(&mu, dt, es, a.u, Lr, a.dim, a.batch, TC, 8, sw128) &&
+             make_map_3d(&mdl, dt, es, a.delta, Lr, a.dim, a.batch, TC, 8, sw128);
+        if (ok && a.z) ok = make_map_3d(&mz, dt, es, a.z, Lr, a.dim, a.batch, TC, 8, sw128);
+        if (!a.z) mz = mu;
+    }
     if (!ok) return SSM_ERR_LAUNCH;
     ssm::SeqParams p{};
     p.A = a.A;
@@ -127,6 +137,9 @@ ssm_status_t launch_seq(const FwdArgs& a, const SeqPlan& pl) {
     p.u_out = a.conv.u_out;
     p.conv_k = a.conv.k;
     p.y_vec = a.y_vec;
+    p.u_rows = a.u;
+    p.dl_rows = a.delta;
+    p.z_rows = a.z;
     p.ckpt = a.ckpt;
     p.nseg = static_cast<int>((a.L + 7) / 8);
     if (a.L >= (1LL << 31) - 1024) return SSM_ERR_UNSUPPORTED;
@@ -143,10 +156,17 @@ ssm_status_t launch_seq(const FwdArgs& a, const SeqPlan& pl) {
     cfg.attrs = attr;
     cfg.numAttrs = a.pdl ? 1 : 0;
     cudaError_t e;
-    switch (pl.stages) {
-        case 2: e = cudaLaunchKernelEx(&cfg, ssm::scan_fwd_seq_kernel<IO, G, CPL, 2, ZOH, CONV, CK>, mu, mdl, mz, mbc, p); break;
-        case 3: e = cudaLaunchKernelEx(&cfg, ssm::scan_fwd_seq_kernel<IO, G, CPL, 3, ZOH, CONV, CK>, mu, mdl, mz, mbc, p); break;
-        default: e = cudaLaunchKernelEx(&cfg, ssm::scan_fwd_seq_kernel<IO, G, CPL, 4, ZOH, CONV, CK>, mu, mdl, mz, mbc, p); break;
+    if constexpr (GA) {
+        if (pl.stages == 3)
+            e = cudaLaunchKernelEx(&cfg, ssm::scan_fwd_seq_kernel<IO, G, CPL, 3, ZOH, CONV, CK, true>, mu, mdl, mz, mbc, p);
+        else
+            e = cudaLaunchKernelEx(&cfg, ssm::scan_fwd_seq_kernel<IO, G, CPL, 4, ZOH, CONV, CK, true>, mu, mdl, mz, mbc, p);
+    } else {
+        switch (pl.stages) {
+            case 2: e = cudaLaunchKernelEx(&cfg, ssm::scan_fwd_seq_kernel<IO, G, CPL, 2, ZOH, CONV, CK>, mu, mdl, mz, mbc, p); break;
+            case 3: e = cudaLaunchKernelEx(&cfg, ssm::scan_fwd_seq_kernel<IO, G, CPL, 3, ZOH, CONV, CK>, mu, mdl, mz, mbc, p); break;
+            default: e = cudaLaunchKernelEx(&cfg, ssm::scan_fwd_seq_kernel<IO, G, CPL, 4, ZOH, CONV, CK>, mu, mdl, mz, mbc, p); break;
+        }
     }
     if (e != cudaSuccess) {
         (void)cudaGetLastError();
@@ -217,5 +237,31 @@ ssm_status_t launch_seq_ckpt(const FwdArgs& a, const ssm_fwd_options_t& o) {
 }
 extern template ssm_status_t launch_seq_ckpt<__nv_bfloat16>(const FwdArgs&, const ssm_fwd_options_t&);
 extern template ssm_status_t launch_seq_ckpt<float>(const FwdArgs&, const ssm_fwd_options_t&);
+
+// Rows of u / delta / z (or x) whose byte length is not a multiple of 16: the GA kernels, which
+// gather the rows themselves (4 or 8 lanes per channel, one channel per lane), for every
+// discretisation / prologue combination without checkpoints.  Instantiated only in
+// fwd_seq_gather_*.cu.
+template <typename IO, bool ZOH, bool CONV>
+ssm_status_t launch_gather_g(const FwdArgs& a, const ssm_fwd_options_t& o) {
+    const SeqPlan p4 = plan_seq<IO, 4, 1, ZOH, CONV, false, true>(a);
+    if constexpr (sizeof(IO) == 2) {
+        const SeqPlan p8 = plan_seq<IO, 8, 1, ZOH, CONV, false, true>(a);
+        const bool use8 = o.lanes_per_channel == 8 ||
+                          (o.lanes_per_channel == 0 && predict_seq<IO, 8, 1>(a, p8) < predict_seq<IO, 4, 1>(a, p4));
+        if (use8) return launch_seq<IO, 8, 1, ZOH, CONV, false, true>(a, p8);
+    }
+    return launch_seq<IO, 4, 1, ZOH, CONV, false, true>(a, p4);
+}
+template <typename IO>
+ssm_status_t launch_seq_gather(const FwdArgs& a, const ssm_fwd_options_t& o) {
+    if (o.lanes_per_channel != 0 && o.lanes_per_channel != 4 && o.lanes_per_channel != 8) return SSM_ERR_UNSUPPORTED;
+    if (a.zoh && a.conv.k > 0) return launch_gather_g<IO, true, true>(a, o);
+    if (a.zoh) return launch_gather_g<IO, true, false>(a, o);
+    if (a.conv.k > 0) return launch_gather_g<IO, false, true>(a, o);
+    return launch_gather_g<IO, false, false>(a, o);
+}
+extern template ssm_status_t launch_seq_gather<__nv_bfloat16>(const FwdArgs&, const ssm_fwd_options_t&);
+extern template ssm_status_t launch_seq_gather<float>(const FwdArgs&, const ssm_fwd_options_t&);
 
 }  // namespace ssmh

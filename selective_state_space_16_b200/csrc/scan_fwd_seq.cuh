@@ -71,8 +71,13 @@ struct SeqParams {
     void* u_out;               // (batch, dim, L) IO: the conv output, or null
     int conv_k;                // 1 .. 4
     // y rows are 16-byte aligned (L * sizeof(IO) a multiple of 16): vector stores; else
-    // element stores (the inputs were then staged into padded rows, see pad_rows_kernel)
+    // element stores
     int y_vec;
+    // u / delta / z themselves, for the GA kernels (rows whose byte length is not a multiple of
+    // 16, which TMA cannot address: see gather_copy); their tensor maps are then unused
+    const void* u_rows;
+    const void* dl_rows;
+    const void* z_rows;
     // checkpoints for the backward, or null: (batch, nseg, dim, 16) fp32, the state at the
     // start of every 8-step segment (h before step 8s), nseg = ceil(L / 8)
     float* ckpt;
@@ -107,6 +112,8 @@ struct SeqCfg {
     __host__ __device__ static constexpr int smem_bytes(int max_tiles, int stages) {
         return stages * stage_bytes(max_tiles) + 1024;  // +1024: alignment slack
     }
+    // GA kernels: one 8-byte word per u / delta / z row of a round after the ring (gather_row_info)
+    __host__ __device__ static constexpr int gather_info_bytes(int max_tiles) { return max_tiles * 8 * 3 * 8; }
 };
 
 __device__ __forceinline__ float2 f2(float x, float y) { return make_float2(x, y); }
@@ -151,6 +158,107 @@ __device__ __forceinline__ void store_run(IO* dst, const float (&v)[N]) {
     }
 }
 
+// Gathered rows (GA kernels: rows of u / delta / z whose byte length is not a multiple of 16,
+// which TMA cannot address).  Every consumer warp stages its own channels' rows itself, so
+// the copies are spread over all warps (a single warp issuing them for the whole CTA fell
+// behind the consumers):
+//  * Row q of a round (tensor q / (nt * 8): u, delta, z; channel q % (nt * 8) of the round) is
+//    described by one word set up at the start of the round, the address of its step 0
+//    (0: no such row).  Its bytes sh = address & 15 before step 0 are the row's offset from the
+//    16-byte grid; the window of stage k is the 128 bytes from (address & ~15) + k * 128.
+//  * gather_copy copies a stage's windows with cp.async into the rows' 128-byte slots of the
+//    tile area, unswizzled, three stages ahead.  Chunks holding no byte of the row's steps
+//    0 .. L - 1 are zero-filled, not read (so nothing outside the caller's arrays, rounded to
+//    16 bytes, is read).  One more stage is copied past the last (the chunks holding the last
+//    step's bytes beyond the last window).
+//  * gather_align, once stage k and k + 1 have landed, shifts the warp's rows of stage k into
+//    place: lane (sub, c) takes window chunks c and c + 1 (chunk 8 is chunk 0 of the next
+//    stage's window, not yet shifted), extracts bytes sh .. sh + 15 and writes them where the
+//    128-byte-swizzled TMA box would have put chunk c (row r of a tile: ((c ^ r) << 4)).
+//    Steps at or past L come out zero, as TMA fills them.
+template <typename IO>
+__device__ __forceinline__ uint64_t gather_row_info(const SeqParams& p, int q, int rows, int j0, int b_first) {
+    const int tq = q >= rows ? (q >= 2 * rows ? 2 : 1) : 0;
+    const int rr = q - tq * rows;
+    const int jt = j0 + (rr >> 3);  // the round's tiles span at most two batch rows
+    const int second = jt >= p.tiles_per_batch ? 1 : 0;
+    const int b = b_first + second;
+    const int d = (jt - second * p.tiles_per_batch) * 8 + (rr & 7);
+    if (d >= p.dim || b >= p.batch) return 0;
+    const uint8_t* base = static_cast<const uint8_t*>(tq == 0 ? p.u_rows : tq == 1 ? p.dl_rows : p.z_rows);
+    return reinterpret_cast<uint64_t>(base + (static_cast<long long>(b) * p.dim + d) * p.L *
+                                                 static_cast<long long>(IoTraits<IO>::kBytes));
+}
+
+// Consumer warp `warp`: copy its rows' windows of stage k (0 <= k <= the number of stages) into
+// the slot st.  row_bytes = L * sizeof(IO).
+template <int CPW, int NT>
+__device__ __forceinline__ void gather_copy(uint8_t* st, const uint64_t* info, const SeqParams& p, int rows,
+                                            long long k, long long row_bytes, int warp, int lane) {
+    const int sub = lane >> 3, c = lane & 7;
+    const int tile_area = p.max_tiles * 1024;
+    const uint8_t* any = static_cast<const uint8_t*>(p.u_rows);  // (zero-fill: not read)
+#pragma unroll
+    for (int r0 = 0; r0 < CPW * NT; r0 += 4) {
+        const int tq = r0 / CPW;  // (CPW is a multiple of 4: the 4 rows of a pass share a tensor)
+        const int cl = warp * CPW + r0 % CPW + sub;
+        if (cl < rows && dcheck(p.hdr, tq * tile_area + cl * 128 + 128 <= 3 * tile_area, kSiteSeqTma, cl)) {
+            const uint64_t at = info[tq * rows + cl];
+            const long long sh = static_cast<long long>(at & 15u);
+            const bool need = at != 0 && k * 128 - sh + c * 16 < row_bytes;  // the chunk holds a step byte
+            const uint8_t* src = need ? reinterpret_cast<const uint8_t*>(at - sh) + k * 128 + c * 16 : any;
+            cp_async_16(st + tq * tile_area + cl * 128 + c * 16, src, need ? 16u : 0u);
+        }
+    }
+}
+
+// Consumer warp `warp`: shift its rows of the landed stage st into place (nx_st: the slot of
+// the next stage, also landed; nbytes: bytes of the stage's steps in a row).  Lane c reads the
+// 24 bytes from window byte 16c + (sh & 8) as three 8-byte words (those past byte 128 from the
+// next stage's window), keeps the words from (sh & 4) on and funnel-shifts by sh & 3.
+template <int CPW, int NT>
+__device__ __forceinline__ void gather_align(uint8_t* st, const uint8_t* nx_st, const uint64_t* info,
+                                             const SeqParams& p, int rows, int nbytes, int warp, int lane) {
+    const int sub = lane >> 3, c = lane & 7;
+    const int keep = nbytes - c * 16;  // bytes of this lane's chunk inside the row's steps
+    const int tile_area = p.max_tiles * 1024;
+    const long long nx_delta = nx_st - st;
+#pragma unroll
+    for (int r0 = 0; r0 < CPW * NT; r0 += 4) {
+        const int tq = r0 / CPW;
+        const int cl = warp * CPW + r0 % CPW + sub;  // channel of the round
+        const bool mine = cl < rows && dcheck(p.hdr, tq * tile_area + cl * 128 + 128 <= 3 * tile_area, kSiteSeqTma, cl);
+        const uint64_t at = mine ? info[tq * rows + cl] : 0;
+        const uint32_t sh = static_cast<uint32_t>(at & 15u);
+        uint8_t* rowp = st + tq * tile_area + cl * 128;
+        uint2 w[3] = {make_uint2(0u, 0u), make_uint2(0u, 0u), make_uint2(0u, 0u)};
+        if (mine) {
+#pragma unroll
+            for (int i = 0; i < 3; ++i) {
+                const int b = c * 16 + static_cast<int>(sh & 8u) + 8 * i;  // window byte (8-aligned)
+                const uint8_t* src = rowp + (b < 128 ? b : b - 128 + nx_delta);
+                w[i] = *reinterpret_cast<const uint2*>(src);
+            }
+        }
+        __syncwarp();  // every lane has read its words before any lane rewrites the row
+        const uint32_t x[6] = {w[0].x, w[0].y, w[1].x, w[1].y, w[2].x, w[2].y};
+        uint32_t u5[5], o[4];
+#pragma unroll
+        for (int i = 0; i < 5; ++i) u5[i] = (sh & 4u) ? x[i + 1] : x[i];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) o[m] = __funnelshift_r(u5[m], u5[m + 1], (sh & 3u) * 8u);
+        if (keep < 16) {
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int kb = keep - 4 * m;
+                o[m] = kb >= 4 ? o[m] : kb <= 0 ? 0u : o[m] & ((1u << (8 * kb)) - 1u);
+            }
+        }
+        if (mine) *reinterpret_cast<uint4*>(rowp + ((c ^ (cl & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    __syncwarp();
+}
+
 // Consumer warp of the sequential kernel (HZ: the z gate is present).
 //
 // Lane (cg, nl) holds the NC chains n = nl*NC .. of the channels cg + c*CW (c < CPL) of
@@ -159,7 +267,7 @@ __device__ __forceinline__ void store_run(IO* dst, const float (&v)[N]) {
 // of a stage are unrolled (compile-time shared-memory offsets) with ping-pong step-size
 // buffers: the step sizes of group g+1 (for the last group: group 0 of the next stage,
 // after waiting for it) are computed while group g is scanned.
-template <typename IO, int G, int CPL, int S, bool HZ, bool ZOH, bool CONV, bool CK>
+template <typename IO, int G, int CPL, int S, bool HZ, bool ZOH, bool CONV, bool CK, bool GA>
 __device__ __forceinline__ void seq_consumer(uint8_t* smem, uint64_t* full_bar, uint64_t* empty_bar,
                                              const int* abort_flag, const SeqParams& p, long long r_begin, int nt,
                                              int b_first, int stage_bytes, int nstages, int L32) {
@@ -441,8 +549,32 @@ __device__ __forceinline__ void seq_consumer(uint8_t* smem, uint64_t* full_bar, 
     const uint8_t* st = smem;
     int slot = 0;
     uint32_t parity = 0;
+    // GA: this warp's rows, copied three stages ahead (the copies of stage k land in a cp.async
+    // group of their own), shifted into place when a stage and the next have landed
+    const uint64_t* ginfo = reinterpret_cast<const uint64_t*>(smem + S * stage_bytes);
+    auto issue_stage = [&](int kk) {
+        if constexpr (GA) {
+            if (kk <= nstages) {  // (stage nstages: the chunks past the last window)
+                gather_copy<CPW, HZ ? 3 : 2>(smem + (kk % S) * stage_bytes, ginfo, p, nt * 8, kk,
+                                             p.L * static_cast<long long>(ES), warp, lane);
+                cp_async_commit();
+            }
+        }
+    };
+    auto align_stage = [&](int kk) {
+        if constexpr (GA) {
+            cp_async_wait<0>();
+            __syncwarp();
+            gather_align<CPW, HZ ? 3 : 2>(smem + (kk % S) * stage_bytes, smem + ((kk + 1) % S) * stage_bytes, ginfo,
+                                          p, nt * 8, min(TC, L32 - kk * TC) * ES, warp, lane);
+        }
+    };
+    issue_stage(0);
+    issue_stage(1);
+    issue_stage(2);
     bool alive = wait_full(0, 0, 0);
     if (alive) {
+        align_stage(0);
         conv_stage(smem, 0);
         prologue(st, 0, 0, spA);
     }
@@ -458,6 +590,7 @@ __device__ __forceinline__ void seq_consumer(uint8_t* smem, uint64_t* full_bar, 
                 const int sn = slot + 1 == S ? 0 : slot + 1;
                 alive = wait_full(sn, slot + 1 == S ? parity ^ 1u : parity, k + 1);
                 if (alive) {
+                    align_stage(k + 1);
                     conv_stage(smem + sn * stage_bytes, tk + TC);
                     prologue(smem + sn * stage_bytes, 0, tk + TC, spA);
                 }
@@ -469,6 +602,7 @@ __device__ __forceinline__ void seq_consumer(uint8_t* smem, uint64_t* full_bar, 
         // The stage is consumed: release it to the producer.
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty_bar[slot]);
+        issue_stage(k + 3);  // (into the slot of stage k + 3 - S, which this warp is done with)
         if (++slot == S) {
             slot = 0;
             parity ^= 1u;
@@ -501,7 +635,7 @@ __device__ __forceinline__ void seq_consumer(uint8_t* smem, uint64_t* full_bar, 
         }
 }
 
-template <typename IO, int G, int CPL, int S, bool ZOH = false, bool CONV = false, bool CK = false>
+template <typename IO, int G, int CPL, int S, bool ZOH = false, bool CONV = false, bool CK = false, bool GA = false>
 __global__ void __launch_bounds__((SeqCfg<IO, G, CPL>::kMaxWarps + 1) * 32, 1)
 scan_fwd_seq_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_dl,
                     const __grid_constant__ CUtensorMap map_z, const __grid_constant__ CUtensorMap map_bc,
@@ -509,6 +643,7 @@ scan_fwd_seq_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_cons
     using Cfg = SeqCfg<IO, G, CPL>;
     constexpr int TC = Cfg::kTC, TPW = Cfg::kTPW;
     static_assert(S >= 2 && S <= 8, "ring depth");
+    static_assert(!GA || (S >= 3 && CPL == 1), "gathered rows: copies run three stages ahead of the scan");
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t full_bar[S], empty_bar[S];
@@ -518,6 +653,7 @@ scan_fwd_seq_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_cons
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
     const int stage_bytes = Cfg::stage_bytes(p.max_tiles);
+    uint64_t* ginfo = reinterpret_cast<uint64_t*>(smem + S * stage_bytes);  // (GA)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int producer_warp = blockDim.x / 32 - 1;
     const int L32 = static_cast<int>(p.L);  // the host launches this kernel for L < 2^31 - 1024 only
@@ -546,18 +682,27 @@ scan_fwd_seq_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_cons
             abort_flag = 0;
             mbar_fence_init();
         }
+        if constexpr (GA) {
+            const int rows = nt * 8;
+            const int j0 = static_cast<int>(r_begin - static_cast<long long>(b_first) * p.tiles_per_batch);
+            for (int q = threadIdx.x; q < rows * (p.has_z ? 3 : 2); q += blockDim.x)
+                ginfo[q] = gather_row_info<IO>(p, q, rows, j0, b_first);
+        }
         __syncthreads();
 
         if (warp == producer_warp) {
             // ------------------------------------------------------------ producer
             if (lane == 0) {
                 if (r_begin == t_begin) {
-                    tma_prefetch_map(&map_u);
-                    tma_prefetch_map(&map_dl);
+                    if constexpr (!GA) {
+                        tma_prefetch_map(&map_u);
+                        tma_prefetch_map(&map_dl);
+                        if (p.has_z) tma_prefetch_map(&map_z);
+                    }
                     tma_prefetch_map(&map_bc);
-                    if (p.has_z) tma_prefetch_map(&map_z);
                 }
-                const uint32_t bytes = nt * (p.has_z ? 3u : 2u) * Cfg::kTileBytes + nb * Cfg::kBC;
+                // (GA: the consumer warps copy u / delta / z themselves)
+                const uint32_t bytes = (GA ? 0u : nt * (p.has_z ? 3u : 2u) * Cfg::kTileBytes) + nb * Cfg::kBC;
                 for (int k = 0; k < nstages; ++k) {
                     const int s = k % S;
                     if (k >= S && !mbar_wait_sleep(&empty_bar[s], ((k / S) - 1) & 1, p.wait_limit)) {
@@ -576,7 +721,7 @@ scan_fwd_seq_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_cons
                     }
                     fence_proxy_async_smem();
                     mbar_arrive_expect_tx(&full_bar[s], bytes);
-                    for (int j = 0; j < nt; ++j) {
+                    for (int j = 0; j < (GA ? 0 : nt); ++j) {
                         const long long tile = r_begin + j;
                         const int b = static_cast<int>(tile / p.tiles_per_batch);
                         const int dd = static_cast<int>(tile % p.tiles_per_batch) * 8;
@@ -595,11 +740,11 @@ scan_fwd_seq_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_cons
             }
         } else if (warp < nwarps) {
             if (p.has_z)
-                seq_consumer<IO, G, CPL, S, true, ZOH, CONV, CK>(smem, full_bar, empty_bar, &abort_flag, p, r_begin, nt,
-                                                             b_first, stage_bytes, nstages, L32);
+                seq_consumer<IO, G, CPL, S, true, ZOH, CONV, CK, GA>(smem, full_bar, empty_bar, &abort_flag, p, r_begin,
+                                                                 nt, b_first, stage_bytes, nstages, L32);
             else
-                seq_consumer<IO, G, CPL, S, false, ZOH, CONV, CK>(smem, full_bar, empty_bar, &abort_flag, p, r_begin, nt,
-                                                              b_first, stage_bytes, nstages, L32);
+                seq_consumer<IO, G, CPL, S, false, ZOH, CONV, CK, GA>(smem, full_bar, empty_bar, &abort_flag, p, r_begin,
+                                                                  nt, b_first, stage_bytes, nstages, L32);
         }
         // Every warp leaves the round before the barriers are re-initialised for the next.
         __syncthreads();

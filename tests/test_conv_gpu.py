@@ -59,16 +59,19 @@ def test_conv_scan_variants(cuda_device, io, algo, lanes):
 
 @pytest.mark.parametrize("io,L", [("bf16", 63), ("bf16", 1001), ("f32", 1001), ("bf16", 2047)])
 def test_conv_scan_unaligned_rows(cuda_device, io, L):
-    # rows of x that are not 16-byte multiples: x is staged in padded rows like u (u_out and
-    # y are stored element by element, the conv state out read from the caller's x)
+    # rows of x that are not 16-byte multiples: x is staged like u, by a padded copy (the
+    # default at this shape) or gathered by the kernel itself (the sequential kernel asked for
+    # explicitly); u_out and y are stored element by element, the conv state out read from the
+    # caller's x
     inp = workloads.scan_inputs(2, 72, L, io=io, seed=140 + L)
     conv = workloads.conv_inputs(2, 72, 4, seed=141, with_state=True)
-    y, last, u_out, st = _gpu_conv_scan(inp, conv)
     y_ref, last_ref, u_ref, x_next = _oracle_conv_scan(inp, conv)
-    assert_close(u_out, u_ref, io, f"conv L={L} u")
-    assert_close(y, y_ref, io, f"conv L={L} y")
-    assert_close(last, last_ref, io, f"conv L={L} last_state")
-    assert torch.equal(st.cpu().double(), torch.from_numpy(x_next)), "conv state out"
+    for opts in (dict(), dict(algo="sequential")):
+        y, last, u_out, st = _gpu_conv_scan(inp, conv, **opts)
+        assert_close(u_out, u_ref, io, f"conv L={L} {opts} u")
+        assert_close(y, y_ref, io, f"conv L={L} {opts} y")
+        assert_close(last, last_ref, io, f"conv L={L} {opts} last_state")
+        assert torch.equal(st.cpu().double(), torch.from_numpy(x_next)), f"conv state out {opts}"
 
 
 @pytest.mark.parametrize("K", [1, 2, 3])

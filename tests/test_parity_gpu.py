@@ -56,18 +56,40 @@ def test_forward_edge_lengths(cuda_device, L):
 
 
 @pytest.mark.parametrize("io,L", [("f32", 1001), ("f32", 1002), ("bf16", 1001), ("bf16", 1004)])
-def test_forward_unaligned_rows_padded(cuda_device, io, L):
-    # L * sizeof(element) not a multiple of 16: u, delta, z are staged into padded rows in the
-    # workspace and the sequential kernel runs on them (also with the zero-order hold)
+def test_forward_unaligned_rows(cuda_device, io, L):
+    # L * sizeof(element) not a multiple of 16 (every row a different offset from the 16-byte
+    # grid): at this small shape the default copies u, delta, z into padded rows in the
+    # workspace; the sequential kernel requested explicitly gathers the rows itself (4 and 8
+    # lanes per channel), and 2 lanes per channel fall back to the padded copy.
     inp = workloads.scan_inputs(2, 100, L, io=io, seed=70 + L)
     check_forward(inp, what=f"padded rows {io} L={L}")
-    check_forward(inp, algo="sequential", lanes_per_channel=4, what=f"padded rows {io} L={L} 4 lanes")
+    check_forward(inp, algo="sequential", lanes_per_channel=4, what=f"gathered rows {io} L={L} 4 lanes")
+    check_forward(inp, algo="sequential", what=f"gathered rows {io} L={L}")
+    if io == "bf16":
+        check_forward(inp, algo="sequential", lanes_per_channel=8, what=f"gathered rows {io} L={L} 8 lanes")
+    check_forward(inp, algo="sequential", lanes_per_channel=2, what=f"padded rows {io} L={L} 2 lanes")
+
+
+@pytest.mark.parametrize("L", [1, 7, 9, 63, 65, 127, 129, 193])
+def test_forward_gathered_rows_short_and_ragged(cuda_device, L):
+    # gathered rows around the stage length (64 bf16 steps) and the copies one stage past
+    # the last; 20 channels (a partial 8-channel tile), with and without the z gate
+    for with_z in (True, False):
+        inp = workloads.scan_inputs(3, 20, L, io="bf16", seed=80 + L, with_z=with_z)
+        check_forward(inp, algo="sequential", what=f"gathered rows L={L} z={with_z}")
 
 
 def test_forward_unaligned_headline_full_size(cuda_device):
-    # the Mamba-2.8B layer shape one step short of 2048: every row starts 2 bytes off the last
+    # the Mamba-2.8B layer shape one step short of 2048: every row starts 2 bytes off the last.
+    # The default gathers the rows in the kernel at this shape.  Storing checkpoints takes the
+    # padded copy instead; with the same lanes per channel both stage the same values and run
+    # the same arithmetic, so y and the final state agree bit for bit.
     inp = workloads.scan_inputs(4, 5120, 2047, io="bf16", seed=71)
     check_forward(inp, what="b4 d5120 L2047")
+    y_ga, last_ga = gpu_forward(inp, lanes_per_channel=4)
+    ck = torch.empty(4, (2047 + 7) // 8, 5120, 16, device="cuda")
+    y_pad, last_pad = gpu_forward(inp, lanes_per_channel=4, checkpoints=ck)
+    assert torch.equal(y_ga, y_pad) and torch.equal(last_ga, last_pad)
 
 
 def test_forward_empty_sequence_gives_zero_state(cuda_device):

@@ -53,6 +53,15 @@ def test_zoh_forward_variants(cuda_device, io, algo, lanes):
     check_zoh(inp, f"zoh {algo}/{lanes}/{io}", algo=algo, lanes_per_channel=lanes)
 
 
+@pytest.mark.parametrize("io,lanes", [("f32", 4), ("bf16", 4), ("bf16", 8)])
+def test_zoh_unaligned_rows(cuda_device, io, lanes):
+    # rows that are not 16-byte multiples: gathered by the sequential kernel itself, or (by
+    # default at this small shape) staged from a padded copy
+    inp = workloads.scan_inputs(2, 40, 333, io=io, dt_min=1e-5, dt_max=1.0, seed=90)
+    check_zoh(inp, f"zoh gathered rows {io}/{lanes}", algo="sequential", lanes_per_channel=lanes)
+    check_zoh(inp, f"zoh padded rows {io}", lanes_per_channel=lanes)
+
+
 def test_zoh_tiny_steps_fp32(cuda_device):
     # every Delta A far below 1/16: the series branch only, where exp(Delta A) - 1 would cancel
     inp = workloads.scan_inputs(1, 64, 512, io="f32", dt_min=1e-7, dt_max=1e-5, seed=72)
