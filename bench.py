@@ -408,8 +408,9 @@ def measure_decode(ssm, stream, pk, steps=None):
 
 
 def measure_unaligned(ssm, stream, pk, steps=10):
-    """Headline shape at L = 2047 (rows not a multiple of 16 bytes: u, delta, z are staged
-    into padded rows in the workspace) against L = 2048 on the same inputs' distribution."""
+    """Headline shape at L = 2047 (rows not a multiple of 16 bytes, which TMA cannot address:
+    at this shape the sequential kernel gathers them itself) against L = 2048 on the same
+    inputs' distribution."""
     out = {"workload": "mamba2p8b_b4_d5120", "unit": UNIT}
     for L in (2048, 2047):
         inp = workloads.scan_inputs(4, 5120, L, io="bf16", seed=1002)
@@ -714,7 +715,7 @@ def run_gpu(args, world, rank, local):
 
 
 def run_profile_workload(args):
-    """Run only the long-sequence scan or the decode chain (for profiler captures)."""
+    """Run only one of the extra workloads (for profiler captures)."""
     import selective_state_space_16_b200 as ssm
     torch.cuda.set_device(0)
     stream = torch.cuda.Stream()
@@ -725,6 +726,8 @@ def run_profile_workload(args):
         out = measure_backward(ssm, stream, pk, steps=args.steps)
     elif args.workload == "wide":
         out = measure_wide(ssm, stream, pk, steps=args.steps, only=args.dstate)
+    elif args.workload == "unaligned":
+        out = measure_unaligned(ssm, stream, pk, steps=args.steps)
     else:
         w = workloads.WORKLOADS[4]
         out = measure_decode(ssm, stream, pk, steps=args.steps)
@@ -741,8 +744,10 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-extra", action="store_true")
-    ap.add_argument("--workload", default="headline", choices=["headline", "long", "decode", "backward", "wide"],
-                    help="profiling runs: 'long' / 'decode' / 'backward' / 'wide' run only that workload a few times")
+    ap.add_argument("--workload", default="headline",
+                    choices=["headline", "long", "decode", "backward", "wide", "unaligned"],
+                    help="profiling runs: 'long' / 'decode' / 'backward' / 'wide' / 'unaligned' run only that "
+                         "workload a few times")
     ap.add_argument("--dstate", type=int, default=None, choices=[32, 64, 128, 256],
                     help="with --workload wide: that d_state only")
     args = ap.parse_args()
