@@ -190,71 +190,108 @@ __device__ __forceinline__ uint64_t gather_row_info(const SeqParams& p, int q, i
                                                  static_cast<long long>(IoTraits<IO>::kBytes));
 }
 
+// Shared-memory accesses of the gathering code by 32-bit shared-window address.
+__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint64_t lds_u64(uint32_t a) {
+    uint64_t v;
+    asm volatile("ld.shared.u64 %0, [%1];" : "=l"(v) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint2 lds_v2(uint32_t a) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ void sts_v4(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
+}
+__device__ __forceinline__ void cp_async_16_to(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+
 // Consumer warp `warp`: copy its rows' windows of stage k (0 <= k <= the number of stages) into
-// the slot st.  row_bytes = L * sizeof(IO).
+// the slot at shared address st (info: shared address of the row words; row_bytes = L *
+// sizeof(IO)).  Pass r0 handles rows r0 .. r0 + 3 of the warp (tensor r0 / CPW), lane (sub, c)
+// chunk c of row r0 + sub.
 template <int CPW, int NT>
-__device__ __forceinline__ void gather_copy(uint8_t* st, const uint64_t* info, const SeqParams& p, int rows,
-                                            long long k, long long row_bytes, int warp, int lane) {
+__device__ __forceinline__ void gather_copy(uint32_t st, uint32_t info, const SeqParams& p, int rows, int k,
+                                            long long row_bytes, int warp, int lane) {
     const int sub = lane >> 3, c = lane & 7;
-    const int tile_area = p.max_tiles * 1024;
+    const uint32_t tile_area = static_cast<uint32_t>(p.max_tiles) * 1024u;
+    const int first = warp * CPW + sub;  // the lane's channel of the round in pass 0
+    const uint32_t dst0 = st + first * 128 + c * 16;
+    const uint32_t inf0 = info + first * 8;
+    const long long rem = row_bytes - static_cast<long long>(k) * 128;  // row bytes from the window's t = 128k/size
+    const long long kc = static_cast<long long>(k) * 128 + c * 16;
+    const bool whole = rem >= 144;  // every chunk of every window holds step bytes (warp-uniform)
     const uint8_t* any = static_cast<const uint8_t*>(p.u_rows);  // (zero-fill: not read)
+    // (every row a warp of a GA kernel covers is one of the round's: one channel per lane, and
+    // the warps cover whole 8-channel tiles)
 #pragma unroll
     for (int r0 = 0; r0 < CPW * NT; r0 += 4) {
-        const int tq = r0 / CPW;  // (CPW is a multiple of 4: the 4 rows of a pass share a tensor)
-        const int cl = warp * CPW + r0 % CPW + sub;
-        if (cl < rows && dcheck(p.hdr, tq * tile_area + cl * 128 + 128 <= 3 * tile_area, kSiteSeqTma, cl)) {
-            const uint64_t at = info[tq * rows + cl];
-            const long long sh = static_cast<long long>(at & 15u);
-            const bool need = at != 0 && k * 128 - sh + c * 16 < row_bytes;  // the chunk holds a step byte
-            const uint8_t* src = need ? reinterpret_cast<const uint8_t*>(at - sh) + k * 128 + c * 16 : any;
-            cp_async_16(st + tq * tile_area + cl * 128 + c * 16, src, need ? 16u : 0u);
+        const int tq = r0 / CPW, rc = r0 % CPW;  // (CPW is a multiple of 4: a pass stays in one tensor)
+        if (dcheck(p.hdr, first + rc < rows, kSiteSeqTma, first + rc)) {
+            const uint64_t at = lds_u64(inf0 + (tq * rows + rc) * 8);
+            const int sh = static_cast<int>(at & 15u);
+            const bool need = at != 0 && (whole || c * 16 - sh < rem);  // the chunk holds a step byte
+            const uint8_t* src = need ? reinterpret_cast<const uint8_t*>((at & ~uint64_t(15)) + kc) : any;
+            cp_async_16_to(dst0 + tq * tile_area + rc * 128, src, need ? 16u : 0u);
         }
     }
 }
 
-// Consumer warp `warp`: shift its rows of the landed stage st into place (nx_st: the slot of
-// the next stage, also landed; nbytes: bytes of the stage's steps in a row).  Lane c reads the
-// 24 bytes from window byte 16c + (sh & 8) as three 8-byte words (those past byte 128 from the
-// next stage's window), keeps the words from (sh & 4) on and funnel-shifts by sh & 3.
+// Consumer warp `warp`: shift its rows of the landed stage at shared address st into place (nx_st:
+// the slot of the next stage, also landed; nbytes: bytes of the stage's steps in a row).  Lane
+// c reads the 24 bytes from window byte 16c + (sh & 8) as three 8-byte words (those from byte
+// 128 on are the next stage's window), keeps the words from (sh & 4) on and funnel-shifts by
+// sh & 3.
 template <int CPW, int NT>
-__device__ __forceinline__ void gather_align(uint8_t* st, const uint8_t* nx_st, const uint64_t* info,
-                                             const SeqParams& p, int rows, int nbytes, int warp, int lane) {
+__device__ __forceinline__ void gather_align(uint32_t st, uint32_t nx_st, uint32_t info, const SeqParams& p, int rows,
+                                             int nbytes, int warp, int lane) {
     const int sub = lane >> 3, c = lane & 7;
     const int keep = nbytes - c * 16;  // bytes of this lane's chunk inside the row's steps
-    const int tile_area = p.max_tiles * 1024;
-    const long long nx_delta = nx_st - st;
+    const uint32_t tile_area = static_cast<uint32_t>(p.max_tiles) * 1024u;
+    const int first = warp * CPW + sub;
+    const uint32_t row0 = st + first * 128;
+    const uint32_t inf0 = info + first * 8;
+    const bool is7 = c == 7;
+    const uint32_t nxd = nx_st - st - 128u;  // window byte 128 + j of a row -> byte j of its next window
+    const uint32_t add2 = is7 ? nxd : 0u;
+    const bool last = nbytes < 128;  // (warp-uniform) the row's last window: zero the steps past L
 #pragma unroll
     for (int r0 = 0; r0 < CPW * NT; r0 += 4) {
-        const int tq = r0 / CPW;
-        const int cl = warp * CPW + r0 % CPW + sub;  // channel of the round
-        const bool mine = cl < rows && dcheck(p.hdr, tq * tile_area + cl * 128 + 128 <= 3 * tile_area, kSiteSeqTma, cl);
-        const uint64_t at = mine ? info[tq * rows + cl] : 0;
-        const uint32_t sh = static_cast<uint32_t>(at & 15u);
-        uint8_t* rowp = st + tq * tile_area + cl * 128;
-        uint2 w[3] = {make_uint2(0u, 0u), make_uint2(0u, 0u), make_uint2(0u, 0u)};
+        const int tq = r0 / CPW, rc = r0 % CPW;
+        const bool mine = dcheck(p.hdr, first + rc < rows, kSiteSeqTma, first + rc);
+        const uint32_t rowp = row0 + tq * tile_area + rc * 128;
+        uint32_t sh = 0;
+        uint2 w0 = make_uint2(0u, 0u), w1 = w0, w2 = w0;
         if (mine) {
-#pragma unroll
-            for (int i = 0; i < 3; ++i) {
-                const int b = c * 16 + static_cast<int>(sh & 8u) + 8 * i;  // window byte (8-aligned)
-                const uint8_t* src = rowp + (b < 128 ? b : b - 128 + nx_delta);
-                w[i] = *reinterpret_cast<const uint2*>(src);
-            }
+            sh = lds_u32(inf0 + (tq * rows + rc) * 8) & 15u;  // (the row word's low half)
+            const uint32_t la = rowp + c * 16 + (sh & 8u);
+            const uint32_t add1 = (is7 && (sh & 8u)) ? nxd : 0u;
+            w0 = lds_v2(la);
+            w1 = lds_v2(la + 8 + add1);
+            w2 = lds_v2(la + 16 + add2);
         }
         __syncwarp();  // every lane has read its words before any lane rewrites the row
-        const uint32_t x[6] = {w[0].x, w[0].y, w[1].x, w[1].y, w[2].x, w[2].y};
+        const uint32_t x[6] = {w0.x, w0.y, w1.x, w1.y, w2.x, w2.y};
         uint32_t u5[5], o[4];
 #pragma unroll
         for (int i = 0; i < 5; ++i) u5[i] = (sh & 4u) ? x[i + 1] : x[i];
 #pragma unroll
         for (int m = 0; m < 4; ++m) o[m] = __funnelshift_r(u5[m], u5[m + 1], (sh & 3u) * 8u);
-        if (keep < 16) {
+        if (last) {
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 const int kb = keep - 4 * m;
                 o[m] = kb >= 4 ? o[m] : kb <= 0 ? 0u : o[m] & ((1u << (8 * kb)) - 1u);
             }
         }
-        if (mine) *reinterpret_cast<uint4*>(rowp + ((c ^ (cl & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+        if (mine) sts_v4(rowp + ((c ^ ((first + rc) & 7)) << 4), o[0], o[1], o[2], o[3]);
     }
     __syncwarp();
 }
@@ -536,6 +573,9 @@ __device__ __forceinline__ void seq_consumer(uint8_t* smem, uint64_t* full_bar, 
                        kSiteSeqY, t0)) {
                 if (p.y_vec && t0 + PER <= L32) {
                     store_run<IO, PER>(yrow[c] + t0, yo);
+                } else if (GA && t0 + PER <= L32) {  // (rows not 16-byte aligned: element stores)
+#pragma unroll
+                    for (int r = 0; r < PER; ++r) yrow[c][t0 + r] = IoTraits<IO>::from_f32(yo[r]);
                 } else {
 #pragma unroll
                     for (int r = 0; r < PER; ++r)
@@ -551,11 +591,12 @@ __device__ __forceinline__ void seq_consumer(uint8_t* smem, uint64_t* full_bar, 
     uint32_t parity = 0;
     // GA: this warp's rows, copied three stages ahead (the copies of stage k land in a cp.async
     // group of their own), shifted into place when a stage and the next have landed
-    const uint64_t* ginfo = reinterpret_cast<const uint64_t*>(smem + S * stage_bytes);
+    const uint32_t smem_s = smem_u32(smem);
+    const uint32_t ginfo = smem_s + S * stage_bytes;
     auto issue_stage = [&](int kk) {
         if constexpr (GA) {
             if (kk <= nstages) {  // (stage nstages: the chunks past the last window)
-                gather_copy<CPW, HZ ? 3 : 2>(smem + (kk % S) * stage_bytes, ginfo, p, nt * 8, kk,
+                gather_copy<CPW, HZ ? 3 : 2>(smem_s + (kk % S) * stage_bytes, ginfo, p, nt * 8, kk,
                                              p.L * static_cast<long long>(ES), warp, lane);
                 cp_async_commit();
             }
@@ -565,8 +606,8 @@ __device__ __forceinline__ void seq_consumer(uint8_t* smem, uint64_t* full_bar, 
         if constexpr (GA) {
             cp_async_wait<0>();
             __syncwarp();
-            gather_align<CPW, HZ ? 3 : 2>(smem + (kk % S) * stage_bytes, smem + ((kk + 1) % S) * stage_bytes, ginfo,
-                                          p, nt * 8, min(TC, L32 - kk * TC) * ES, warp, lane);
+            gather_align<CPW, HZ ? 3 : 2>(smem_s + (kk % S) * stage_bytes, smem_s + ((kk + 1) % S) * stage_bytes,
+                                          ginfo, p, nt * 8, min(TC, L32 - kk * TC) * ES, warp, lane);
         }
     };
     issue_stage(0);
