@@ -34,7 +34,10 @@
 // boxes use the 128-byte swizzle, so the per-lane 16-byte reads of one column hit
 // distinct banks; B/C are read as broadcasts.  The kernel may be launched as a
 // programmatic dependent of the B/C transpose before it: the producer waits for that
-// grid only before its first B/C copy.
+// grid only before its first B/C copy.  Rows whose byte length is not a multiple of 16
+// cannot be staged by TMA: the GA kernels leave u / delta / z to the consumer warps, which
+// copy their own rows' 16-byte-aligned windows and shift them into the same tile layout
+// (gather_copy, gather_align); the producer then streams only the B/C rows.
 //
 // Checkpoints (CK kernels, for the backward: [Tech] 四.1, keep a little in the forward
 // pass): after every group of steps that ends on a multiple of 8, each lane also stores
