@@ -76,7 +76,11 @@ ssm_status_t launch_forward(const FwdArgs& a, const ssm_fwd_options_t& o) {
         FwdArgs g = a;
         g.y_vec = 0;
         g.pdl = true;  // launched right after the B/C pack
-        return launch_seq_gather<IO>(g, o);
+        const ssm_status_t sg = launch_seq_gather<IO>(g, o);
+        if (sg != SSM_ERR_UNSUPPORTED) return sg;
+        // no gathering plan fits (shared memory): the padded copy, or without room for it the
+        // direct kernel
+        return a.pad_ok ? launch_forward_padded<IO>(a, o) : launch_direct<IO>(a);
     }
     if (!tma_ok) algo = SSM_ALGO_DIRECT;
     if (a.ckpt && algo == SSM_ALGO_DIRECT) return SSM_ERR_UNSUPPORTED;  // checkpoints: sequential kernel only

@@ -44,12 +44,17 @@ SeqPlan plan_seq(const FwdArgs& a) {
     // (tiles are handed out in whole-warp units of kTPW tiles).
     const int tiles_cap = std::min(Cfg::kMaxWarps * Cfg::kCPW / 8 / Cfg::kTPW * Cfg::kTPW,
                                    pl.tiles_per_batch + Cfg::kTPW);
-    for (int per_sm = 1; per_sm <= 2 && !pl.ok; ++per_sm) {
+    // Attempts: one CTA per SM in one round; two per SM (several rounds when needed); one per SM
+    // in several rounds (shapes with more tiles than two CTAs' warps hold, e.g. b8 d5120, where
+    // two CTAs of that size do not fit an SM's registers; the GA kernels' ring needs three
+    // stages, which two CTAs per SM do not leave room for).
+    for (int at = 0; at < 3 && !pl.ok; ++at) {
+        const int per_sm = at == 1 ? 2 : 1;
         const long long ctas = std::min<long long>(pl.total_tiles, static_cast<long long>(a.sm_count) * per_sm);
         const long long units = pl.total_tiles / Cfg::kTPW;  // tiles in whole-warp units
         int mt = static_cast<int>((units + ctas - 1) / ctas) * Cfg::kTPW;
         if (mt > tiles_cap) {
-            if (per_sm == 1) continue;
+            if (at == 0) continue;
             mt = tiles_cap;  // several rounds per CTA
         }
         const int budget = (228 * 1024) / per_sm - 1024 - 256;  // per-CTA reserve and static barriers

@@ -654,6 +654,7 @@ __device__ __forceinline__ void seq_consumer(uint8_t* smem, uint64_t* full_bar, 
         st = smem + slot * stage_bytes;
     }
 
+    if constexpr (GA) cp_async_wait<0>();  // (after a timeout: no copy may land in the next round)
     if constexpr (CONV) {
         // the last conv_k - 1 inputs (from x, or from conv_in when the sequence is shorter)
         const int K = p.conv_k;

@@ -70,6 +70,18 @@ def test_forward_unaligned_rows(cuda_device, io, L):
     check_forward(inp, algo="sequential", lanes_per_channel=2, what=f"padded rows {io} L={L} 2 lanes")
 
 
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+@pytest.mark.parametrize("L", [160, 131])
+def test_forward_more_tiles_than_one_round(cuda_device, io, L):
+    # b8 d5120 (40960 channels): more 8-channel tiles than the CTAs' warps hold at once, so each
+    # CTA stages them in several rounds; TMA-staged rows (L 160) and gathered rows (L 131, the
+    # row words set up again for every round); checked on sampled channels
+    inp = workloads.scan_inputs(8, 5120, L, io=io, seed=95)
+    rng = np.random.default_rng(95)
+    channels = np.sort(rng.choice(8 * 5120, 512, replace=False))
+    check_forward(inp, channels=channels, what=f"b8 d5120 L{L} {io}, several rounds")
+
+
 @pytest.mark.parametrize("L", [1, 7, 9, 63, 65, 127, 129, 193])
 def test_forward_gathered_rows_short_and_ragged(cuda_device, L):
     # gathered rows around the stage length (64 bf16 steps) and the copies one stage past
