@@ -121,8 +121,9 @@ def use_debug_library():
     if not os.path.exists(DEBUG_LIB_PATH):
         raise ImportError(f"{DEBUG_LIB_PATH} is missing; build it with build.py --debug")
     debug = _declare(ctypes.CDLL(DEBUG_LIB_PATH))
+    base = load()  # (before taking the lock, which load() takes itself)
     with _lock:
-        saved = load() if _lib is None else _lib
+        saved = _lib if _lib is not None else base
         _lib = debug
     try:
         yield debug

@@ -62,6 +62,24 @@ def test_debug_library_builds_and_exports_every_declared_symbol():
     assert dbg.ssm_abi_version() == 3
 
 
+def test_debug_library_switch_as_first_call():
+    # Entering use_debug_library() before anything else has loaded the release library must
+    # not deadlock (it loads that library too, and both take the module's lock); run in a
+    # fresh process, bounded by a timeout.
+    if not os.path.exists(binding.DEBUG_LIB_PATH):
+        pytest.skip("debug library not built")
+    import subprocess
+    import sys
+    code = ("from selective_state_space_16_b200 import binding\n"
+            "with binding.use_debug_library() as lib:\n"
+            "    assert binding.load() is lib\n"
+            "assert binding.load() is not lib\n"
+            "print('switched')\n")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and "switched" in r.stdout, r.stderr
+
+
 def test_workspace_size(lib):
     f = binding.ssm_selective_scan_workspace_size
     assert f(4, 5120, 16, 2048) % 256 == 0
