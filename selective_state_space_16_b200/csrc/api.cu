@@ -28,9 +28,10 @@ template <typename IO>
 constexpr int chunk_steps() { return 128 / static_cast<int>(sizeof(IO)); }
 
 // Rows of u / delta / z (or x, with the conv prologue) whose byte length is not a multiple of
-// 16: TMA cannot address them, so they are copied into padded rows in the workspace and the
-// sequential kernel stages those; y (and u_out) go straight to the caller's rows with element
-// stores.
+// 16, which TMA cannot address, staged the second of two ways (the first: the GA kernels gather
+// them themselves, see launch_forward): copied into padded rows in the workspace, which the
+// sequential kernel then stages with TMA; y (and u_out) go straight to the caller's rows with
+// element stores.
 template <typename IO>
 ssm_status_t launch_forward_padded(const FwdArgs& a, const ssm_fwd_options_t& o) {
     constexpr int64_t E = 16 / static_cast<int64_t>(sizeof(IO));
